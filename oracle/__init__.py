@@ -1,0 +1,163 @@
+"""CPU oracle for the FP8 W8A8 linear layer (ctypes wrapper over fp8_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: tests/, __graft_entry__.smoke() and bench.py's
+CPU-baseline leg are the only callers.  The GPU product path never imports
+this package and must not be routed through it.
+
+Arrays are numpy: bf16 tensors travel as their uint16 bit patterns, codes as
+uint8, scales as float32.  See fp8_oracle.c for what each function computes
+and which page passage it follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp8_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+CHANNEL_TOKEN = 0
+BLOCK128 = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile fp8_oracle.c into liboracle.so (gcc, no fast-math, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+               "-fno-fast-math", "-ffp-contract=off", "-fvisibility=hidden",
+               _SRC, "-o", _LIB + ".tmp", "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int64
+        _lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+        _lib.orc_e4m3_decode.restype = ctypes.c_double
+        _lib.orc_e5m2_decode.argtypes = [ctypes.c_uint8]
+        _lib.orc_e5m2_decode.restype = ctypes.c_double
+        _lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        _lib.orc_e4m3_encode.restype = ctypes.c_uint8
+        _lib.orc_e4m3_encode_n.argtypes = [P, I, P]
+        _lib.orc_e4m3_encode_n.restype = None
+        for f in ("orc_quant_rows", "orc_quant_groups128", "orc_quant_blocks128"):
+            getattr(_lib, f).argtypes = [P, I, I, I, P, I, P]
+            getattr(_lib, f).restype = None
+        _lib.orc_linear.argtypes = [P, P, P, P, I, I, I, I, I, ctypes.c_int, P]
+        _lib.orc_linear.restype = None
+        _lib.orc_linear_at.argtypes = [P, P, P, P, I, I, I, ctypes.c_int, P, P, I, P]
+        _lib.orc_linear_at.restype = None
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bits(x) -> np.ndarray:
+    """bf16 torch tensor or uint16 array -> C-contiguous uint16 numpy array."""
+    if hasattr(x, "view") and hasattr(x, "dtype") and str(x.dtype) == "torch.bfloat16":
+        import torch
+        x = x.detach().cpu().contiguous().view(torch.uint16).numpy()
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    return x
+
+
+def e4m3_decode(code: int) -> float:
+    return lib().orc_e4m3_decode(int(code) & 0xFF)
+
+
+def e5m2_decode(code: int) -> float:
+    return lib().orc_e5m2_decode(int(code) & 0xFF)
+
+
+def e4m3_encode(v: float) -> int:
+    return int(lib().orc_e4m3_encode(float(v)))
+
+
+def e4m3_encode_array(v: np.ndarray) -> np.ndarray:
+    """Encode each float32 of v (scale 1) through the oracle's encoder."""
+    v = np.ascontiguousarray(v, dtype=np.float32).ravel()
+    out = np.empty(v.shape, np.uint8)
+    lib().orc_e4m3_encode_n(_p(v), v.size, _p(out))
+    return out
+
+
+def quant_rows(x):
+    """One amax/448 scale per row.  x: bf16 [R, K] -> (codes u8 [R, K], scales f32 [R])."""
+    xb = _bits(x)
+    R, K = xb.shape
+    q = np.empty((R, K), np.uint8)
+    s = np.empty((R,), np.float32)
+    lib().orc_quant_rows(_p(xb), R, K, K, _p(q), K, _p(s))
+    return q, s
+
+
+def quant_groups128(x):
+    """One scale per 128-group of each row.  -> (codes [M, K], scales [M, K/128])."""
+    xb = _bits(x)
+    M, K = xb.shape
+    assert K % 128 == 0
+    q = np.empty((M, K), np.uint8)
+    s = np.empty((M, K // 128), np.float32)
+    lib().orc_quant_groups128(_p(xb), M, K, K, _p(q), K, _p(s))
+    return q, s
+
+
+def quant_blocks128(w):
+    """One scale per 128x128 tile.  -> (codes [N, K], scales [ceil(N/128), K/128])."""
+    wb = _bits(w)
+    N, K = wb.shape
+    assert K % 128 == 0
+    q = np.empty((N, K), np.uint8)
+    s = np.empty(((N + 127) // 128, K // 128), np.float32)
+    lib().orc_quant_blocks128(_p(wb), N, K, K, _p(q), K, _p(s))
+    return q, s
+
+
+def quant_weight(w, mode: int):
+    return quant_rows(w) if mode == CHANNEL_TOKEN else quant_blocks128(w)
+
+
+def quant_act(x, mode: int):
+    return quant_rows(x) if mode == CHANNEL_TOKEN else quant_groups128(x)
+
+
+def linear(xq, xs, wq, ws, mode: int) -> np.ndarray:
+    """Exact layer output Y [M, N] (fp32) from codes and scales."""
+    xq = np.ascontiguousarray(xq, np.uint8)
+    wq = np.ascontiguousarray(wq, np.uint8)
+    xs = np.ascontiguousarray(xs, np.float32)
+    ws = np.ascontiguousarray(ws, np.float32)
+    M, K = xq.shape
+    N = wq.shape[0]
+    y = np.empty((M, N), np.float32)
+    lib().orc_linear(_p(xq), _p(xs), _p(wq), _p(ws), M, N, K, K, K, mode, _p(y))
+    return y
+
+
+def linear_at(xq, xs, wq, ws, mode: int, ms, ns) -> np.ndarray:
+    """Exact outputs Y[ms[i], ns[i]] only."""
+    xq = np.ascontiguousarray(xq, np.uint8)
+    wq = np.ascontiguousarray(wq, np.uint8)
+    xs = np.ascontiguousarray(xs, np.float32)
+    ws = np.ascontiguousarray(ws, np.float32)
+    ms = np.ascontiguousarray(ms, np.int64)
+    ns = np.ascontiguousarray(ns, np.int64)
+    K = xq.shape[1]
+    y = np.empty(ms.shape, np.float32)
+    lib().orc_linear_at(_p(xq), _p(xs), _p(wq), _p(ws), K, K, K, mode,
+                        _p(ms), _p(ns), ms.size, _p(y))
+    return y

@@ -1,0 +1,267 @@
+/*
+ * fp8_oracle.c -- plain CPU oracle for the FP8 W8A8 linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * CPU-baseline leg of bench.py may load this library.  The GPU library
+ * never links, includes or calls it, and it shares no code with the GPU
+ * path (no common headers, tables or helpers).
+ *
+ * What it computes, and where the pages say so:
+ *
+ *   [P1] "Llama 3 精读实录：FP8 量化与长上下文实测的完整记录", section 2.1
+ *        (两种 FP8 格式的本质区别): E4M3 = 4 exponent bits and 3 mantissa
+ *        bits, largest value 448; E5M2 = 5 and 2, largest 57344; inference
+ *        uses E4M3 for weights and activations.
+ *   [P2] "Llama-3.1-8B-Instruct-FP8-Dynamic" explainer, section "FP8 动态量化"
+ *        table: weights 8-bit float, one scale per output channel from a
+ *        minmax observer; input activations 8-bit float, dynamic, one scale
+ *        per token; lm_head not quantized.
+ *   [P4] "Llama-3.1-70B-FP8-Dynamic" explainer, section 1.2 (名字里的
+ *        "Dynamic"): the same scheme; FAQ Q2: activations quantized per token
+ *        at inference time.
+ *   [P5] "Llama-3.2-3B-Instruct-FP8-Block" explainer, quantization_config
+ *        table: weight block_structure [128, 128]; input activations in
+ *        dynamic groups of 128; lm_head ignored.
+ *
+ * Readings taken where the pages leave a step open (each listed in the
+ * design notes):
+ *   - E4M3 is the "FN" variant: no infinities, codes 0x7F/0xFF are NaN.  It is
+ *     the variant whose largest finite value is the 448 that [P1] prints.
+ *   - A symmetric minmax observer gives amax = max|x| over the unit and
+ *     scale s = amax / 448, one IEEE fp32 division.  amax == 0 gives s = 1.
+ *   - The code of x is E4M3(fl32(x / s)): an IEEE fp32 quotient, then the
+ *     nearest E4M3 value, ties to the even mantissa, saturating at +-448,
+ *     sign kept (a negative value that rounds to zero is -0, code 0x80).
+ *   - The layer output is y[m,n] = sum_k deq(xq[m,k]) * deq(wq[n,k]) with
+ *     deq(q) = E4M3value(q) * scale; block mode sums per 128-wide K slice
+ *     with that slice's two scales.  It is computed here EXACTLY: every finite
+ *     E4M3 value is an integer multiple of 2^-9, so the dot product of codes is
+ *     an exact int64 sum, scaled once in double and rounded to fp32.
+ *
+ * The E4M3 encoder is a nearest-value search over the table of the 127
+ * non-negative finite E4M3 values (built from the decoder), not bit
+ * manipulation: it is written to be independent of how a GPU converts.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORC_EXPORT __attribute__((visibility("default")))
+
+/* ---------------------------------------------------------------- formats */
+
+/* E4M3FN decode from the bit fields: s.eeee.mmm, exponent bias 7. */
+ORC_EXPORT double orc_e4m3_decode(uint8_t code) {
+    int s = (code >> 7) & 1;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;                 /* the only NaN pattern   */
+    if (e == 0) mag = ldexp((double)m, -9);            /* subnormal: m * 2^-9    */
+    else mag = ldexp(1.0 + m / 8.0, e - 7);            /* (1 + m/8) * 2^(e-7)    */
+    return s ? -mag : mag;
+}
+
+/* E5M2 decode (IEEE-like: exponent bias 15, inf and NaN at exponent 31).
+ * Used only to check the format facts [P1] prints. */
+ORC_EXPORT double orc_e5m2_decode(uint8_t code) {
+    int s = (code >> 7) & 1;
+    int e = (code >> 2) & 0x1F;
+    int m = code & 0x3;
+    double mag;
+    if (e == 31) mag = (m == 0) ? INFINITY : NAN;
+    else if (e == 0) mag = ldexp((double)m, -16);
+    else mag = ldexp(1.0 + m / 4.0, e - 15);
+    return s ? -mag : mag;
+}
+
+static double g_mag[127];     /* value of code c, c = 0x00 .. 0x7E, ascending */
+static int g_mag_ready = 0;
+
+static void build_mag_table(void) {
+    if (g_mag_ready) return;
+    for (int c = 0; c < 127; ++c) g_mag[c] = orc_e4m3_decode((uint8_t)c);
+    g_mag_ready = 1;
+}
+
+/* Nearest E4M3 code to a finite float: bisection for the two neighbouring
+ * table values, then the closer one; an exact tie goes to the code whose
+ * mantissa LSB (= code LSB) is 0.  Values beyond 448 have only one neighbour
+ * (448), which is saturation.  The sign bit is copied from v. */
+ORC_EXPORT uint8_t orc_e4m3_encode(float v) {
+    build_mag_table();
+    double a = fabs((double)v);
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    uint8_t c;
+    if (a >= g_mag[126]) {
+        c = 126;
+    } else {
+        int lo = 0, hi = 126;                 /* g_mag[lo] <= a < g_mag[hi] */
+        while (hi - lo > 1) {
+            int mid = (lo + hi) / 2;
+            if (g_mag[mid] <= a) lo = mid; else hi = mid;
+        }
+        double dl = a - g_mag[lo], dh = g_mag[hi] - a;
+        if (dl < dh) c = (uint8_t)lo;
+        else if (dh < dl) c = (uint8_t)hi;
+        else c = (uint8_t)((lo & 1) ? hi : lo);
+    }
+    return (uint8_t)(c | sign);
+}
+
+/* Encode n floats (scale 1), for sweeps over many values. */
+ORC_EXPORT void orc_e4m3_encode_n(const float* v, int64_t n, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_encode(v[i]);
+}
+
+static inline float bf16_to_float(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* ----------------------------------------------------------- quantization */
+
+/* Scale of one unit from its amax: s = fl32(amax / 448), or 1 when amax = 0. */
+static float scale_from_amax(float amax) {
+    volatile float num = amax;            /* keep it an IEEE single division */
+    if (amax == 0.0f) return 1.0f;
+    return num / 448.0f;
+}
+
+static inline uint8_t code_of(float x, float s) {
+    volatile float q = x / s;             /* fp32 quotient, RNE */
+    return orc_e4m3_encode(q);
+}
+
+/* One scale per row: per-token activations [P2, P4] and per-output-channel
+ * weights [P2] are the same operation on X[M,K] and on W[N,K].
+ * x: bf16 bits [rows, ld], q: [rows, ldq], s: [rows]. */
+ORC_EXPORT void orc_quant_rows(const uint16_t* x, int64_t rows, int64_t K, int64_t ld,
+                               uint8_t* q, int64_t ldq, float* s) {
+    for (int64_t r = 0; r < rows; ++r) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(bf16_to_float(x[r * ld + k]));
+            if (a > amax) amax = a;
+        }
+        float sr = scale_from_amax(amax);
+        s[r] = sr;
+        for (int64_t k = 0; k < K; ++k) q[r * ldq + k] = code_of(bf16_to_float(x[r * ld + k]), sr);
+    }
+}
+
+/* One scale per 128 consecutive input features of each token [P5].
+ * K must be a multiple of 128.  s: [M, K/128] row-major. */
+ORC_EXPORT void orc_quant_groups128(const uint16_t* x, int64_t M, int64_t K, int64_t ld,
+                                    uint8_t* q, int64_t ldq, float* s) {
+    int64_t G = K / 128;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t g = 0; g < G; ++g) {
+            float amax = 0.0f;
+            for (int64_t k = g * 128; k < g * 128 + 128; ++k) {
+                float a = fabsf(bf16_to_float(x[m * ld + k]));
+                if (a > amax) amax = a;
+            }
+            float sg = scale_from_amax(amax);
+            s[m * G + g] = sg;
+            for (int64_t k = g * 128; k < g * 128 + 128; ++k)
+                q[m * ldq + k] = code_of(bf16_to_float(x[m * ld + k]), sg);
+        }
+    }
+}
+
+/* One scale per 128 x 128 tile of W[N,K] [P5, block_structure [128, 128]].
+ * K must be a multiple of 128; the last row-tile may be shorter than 128
+ * (amax over the rows that exist).  s: [ceil(N/128), K/128] row-major. */
+ORC_EXPORT void orc_quant_blocks128(const uint16_t* w, int64_t N, int64_t K, int64_t ld,
+                                    uint8_t* q, int64_t ldq, float* s) {
+    int64_t NB = (N + 127) / 128, KB = K / 128;
+    for (int64_t nb = 0; nb < NB; ++nb) {
+        int64_t n1 = (nb + 1) * 128 < N ? (nb + 1) * 128 : N;
+        for (int64_t kb = 0; kb < KB; ++kb) {
+            float amax = 0.0f;
+            for (int64_t n = nb * 128; n < n1; ++n)
+                for (int64_t k = kb * 128; k < kb * 128 + 128; ++k) {
+                    float a = fabsf(bf16_to_float(w[n * ld + k]));
+                    if (a > amax) amax = a;
+                }
+            float sb = scale_from_amax(amax);
+            s[nb * KB + kb] = sb;
+            for (int64_t n = nb * 128; n < n1; ++n)
+                for (int64_t k = kb * 128; k < kb * 128 + 128; ++k)
+                    q[n * ldq + k] = code_of(bf16_to_float(w[n * ld + k]), sb);
+        }
+    }
+}
+
+/* ----------------------------------------------------------------- linear */
+
+/* Integer mantissa of a code: E4M3value(c) = ik(c) * 2^-9 exactly. */
+static int32_t g_ik[256];
+static int g_ik_ready = 0;
+
+static void build_ik_table(void) {
+    if (g_ik_ready) return;
+    for (int c = 0; c < 256; ++c) {
+        double v = orc_e4m3_decode((uint8_t)c);
+        g_ik[c] = isnan(v) ? 0 : (int32_t)ldexp(v, 9);
+    }
+    g_ik_ready = 1;
+}
+
+/* Exact sum over k in [k0, k1) of E4M3value(a[k]) * E4M3value(b[k]), times 2^18. */
+static int64_t code_dot(const uint8_t* a, const uint8_t* b, int64_t k0, int64_t k1) {
+    int64_t acc = 0;
+    for (int64_t k = k0; k < k1; ++k) acc += (int64_t)g_ik[a[k]] * (int64_t)g_ik[b[k]];
+    return acc;
+}
+
+/* Channel/token mode: y[m,n] = xs[m] * ws[n] * sum_k x(m,k) w(n,k), the
+ * x_scale[m] * w_scale[n] product applied to the FP8 dot product [P2, P4]. */
+static float linear_channel_one(const uint8_t* xq, const float* xs, const uint8_t* wq,
+                                const float* ws, int64_t K, int64_t ldx, int64_t ldw,
+                                int64_t m, int64_t n) {
+    int64_t S = code_dot(xq + m * ldx, wq + n * ldw, 0, K);
+    return (float)((double)xs[m] * (double)ws[n] * ldexp((double)S, -18));
+}
+
+/* Block mode: sum over 128-wide K slices of the slice's exact dot product
+ * times x_scale[m, kb] * w_scale[n / 128, kb] [P5]. */
+static float linear_block_one(const uint8_t* xq, const float* xs, const uint8_t* wq,
+                              const float* ws, int64_t K, int64_t ldx, int64_t ldw,
+                              int64_t m, int64_t n) {
+    int64_t KB = K / 128;
+    double y = 0.0;
+    for (int64_t kb = 0; kb < KB; ++kb) {
+        int64_t S = code_dot(xq + m * ldx, wq + n * ldw, kb * 128, kb * 128 + 128);
+        y += (double)xs[m * KB + kb] * (double)ws[(n / 128) * KB + kb] * ldexp((double)S, -18);
+    }
+    return (float)y;
+}
+
+/* Full output Y[M,N] (fp32), mode 0 = channel/token, 1 = block-128. */
+ORC_EXPORT void orc_linear(const uint8_t* xq, const float* xs, const uint8_t* wq,
+                           const float* ws, int64_t M, int64_t N, int64_t K,
+                           int64_t ldx, int64_t ldw, int mode, float* y) {
+    build_ik_table();
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n)
+            y[m * N + n] = mode == 0
+                ? linear_channel_one(xq, xs, wq, ws, K, ldx, ldw, m, n)
+                : linear_block_one(xq, xs, wq, ws, K, ldx, ldw, m, n);
+}
+
+/* Selected outputs y[i] = Y[ms[i], ns[i]], for spot checks at full size. */
+ORC_EXPORT void orc_linear_at(const uint8_t* xq, const float* xs, const uint8_t* wq,
+                              const float* ws, int64_t K, int64_t ldx, int64_t ldw, int mode,
+                              const int64_t* ms, const int64_t* ns, int64_t count, float* y) {
+    build_ik_table();
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; ++i)
+        y[i] = mode == 0
+            ? linear_channel_one(xq, xs, wq, ws, K, ldx, ldw, ms[i], ns[i])
+            : linear_block_one(xq, xs, wq, ws, K, ldx, ldw, ms[i], ns[i]);
+}

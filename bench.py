@@ -1,0 +1,491 @@
+#!/usr/bin/env python
+"""Throughput of the B200 FP8 W8A8 linear layer on one workload.
+
+A step is one forward pass of the workload's FP8 linears: every distinct
+activation is quantized (dynamic per-token or per-128-group scales), then
+every GEMM runs.  Weights are quantized once at load time, outside the step
+(that kernel is timed separately and reported under "weight_quant").
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the CPU oracle, timed on a sample
+
+The L2 cache (126 MB) is flushed by a 256 MiB write before every step; each
+step and each kernel launch is timed with CUDA events on the launching stream,
+so the flush is not counted.  With N > 1 (torchrun, one rank per GPU) every
+rank runs its own batch of tokens against replicated weights (token-parallel,
+no collective on the data path): weak scaling, value = all ranks' work over
+the slowest rank's time.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+import zlib
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "llama3.2-3b_mlp_m2048"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP8_OVER_BF16 = 2.0        # nominal dense fp8 / bf16 tensor ratio (4.5 / 2.25 PFLOP/s)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fp8q", choices=["fp8q", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--flush-mib", type=int, default=256)
+    ap.add_argument("--cpu-sample-rows", type=int, default=256,
+                    help="rows of every GEMM the CPU oracle runs for cpu_baseline")
+    ap.add_argument("--ref-sample-rows", type=int, default=32,
+                    help="rows of every GEMM one reference-arm step runs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        p = json.load(open(PEAKS_FILE))
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def metric_for(wl) -> tuple:
+    decode = all(g.M <= 16 for g in wl.gemms)
+    if decode:
+        return "FP8 linear GB/s vs HBM (decode M<=16)", "GB/s"
+    return "FP8 linear TFLOP/s and % of FP8 peak (prefill)", "TFLOP/s"
+
+
+def gemm_bytes(g) -> int:
+    """Algorithmic bytes of one FP8 linear: codes of X and W once, bf16 Y
+    once, and the scales."""
+    if g.mode == synth.CHANNEL_TOKEN:
+        sb = 4 * g.M + 4 * g.N
+    else:
+        sb = 4 * g.M * (g.K // 128) + 4 * ((g.N + 127) // 128) * (g.K // 128)
+    return g.M * g.K + g.N * g.K + 2 * g.M * g.N + sb
+
+
+def quant_bytes(rows, K, mode) -> int:
+    nscale = rows if mode == synth.CHANNEL_TOKEN else rows * (K // 128)
+    return 2 * rows * K + rows * K + 4 * nscale
+
+
+def step_units(wl, unit) -> float:
+    """Work of one step in the metric's unit numerator (flop or byte)."""
+    if unit == "GB/s":
+        xs = {}
+        for g in wl.gemms:
+            xs[g.x] = (g.M, g.K, g.mode)
+        return float(sum(gemm_bytes(g) for g in wl.gemms) + sum(quant_bytes(*v) for v in xs.values()))
+    return float(sum(g.flops for g in wl.gemms))
+
+
+def to_metric(units, seconds, unit):
+    return units / seconds / (1e9 if unit == "GB/s" else 1e12)
+
+
+# ------------------------------------------------------------------ clocks ---
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.err = [], set(), None
+        self.period = period_s
+        self.stop_ev = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report why
+            self.nv, self.err, self.max_mhz = None, f"nvml unavailable: {e}", None
+
+    def _run(self):
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception as e:
+                self.err = str(e)
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv is not None:
+            self.stop_ev.set()
+            self.t.join()
+
+    def summary(self):
+        if self.nv is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples), "error": self.err}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------- GPU arm ---
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def launches_of(g) -> int:
+    return 2 if g.M <= 64 else 1          # decode: GEMM + reduction kernel
+
+
+def run_gpu(args):
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    import fp8_w8a8_quantized_amax_b200 as fq
+    from fp8_w8a8_quantized_amax_b200 import build as fbuild
+    fbuild.build()
+    dev = torch.device("cuda", local)
+    wl = synth.workloads()[args.workload]
+    metric, unit = metric_for(wl)
+    pk = peaks()
+
+    # ---- load time: weights (replicated), quantized once
+    W = {}
+    for g in wl.gemms:
+        w = synth.make_w(g.N, g.K, seed=zlib.crc32(g.name.encode()) % 1000).to(dev) if g.N * g.K <= (1 << 26) \
+            else synth.make_w_device(g.N, g.K, seed=zlib.crc32(g.name.encode()) % 1000, device=dev)
+        W[g.name] = w
+    xs_shapes = {}
+    for g in wl.gemms:
+        xs_shapes.setdefault(g.x, (g.M, g.K, g.mode))
+    X = {k: synth.make_x_device(M, K, seed=1000 * rank + i, device=dev)
+         for i, (k, (M, K, _)) in enumerate(xs_shapes.items())}
+    WQ = {g.name: fq.fp8_quant_weight(W[g.name], g.mode) for g in wl.gemms}
+    XQ = {k: (torch.empty((M, K), dtype=torch.uint8, device=dev),
+              torch.empty(fq.scale_shape_act(M, K, mode), dtype=torch.float32, device=dev))
+          for k, (M, K, mode) in xs_shapes.items()}
+    Y = {g.name: torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev) for g in wl.gemms}
+    WS = {g.name: (torch.empty(fq.fp8_linear_workspace_size(g.M, g.N, g.K, g.mode), dtype=torch.uint8,
+                               device=dev) if g.M <= 64 else None) for g in wl.gemms}
+    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    n_ops = len(xs_shapes) + len(wl.gemms)
+
+    def step(ev=None):
+        i = 0
+        for k, (M, K, mode) in xs_shapes.items():
+            fq.fp8_quant_act(X[k], mode, out=XQ[k])
+            if ev is not None:
+                ev[i].record(stream)
+            i += 1
+        for g in wl.gemms:
+            xq, xsc = XQ[g.x]
+            wq, wsc = WQ[g.name]
+            fq.fp8_linear(xq, xsc, wq, wsc, g.mode, out=Y[g.name], workspace=WS[g.name])
+            if ev is not None:
+                ev[i].record(stream)
+            i += 1
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert fq.device_error(clear=True) == 0
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ops + 1)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for s in range(args.steps):
+            flush.zero_()
+            events[s][0].record(stream)
+            step(events[s][1:])
+        torch.cuda.synchronize()
+    barrier(world)
+    step_ms = [events[s][0].elapsed_time(events[s][n_ops]) for s in range(args.steps)]
+    op_ms = np.array([[events[s][i].elapsed_time(events[s][i + 1]) for i in range(n_ops)]
+                      for s in range(args.steps)]).mean(axis=0)
+    total_s = sum(step_ms) / 1e3
+    total_s = max_over_ranks(total_s, world)
+    units = step_units(wl, unit) * args.steps
+    value = to_metric(sum_over_ranks(units, world), total_s, unit)
+    err = fq.device_error(clear=True)
+
+    # ---- per-kernel detail and the dominant kernel's roofline
+    names = [f"quant_act[{k}]" for k in xs_shapes] + [g.name for g in wl.gemms]
+    detail = []
+    fp8_peak = pk["bf16_tflops"] * FP8_OVER_BF16
+    for i, (k, (M, K, mode)) in enumerate(xs_shapes.items()):
+        b = quant_bytes(M, K, mode)
+        detail.append({"op": names[i], "kernel": "quant_rows" if mode == 0 else "quant_groups128",
+                       "ms": round(float(op_ms[i]), 5), "GB/s": round(b / (op_ms[i] / 1e3) / 1e9, 1),
+                       "frac_hbm": round(b / (op_ms[i] / 1e3) / 1e9 / pk["hbm_gbs"], 3)})
+    for j, g in enumerate(wl.gemms):
+        t = op_ms[len(xs_shapes) + j] / 1e3
+        kern = ("gemm_decode+reduce" if g.M <= 64 else
+                ("gemm_block" if g.mode == synth.BLOCK128 else "gemm_channel"))
+        detail.append({"op": g.name, "kernel": kern, "M": g.M, "N": g.N, "K": g.K, "mode": g.mode,
+                       "ms": round(float(op_ms[len(xs_shapes) + j]), 5),
+                       "TFLOP/s": round(g.flops / t / 1e12, 1),
+                       "GB/s": round(gemm_bytes(g) / t / 1e9, 1),
+                       "frac_fp8_peak": round(g.flops / t / 1e12 / fp8_peak, 3),
+                       "frac_hbm": round(gemm_bytes(g) / t / 1e9 / pk["hbm_gbs"], 3)})
+    gemm_ops = detail[len(xs_shapes):]
+    dom = max(gemm_ops, key=lambda d: d["ms"])
+    gsel = [g for g in wl.gemms if g.name == dom["op"]][0]
+    if unit == "TFLOP/s":
+        roof = {"kernel": dom["kernel"], "bound": "tensor", "achieved": dom["TFLOP/s"],
+                "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                "frac": round(dom["TFLOP/s"] / fp8_peak, 3),
+                "peak_basis": f"{pk['source']} bf16 burst {pk['bf16_tflops']} TFLOP/s x {FP8_OVER_BF16} "
+                              "(nominal fp8/bf16 dense ratio)",
+                "algorithmic": f"2*M*N*K = {gsel.flops} flop per launch", "traffic": None}
+    else:
+        roof = {"kernel": dom["kernel"], "bound": "hbm", "achieved": dom["GB/s"], "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": round(dom["GB/s"] / pk["hbm_gbs"], 3),
+                "peak_basis": f"{pk['source']} HBM copy bandwidth",
+                "algorithmic": f"M*K + N*K + 2*M*N + scales = {gemm_bytes(gsel)} bytes per launch",
+                "traffic": None}
+    tfile = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tfile):
+        try:
+            tr = json.load(open(tfile)).get(f"{args.workload}:{dom['op']}")
+            if tr:
+                roof["traffic"] = tr
+        except Exception:
+            pass
+
+    # ---- weight quantization (load-time kernel) timed alone
+    wq_ms = []
+    g0 = max(wl.gemms, key=lambda g: g.N * g.K)
+    for _ in range(3):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fq.fp8_quant_weight(W[g0.name], g0.mode, out=WQ[g0.name])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        wq_ms.append(e0.elapsed_time(e1))
+    wqb = quant_bytes(g0.N, g0.K, 0) if g0.mode == 0 else (3 * g0.N * g0.K + 4 * ((g0.N + 127) // 128) * (g0.K // 128))
+    weight_quant = {"shape": [g0.N, g0.K], "mode": g0.mode, "ms": round(min(wq_ms), 5),
+                    "GB/s": round(wqb / (min(wq_ms) / 1e3) / 1e9, 1),
+                    "frac_hbm": round(wqb / (min(wq_ms) / 1e3) / 1e9 / pk["hbm_gbs"], 3)}
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Xh = {k: X[k].cpu().pin_memory() for k in X}
+        Yh = {g.name: torch.empty((g.M, g.N), dtype=torch.bfloat16).pin_memory() for g in wl.gemms}
+        Xd = {k: torch.empty_like(X[k]) for k in X}
+
+        def e2e_step():
+            for k in X:
+                Xd[k].copy_(Xh[k], non_blocking=True)
+            for k, (M, K, mode) in xs_shapes.items():
+                fq.fp8_quant_act(Xd[k], mode, out=XQ[k])
+            for g in wl.gemms:
+                xq, xsc = XQ[g.x]
+                wq, wsc = WQ[g.name]
+                fq.fp8_linear(xq, xsc, wq, wsc, g.mode, out=Y[g.name], workspace=WS[g.name])
+                Yh[g.name].copy_(Y[g.name], non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e_ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+            e_ms.append((a, b))
+        torch.cuda.synchronize()
+        barrier(world)
+        et = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ms) / 1e3, world)
+        e2e = {"value": round(to_metric(sum_over_ranks(units, world), et, unit), 3), "unit": unit,
+               "h2d_bytes_per_step": int(sum(x.numel() * 2 for x in X.values())),
+               "d2h_bytes_per_step": int(sum(y.numel() * 2 for y in Y.values())),
+               "ms_per_step": round(et * 1e3 / args.steps, 4),
+               "path": "pinned host X -> device, fp8_quant_act, fp8_linear, device Y -> pinned host"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, unit, args.cpu_sample_rows)
+
+    if rank == 0:
+        line = {
+            "metric": metric, "value": round(value, 3), "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_s * 1e3 / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8_e4m3 (fp32 accumulate, bf16 out)", "data": "synthetic",
+            "config": {"workload": wl.name,
+                       "gemms": [f"{g.name}:{g.M}x{g.K}->{g.N}:{'channel' if g.mode == 0 else 'block128'}"
+                                 for g in wl.gemms],
+                       "step": "quantize each activation + every FP8 GEMM; weights quantized at load",
+                       "l2": f"flushed ({args.flush_mib} MiB write) before every step, outside the timed events",
+                       "parallelism": "single GPU" if world == 1 else f"token-parallel x{world}, weights replicated"},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g) for g in wl.gemms)),
+            "clocks": clk.summary(), "detail": detail, "weight_quant": weight_quant,
+            "device_error": err, "gpu": torch.cuda.get_device_name(dev),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ----------------------------------------------------------- CPU oracle ---
+
+def oracle_sample(wl, rows, w_cache=None):
+    """Run the oracle on `rows` rows of every GEMM (all N, all K); returns
+    (seconds, rows used per GEMM, threads)."""
+    import oracle
+    oracle.build()
+    if w_cache is None:
+        w_cache = {}
+    for g in wl.gemms:
+        if g.name not in w_cache:
+            w = synth.make_w(g.N, g.K, seed=zlib.crc32(g.name.encode()) % 1000)
+            w_cache[g.name] = oracle.quant_weight(w, g.mode)
+    xs = {}
+    for g in wl.gemms:
+        if g.x not in xs:
+            xs[g.x] = synth.make_x(min(rows, g.M), g.K, seed=7)
+    t0 = time.perf_counter()
+    q = {}
+    for g in wl.gemms:
+        if g.x not in q:
+            q[g.x] = oracle.quant_act(xs[g.x], g.mode)
+    for g in wl.gemms:
+        xq, xsc = q[g.x]
+        wq, wsc = w_cache[g.name]
+        oracle.linear(xq, xsc, wq, wsc, g.mode)
+    return time.perf_counter() - t0, w_cache
+
+
+def omp_threads():
+    n = os.environ.get("OMP_NUM_THREADS")
+    if n and n.isdigit():
+        return int(n)
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, unit, rows, w_cache=None):
+    secs, _ = oracle_sample(wl, rows, w_cache)
+    # linear extrapolation in M of the sampled rows to the whole workload
+    frac = sum(min(rows, g.M) * g.N * g.K for g in wl.gemms) / sum(g.M * g.N * g.K for g in wl.gemms)
+    full_s = secs / frac
+    return {"value": round(to_metric(step_units(wl, unit), full_s, unit), 6), "unit": unit,
+            "cores": omp_threads(), "kind": "oracle",
+            "sample": f"first {rows} token rows of every GEMM (all N, all K): activation quantization + "
+                      f"exact int64 GEMM, {secs:.2f} s, extrapolated linearly in M (weights quantized "
+                      "before timing, as in the GPU step)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = synth.workloads()[args.workload]
+    metric, unit = metric_for(wl)
+    rows = args.ref_sample_rows
+    cache = {}
+    for _ in range(args.warmup):
+        oracle_sample(wl, rows, cache)
+    secs = [oracle_sample(wl, rows, cache)[0] for _ in range(args.steps)]
+    frac = sum(min(rows, g.M) * g.N * g.K for g in wl.gemms) / sum(g.M * g.N * g.K for g in wl.gemms)
+    full = sum(secs) / frac
+    value = to_metric(step_units(wl, unit) * args.steps, full, unit)
+    sample = (f"first {rows} token rows of every GEMM per step (all N, all K), extrapolated linearly "
+              "in M to the whole workload")
+    line = {"impl": "reference", "metric": metric, "value": round(value, 6), "unit": unit,
+            "n_gpus": int(os.environ.get("WORLD_SIZE", args.gpus)), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(full * 1e3 / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int64 exact dot products, f64 scaling", "data": "synthetic",
+            "config": {"workload": wl.name, "parallelism": "host cores (oracle)"},
+            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": omp_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

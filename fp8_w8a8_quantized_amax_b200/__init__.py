@@ -1,0 +1,183 @@
+"""B200 (sm_100a) FP8 W8A8 linear layer: Python binding of libfp8q.so.
+
+The functions here carry the names of the C entry points declared in
+include/fp8q.h and only marshal arguments: torch tensors supply device memory
+and the current CUDA stream, every step of the computation runs in the
+library's CUDA kernels.  There is no CPU fallback; without the built library
+(or without a GPU) the calls raise.
+
+    Wq, w_scale = fp8_quant_weight(W, mode)      # once per layer
+    Xq, x_scale = fp8_quant_act(X, mode)         # every forward
+    Y = fp8_linear(Xq, x_scale, Wq, w_scale, mode)
+
+mode: CHANNEL_TOKEN (per-output-channel weights, per-token activations, the
+FP8-Dynamic scheme) or BLOCK128 (128x128 weight blocks, 128-groups of
+activations, the FP8-Block scheme).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+from .policy import DEFAULT_IGNORE, should_quantize  # noqa: F401
+
+CHANNEL_TOKEN = 0
+BLOCK128 = 1
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_UNSUPPORTED = 2
+ERR_MISALIGNED = 3
+ERR_CUDA = 4
+ERR_DEVICE_TIMEOUT = 5
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8q.so")
+
+_lib = None
+
+
+class FP8QError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfp8q.so (built in-tree by build.py); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libfp8q.so not built ({LIB_PATH}); run "
+                              "python -m fp8_w8a8_quantized_amax_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+        L.fp8_quant_weight.argtypes = [P, I, I, I, ctypes.c_int, P, I, P, P]
+        L.fp8_quant_weight.restype = ctypes.c_int
+        L.fp8_quant_act.argtypes = [P, I, I, I, ctypes.c_int, P, I, P, P]
+        L.fp8_quant_act.restype = ctypes.c_int
+        L.fp8_linear.argtypes = [P, P, P, P, I, I, I, ctypes.c_int, P, I, P, S, P]
+        L.fp8_linear.restype = ctypes.c_int
+        L.fp8_linear_workspace_size.argtypes = [I, I, I, ctypes.c_int]
+        L.fp8_linear_workspace_size.restype = S
+        L.fp8q_status_string.argtypes = [ctypes.c_int]
+        L.fp8q_status_string.restype = ctypes.c_char_p
+        L.fp8q_device_error.argtypes = [ctypes.c_int]
+        L.fp8q_device_error.restype = ctypes.c_int
+        L.fp8q_version.argtypes = []
+        L.fp8q_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().fp8q_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != OK:
+        raise FP8QError(status, what)
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _require_cuda(t: torch.Tensor, name: str, dtype) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be 2-D with unit stride in the last dimension")
+
+
+def scale_shape_weight(N: int, K: int, mode: int) -> Tuple[int, ...]:
+    return (N,) if mode == CHANNEL_TOKEN else ((N + 127) // 128, K // 128)
+
+
+def scale_shape_act(M: int, K: int, mode: int) -> Tuple[int, ...]:
+    return (M,) if mode == CHANNEL_TOKEN else (M, K // 128)
+
+
+def fp8_quant_weight(W: torch.Tensor, mode: int = CHANNEL_TOKEN,
+                     out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
+    """W bf16 [N, K] -> (Wq uint8 [N, K] E4M3 codes, w_scale fp32 [N] or [N/128, K/128])."""
+    _require_cuda(W, "W", torch.bfloat16)
+    N, K = W.shape
+    if out is None:
+        Wq = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+        ws = torch.empty(scale_shape_weight(N, K, mode), dtype=torch.float32, device=W.device)
+    else:
+        Wq, ws = out
+    st = lib().fp8_quant_weight(_ptr(W), N, K, W.stride(0), int(mode), _ptr(Wq), Wq.stride(0),
+                                _ptr(ws), _stream(W))
+    _check(st, "fp8_quant_weight")
+    return Wq, ws
+
+
+def fp8_quant_act(X: torch.Tensor, mode: int = CHANNEL_TOKEN,
+                  out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
+    """X bf16 [M, K] -> (Xq uint8 [M, K], x_scale fp32 [M] or [M, K/128])."""
+    _require_cuda(X, "X", torch.bfloat16)
+    M, K = X.shape
+    if out is None:
+        Xq = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+        xs = torch.empty(scale_shape_act(M, K, mode), dtype=torch.float32, device=X.device)
+    else:
+        Xq, xs = out
+    st = lib().fp8_quant_act(_ptr(X), M, K, X.stride(0), int(mode), _ptr(Xq), Xq.stride(0),
+                             _ptr(xs), _stream(X))
+    _check(st, "fp8_quant_act")
+    return Xq, xs
+
+
+def fp8_linear_workspace_size(M: int, N: int, K: int, mode: int = CHANNEL_TOKEN) -> int:
+    return int(lib().fp8_linear_workspace_size(M, N, K, int(mode)))
+
+
+def fp8_linear(Xq: torch.Tensor, x_scale: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+               mode: int = CHANNEL_TOKEN, out: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y bf16 [M, N] = dequant(Xq) . dequant(Wq)^T.  Workspace (small-M path) is
+    taken from torch's caching allocator unless given."""
+    _require_cuda(Xq, "Xq", torch.uint8)
+    _require_cuda(Wq, "Wq", torch.uint8)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K:
+        raise ValueError("Xq and Wq disagree on K")
+    if not (Xq.is_contiguous() and Wq.is_contiguous()):
+        raise ValueError("Xq and Wq must be contiguous")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    need = fp8_linear_workspace_size(M, N, K, mode)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Xq.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().fp8_linear(_ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), M, N, K, int(mode),
+                          _ptr(out), out.stride(0), _ptr(workspace), wbytes, _stream(Xq))
+    _check(st, "fp8_linear")
+    return out
+
+
+def device_error(clear: bool = True) -> int:
+    """Device-side error word (nonzero after a kernel gave up waiting)."""
+    return int(lib().fp8q_device_error(1 if clear else 0))
+
+
+def version() -> int:
+    return int(lib().fp8q_version())
+
+
+# Short aliases.
+quant_weight = fp8_quant_weight
+quant_act = fp8_quant_act
+linear = fp8_linear

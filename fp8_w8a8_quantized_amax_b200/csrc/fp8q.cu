@@ -1,0 +1,338 @@
+// fp8q.cu -- C ABI of libfp8q.so: argument checks, tensor maps, dispatch.
+//
+// All device work lives in the kernels included below; this file only checks
+// arguments (before anything touches CUDA), builds TMA descriptors, picks a
+// kernel and launch shape, and maps errors to fp8q_status.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "../../include/fp8q.h"
+#include "gemm_decode.cuh"
+#include "gemm_prefill.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
+
+namespace {
+
+using fp8q::decode::Params;
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kInt32Max = 2147483647;
+
+// ------------------------------------------------------------ device info ---
+
+struct DeviceInfo {
+  int sms = 0;
+  bool ready = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+fp8q_status current_device(int* dev, int* sms) {
+  if (cudaGetDevice(dev) != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (*dev < 0 || *dev >= kMaxDevices) return FP8Q_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[*dev];
+  if (!d.ready) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess) return FP8Q_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess) return FP8Q_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess) return FP8Q_ERR_CUDA;
+    if (major != 10 || minor != 0) return FP8Q_ERR_UNSUPPORTED;   // built for sm_100a only
+    d.ready = true;
+  }
+  *sms = d.sms;
+  return FP8Q_OK;
+}
+
+// Opt a kernel in to large dynamic shared memory, once per (kernel, device).
+struct SmemOptIn {
+  const void* fn;
+  int dev;
+};
+SmemOptIn g_optin[256];
+int g_noptin = 0;
+std::mutex g_optin_mu;
+
+template <typename K>
+fp8q_status ensure_smem(K kernel, int bytes, int dev) {
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  std::lock_guard<std::mutex> lk(g_optin_mu);
+  for (int i = 0; i < g_noptin; ++i)
+    if (g_optin[i].fn == fn && g_optin[i].dev == dev) return FP8Q_OK;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
+  if (g_noptin < 256) g_optin[g_noptin++] = {fn, dev};
+  return FP8Q_OK;
+}
+
+template <typename... KArgs, typename... Args>
+fp8q_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, void* stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ tensor maps ---
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+fp8q_status get_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+// Row-major uint8 matrix [rows, cols] with row stride `ld` bytes, tiles of
+// box_rows x 128 bytes, 128-byte swizzle (the layout tcgen05 descriptors expect).
+fp8q_status tmap_u8_sw128(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                          uint32_t box_rows) {
+  if (get_encode() != FP8Q_OK) return FP8Q_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
+  cuuint32_t box[2] = {128u, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// ------------------------------------------------------------ quantization ---
+
+fp8q_status check_quant_args(const void* src, int64_t rows, int64_t K, int64_t ld, int mode, const uint8_t* q,
+                             int64_t ldq, const float* s) {
+  if (mode != FP8Q_CHANNEL_TOKEN && mode != FP8Q_BLOCK128) return FP8Q_ERR_INVALID_ARG;
+  if (rows < 0 || K <= 0 || ld < K || ldq < K) return FP8Q_ERR_INVALID_ARG;
+  if (K % 16 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (mode == FP8Q_BLOCK128 && K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (rows == 0) return FP8Q_OK;
+  if (!src || !q || !s) return FP8Q_ERR_INVALID_ARG;
+  if (ld % 8 != 0 || ldq % 16 != 0) return FP8Q_ERR_MISALIGNED;
+  if (!aligned(src, 16) || !aligned(q, 16) || !aligned(s, 4)) return FP8Q_ERR_MISALIGNED;
+  if (rows > kInt32Max || K > kInt32Max) return FP8Q_ERR_UNSUPPORTED;
+  return FP8Q_OK;
+}
+
+fp8q_status launch_rows(const uint16_t* x, int64_t rows, int K, int64_t ldx, uint8_t* q, int64_t ldq, float* s,
+                        void* stream) {
+  const int nvec = K / 8;
+  int T = 32 * ((nvec + 32 * 8 - 1) / (32 * 8));
+  if (T > 1024) T = 1024;
+  const int need = (nvec + T - 1) / T;
+  const dim3 grid(static_cast<unsigned>(rows));
+  const dim3 block(T);
+  if (need <= 1) return launch(fp8q::quant_rows_kernel<1>, grid, block, 0, stream, x, K, ldx, q, ldq, s);
+  if (need <= 2) return launch(fp8q::quant_rows_kernel<2>, grid, block, 0, stream, x, K, ldx, q, ldq, s);
+  if (need <= 4) return launch(fp8q::quant_rows_kernel<4>, grid, block, 0, stream, x, K, ldx, q, ldq, s);
+  if (need <= 8) return launch(fp8q::quant_rows_kernel<8>, grid, block, 0, stream, x, K, ldx, q, ldq, s);
+  if (need <= 16) return launch(fp8q::quant_rows_kernel<16>, grid, block, 0, stream, x, K, ldx, q, ldq, s);
+  return FP8Q_ERR_UNSUPPORTED;   // K > 131072
+}
+
+// ------------------------------------------------------------------ linear ---
+
+constexpr int kPrefillBN = 256;
+constexpr int kPrefillStages = 4;
+constexpr int kBlockStages = 6;
+constexpr int kDecodeStages = 8;
+constexpr int kDecodeMaxM = 64;
+
+int decode_nx(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
+
+void decode_shape(int64_t M, int64_t N, int64_t K, int sms, int* n_tiles, int64_t* total, int* G, int* nx) {
+  const int KB = static_cast<int>((K + 127) / 128);
+  *n_tiles = static_cast<int>((N + 127) / 128);
+  *total = static_cast<int64_t>(*n_tiles) * KB;
+  *G = static_cast<int>(*total < sms ? *total : sms);
+  *nx = decode_nx(M);
+}
+
+size_t decode_workspace_bytes(int n_tiles, int G, int nx) {
+  return static_cast<size_t>(n_tiles + G - 1) * nx * 128 * sizeof(float);
+}
+
+fp8q_status check_linear_args(const uint8_t* Xq, const float* xs, const uint8_t* Wq, const float* ws, int64_t M,
+                              int64_t N, int64_t K, int mode, const void* Y, int64_t ldy) {
+  if (mode != FP8Q_CHANNEL_TOKEN && mode != FP8Q_BLOCK128) return FP8Q_ERR_INVALID_ARG;
+  if (M < 0 || N <= 0 || K <= 0 || ldy < N) return FP8Q_ERR_INVALID_ARG;
+  if (K % 16 != 0 || N % 16 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (mode == FP8Q_BLOCK128 && K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (M == 0) return FP8Q_OK;
+  if (!Xq || !xs || !Wq || !ws || !Y) return FP8Q_ERR_INVALID_ARG;
+  if (ldy % 8 != 0) return FP8Q_ERR_MISALIGNED;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(Y, 16) || !aligned(xs, 4) || !aligned(ws, 4))
+    return FP8Q_ERR_MISALIGNED;
+  if (M > kInt32Max || N > kInt32Max || K > kInt32Max) return FP8Q_ERR_UNSUPPORTED;
+  return FP8Q_OK;
+}
+
+template <int NX>
+fp8q_status launch_decode_nx(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p, int mode, int dev,
+                             void* Y, int64_t ldy, void* stream) {
+  using L = fp8q::decode::Layout<NX, kDecodeStages>;
+  fp8q_status st;
+  if (mode == FP8Q_BLOCK128) {
+    auto k = fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, true>;
+    if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
+    if ((st = launch(k, dim3(p.G), dim3(192), L::kBytes, stream, tw, tx, p)) != FP8Q_OK) return st;
+    return launch(fp8q::decode::decode_reduce_kernel<true>, dim3(p.n_tiles, p.M), dim3(128), 0, stream, p, NX,
+                  static_cast<__nv_bfloat16*>(Y), ldy);
+  }
+  auto k = fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, false>;
+  if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
+  if ((st = launch(k, dim3(p.G), dim3(192), L::kBytes, stream, tw, tx, p)) != FP8Q_OK) return st;
+  return launch(fp8q::decode::decode_reduce_kernel<false>, dim3(p.n_tiles, p.M), dim3(128), 0, stream, p, NX,
+                static_cast<__nv_bfloat16*>(Y), ldy);
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8q_status fp8_quant_weight(const void* W_bf16, int64_t N, int64_t K, int64_t ldw, int mode, uint8_t* Wq,
+                             int64_t ldwq, float* w_scale, void* stream) {
+  fp8q_status st = check_quant_args(W_bf16, N, K, ldw, mode, Wq, ldwq, w_scale);
+  if (st != FP8Q_OK || N == 0) return st;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
+  const uint16_t* w = static_cast<const uint16_t*>(W_bf16);
+  if (mode == FP8Q_CHANNEL_TOKEN) return launch_rows(w, N, static_cast<int>(K), ldw, Wq, ldwq, w_scale, stream);
+  const int64_t NB = (N + 127) / 128;
+  if (NB > 65535) return FP8Q_ERR_UNSUPPORTED;
+  return launch(fp8q::quant_blocks128_kernel, dim3(static_cast<unsigned>(K / 128), static_cast<unsigned>(NB)),
+                dim3(256), 0, stream, w, N, static_cast<int>(K / 128), ldw, Wq, ldwq, w_scale);
+}
+
+fp8q_status fp8_quant_act(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, int mode, uint8_t* Xq,
+                          int64_t ldxq, float* x_scale, void* stream) {
+  fp8q_status st = check_quant_args(X_bf16, M, K, ldx, mode, Xq, ldxq, x_scale);
+  if (st != FP8Q_OK || M == 0) return st;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
+  const uint16_t* x = static_cast<const uint16_t*>(X_bf16);
+  if (mode == FP8Q_CHANNEL_TOKEN) return launch_rows(x, M, static_cast<int>(K), ldx, Xq, ldxq, x_scale, stream);
+  constexpr int GPT = 4;
+  const int G = static_cast<int>(K / 128);
+  const int64_t total = M * G;
+  int64_t grid = (total + 16 * GPT - 1) / (16 * GPT);
+  if (grid > static_cast<int64_t>(sms) * 16) grid = static_cast<int64_t>(sms) * 16;
+  return launch(fp8q::quant_groups128_kernel<GPT>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream, x, M,
+                G, ldx, Xq, ldxq, x_scale);
+}
+
+size_t fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int mode) {
+  if (mode != FP8Q_CHANNEL_TOKEN && mode != FP8Q_BLOCK128) return 0;
+  if (M <= 0 || M > kDecodeMaxM || N <= 0 || K <= 0) return 0;
+  int dev, sms;
+  if (current_device(&dev, &sms) != FP8Q_OK) return 0;
+  int n_tiles, G, nx;
+  int64_t total;
+  decode_shape(M, N, K, sms, &n_tiles, &total, &G, &nx);
+  return decode_workspace_bytes(n_tiles, G, nx);
+}
+
+fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq, const float* w_scale, int64_t M,
+                       int64_t N, int64_t K, int mode, void* Y_bf16, int64_t ldy, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  fp8q_status st = check_linear_args(Xq, x_scale, Wq, w_scale, M, N, K, mode, Y_bf16, ldy);
+  if (st != FP8Q_OK || M == 0) return st;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
+  const int KB = static_cast<int>((K + 127) / 128);
+
+  if (M <= kDecodeMaxM) {
+    int n_tiles, G, nx;
+    int64_t total;
+    decode_shape(M, N, K, sms, &n_tiles, &total, &G, &nx);
+    if (!workspace || workspace_bytes < decode_workspace_bytes(n_tiles, G, nx)) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return FP8Q_ERR_MISALIGNED;
+    CUtensorMap tw, tx;
+    if ((st = tmap_u8_sw128(&tw, Wq, N, K, K, 128)) != FP8Q_OK) return st;
+    if ((st = tmap_u8_sw128(&tx, Xq, M, K, K, static_cast<uint32_t>(nx))) != FP8Q_OK) return st;
+    Params p;
+    p.xs = x_scale;
+    p.ws = w_scale;
+    p.part = static_cast<float*>(workspace);
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.KB = KB;
+    p.n_tiles = n_tiles;
+    p.total = total;
+    p.G = G;
+    if (nx == 16) return launch_decode_nx<16>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
+    if (nx == 32) return launch_decode_nx<32>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
+    return launch_decode_nx<64>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
+  }
+
+  fp8q::prefill::Params p;
+  p.xs = x_scale;
+  p.ws = w_scale;
+  p.y = static_cast<__nv_bfloat16*>(Y_bf16);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.ldy = ldy;
+  p.KB = KB;
+  const int BN = mode == FP8Q_BLOCK128 ? 128 : kPrefillBN;
+  p.num_m = static_cast<int>((M + 127) / 128);
+  p.num_n = static_cast<int>((N + BN - 1) / BN);
+  p.num_tiles = p.num_m * p.num_n;
+  p.group_m = p.num_m < 16 ? p.num_m : 16;
+  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  CUtensorMap ta, tb;
+  if ((st = tmap_u8_sw128(&ta, Xq, M, K, K, 128)) != FP8Q_OK) return st;
+  if ((st = tmap_u8_sw128(&tb, Wq, N, K, K, static_cast<uint32_t>(BN))) != FP8Q_OK) return st;
+  if (mode == FP8Q_BLOCK128) {
+    using L = fp8q::prefill::BlockLayout<kBlockStages>;
+    auto k = fp8q::prefill::gemm_block_kernel<kBlockStages>;
+    if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
+    return launch(k, dim3(grid), dim3(320), L::kBytes, stream, ta, tb, p);
+  }
+  using L = fp8q::prefill::ChannelLayout<kPrefillBN, kPrefillStages>;
+  auto k = fp8q::prefill::gemm_channel_kernel<kPrefillBN, kPrefillStages>;
+  if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
+  return launch(k, dim3(grid), dim3(192), L::kBytes, stream, ta, tb, p);
+}
+
+const char* fp8q_status_string(int status) {
+  switch (status) {
+    case FP8Q_OK: return "FP8Q_OK";
+    case FP8Q_ERR_INVALID_ARG: return "FP8Q_ERR_INVALID_ARG: invalid argument";
+    case FP8Q_ERR_UNSUPPORTED: return "FP8Q_ERR_UNSUPPORTED: outside what the kernels cover";
+    case FP8Q_ERR_MISALIGNED: return "FP8Q_ERR_MISALIGNED: pointer or stride not 16-byte aligned";
+    case FP8Q_ERR_CUDA: return "FP8Q_ERR_CUDA: a CUDA call failed";
+    case FP8Q_ERR_DEVICE_TIMEOUT: return "FP8Q_ERR_DEVICE_TIMEOUT: a kernel gave up waiting";
+    default: return "FP8Q: unknown status";
+  }
+}
+
+int fp8q_device_error(int clear) {
+  int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  if (cudaMemcpyFromSymbol(&v, fp8q::g_device_error, sizeof(int)) != cudaSuccess) return -1;
+  if (clear) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(fp8q::g_device_error, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
+}
+
+int fp8q_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,227 @@
+// gemm_decode.cuh -- FP8 linear for small M (decode, M <= 64): HBM-bound weight stream.
+//
+// Swap-AB: a 128-row slice of Wq is the tcgen05 "A" operand (UMMA M = 128)
+// and the M tokens, padded with zero rows to NX in {16, 32, 64}, are "B"
+// (UMMA N = NX), so the accumulator D[n, m] sits in TMEM with lane = output
+// channel and column = token.
+//
+// Stream-K: the (weight tile t, K block kb) pairs, t-major, form one list of
+// T = n_tiles * KB steps that is cut into G equal contiguous ranges, one per
+// CTA (G <= #SMs, every range non-empty).  A CTA walks its range; each run of
+// steps inside one weight tile is a "segment", whose fp32 partial
+// D[n, m] (already multiplied by the block scales in block mode) goes to
+// workspace slot (t + c) -- slots are unique because a CTA's tiles increase
+// with c.  The reduction kernel adds the segments of each tile in CTA order
+// (deterministic), applies the channel scales in channel mode, and writes
+// bf16.  Partial traffic is (n_tiles + G) * NX * 512 bytes, small next to the
+// N * K weight bytes.
+//
+// Roles: warp 0 TMA (W tile 128 x 128 B evict-first + X tile NX x 128 B),
+// warp 1 TMEM allocation + MMA issue (one TMEM slot of NX columns per step,
+// 4 slots), warps 2..5 fold each slot into registers and write segments.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace fp8q {
+namespace decode {
+
+constexpr int BK = 128;
+constexpr int UMMA_K = 32;
+constexpr int kSlots = 4;
+
+struct Params {
+  const float* xs;
+  const float* ws;
+  float* part;        // workspace: [(n_tiles + G - 1)][NX][128] fp32
+  int M, N, K, KB;
+  int n_tiles;
+  int64_t total;      // n_tiles * KB
+  int G;              // CTAs
+};
+
+__host__ __device__ __forceinline__ int64_t range_begin(int64_t c, int64_t total, int64_t G) {
+  return c * total / G;
+}
+
+// Largest CTA index c whose range starts at or before step x.
+__host__ __device__ __forceinline__ int cta_of_step(int64_t x, int64_t total, int64_t G) {
+  return static_cast<int>(((x + 1) * G - 1) / total);
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+}
+
+template <int NX, int STAGES>
+struct Layout {
+  static constexpr int kW = 128 * BK;
+  static constexpr int kX = NX * BK;
+  static constexpr int kBarOff = STAGES * (kW + kX);
+  static constexpr int kBytes = kBarOff + 256 + 1024;
+  static constexpr uint32_t kTmemCols = (kSlots * NX) < 32 ? 32 : (kSlots * NX);
+};
+
+template <int NX, int STAGES, bool BLOCK>
+__global__ void __launch_bounds__(192, 1)
+    gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                       const Params p) {
+  using L = Layout<NX, STAGES>;
+  static_assert(NX % 16 == 0 && NX >= 16 && NX <= 64, "token tile");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sW = smem;
+  uint8_t* sX = smem + STAGES * L::kW;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* sfull = empty + STAGES;
+  uint64_t* sempty = sfull + kSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + kSlots);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+  const int64_t b = range_begin(c, p.total, p.G);
+  const int64_t e = range_begin(c + 1, p.total, p.G);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < kSlots; ++a) {
+      mbar_init(&sfull[a], 1);
+      mbar_init(&sempty[a], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int64_t s = b; s < e; ++s) {
+        const int t = static_cast<int>(s / p.KB);
+        const int kb = static_cast<int>(s - static_cast<int64_t>(t) * p.KB);
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) { ok = false; break; }
+        mbar_arrive_expect_tx(&full[stage], L::kW + L::kX);
+        tma_load_2d(sW + stage * L::kW, &tmW, &full[stage], kb * BK, t * 128, pol_w);
+        tma_load_2d(sX + stage * L::kX, &tmX, &full[stage], kb * BK, 0, pol_x);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      for (int i = 0; ok && i < STAGES; ++i) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) break;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(128, NX);
+      int stage = 0, slot = 0;
+      uint32_t phase = 0, sphase = 0;
+      for (int64_t s = b; s < e; ++s) {
+        if (!mbar_wait(&sempty[slot], sphase ^ 1u, abort_flag, kErrWaitTmemEmpty)) break;
+        if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + slot * NX;
+        const uint32_t a0 = smem_u32(sW + stage * L::kW);
+        const uint32_t b0 = smem_u32(sX + stage * L::kX);
+#pragma unroll
+        for (int k = 0; k < BK / UMMA_K; ++k)
+          mma_e4m3(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + k * UMMA_K), idesc, k != 0);
+        mma_commit(&empty[stage]);
+        mma_commit(&sfull[slot]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int nl = quarter * 32 + lane;          // output channel within the tile
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    float acc[NX];
+#pragma unroll
+    for (int j = 0; j < NX; ++j) acc[j] = 0.0f;
+    int slot = 0;
+    uint32_t sphase = 0;
+    for (int64_t s = b; s < e; ++s) {
+      const int t = static_cast<int>(s / p.KB);
+      const int kb = static_cast<int>(s - static_cast<int64_t>(t) * p.KB);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sfull[slot], sphase, abort_flag, kErrWaitTmemFull))) break;
+      tc_fence_after();
+      uint32_t r[NX];
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < NX; j += 16) tmem_ld_32x32b_x16(tmem_base + lane_addr + slot * NX + j,
+                                                           *reinterpret_cast<uint32_t(*)[16]>(&r[j]));
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&sempty[slot]);
+      if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
+      if constexpr (BLOCK) {
+        const float wsf = __ldg(p.ws + static_cast<int64_t>(t) * p.KB + kb);
+#pragma unroll
+        for (int j = 0; j < NX; ++j) {
+          const float f = j < p.M ? __ldg(p.xs + static_cast<int64_t>(j) * p.KB + kb) * wsf : 0.0f;
+          acc[j] = fmaf(__uint_as_float(r[j]), f, acc[j]);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < NX; ++j) acc[j] += __uint_as_float(r[j]);
+      }
+      if (s + 1 == e || kb + 1 == p.KB) {        // segment ends: publish it
+        float* dst = p.part + (static_cast<int64_t>(t) + c) * NX * 128 + nl;
+#pragma unroll
+        for (int j = 0; j < NX; ++j) {
+          if (j < p.M) dst[j * 128] = acc[j];
+          acc[j] = 0.0f;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+// Sum the segments of every weight tile in CTA order and write bf16 output.
+// grid (n_tiles, M), 128 threads: thread = output channel within the tile.
+template <bool BLOCK>
+__global__ void __launch_bounds__(128) decode_reduce_kernel(const Params p, int nx, __nv_bfloat16* __restrict__ y,
+                                                            int64_t ldy) {
+  const int t = blockIdx.x;
+  const int m = blockIdx.y;
+  const int nl = threadIdx.x;
+  const int n = t * 128 + nl;
+  const int c0 = cta_of_step(static_cast<int64_t>(t) * p.KB, p.total, p.G);
+  const int c1 = cta_of_step(static_cast<int64_t>(t + 1) * p.KB - 1, p.total, p.G);
+  float sum = 0.0f;
+  for (int c = c0; c <= c1; ++c) sum += p.part[((static_cast<int64_t>(t) + c) * nx + m) * 128 + nl];
+  if (n < p.N) {
+    const float v = BLOCK ? sum : sum * __ldg(p.xs + m) * __ldg(p.ws + n);
+    y[static_cast<int64_t>(m) * ldy + n] = __float2bfloat16_rn(v);
+  }
+}
+
+}  // namespace decode
+}  // namespace fp8q

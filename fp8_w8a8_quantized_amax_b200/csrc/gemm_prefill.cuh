@@ -1,0 +1,389 @@
+// gemm_prefill.cuh -- persistent, warp-specialised tcgen05 FP8 GEMM for M > 64.
+//
+//   Y[m, n] = bf16( sum_k E4M3(Xq[m,k]) E4M3(Wq[n,k]) * x_scale[m] * w_scale[n] )   (channel mode)
+//   Y[m, n] = bf16( sum_kb x_scale[m,kb] w_scale[n/128,kb] sum_{k in kb} ... )        (block mode)
+//
+// Roles inside one CTA (one CTA per SM, tiles handed out round-robin):
+//   warp 0      TMA producer: Xq and Wq tiles of 128 K-bytes into a ring of
+//               shared-memory stages (128-byte swizzle), one mbarrier per stage.
+//   warp 1      allocates tensor memory, then one thread issues tcgen05.mma
+//               (E4M3 x E4M3 -> fp32 in TMEM) and tcgen05.commit to release
+//               stages and to publish finished accumulators.
+//   warps 2..   epilogue: tcgen05.ld the fp32 accumulator, apply the scales,
+//               round to bf16 (RNE) and store.
+// Channel mode: tile 128 x 256, two TMEM accumulators of 256 columns, so the
+// epilogue of one tile overlaps the main loop of the next.
+// Block mode: tile 128 x 128 (one weight block wide).  Every 128-wide K slice
+// is accumulated into its own TMEM slot (4 slots of 128 columns); 8 epilogue
+// warps fold each slot into fp32 registers with that slice's scale product.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace fp8q {
+namespace prefill {
+
+constexpr int BM = 128;       // rows of X per tile (UMMA M)
+constexpr int BK = 128;       // K bytes per stage: one 128-byte swizzle row
+constexpr int UMMA_K = 32;    // K of one tcgen05.mma for 8-bit operands
+
+struct Params {
+  const float* xs;
+  const float* ws;
+  __nv_bfloat16* y;
+  int M, N, K;
+  int64_t ldy;
+  int KB;          // ceil(K / 128)
+  int num_m, num_n, num_tiles, group_m;
+};
+
+// Tile order: groups of `group_m` row-blocks, column-blocks within a group,
+// so that the tiles in flight at one time share operands in L2.
+__device__ __forceinline__ void tile_coords(const Params& p, int t, int& mb, int& nb) {
+  const int per_group = p.group_m * p.num_n;
+  const int g = t / per_group;
+  const int first_m = g * p.group_m;
+  const int gm = min(p.group_m, p.num_m - first_m);
+  const int r = t - g * per_group;
+  mb = first_m + r % gm;
+  nb = r / gm;
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+}
+
+template <int BN, int STAGES>
+struct ChannelLayout {
+  static constexpr int kA = BM * BK;
+  static constexpr int kB = BN * BK;
+  static constexpr int kBarOff = STAGES * (kA + kB);
+  static constexpr int kBytes = kBarOff + 256 + 1024;   // + barriers + alignment slack
+};
+
+// ------------------------------------------------------------- channel ---
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+    gemm_channel_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const Params p) {
+  using L = ChannelLayout<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * L::kA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr uint32_t kTmemCols = 2 * BN;   // 512
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+        int mb, nb;
+        tile_coords(p, t, mb, nb);
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], L::kA + L::kB);
+          tma_load_2d(sA + stage * L::kA, &tmA, &full[stage], kb * BK, mb * BM, pol);
+          tma_load_2d(sB + stage * L::kB, &tmB, &full[stage], kb * BK, nb * BN, pol);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Tail: wait until the MMA has released every stage, so that no
+      // tcgen05.commit arrival is still in flight when the CTA exits.
+      for (int i = 0; ok && i < STAGES; ++i) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) break;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, kErrWaitTmemEmpty)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * BN;
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * L::kA);
+          const uint32_t b0 = smem_u32(sB + stage * L::kB);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k)
+            mma_e4m3(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + k * UMMA_K), idesc,
+                     (kb | k) != 0);
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) mma_commit(&tfull[acc]);
+      }
+    }
+  } else {
+    // Epilogue: warp w may read TMEM lanes 32*(w%4) .. +31.
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    int it = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++it) {
+      int mb, nb;
+      tile_coords(p, t, mb, nb);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrWaitTmemFull))) break;
+      tc_fence_after();
+      const int m = mb * BM + row;
+      const bool row_ok = m < p.M;
+      const float xsm = row_ok ? __ldg(p.xs + m) : 0.0f;
+      __nv_bfloat16* yrow = p.y + static_cast<int64_t>(m) * p.ldy;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tmem_base + lane_addr + acc * BN + c, r);
+        tmem_ld_wait();
+        const int n0 = nb * BN + c;
+        if (row_ok) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            if (n0 + j < p.N) {
+              const float* wsp = p.ws + n0 + j;
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(r[j + 0]) * xsm * __ldg(wsp + 0),
+                                __uint_as_float(r[j + 1]) * xsm * __ldg(wsp + 1));
+              o.y = pack_bf16x2(__uint_as_float(r[j + 2]) * xsm * __ldg(wsp + 2),
+                                __uint_as_float(r[j + 3]) * xsm * __ldg(wsp + 3));
+              o.z = pack_bf16x2(__uint_as_float(r[j + 4]) * xsm * __ldg(wsp + 4),
+                                __uint_as_float(r[j + 5]) * xsm * __ldg(wsp + 5));
+              o.w = pack_bf16x2(__uint_as_float(r[j + 6]) * xsm * __ldg(wsp + 6),
+                                __uint_as_float(r[j + 7]) * xsm * __ldg(wsp + 7));
+              *reinterpret_cast<uint4*>(yrow + n0 + j) = o;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// --------------------------------------------------------------- block ---
+template <int STAGES>
+struct BlockLayout {
+  static constexpr int BN = 128;
+  static constexpr int kA = BM * BK;
+  static constexpr int kB = BN * BK;
+  static constexpr int kSlots = 4;
+  static constexpr int kBarOff = STAGES * (kA + kB);
+  static constexpr int kBytes = kBarOff + 256 + 1024;
+};
+
+template <int STAGES>
+__global__ void __launch_bounds__(320, 1)
+    gemm_block_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const Params p) {
+  using L = BlockLayout<STAGES>;
+  constexpr int BN = L::BN;
+  constexpr int kSlots = L::kSlots;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * L::kA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* sfull = empty + STAGES;
+  uint64_t* sempty = sfull + kSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + kSlots);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr uint32_t kTmemCols = kSlots * BN;   // 512
+  constexpr int kEpiThreads = 256;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < kSlots; ++a) {
+      mbar_init(&sfull[a], 1);
+      mbar_init(&sempty[a], kEpiThreads);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+        int mb, nb;
+        tile_coords(p, t, mb, nb);
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], L::kA + L::kB);
+          tma_load_2d(sA + stage * L::kA, &tmA, &full[stage], kb * BK, mb * BM, pol);
+          tma_load_2d(sB + stage * L::kB, &tmB, &full[stage], kb * BK, nb * BN, pol);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      for (int i = 0; ok && i < STAGES; ++i) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) break;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      int stage = 0, slot = 0;
+      uint32_t phase = 0, sphase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!mbar_wait(&sempty[slot], sphase ^ 1u, abort_flag, kErrWaitTmemEmpty)) { ok = false; break; }
+          if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem_base + slot * BN;
+          const uint32_t a0 = smem_u32(sA + stage * L::kA);
+          const uint32_t b0 = smem_u32(sB + stage * L::kB);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k)
+            mma_e4m3(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + k * UMMA_K), idesc, k != 0);
+          mma_commit(&empty[stage]);
+          mma_commit(&sfull[slot]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
+        }
+      }
+    }
+  } else {
+    // 8 epilogue warps: two per TMEM lane quarter, each owning 64 columns.
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    int slot = 0;
+    uint32_t sphase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+      int mb, nb;
+      tile_coords(p, t, mb, nb);
+      const int m = mb * BM + row;
+      const bool row_ok = m < p.M;
+      const float* xsrow = p.xs + static_cast<int64_t>(m) * p.KB;
+      const float* wsrow = p.ws + static_cast<int64_t>(nb) * p.KB;
+      float acc[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+      float f_next = row_ok ? __ldg(xsrow) * __ldg(wsrow) : 0.0f;
+      for (int kb = 0; kb < p.KB; ++kb) {
+        const float f = f_next;
+        if (kb + 1 < p.KB) f_next = row_ok ? __ldg(xsrow + kb + 1) * __ldg(wsrow + kb + 1) : 0.0f;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sfull[slot], sphase, abort_flag, kErrWaitTmemFull))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t r0[32], r1[32];
+        __syncwarp();
+        const uint32_t a = tmem_base + lane_addr + slot * BN + half * 64;
+        tmem_ld_32x32b_x32(a, r0);
+        tmem_ld_32x32b_x32(a + 32, r1);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&sempty[slot]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          acc[j] = fmaf(__uint_as_float(r0[j]), f, acc[j]);
+          acc[32 + j] = fmaf(__uint_as_float(r1[j]), f, acc[32 + j]);
+        }
+        if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
+      }
+      if (!ok) break;
+      if (row_ok) {
+        __nv_bfloat16* yrow = p.y + static_cast<int64_t>(m) * p.ldy;
+        const int n0 = nb * BN + half * 64;
+#pragma unroll
+        for (int j = 0; j < 64; j += 8) {
+          if (n0 + j < p.N) {
+            uint4 o;
+            o.x = pack_bf16x2(acc[j + 0], acc[j + 1]);
+            o.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
+            o.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
+            o.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
+            *reinterpret_cast<uint4*>(yrow + n0 + j) = o;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace prefill
+}  // namespace fp8q

@@ -1,0 +1,163 @@
+// quant.cuh -- bf16 -> E4M3 quantization kernels (HBM-bound).
+//
+// Every unit (a row, a 128-group of a row, a 128x128 block) is read once into
+// registers with 16-byte loads, its amax found, and its codes written:
+//   scale = amax / 448 (IEEE fp32 division; 1 when amax == 0)
+//   code  = cvt.rn.satfinite.e4m3(x / scale)   (IEEE fp32 quotient first)
+// The amax runs on the packed bf16 bit patterns: with the sign bit cleared,
+// non-negative bf16 values order exactly like their 16-bit patterns, so an
+// unsigned SIMD max over halfwords (__vmaxu2) is an exact max of |x|.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace fp8q {
+
+constexpr uint32_t kAbsMask2 = 0x7FFF7FFFu;
+
+__device__ __forceinline__ uint32_t absmax_bits_vec(const uint4& v, uint32_t acc) {
+  acc = __vmaxu2(acc, v.x & kAbsMask2);
+  acc = __vmaxu2(acc, v.y & kAbsMask2);
+  acc = __vmaxu2(acc, v.z & kAbsMask2);
+  acc = __vmaxu2(acc, v.w & kAbsMask2);
+  return acc;
+}
+
+__device__ __forceinline__ uint32_t fold_halves(uint32_t m2) { return max(m2 & 0xFFFFu, m2 >> 16); }
+
+__device__ __forceinline__ float amax_bits_to_float(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+
+__device__ __forceinline__ float scale_of(float amax) { return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f); }
+
+// 8 bf16 (one uint4) -> 8 codes (one uint2), each x / scale in IEEE fp32.
+__device__ __forceinline__ uint2 encode_vec(const uint4& v, float sc) {
+  uint2 o;
+  o.x = cvt_e4m3x2(__fdiv_rn(bf16lo(v.x), sc), __fdiv_rn(bf16hi(v.x), sc)) |
+        (cvt_e4m3x2(__fdiv_rn(bf16lo(v.y), sc), __fdiv_rn(bf16hi(v.y), sc)) << 16);
+  o.y = cvt_e4m3x2(__fdiv_rn(bf16lo(v.z), sc), __fdiv_rn(bf16hi(v.z), sc)) |
+        (cvt_e4m3x2(__fdiv_rn(bf16lo(v.w), sc), __fdiv_rn(bf16hi(v.w), sc)) << 16);
+  return o;
+}
+
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+
+// ---------------------------------------------------------------- rows ---
+// One CTA per row (per token of X, or per output channel of W).  Thread t
+// holds vectors t, t + T, ..., t + (VPT-1) T of the row, T = blockDim.x.
+template <int VPT>
+__global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __restrict__ x, int K, int64_t ldx,
+                                                         uint8_t* __restrict__ q, int64_t ldq,
+                                                         float* __restrict__ s) {
+  __shared__ uint32_t red[32];
+  const int64_t r = blockIdx.x;
+  const int nvec = K >> 3;
+  const int T = blockDim.x;
+  const uint16_t* xr = x + r * ldx;
+  uint4 v[VPT];
+  uint32_t m2 = 0;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = threadIdx.x + i * T;
+    if (idx < nvec) {
+      v[i] = ld_stream16(xr + idx * 8);
+      m2 = absmax_bits_vec(v[i], m2);
+    }
+  }
+  uint32_t m = __reduce_max_sync(0xFFFFFFFFu, fold_halves(m2));
+  if (T > 32) {
+    const int warp = threadIdx.x >> 5, nw = T >> 5;
+    if (lane_id() == 0) red[warp] = m;
+    __syncthreads();
+    m = lane_id() < nw ? red[lane_id()] : 0u;
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+  }
+  const float sc = scale_of(amax_bits_to_float(m));
+  if (threadIdx.x == 0) s[r] = sc;
+  uint8_t* qr = q + r * ldq;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = threadIdx.x + i * T;
+    if (idx < nvec) *reinterpret_cast<uint2*>(qr + idx * 8) = encode_vec(v[i], sc);
+  }
+}
+
+// ----------------------------------------------------------- groups 128 ---
+// Groups of 128 features: 16 consecutive lanes (a half warp) own one group,
+// one 16-byte vector each.  Each half warp walks GPT groups, strided by the
+// number of half warps in the grid, with all loads issued before any reduce.
+template <int GPT>
+__global__ void __launch_bounds__(256) quant_groups128_kernel(const uint16_t* __restrict__ x, int64_t M, int G,
+                                                             int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
+                                                             float* __restrict__ s) {
+  const int64_t total = M * static_cast<int64_t>(G);
+  const int sub = threadIdx.x & 15;
+  const uint32_t half_mask = 0xFFFFu << (threadIdx.x & 16);
+  const int64_t nhalf = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 4);
+  const int64_t h = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+  for (int64_t base = h; base < total; base += nhalf * GPT) {
+    uint4 v[GPT];
+#pragma unroll
+    for (int i = 0; i < GPT; ++i) {
+      const int64_t gi = base + i * nhalf;
+      if (gi < total) {
+        const int64_t m = gi / G, g = gi - m * G;
+        v[i] = ld_stream16(x + m * ldx + g * 128 + sub * 8);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < GPT; ++i) {
+      const int64_t gi = base + i * nhalf;
+      if (gi < total) {  // uniform across the half warp
+        uint32_t mm = fold_halves(absmax_bits_vec(v[i], 0u));
+        mm = max(mm, __shfl_xor_sync(half_mask, mm, 8, 16));
+        mm = max(mm, __shfl_xor_sync(half_mask, mm, 4, 16));
+        mm = max(mm, __shfl_xor_sync(half_mask, mm, 2, 16));
+        mm = max(mm, __shfl_xor_sync(half_mask, mm, 1, 16));
+        const float sc = scale_of(amax_bits_to_float(mm));
+        const int64_t m = gi / G, g = gi - m * G;
+        if (sub == 0) s[gi] = sc;
+        *reinterpret_cast<uint2*>(q + m * ldq + g * 128 + sub * 8) = encode_vec(v[i], sc);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------- blocks 128 ---
+// One CTA of 256 threads per 128 x 128 block of W.  Thread t owns the
+// 16-byte vector (t % 16) of rows t/16 + 16 i, i < 8.  Rows past N are absent
+// (the last row-block may be short) and take no part in the amax.
+__global__ void __launch_bounds__(256) quant_blocks128_kernel(const uint16_t* __restrict__ w, int64_t N, int KB,
+                                                             int64_t ldw, uint8_t* __restrict__ q, int64_t ldq,
+                                                             float* __restrict__ s) {
+  __shared__ uint32_t red[8];
+  const int kb = blockIdx.x;
+  const int64_t nb = blockIdx.y;
+  const int vc = threadIdx.x & 15;
+  const int r0 = threadIdx.x >> 4;
+  uint4 v[8];
+  uint32_t m2 = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t row = nb * 128 + r0 + 16 * i;
+    if (row < N) {
+      v[i] = ld_stream16(w + row * ldw + kb * 128 + vc * 8);
+      m2 = absmax_bits_vec(v[i], m2);
+    }
+  }
+  uint32_t m = __reduce_max_sync(0xFFFFFFFFu, fold_halves(m2));
+  if (lane_id() == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = lane_id() < 8 ? red[lane_id()] : 0u;
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  const float sc = scale_of(amax_bits_to_float(m));
+  if (threadIdx.x == 0) s[nb * KB + kb] = sc;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t row = nb * 128 + r0 + 16 * i;
+    if (row < N) *reinterpret_cast<uint2*>(q + row * ldq + kb * 128 + vc * 8) = encode_vec(v[i], sc);
+  }
+}
+
+}  // namespace fp8q

@@ -1,0 +1,145 @@
+/*
+ * fp8q.h -- C ABI of the B200 (sm_100a) FP8 W8A8 linear layer library, libfp8q.so.
+ *
+ * The layer is the one Llama-3.x "FP8-Dynamic" and "FP8-Block" checkpoints use:
+ *
+ *   - Weights are E4M3 codes with one scale per output channel, taken from a
+ *     minmax observer ("Llama-3.1-8B-Instruct-FP8-Dynamic" explainer, FP8 动态量化
+ *     table, weights row; "Llama-3.1-70B-FP8-Dynamic" explainer, section 1.2), or
+ *     one scale per 128 x 128 block ("Llama-3.2-3B-Instruct-FP8-Block" explainer,
+ *     quantization_config table, block_structure [128, 128]).
+ *   - Activations are quantized at run time, one dynamic scale per token (the
+ *     FP8-Dynamic table's input_activations row; 70B explainer FAQ Q2), or one
+ *     per group of 128 input features (FP8-Block table, input activations row).
+ *   - E4M3 has 4 exponent and 3 mantissa bits and tops out at 448 ("Llama 3 精读实录",
+ *     section 2.1).  Codes are the E4M3FN bit patterns (no infinities; 0x7F and
+ *     0xFF are NaN and never produced for finite input).
+ *   - lm_head stays in high precision: it is not passed to this library (same
+ *     tables, ignore row).
+ *
+ * Arithmetic, identical on every path:
+ *   amax  = max |x| over the unit (row, 128-group or 128x128 block), exact in fp32
+ *   scale = amax / 448 as one IEEE fp32 division; 1.0 when amax == 0
+ *   code  = E4M3(x / scale): IEEE fp32 quotient, then round to nearest even,
+ *           saturating to +-448, sign kept (-0 is 0x80)
+ *   Y[m,n] = bf16_rne( acc[m,n] * x_scale[m] * w_scale[n] ),
+ *           acc = fp32 sum over k of E4M3(xq[m,k]) * E4M3(wq[n,k]) (channel mode)
+ *   Y[m,n] = bf16_rne( sum_kb  x_scale[m,kb] * w_scale[n/128,kb] * acc_kb[m,n] )
+ *           with acc_kb the fp32 sum over the 128-wide K slice kb (block mode)
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers owned by the caller.  The library
+ *     never allocates, frees or synchronizes; work is enqueued on `stream`
+ *     (a cudaStream_t passed as void*; NULL is the legacy default stream).
+ *   - Matrices are row-major; ld* arguments are row strides in ELEMENTS.
+ *   - Arguments are checked before anything is launched.  A bad argument
+ *     returns an error status and launches nothing.  A launch failure returns
+ *     FP8Q_ERR_CUDA.  Errors that happen later on the device surface at the
+ *     caller's next synchronization; a kernel whose internal wait runs out
+ *     (about 4 s, which only a broken machine reaches) sets a device-side
+ *     error word that fp8q_device_error() reads.
+ *   - The calls are thread-safe; they keep no state between calls other than
+ *     the device error word and a cached device-attribute table.
+ */
+#ifndef FP8Q_H_
+#define FP8Q_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FP8Q_API __attribute__((visibility("default")))
+#else
+#define FP8Q_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8Q_OK = 0,
+    FP8Q_ERR_INVALID_ARG = 1,     /* null pointer, negative size, bad mode, ...        */
+    FP8Q_ERR_UNSUPPORTED = 2,     /* valid but outside what the kernels cover          */
+    FP8Q_ERR_MISALIGNED = 3,      /* pointer or stride breaks a 16-byte requirement     */
+    FP8Q_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed                  */
+    FP8Q_ERR_DEVICE_TIMEOUT = 5   /* a kernel gave up waiting (see fp8q_device_error)   */
+} fp8q_status;
+
+typedef enum {
+    FP8Q_CHANNEL_TOKEN = 0,       /* W: one scale per output channel; X: one per token  */
+    FP8Q_BLOCK128 = 1             /* W: one per 128x128 block;  X: one per 128-group     */
+} fp8q_mode;
+
+/*
+ * fp8_quant_weight -- quantize a bf16 weight W[N, K] (nn.Linear layout, out x in).
+ *
+ *   W_bf16   [N, ldw] bf16, read-only.  ldw >= K, (ldw * 2) % 16 == 0, 16-byte aligned.
+ *   Wq       [N, ldwq] uint8 E4M3 codes, written.  ldwq >= K, ldwq % 16 == 0, 16-byte aligned.
+ *   w_scale  fp32, written:  [N]                              (FP8Q_CHANNEL_TOKEN)
+ *                            [ceil(N/128), K/128] row-major   (FP8Q_BLOCK128)
+ *   Requirements: N >= 0, K > 0, K % 16 == 0; K % 128 == 0 in block mode.
+ *   In block mode the last row-block may hold fewer than 128 rows; its amax
+ *   covers the rows that exist.
+ */
+FP8Q_API fp8q_status fp8_quant_weight(const void* W_bf16, int64_t N, int64_t K, int64_t ldw, int mode,
+                             uint8_t* Wq, int64_t ldwq, float* w_scale, void* stream);
+
+/*
+ * fp8_quant_act -- quantize bf16 activations X[M, K] (one row per token).
+ *
+ *   X_bf16   [M, ldx] bf16, read-only.  Same stride/alignment rules as W.
+ *   Xq       [M, ldxq] uint8 codes, written.
+ *   x_scale  fp32, written:  [M]                  (FP8Q_CHANNEL_TOKEN, per token)
+ *                            [M, K/128] row-major (FP8Q_BLOCK128, per 128-group)
+ *   Requirements: M >= 0 (M == 0 is a no-op), K > 0, K % 16 == 0;
+ *   K % 128 == 0 in block mode.
+ */
+FP8Q_API fp8q_status fp8_quant_act(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, int mode,
+                          uint8_t* Xq, int64_t ldxq, float* x_scale, void* stream);
+
+/*
+ * fp8_linear -- Y[M, N] = dequant(Xq) . dequant(Wq)^T in bf16, on tcgen05 tensor cores.
+ *
+ *   Xq        [M, K] uint8 codes, contiguous (row stride K), 16-byte aligned.
+ *   x_scale   [M] or [M, K/128] fp32 (as written by fp8_quant_act in `mode`).
+ *   Wq        [N, K] uint8 codes, contiguous, 16-byte aligned.
+ *   w_scale   [N] or [ceil(N/128), K/128] fp32 (as written by fp8_quant_weight).
+ *   Y_bf16    [M, ldy] bf16, written.  ldy >= N, (ldy * 2) % 16 == 0, 16-byte aligned.
+ *   workspace device scratch of at least fp8_linear_workspace_size(M, N, K, mode)
+ *             bytes, 256-byte aligned (may be NULL when that size is 0).  It holds
+ *             fp32 split-K partial sums of the small-M (decode) path; its contents
+ *             need no initialisation and are garbage afterwards.  Two calls that
+ *             run concurrently must not share one workspace.
+ *   Requirements: M >= 0 (M == 0 is a no-op), N > 0, K > 0, K % 16 == 0,
+ *   N % 16 == 0; K % 128 == 0 in block mode.  The mode must be the one both
+ *   operands were quantized with.
+ *   Dispatch: M <= 64 takes the decode kernel (weights streamed once, swap-AB,
+ *   stream-K split over all SMs, then a reduction kernel); larger M takes the
+ *   persistent warp-specialised prefill kernel (no workspace).
+ */
+FP8Q_API fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq,
+                       const float* w_scale, int64_t M, int64_t N, int64_t K, int mode,
+                       void* Y_bf16, int64_t ldy, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/* Bytes of workspace fp8_linear needs for this problem on the current device
+ * (0 for the prefill path).  Returns 0 for invalid arguments as well. */
+FP8Q_API size_t fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int mode);
+
+/* Human-readable name of a status code (static string, never NULL). */
+FP8Q_API const char* fp8q_status_string(int status);
+
+/* Reads the device-side error word of the current device: 0 when no kernel
+ * has given up waiting, otherwise a nonzero code naming the wait site.  It
+ * synchronizes the device.  clear != 0 resets the word to 0 afterwards. */
+FP8Q_API int fp8q_device_error(int clear);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+FP8Q_API int fp8q_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H_ */

@@ -83,6 +83,7 @@ class Gemm:
     K: int
     N: int
     mode: int = CHANNEL_TOKEN
+    x: str = ""          # which activation it reads; GEMMs naming the same one share it
 
     @property
     def flops(self) -> int:
@@ -99,22 +100,26 @@ class Workload:
 def workloads() -> dict:
     """The five workloads, keyed by name."""
     w = {}
-    w["tiny_16x256x512"] = Workload("tiny_16x256x512", [Gemm("tiny", 16, 256, 512)], tiny=True)
+    w["tiny_16x256x512"] = Workload("tiny_16x256x512", [Gemm("tiny", 16, 256, 512, x="x")], tiny=True)
     w["llama3.2-3b_mlp_m2048"] = Workload(
         "llama3.2-3b_mlp_m2048",
-        [Gemm("gate_proj", 2048, 3072, 8192), Gemm("up_proj", 2048, 3072, 8192)])
+        [Gemm("gate_proj", 2048, 3072, 8192, x="mlp_in"), Gemm("up_proj", 2048, 3072, 8192, x="mlp_in")])
     w["llama3.1-8b_layer_m8192"] = Workload(
         "llama3.1-8b_layer_m8192",
-        [Gemm("q_proj", 8192, 4096, 4096), Gemm("k_proj", 8192, 4096, 1024),
-         Gemm("v_proj", 8192, 4096, 1024), Gemm("o_proj", 8192, 4096, 4096),
-         Gemm("gate_proj", 8192, 4096, 14336), Gemm("up_proj", 8192, 4096, 14336),
-         Gemm("down_proj", 8192, 14336, 4096)])
+        [Gemm("q_proj", 8192, 4096, 4096, x="attn_in"), Gemm("k_proj", 8192, 4096, 1024, x="attn_in"),
+         Gemm("v_proj", 8192, 4096, 1024, x="attn_in"), Gemm("o_proj", 8192, 4096, 4096, x="attn_out"),
+         Gemm("gate_proj", 8192, 4096, 14336, x="mlp_in"), Gemm("up_proj", 8192, 4096, 14336, x="mlp_in"),
+         Gemm("down_proj", 8192, 14336, 4096, x="mlp_act")])
     w["llama3.2-3b_block128"] = Workload(
         "llama3.2-3b_block128",
-        [Gemm(f"gate_proj_m{m}", m, 3072, 8192, BLOCK128) for m in (1, 16, 4096)])
+        [Gemm(f"gate_proj_m{m}", m, 3072, 8192, BLOCK128, x=f"mlp_in_m{m}") for m in (1, 16, 4096)])
     g70 = []
     for m in (1, 8, 64, 512, 8192):
-        g70 += [Gemm(f"gate_proj_m{m}", m, 8192, 28672), Gemm(f"up_proj_m{m}", m, 8192, 28672),
-                Gemm(f"down_proj_m{m}", m, 28672, 8192), Gemm(f"qkv_proj_m{m}", m, 8192, 10240)]
+        g70 += [Gemm(f"gate_proj_m{m}", m, 8192, 28672, x=f"mlp_in_m{m}"),
+                Gemm(f"up_proj_m{m}", m, 8192, 28672, x=f"mlp_in_m{m}"),
+                Gemm(f"down_proj_m{m}", m, 28672, 8192, x=f"mlp_act_m{m}"),
+                Gemm(f"qkv_proj_m{m}", m, 8192, 10240, x=f"attn_in_m{m}")]
     w["llama3.1-70b_sweep"] = Workload("llama3.1-70b_sweep", g70)
+    for m in (1, 8, 64, 512, 8192):   # one M of the sweep at a time
+        w[f"llama3.1-70b_m{m}"] = Workload(f"llama3.1-70b_m{m}", [g for g in g70 if g.M == m])
     return w

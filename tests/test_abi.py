@@ -1,0 +1,150 @@
+"""The C-ABI library: it loads, exports every function include/fp8q.h declares,
+and rejects bad arguments before touching CUDA (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import fp8_w8a8_quantized_amax_b200 as fq
+from fp8_w8a8_quantized_amax_b200 import build as fbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", h) for h in os.listdir(os.path.join(ROOT, "include"))
+           if h.endswith(".h")]
+
+
+def declared_functions():
+    names = []
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*FP8Q_API\s+[^;(]*?\b(fp8\w*)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    fbuild.build()
+    return fq.lib()
+
+
+def test_header_declares_the_three_entry_points():
+    d = declared_functions()
+    for n in ("fp8_quant_weight", "fp8_quant_act", "fp8_linear"):
+        assert n in d
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", fq.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT\s+(\w+)", out))
+    for n in declared_functions():
+        assert n in exported, n
+        assert getattr(L, n) is not None
+
+
+def test_library_exports_nothing_else_public(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", fq.LIB_PATH], capture_output=True, text=True).stdout
+    ours = {s for s in re.findall(r"\bT\s+(\w+)", out) if s.startswith("fp8")}
+    assert ours == set(declared_functions())
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert fq.status_string(s).startswith("FP8Q")
+    assert "unknown" in fq.status_string(99)
+
+
+def test_version(L):
+    assert fq.version() >= 100
+
+
+P = 0x10000          # a 16-byte aligned dummy address (never dereferenced here)
+BAD = 0x10001        # misaligned
+
+
+def q_act(L, x=P, M=4, K=256, ldx=256, mode=0, q=P, ldq=256, s=P):
+    return L.fp8_quant_act(x, M, K, ldx, mode, q, ldq, s, None)
+
+
+def q_w(L, w=P, N=4, K=256, ldw=256, mode=0, q=P, ldq=256, s=P):
+    return L.fp8_quant_weight(w, N, K, ldw, mode, q, ldq, s, None)
+
+
+def lin(L, M=4, N=64, K=256, mode=0, y=P, ldy=64, xq=P, xs=P, wq=P, ws=P, wsp=P, wsb=1 << 30):
+    return L.fp8_linear(xq, xs, wq, ws, M, N, K, mode, y, ldy, wsp, wsb, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(mode=2), fq.ERR_INVALID_ARG),
+    (dict(mode=-1), fq.ERR_INVALID_ARG),
+    (dict(K=0), fq.ERR_INVALID_ARG),
+    (dict(K=24, ldx=24, ldq=32), fq.ERR_INVALID_ARG),        # K % 16
+    (dict(M=-1), fq.ERR_INVALID_ARG),
+    (dict(ldx=128), fq.ERR_INVALID_ARG),                     # ld < K
+    (dict(ldq=128), fq.ERR_INVALID_ARG),
+    (dict(x=None), fq.ERR_INVALID_ARG),
+    (dict(q=None), fq.ERR_INVALID_ARG),
+    (dict(s=None), fq.ERR_INVALID_ARG),
+    (dict(x=BAD), fq.ERR_MISALIGNED),
+    (dict(q=P + 8), fq.ERR_MISALIGNED),
+    (dict(ldx=260), fq.ERR_MISALIGNED),
+    (dict(ldq=264), fq.ERR_MISALIGNED),
+    (dict(mode=1, K=192, ldx=192, ldq=192), fq.ERR_INVALID_ARG),   # block mode needs K % 128
+    (dict(M=0, x=None, q=None, s=None), fq.OK),              # empty input is a no-op
+])
+def test_quant_act_argument_checks(L, kw, want):
+    assert q_act(L, **kw) == want
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(mode=3), fq.ERR_INVALID_ARG),
+    (dict(N=-2), fq.ERR_INVALID_ARG),
+    (dict(w=None), fq.ERR_INVALID_ARG),
+    (dict(w=BAD), fq.ERR_MISALIGNED),
+    (dict(mode=1, K=64, ldw=64, ldq=64), fq.ERR_INVALID_ARG),
+    (dict(N=0, w=None, q=None, s=None), fq.OK),
+])
+def test_quant_weight_argument_checks(L, kw, want):
+    assert q_w(L, **kw) == want
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(mode=5), fq.ERR_INVALID_ARG),
+    (dict(N=0), fq.ERR_INVALID_ARG),
+    (dict(N=24, ldy=24), fq.ERR_INVALID_ARG),               # N % 16
+    (dict(K=40), fq.ERR_INVALID_ARG),                       # K % 16
+    (dict(K=272, mode=1), fq.ERR_INVALID_ARG),              # block: K % 128
+    (dict(ldy=32), fq.ERR_INVALID_ARG),                     # ldy < N
+    (dict(ldy=68), fq.ERR_MISALIGNED),
+    (dict(y=BAD), fq.ERR_MISALIGNED),
+    (dict(xq=P + 4), fq.ERR_MISALIGNED),
+    (dict(wq=None), fq.ERR_INVALID_ARG),
+    (dict(xs=None), fq.ERR_INVALID_ARG),
+    (dict(M=-3), fq.ERR_INVALID_ARG),
+    (dict(M=0, xq=None, xs=None, wq=None, ws=None, y=None), fq.OK),
+])
+def test_linear_argument_checks(L, kw, want):
+    assert lin(L, **kw) == want
+
+
+def test_workspace_size_is_zero_for_invalid_or_prefill(L):
+    assert L.fp8_linear_workspace_size(0, 64, 256, 0) == 0
+    assert L.fp8_linear_workspace_size(128, 64, 256, 0) == 0
+    assert L.fp8_linear_workspace_size(4, 64, 256, 9) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="needs a machine without a CUDA device")
+def test_valid_arguments_without_a_gpu_report_cuda_error(L):
+    assert q_act(L) == fq.ERR_CUDA
+    assert q_w(L) == fq.ERR_CUDA
+    assert lin(L) == fq.ERR_CUDA
+
+
+def test_binding_refuses_cpu_tensors(L):
+    with pytest.raises(ValueError):
+        fq.fp8_quant_act(torch.zeros(4, 256, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        fq.fp8_quant_weight(torch.zeros(4, 256, dtype=torch.bfloat16))

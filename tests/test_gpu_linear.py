@@ -1,0 +1,197 @@
+"""GPU FP8 linear (tcgen05 prefill, swap-AB stream-K decode) vs the exact oracle.
+
+Both sides start from the same bf16 inputs; each quantizes with its own code
+(the codes were shown bit-exact separately), and the outputs must agree
+within 4e-3 * max|y_ref| + 1 bf16 ulp elementwise.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import fp8_w8a8_quantized_amax_b200 as fq
+from tests import _parity as P
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from fp8_w8a8_quantized_amax_b200 import build
+    build.build()
+    fq.device_error(clear=True)
+    yield
+    assert fq.device_error(clear=True) == 0
+
+
+def run_gpu(x, w, mode, ldy_pad=0):
+    xd, wd = x.to(DEV), w.to(DEV)
+    wq, ws = fq.fp8_quant_weight(wd, mode)
+    xq, xs = fq.fp8_quant_act(xd, mode)
+    M, N = x.shape[0], w.shape[0]
+    out = None
+    if ldy_pad:
+        out = torch.full((M, N + ldy_pad), 7.0, dtype=torch.bfloat16, device=DEV)[:, :N]
+    y = fq.fp8_linear(xq, xs, wq, ws, mode, out=out)
+    torch.cuda.synchronize()
+    return y, (xq, xs, wq, ws)
+
+
+def check_full(M, N, K, mode, seed=0, ldy_pad=0):
+    x = synth.make_x(M, K, seed=seed)
+    w = synth.make_w(N, K, seed=seed)
+    y, (xq, xs, wq, ws) = run_gpu(x, w, mode, ldy_pad)
+    rxq, rxs = oracle.quant_act(x, mode)
+    rwq, rws = oracle.quant_weight(w, mode)
+    P.assert_codes_equal(xq, rxq, "xq")
+    P.assert_codes_equal(wq, rwq, "wq")
+    yref = oracle.linear(rxq, rxs, rwq, rws, mode)
+    P.assert_y_close(y.float().cpu().numpy(), yref, what=f"Y {M}x{N}x{K} mode {mode}")
+    return y
+
+
+# ----------------------------------------------------------- prefill path ---
+
+@pytest.mark.parametrize("M,N,K", [
+    (65, 16, 16),          # smallest prefill problem: one partial tile everywhere
+    (200, 320, 272),       # ragged M, N (BN=256) and K (128-byte blocks)
+    (129, 512, 256),
+    (384, 768, 1024),      # several tiles in both dimensions, 8 K blocks
+    (2048, 2560, 256),     # 160 tiles > 148 SMs: persistent loop, both accumulators
+])
+def test_prefill_channel(M, N, K):
+    check_full(M, N, K, fq.CHANNEL_TOKEN, seed=M)
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (200, 384, 384),
+    (130, 144, 256),       # a partial 128-row weight block
+    (1024, 3072, 512),     # 192 tiles > 148 SMs
+])
+def test_prefill_block(M, N, K):
+    check_full(M, N, K, fq.BLOCK128, seed=N)
+
+
+def test_prefill_output_stride():
+    check_full(150, 256, 256, fq.CHANNEL_TOKEN, ldy_pad=64)
+
+
+# ------------------------------------------------------------ decode path ---
+
+@pytest.mark.parametrize("M", [1, 2, 8, 16, 17, 31, 32, 33, 64])
+def test_decode_channel_stream_k(M):
+    # 8 weight tiles x 32 K blocks = 256 steps over at most 148 CTAs: segments
+    # cross tile boundaries
+    check_full(M, 1024, 4096, fq.CHANNEL_TOKEN, seed=M)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 400, 1040), (5, 16, 16), (64, 4096, 128)])
+def test_decode_channel_ragged(M, N, K):
+    check_full(M, N, K, fq.CHANNEL_TOKEN, seed=N)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 272, 384), (16, 1024, 2048), (40, 512, 1024), (64, 256, 128)])
+def test_decode_block(M, N, K):
+    check_full(M, N, K, fq.BLOCK128, seed=K)
+
+
+def test_decode_output_stride():
+    check_full(3, 512, 512, fq.CHANNEL_TOKEN, ldy_pad=32)
+
+
+def test_zero_activations_give_zero():
+    x = torch.zeros(70, 256, dtype=torch.bfloat16)
+    w = synth.make_w(128, 256)
+    for M in (70, 4):
+        y, _ = run_gpu(x[:M], w, fq.CHANNEL_TOKEN)
+        assert torch.all(y == 0)
+
+
+def test_empty_m():
+    xq = torch.empty(0, 256, dtype=torch.uint8, device=DEV)
+    xs = torch.empty(0, dtype=torch.float32, device=DEV)
+    wq = torch.zeros(64, 256, dtype=torch.uint8, device=DEV)
+    ws = torch.ones(64, dtype=torch.float32, device=DEV)
+    assert fq.fp8_linear(xq, xs, wq, ws).shape == (0, 64)
+
+
+def test_workspace_too_small_is_rejected():
+    xq = torch.zeros(4, 256, dtype=torch.uint8, device=DEV)
+    xs = torch.ones(4, dtype=torch.float32, device=DEV)
+    wq = torch.zeros(256, 256, dtype=torch.uint8, device=DEV)
+    ws = torch.ones(256, dtype=torch.float32, device=DEV)
+    small = torch.empty(16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(fq.FP8QError) as e:
+        fq.fp8_linear(xq, xs, wq, ws, workspace=small)
+    assert e.value.status == fq.ERR_INVALID_ARG
+
+
+def test_repeat_calls_are_deterministic():
+    x = synth.make_x(8, 2048, seed=3).to(DEV)
+    w = synth.make_w(2048, 2048, seed=3).to(DEV)
+    wq, ws = fq.fp8_quant_weight(w)
+    xq, xs = fq.fp8_quant_act(x)
+    y0 = fq.fp8_linear(xq, xs, wq, ws)
+    for _ in range(3):
+        assert torch.equal(fq.fp8_linear(xq, xs, wq, ws), y0)
+
+
+# ------------------------------------------------ full workload sizes, sampled ---
+
+def _sample(n, k, seed):
+    rng = np.random.default_rng(seed)
+    return np.array(sorted(set([0, n - 1]) | set(rng.integers(0, n, k).tolist())))
+
+
+def _check_sampled(g: synth.Gemm, seed=0):
+    x = synth.make_x_device(g.M, g.K, seed=seed)
+    w = synth.make_w_device(g.N, g.K, seed=seed)
+    mode = g.mode
+    wq, ws = fq.fp8_quant_weight(w, mode)
+    xq, xs = fq.fp8_quant_act(x, mode)
+    y = fq.fp8_linear(xq, xs, wq, ws, mode)
+    torch.cuda.synchronize()
+    ms = _sample(g.M, 30, seed + 1)
+    nblocks = _sample(g.N // 128, 2, seed + 2)          # whole 128-row weight blocks
+    ns = np.concatenate([np.arange(b * 128, b * 128 + 128) for b in nblocks])
+    xsub = x[torch.as_tensor(ms, device=DEV)].cpu()
+    rxq, rxs = oracle.quant_act(xsub, mode)
+    P.assert_codes_equal(xq[torch.as_tensor(ms, device=DEV)], rxq, f"{g.name} xq")
+    rwq, rws = [], []
+    for b in nblocks:
+        q, s = oracle.quant_weight(w[b * 128:(b + 1) * 128].cpu(), mode)
+        rwq.append(q)
+        rws.append(s)
+    rwq = np.concatenate(rwq)
+    rws = np.concatenate(rws)
+    P.assert_codes_equal(wq[torch.as_tensor(ns, device=DEV)], rwq, f"{g.name} wq")
+    yref = oracle.linear(rxq, rxs, rwq, rws, mode)
+    ygpu = y[torch.as_tensor(ms, device=DEV)][:, torch.as_tensor(ns, device=DEV)].float().cpu().numpy()
+    # the tolerance's first term uses the largest |y| of the sampled outputs
+    P.assert_y_close(ygpu, yref, what=f"{g.name} M={g.M} K={g.K} N={g.N}")
+
+
+ALL = synth.workloads()
+FULL = [g for name in ("llama3.2-3b_mlp_m2048", "llama3.1-8b_layer_m8192", "llama3.2-3b_block128",
+                       "llama3.1-70b_sweep") for g in ALL[name].gemms]
+
+
+@pytest.mark.parametrize("g", FULL, ids=[f"{g.name}-{g.M}x{g.K}x{g.N}-m{g.mode}" for g in FULL])
+def test_full_size_sampled(g):
+    _check_sampled(g)
+
+
+def test_tiny_workload_in_full():
+    g = ALL["tiny_16x256x512"].gemms[0]
+    x = synth.make_x(g.M, g.K, seed=0, n_out=2)
+    w = synth.make_w(g.N, g.K, seed=0)
+    y, (xq, xs, wq, ws) = run_gpu(x, w, fq.CHANNEL_TOKEN)
+    rxq, rxs = oracle.quant_rows(x)
+    rwq, rws = oracle.quant_rows(w)
+    P.assert_codes_equal(xq, rxq, "tiny xq")
+    P.assert_scales_equal(xs, rxs, "tiny xs")
+    P.assert_codes_equal(wq, rwq, "tiny wq")
+    P.assert_scales_equal(ws, rws, "tiny ws")
+    P.assert_y_close(y.float().cpu().numpy(), oracle.linear(rxq, rxs, rwq, rws, 0), what="tiny")

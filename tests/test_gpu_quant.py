@@ -1,0 +1,142 @@
+"""GPU quantize kernels vs the oracle: codes and scales bit-exact.
+
+Per-token / per-channel (one amax/448 scale per row), per-128-group and
+per-128x128-block schemes of the FP8-Dynamic and FP8-Block checkpoints.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import fp8_w8a8_quantized_amax_b200 as fq
+from tests import _parity as P
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from fp8_w8a8_quantized_amax_b200 import build
+    build.build()
+    fq.device_error(clear=True)
+    yield
+    assert fq.device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (3, 48), (17, 256), (129, 384), (64, 3072), (5, 4096),
+                                 (2, 14336), (3, 28672), (2, 65536 + 16), (1, 131072)])
+def test_rows_bit_exact(M, K):
+    x = synth.make_x(M, K, seed=M + K)
+    q, s = fq.fp8_quant_act(x.to(DEV), fq.CHANNEL_TOKEN)
+    rq, rs = oracle.quant_rows(x)
+    P.assert_codes_equal(q, rq, f"rows {M}x{K}")
+    P.assert_scales_equal(s, rs, f"rows {M}x{K}")
+
+
+@pytest.mark.parametrize("M,K", [(1, 128), (5, 384), (33, 3072), (300, 256)])
+def test_groups_bit_exact(M, K):
+    x = synth.make_x(M, K, seed=7 * M + K)
+    q, s = fq.fp8_quant_act(x.to(DEV), fq.BLOCK128)
+    rq, rs = oracle.quant_groups128(x)
+    assert tuple(s.shape) == (M, K // 128)
+    P.assert_codes_equal(q, rq, f"groups {M}x{K}")
+    P.assert_scales_equal(s, rs, f"groups {M}x{K}")
+
+
+@pytest.mark.parametrize("N,K", [(128, 128), (300, 256), (1000, 384), (64, 512)])
+def test_blocks_bit_exact(N, K):
+    w = synth.make_w(N, K, seed=N + K)
+    q, s = fq.fp8_quant_weight(w.to(DEV), fq.BLOCK128)
+    rq, rs = oracle.quant_blocks128(w)
+    assert tuple(s.shape) == ((N + 127) // 128, K // 128)
+    P.assert_codes_equal(q, rq, f"blocks {N}x{K}")
+    P.assert_scales_equal(s, rs, f"blocks {N}x{K}")
+
+
+def test_channel_weight_is_per_row():
+    w = synth.make_w(777, 512, seed=3)
+    q, s = fq.fp8_quant_weight(w.to(DEV), fq.CHANNEL_TOKEN)
+    rq, rs = oracle.quant_rows(w)
+    P.assert_codes_equal(q, rq, "channel weight")
+    P.assert_scales_equal(s, rs, "channel weight")
+
+
+def test_special_values():
+    K = 256
+    x = torch.zeros(8, K, dtype=torch.bfloat16)
+    x[1, 3] = -0.0                        # only a negative zero
+    x[2, :] = 1e-30                       # everything tiny (scale ~2e-33)
+    x[3, 0] = 3.0e38                      # huge amax, the rest flushed to +-0
+    x[3, 1:] = -1.0
+    x[4, :] = torch.linspace(-448, 448, K)
+    x[5, ::2] = 1.0
+    x[5, 1::2] = -1.0
+    x[6, 7] = 2.0 ** -133                 # smallest bf16 subnormal as the amax
+    x[7] = synth.make_x(1, K, seed=9)[0]
+    x[7, 5] = -x[7].abs().max()           # negative amax
+    for mode in (fq.CHANNEL_TOKEN, fq.BLOCK128):
+        q, s = fq.fp8_quant_act(x.to(DEV), mode)
+        rq, rs = oracle.quant_act(x, mode)
+        P.assert_codes_equal(q, rq, f"special mode {mode}")
+        P.assert_scales_equal(s, rs, f"special mode {mode}")
+
+
+def test_strided_input_and_output():
+    M, K = 37, 384
+    big = synth.make_x(M, 1024, seed=5).to(DEV)
+    x = big[:, 128:128 + K]               # row stride 1024 elements
+    qbuf = torch.full((M, 512), 0xAB, dtype=torch.uint8, device=DEV)
+    q = qbuf[:, :K]
+    s = torch.empty(M, dtype=torch.float32, device=DEV)
+    fq.fp8_quant_act(x, fq.CHANNEL_TOKEN, out=(q, s))
+    rq, rs = oracle.quant_rows(x.cpu().contiguous())
+    P.assert_codes_equal(q, rq, "strided")
+    P.assert_scales_equal(s, rs, "strided")
+    assert torch.all(qbuf[:, K:] == 0xAB)     # nothing written past K
+
+
+def test_empty_rows():
+    x = torch.empty(0, 256, dtype=torch.bfloat16, device=DEV)
+    q, s = fq.fp8_quant_act(x)
+    assert q.shape == (0, 256) and s.shape == (0,)
+
+
+def _sampled_rows(n, k=24, seed=0):
+    rng = np.random.default_rng(seed)
+    r = set([0, n - 1]) | set(rng.integers(0, n, k).tolist())
+    return np.array(sorted(r))
+
+
+@pytest.mark.parametrize("M,K", [(8192, 4096), (8192, 14336), (8192, 28672), (2048, 3072)])
+def test_full_size_activation_rows(M, K):
+    x = synth.make_x_device(M, K, seed=11)
+    q, s = fq.fp8_quant_act(x, fq.CHANNEL_TOKEN)
+    rows = _sampled_rows(M)
+    rq, rs = P.oracle_rows_for(x.cpu(), rows, fq.CHANNEL_TOKEN)
+    P.assert_codes_equal(q[torch.as_tensor(rows, device=DEV)], rq, f"act {M}x{K}")
+    P.assert_scales_equal(s[torch.as_tensor(rows, device=DEV)], rs, f"act {M}x{K}")
+
+
+@pytest.mark.parametrize("N,K", [(28672, 8192), (8192, 28672), (10240, 8192), (14336, 4096)])
+def test_full_size_weight_rows(N, K):
+    w = synth.make_w_device(N, K, seed=13)
+    q, s = fq.fp8_quant_weight(w, fq.CHANNEL_TOKEN)
+    rows = _sampled_rows(N)
+    rq, rs = oracle.quant_rows(w[torch.as_tensor(rows, device=DEV)].cpu())
+    P.assert_codes_equal(q[torch.as_tensor(rows, device=DEV)], rq, f"weight {N}x{K}")
+    P.assert_scales_equal(s[torch.as_tensor(rows, device=DEV)], rs, f"weight {N}x{K}")
+
+
+def test_full_size_block_weight_and_groups():
+    w = synth.make_w(8192, 3072, seed=0)
+    q, s = fq.fp8_quant_weight(w.to(DEV), fq.BLOCK128)
+    rq, rs = oracle.quant_blocks128(w)
+    P.assert_codes_equal(q, rq, "block weight 8192x3072")
+    P.assert_scales_equal(s, rs, "block weight 8192x3072")
+    x = synth.make_x(4096, 3072, seed=0)
+    q, s = fq.fp8_quant_act(x.to(DEV), fq.BLOCK128)
+    rq, rs = oracle.quant_groups128(x)
+    P.assert_codes_equal(q, rq, "groups 4096x3072")
+    P.assert_scales_equal(s, rs, "groups 4096x3072")

@@ -57,7 +57,19 @@ def parse():
                     help="rows of every GEMM one reference-arm step runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", default="",
+                    help="comma-separated GEMM names: restrict the workload to them (profiling)")
     return ap.parse_args()
+
+
+def select(args):
+    wl = synth.workloads()[args.workload]
+    if args.only:
+        keep = set(args.only.split(","))
+        wl = synth.Workload(wl.name + "[" + args.only + "]", [g for g in wl.gemms if g.name in keep])
+        if not wl.gemms:
+            raise SystemExit(f"--only {args.only}: no such GEMM in {args.workload}")
+    return wl
 
 
 def peaks():
@@ -206,7 +218,7 @@ def run_gpu(args):
     from fp8_w8a8_quantized_amax_b200 import build as fbuild
     fbuild.build()
     dev = torch.device("cuda", local)
-    wl = synth.workloads()[args.workload]
+    wl = select(args)
     metric, unit = metric_for(wl)
     pk = peaks()
 
@@ -454,7 +466,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl = synth.workloads()[args.workload]
+    wl = select(args)
     metric, unit = metric_for(wl)
     rows = args.ref_sample_rows
     cache = {}

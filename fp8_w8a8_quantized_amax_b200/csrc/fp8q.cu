@@ -336,3 +336,72 @@ int fp8q_device_error(int clear) {
 int fp8q_version(void) { return 100; }
 
 }  // extern "C"
+
+// ------------------------------------------------- allocation-free variant ---
+//
+// fp8_linear_noalloc: the small-M (M <= 64) linear with its split-K scratch in
+// a fixed array that lives in the library's device image, for callers that
+// cannot allocate device memory when they call (see fp8q.h).
+namespace {
+
+// Largest scratch the allocation-free entry point can use.  Every GPU that
+// loads libfp8q.so reserves this much device memory until the process exits.
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(16) << 20;   // 16 MiB
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, looked up once per device.  Host code
+// must not pass the symbol itself to a kernel: on the host it names a shadow
+// variable, not device memory.
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+fp8q_status noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FP8Q_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FP8Q_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8q_status fp8_linear_noalloc(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq, const float* w_scale,
+                               int64_t M, int64_t N, int64_t K, int mode, void* Y_bf16, int64_t ldy,
+                               void* stream) {
+  fp8q_status st = check_linear_args(Xq, x_scale, Wq, w_scale, M, N, K, mode, Y_bf16, ldy);
+  if (st != FP8Q_OK || M == 0) return st;
+  if (M > kDecodeMaxM) return FP8Q_ERR_UNSUPPORTED;    // the M > 64 path of fp8_linear needs no scratch
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
+  int n_tiles, G, nx;
+  int64_t total;
+  decode_shape(M, N, K, sms, &n_tiles, &total, &G, &nx);
+  if (decode_workspace_bytes(n_tiles, G, nx) > kNoAllocScratchBytes) return FP8Q_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(dev, &scratch)) != FP8Q_OK) return st;
+  CUtensorMap tw, tx;
+  if ((st = tmap_u8_sw128(&tw, Wq, N, K, K, 128)) != FP8Q_OK) return st;
+  if ((st = tmap_u8_sw128(&tx, Xq, M, K, K, static_cast<uint32_t>(nx))) != FP8Q_OK) return st;
+  Params p;
+  p.xs = x_scale;
+  p.ws = w_scale;
+  p.part = static_cast<float*>(scratch);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.KB = static_cast<int>((K + 127) / 128);
+  p.n_tiles = n_tiles;
+  p.total = total;
+  p.G = G;
+  if (nx == 16) return launch_decode_nx<16>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
+  if (nx == 32) return launch_decode_nx<32>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
+  return launch_decode_nx<64>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
+}
+
+}  // extern "C"

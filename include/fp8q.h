@@ -135,6 +135,37 @@ FP8Q_API const char* fp8q_status_string(int status);
  * synchronizes the device.  clear != 0 resets the word to 0 afterwards. */
 FP8Q_API int fp8q_device_error(int clear);
 
+/*
+ * fp8_linear_noalloc -- fp8_linear for M <= 64 without a caller-supplied workspace.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers that
+ * cannot allocate device memory at the moment they call: plugin or enqueue
+ * interfaces that hand over inputs and outputs but no scratch, code that must
+ * not pay cudaMalloc's implicit device synchronisation on its critical path,
+ * and programs whose device-memory budget is fixed before they run.
+ *
+ * Same arguments, requirements and result as fp8_linear, minus the workspace.
+ * The split-K scratch is instead a fixed array of 16 MiB (16777216 bytes)
+ * compiled into the library: every GPU that loads libfp8q.so holds it until the
+ * process exits.  This call allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library routine).
+ *   - M > 64 returns FP8Q_ERR_UNSUPPORTED: call fp8_linear with a NULL workspace
+ *     there, which needs no scratch and allocates nothing either.
+ *   - A problem whose scratch would exceed the array (the size
+ *     fp8_linear_workspace_size reports) returns FP8Q_ERR_UNSUPPORTED.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array, which keeps whatever the last
+ *     call left in it.  Nothing in it needs to start at zero: each call writes
+ *     every partial sum it later reads.  Calls whose kernels overlap on the GPU
+ *     (different streams, or different host threads) race on the array and give
+ *     wrong results; serialise them.
+ */
+FP8Q_API fp8q_status fp8_linear_noalloc(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq,
+                                        const float* w_scale, int64_t M, int64_t N, int64_t K, int mode,
+                                        void* Y_bf16, int64_t ldy, void* stream);
+
 /* Library version: major * 10000 + minor * 100 + patch. */
 FP8Q_API int fp8q_version(void);
 

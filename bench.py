@@ -324,8 +324,9 @@ def run_gpu(args):
     if os.path.exists(tfile):
         try:
             tr = json.load(open(tfile)).get(f"{args.workload}:{dom['op']}")
-            if tr:
-                roof["traffic"] = tr
+            if tr and tr.get("kernel", "").startswith(dom["kernel"]):
+                roof["traffic"] = tr["bytes"]
+                roof["traffic_source"] = tr["summary"]
         except Exception:
             pass
 

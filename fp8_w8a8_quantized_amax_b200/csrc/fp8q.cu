@@ -110,6 +110,21 @@ fp8q_status tmap_u8_sw128(CUtensorMap* m, const void* base, int64_t rows, int64_
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
+// Row-major bf16 matrix [rows, cols], row stride `ld` elements, tiles of
+// box_rows x 32 columns (64 bytes) with the 64-byte swizzle.
+fp8q_status tmap_bf16_sw64(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                           uint32_t box_rows) {
+  if (get_encode() != FP8Q_OK) return FP8Q_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  cuuint32_t box[2] = {32u, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 // ------------------------------------------------------------ quantization ---
@@ -306,8 +321,10 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
   }
   using L = fp8q::prefill::ChannelLayout<kPrefillBN, kPrefillStages>;
   auto k = fp8q::prefill::gemm_channel_kernel<kPrefillBN, kPrefillStages>;
+  CUtensorMap ty;
+  if ((st = tmap_bf16_sw64(&ty, Y_bf16, M, N, ldy, 32)) != FP8Q_OK) return st;
   if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
-  return launch(k, dim3(grid), dim3(192), L::kBytes, stream, ta, tb, p);
+  return launch(k, dim3(grid), dim3(192), L::kBytes, stream, ta, tb, ty, p);
 }
 
 const char* fp8q_status_string(int status) {

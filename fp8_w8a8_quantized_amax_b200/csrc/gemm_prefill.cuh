@@ -10,7 +10,9 @@
 //               (E4M3 x E4M3 -> fp32 in TMEM) and tcgen05.commit to release
 //               stages and to publish finished accumulators.
 //   warps 2..   epilogue: tcgen05.ld the fp32 accumulator, apply the scales,
-//               round to bf16 (RNE) and store.
+//               round to bf16 (RNE) and store.  Channel mode stages each
+//               32 x 32 output chunk in shared memory (64-byte swizzle,
+//               double-buffered per warp) and writes it with a TMA store.
 // Channel mode: tile 128 x 256, two TMEM accumulators of 256 columns, so the
 // epilogue of one tile overlaps the main loop of the next.
 // Block mode: tile 128 x 128 (one weight block wide).  Every 128-wide K slice
@@ -57,15 +59,18 @@ template <int BN, int STAGES>
 struct ChannelLayout {
   static constexpr int kA = BM * BK;
   static constexpr int kB = BN * BK;
-  static constexpr int kBarOff = STAGES * (kA + kB);
-  static constexpr int kBytes = kBarOff + 256 + 1024;   // + barriers + alignment slack
+  static constexpr int kOutChunk = 32 * 32 * 2;                  // 32 rows x 32 bf16 columns
+  static constexpr int kOutOff = STAGES * (kA + kB);             // 4 warps x 2 staging buffers
+  static constexpr int kWsOff = kOutOff + 4 * 2 * kOutChunk;     // 4 warps x BN w_scale values
+  static constexpr int kBarOff = kWsOff + 4 * BN * 4;
+  static constexpr int kBytes = kBarOff + 256 + 1024;            // + barriers + alignment slack
 };
 
 // ------------------------------------------------------------- channel ---
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
     gemm_channel_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const Params p) {
+                        const __grid_constant__ CUtensorMap tmY, const Params p) {
   using L = ChannelLayout<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -95,6 +100,7 @@ __global__ void __launch_bounds__(192, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -158,51 +164,69 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // Epilogue: warp w may read TMEM lanes 32*(w%4) .. +31.
+    // Epilogue: warp w may read TMEM lanes 32*(w%4) .. +31, i.e. tile rows
+    // 32*(w%4) .. +31; each thread owns one row.
+    const int ew = warp - 2;
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    int it = 0;
+    float* ws_s = reinterpret_cast<float*>(smem + L::kWsOff) + ew * BN;
+    uint8_t* out_s = smem + L::kOutOff + ew * 2 * L::kOutChunk;
+    const int swz = (lane >> 1) & 3;         // 64-byte swizzle of this thread's staging row
+    int it = 0, buf = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++it) {
       int mb, nb;
       tile_coords(p, t, mb, nb);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
+      // Scales of this tile, fetched while the main loop still runs.
+      const int m = mb * BM + quarter * 32 + lane;
+      const float xsm = m < p.M ? __ldg(p.xs + m) : 0.0f;
+      float wv[BN / 32];
+#pragma unroll
+      for (int i = 0; i < BN / 32; ++i) {
+        const int n = nb * BN + i * 32 + lane;
+        wv[i] = n < p.N ? __ldg(p.ws + n) : 0.0f;
+      }
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrWaitTmemFull))) break;
       tc_fence_after();
-      const int m = mb * BM + row;
-      const bool row_ok = m < p.M;
-      const float xsm = row_ok ? __ldg(p.xs + m) : 0.0f;
-      __nv_bfloat16* yrow = p.y + static_cast<int64_t>(m) * p.ldy;
+#pragma unroll
+      for (int i = 0; i < BN / 32; ++i) ws_s[i * 32 + lane] = wv[i];
+      __syncwarp();
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         uint32_t r[32];
         __syncwarp();
         tmem_ld_32x32b_x32(tmem_base + lane_addr + acc * BN + c, r);
         tmem_ld_wait();
-        const int n0 = nb * BN + c;
-        if (row_ok) {
-#pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            if (n0 + j < p.N) {
-              const float* wsp = p.ws + n0 + j;
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(r[j + 0]) * xsm * __ldg(wsp + 0),
-                                __uint_as_float(r[j + 1]) * xsm * __ldg(wsp + 1));
-              o.y = pack_bf16x2(__uint_as_float(r[j + 2]) * xsm * __ldg(wsp + 2),
-                                __uint_as_float(r[j + 3]) * xsm * __ldg(wsp + 3));
-              o.z = pack_bf16x2(__uint_as_float(r[j + 4]) * xsm * __ldg(wsp + 4),
-                                __uint_as_float(r[j + 5]) * xsm * __ldg(wsp + 5));
-              o.w = pack_bf16x2(__uint_as_float(r[j + 6]) * xsm * __ldg(wsp + 6),
-                                __uint_as_float(r[j + 7]) * xsm * __ldg(wsp + 7));
-              *reinterpret_cast<uint4*>(yrow + n0 + j) = o;
-            }
-          }
+        if (c + 32 == BN) {              // accumulator fully read: hand it back to the MMA
+          tc_fence_before();
+          mbar_arrive(&tempty[acc]);
         }
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float2 w = *reinterpret_cast<const float2*>(ws_s + c + 2 * j);
+          pk[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * xsm * w.x, __uint_as_float(r[2 * j + 1]) * xsm * w.y);
+        }
+        // The staging buffer written two chunks ago must have been read by its store.
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        uint8_t* sb = out_s + buf * L::kOutChunk;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(sb + lane * 64 + ((q ^ swz) << 4)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        const int row0 = mb * BM + quarter * 32, col0 = nb * BN + c;
+        if (lane == 0 && row0 < p.M && col0 < p.N) {   // the store clips the rest of the box
+          tma_store_2d(&tmY, sb, col0, row0);
+          bulk_commit();
+        }
+        buf ^= 1;
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
     }
+    if (lane == 0) bulk_wait<0>();
   }
 
   tc_fence_before();

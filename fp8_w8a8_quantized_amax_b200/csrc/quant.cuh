@@ -3,7 +3,7 @@
 // Every unit (a row, a 128-group of a row, a 128x128 block) is read once into
 // registers with 16-byte loads, its amax found, and its codes written:
 //   scale = amax / 448 (IEEE fp32 division; 1 when amax == 0)
-//   code  = cvt.rn.satfinite.e4m3(x / scale)   (IEEE fp32 quotient first)
+//   code  = cvt.rn.satfinite.e4m3(x / scale)   (correctly rounded fp32 quotient first)
 // The amax runs on the packed bf16 bit patterns: with the sign bit cleared,
 // non-negative bf16 values order exactly like their 16-bit patterns, so an
 // unsigned SIMD max over halfwords (__vmaxu2) is an exact max of |x|.
@@ -29,13 +29,48 @@ __device__ __forceinline__ float amax_bits_to_float(uint32_t bits16) { return __
 
 __device__ __forceinline__ float scale_of(float amax) { return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f); }
 
+// x / s, correctly rounded (identical to __fdiv_rn), for many x and one s.
+// With y = RN(1/s) and q = RN(x * y) within one ulp of x / s, Markstein's
+// correction step q' = RN(q + RN(x - q*s) * y) -- the residual x - q*s being
+// exact in an FMA -- gives the correctly rounded quotient when nothing
+// underflows or overflows (P. Markstein, "Computation of elementary functions
+// on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990).  Here
+// |x / s| <= 448 * (1 + 2^-23); for s in [2^-60, 2^60] every intermediate of a
+// quotient that can reach a nonzero E4M3 code stays normal, and quotients
+// below 2^-11 encode to a signed zero either way.  Outside that range the
+// plain IEEE division is used.  Three instructions per element instead of a
+// division; the equality with __fdiv_rn is tested over every (amax, x) pair of
+// bf16 values.
+struct Divider {
+  float s, y;
+  bool fast;
+};
+
+__device__ __forceinline__ Divider make_divider(float s) {
+  Divider d;
+  d.s = s;
+  d.fast = s >= 0x1p-60f && s <= 0x1p60f;
+  d.y = __frcp_rn(s);
+  return d;
+}
+
+__device__ __forceinline__ float divide(float x, const Divider& d) {
+  if (d.fast) {
+    const float q = __fmul_rn(x, d.y);
+    const float r = __fmaf_rn(-q, d.s, x);
+    // copysign: for x = -0 the correction step gives +0; the quotient keeps x's sign
+    return copysignf(__fmaf_rn(r, d.y, q), x);
+  }
+  return __fdiv_rn(x, d.s);
+}
+
 // 8 bf16 (one uint4) -> 8 codes (one uint2), each x / scale in IEEE fp32.
-__device__ __forceinline__ uint2 encode_vec(const uint4& v, float sc) {
+__device__ __forceinline__ uint2 encode_vec(const uint4& v, const Divider& d) {
   uint2 o;
-  o.x = cvt_e4m3x2(__fdiv_rn(bf16lo(v.x), sc), __fdiv_rn(bf16hi(v.x), sc)) |
-        (cvt_e4m3x2(__fdiv_rn(bf16lo(v.y), sc), __fdiv_rn(bf16hi(v.y), sc)) << 16);
-  o.y = cvt_e4m3x2(__fdiv_rn(bf16lo(v.z), sc), __fdiv_rn(bf16hi(v.z), sc)) |
-        (cvt_e4m3x2(__fdiv_rn(bf16lo(v.w), sc), __fdiv_rn(bf16hi(v.w), sc)) << 16);
+  o.x = cvt_e4m3x2(divide(bf16lo(v.x), d), divide(bf16hi(v.x), d)) |
+        (cvt_e4m3x2(divide(bf16lo(v.y), d), divide(bf16hi(v.y), d)) << 16);
+  o.y = cvt_e4m3x2(divide(bf16lo(v.z), d), divide(bf16hi(v.z), d)) |
+        (cvt_e4m3x2(divide(bf16lo(v.w), d), divide(bf16hi(v.w), d)) << 16);
   return o;
 }
 
@@ -75,11 +110,12 @@ __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __rest
   }
   const float sc = scale_of(amax_bits_to_float(m));
   if (threadIdx.x == 0) s[r] = sc;
+  const Divider dv = make_divider(sc);
   uint8_t* qr = q + r * ldq;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int idx = threadIdx.x + i * T;
-    if (idx < nvec) *reinterpret_cast<uint2*>(qr + idx * 8) = encode_vec(v[i], sc);
+    if (idx < nvec) *reinterpret_cast<uint2*>(qr + idx * 8) = encode_vec(v[i], dv);
   }
 }
 
@@ -118,7 +154,7 @@ __global__ void __launch_bounds__(256) quant_groups128_kernel(const uint16_t* __
         const float sc = scale_of(amax_bits_to_float(mm));
         const int64_t m = gi / G, g = gi - m * G;
         if (sub == 0) s[gi] = sc;
-        *reinterpret_cast<uint2*>(q + m * ldq + g * 128 + sub * 8) = encode_vec(v[i], sc);
+        *reinterpret_cast<uint2*>(q + m * ldq + g * 128 + sub * 8) = encode_vec(v[i], make_divider(sc));
       }
     }
   }
@@ -153,10 +189,11 @@ __global__ void __launch_bounds__(256) quant_blocks128_kernel(const uint16_t* __
   m = __reduce_max_sync(0xFFFFFFFFu, m);
   const float sc = scale_of(amax_bits_to_float(m));
   if (threadIdx.x == 0) s[nb * KB + kb] = sc;
+  const Divider dv = make_divider(sc);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int64_t row = nb * 128 + r0 + 16 * i;
-    if (row < N) *reinterpret_cast<uint2*>(q + row * ldq + kb * 128 + vc * 8) = encode_vec(v[i], sc);
+    if (row < N) *reinterpret_cast<uint2*>(q + row * ldq + kb * 128 + vc * 8) = encode_vec(v[i], dv);
   }
 }
 

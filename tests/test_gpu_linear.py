@@ -33,9 +33,12 @@ def run_gpu(x, w, mode, ldy_pad=0):
     M, N = x.shape[0], w.shape[0]
     out = None
     if ldy_pad:
-        out = torch.full((M, N + ldy_pad), 7.0, dtype=torch.bfloat16, device=DEV)[:, :N]
+        full = torch.full((M, N + ldy_pad), 7.0, dtype=torch.bfloat16, device=DEV)
+        out = full[:, :N]
     y = fq.fp8_linear(xq, xs, wq, ws, mode, out=out)
     torch.cuda.synchronize()
+    if ldy_pad:
+        assert torch.all(full[:, N:] == 7.0), "columns past N were written"
     return y, (xq, xs, wq, ws)
 
 
@@ -74,8 +77,10 @@ def test_prefill_block(M, N, K):
     check_full(M, N, K, fq.BLOCK128, seed=N)
 
 
-def test_prefill_output_stride():
-    check_full(150, 256, 256, fq.CHANNEL_TOKEN, ldy_pad=64)
+@pytest.mark.parametrize("mode", [0, 1])
+def test_prefill_output_stride(mode):
+    check_full(150, 256, 256, mode, ldy_pad=64)
+    check_full(300, 272, 384, mode, ldy_pad=40)
 
 
 # ------------------------------------------------------------ decode path ---

@@ -140,3 +140,35 @@ def test_full_size_block_weight_and_groups():
     rq, rs = oracle.quant_groups128(x)
     P.assert_codes_equal(q, rq, "groups 4096x3072")
     P.assert_scales_equal(s, rs, "groups 4096x3072")
+
+
+def test_every_bf16_pair_matches_ieee_division():
+    """The quantizer's division (reciprocal + correction step) against torch's
+    IEEE fp32 division and fp8 cast, for every positive finite bf16 amax and
+    every bf16 x with |x| <= amax (both signs, zeros and subnormals included).
+    Row r holds amax_r first, then all 65536 bf16 patterns with those above
+    amax_r replaced by 0."""
+    allv = torch.arange(65536, dtype=torch.int32).to(torch.int16).view(torch.bfloat16).to(DEV)
+    finite = torch.isfinite(allv.float())
+    allv = torch.where(finite, allv, torch.zeros_like(allv))
+    amax_bits = torch.arange(1, 0x7F80, dtype=torch.int32, device=DEV)   # +subnormals .. max finite
+    K = 65536 + 16
+    chunk = 1024
+    for lo in range(0, amax_bits.numel(), chunk):
+        a = amax_bits[lo:lo + chunk].to(torch.int16).view(torch.bfloat16)
+        R = a.numel()
+        x = torch.zeros((R, K), dtype=torch.bfloat16, device=DEV)
+        x[:, 0] = a
+        keep = allv.float().abs()[None, :] <= a.float()[:, None]
+        x[:, 16:] = torch.where(keep, allv[None, :], torch.zeros((), dtype=torch.bfloat16, device=DEV))
+        q, s = fq.fp8_quant_act(x, fq.CHANNEL_TOKEN)
+        # tensor / tensor: an elementwise IEEE division (dividing by a CPU scalar
+        # would become a multiplication by its reciprocal)
+        s_ref = a.float() / torch.full((R,), 448.0, device=DEV)
+        q_ref = (x.float() / s_ref[:, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+        assert torch.equal(s.view(torch.int32), s_ref.view(torch.int32)), f"scales differ in rows {lo}.."
+        bad = (q != q_ref)
+        if bad.any():
+            r, c = bad.nonzero()[0].tolist()
+            raise AssertionError(f"amax {float(a[r])}: x {float(x[r, c])} gives {int(q[r, c]):#04x}, "
+                                 f"IEEE division {int(q_ref[r, c]):#04x} ({int(bad.sum())} differ in this chunk)")

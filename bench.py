@@ -57,6 +57,8 @@ def parse():
                     help="rows of every GEMM one reference-arm step runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every op from Python each step instead of replaying CUDA graphs")
     ap.add_argument("--only", default="",
                     help="comma-separated GEMM names: restrict the workload to them (profiling)")
     return ap.parse_args()
@@ -245,44 +247,86 @@ def run_gpu(args):
 
     n_ops = len(xs_shapes) + len(wl.gemms)
 
-    def step(ev=None):
-        i = 0
+    def make_ops():
+        ops = []
         for k, (M, K, mode) in xs_shapes.items():
-            fq.fp8_quant_act(X[k], mode, out=XQ[k])
-            if ev is not None:
-                ev[i].record(stream)
-            i += 1
+            ops.append(lambda k=k, mode=mode: fq.fp8_quant_act(X[k], mode, out=XQ[k]))
         for g in wl.gemms:
-            xq, xsc = XQ[g.x]
-            wq, wsc = WQ[g.name]
-            fq.fp8_linear(xq, xsc, wq, wsc, g.mode, out=Y[g.name], workspace=WS[g.name])
-            if ev is not None:
-                ev[i].record(stream)
-            i += 1
+            def op(g=g):
+                xq, xsc = XQ[g.x]
+                wq, wsc = WQ[g.name]
+                fq.fp8_linear(xq, xsc, wq, wsc, g.mode, out=Y[g.name], workspace=WS[g.name])
+            ops.append(op)
+        return ops
 
+    ops = make_ops()
     for _ in range(args.warmup):
         flush.zero_()
-        step()
+        for op in ops:
+            op()
     torch.cuda.synchronize()
     assert fq.device_error(clear=True) == 0
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ops + 1)] for _ in range(args.steps)]
+    def capture(fns):
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for f in fns:
+                    f()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        return g
+
+    # The step as one CUDA graph (kernels of consecutive ops overlap their
+    # launch through programmatic dependent launch); each op also as its own
+    # graph, timed alone for the per-kernel figures.
+    if args.eager:
+        step_runner = lambda: [op() for op in ops]
+        op_runners = ops
+    else:
+        step_graph = capture(ops)
+        op_graphs = [capture([op]) for op in ops]
+        step_runner = step_graph.replay
+        op_runners = [g.replay for g in op_graphs]
+        for _ in range(2):
+            step_runner()
+            for r in op_runners:
+                r()
+        torch.cuda.synchronize()
+
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        torch.cuda._sleep(2_000_000)          # lets the host queue ahead of the device
         for s in range(args.steps):
             flush.zero_()
-            events[s][0].record(stream)
-            step(events[s][1:])
+            step_ev[s][0].record(stream)
+            step_runner()
+            step_ev[s][1].record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    step_ms = [events[s][0].elapsed_time(events[s][n_ops]) for s in range(args.steps)]
-    op_ms = np.array([[events[s][i].elapsed_time(events[s][i + 1]) for i in range(n_ops)]
-                      for s in range(args.steps)]).mean(axis=0)
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
     total_s = sum(step_ms) / 1e3
     total_s = max_over_ranks(total_s, world)
     units = step_units(wl, unit) * args.steps
     value = to_metric(sum_over_ranks(units, world), total_s, unit)
+
+    # per-op times: every op timed alone after its own L2 flush
+    op_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_ops)] for _ in range(args.steps)]
+    torch.cuda._sleep(2_000_000)
+    for s in range(args.steps):
+        for i, r in enumerate(op_runners):
+            flush.zero_()
+            op_ev[s][i][0].record(stream)
+            r()
+            op_ev[s][i][1].record(stream)
+    torch.cuda.synchronize()
+    op_ms = np.array([[a.elapsed_time(b) for a, b in row] for row in op_ev]).mean(axis=0)
     err = fq.device_error(clear=True)
 
     # ---- per-kernel detail and the dominant kernel's roofline
@@ -401,6 +445,8 @@ def run_gpu(args):
                                  for g in wl.gemms],
                        "step": "quantize each activation + every FP8 GEMM; weights quantized at load",
                        "l2": f"flushed ({args.flush_mib} MiB write) before every step, outside the timed events",
+                       "launch": "eager" if args.eager else
+                       "step: one CUDA graph replayed per step; per-op detail: each op's own graph, timed alone",
                        "parallelism": "single GPU" if world == 1 else f"token-parallel x{world}, weights replicated"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g) for g in wl.gemms)),

@@ -74,8 +74,14 @@ fp8q_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;
+  // Programmatic dependent launch: the kernel may begin while its stream
+  // predecessor finishes; every kernel here waits (griddepcontrol.wait)
+  // before touching global memory.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
@@ -164,7 +170,8 @@ fp8q_status launch_rows(const uint16_t* x, int64_t rows, int K, int64_t ldx, uin
 constexpr int kPrefillBN = 256;
 constexpr int kPrefillStages = 4;
 constexpr int kBlockStages = 6;
-constexpr int kDecodeStages = 8;
+template <int NX>
+constexpr int decode_stages() { return NX == 16 ? 12 : (NX == 32 ? 10 : 8); }
 constexpr int kDecodeMaxM = 64;
 
 int decode_nx(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
@@ -199,6 +206,7 @@ fp8q_status check_linear_args(const uint8_t* Xq, const float* xs, const uint8_t*
 template <int NX>
 fp8q_status launch_decode_nx(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p, int mode, int dev,
                              void* Y, int64_t ldy, void* stream) {
+  constexpr int kDecodeStages = decode_stages<NX>();
   using L = fp8q::decode::Layout<NX, kDecodeStages>;
   fp8q_status st;
   if (mode == FP8Q_BLOCK128) {

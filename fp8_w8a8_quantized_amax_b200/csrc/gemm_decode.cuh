@@ -17,8 +17,11 @@
 // N * K weight bytes.
 //
 // Roles: warp 0 TMA (W tile 128 x 128 B evict-first + X tile NX x 128 B),
-// warp 1 TMEM allocation + MMA issue (one TMEM slot of NX columns per step,
-// 4 slots), warps 2..5 fold each slot into registers and write segments.
+// warp 1 TMEM allocation + MMA issue, warps 2..5 drain TMEM and write
+// segments.  TMEM holds 4 slots of NX columns.  Channel mode accumulates a
+// whole segment in one slot (drained once per segment); block mode gives
+// every K block its own slot, folded into registers with that block's
+// x_scale * w_scale.
 #pragma once
 
 #include "ptx.cuh"
@@ -58,7 +61,10 @@ struct Layout {
   static constexpr int kW = 128 * BK;
   static constexpr int kX = NX * BK;
   static constexpr int kBarOff = STAGES * (kW + kX);
-  static constexpr int kBytes = kBarOff + 256 + 1024;
+  static constexpr int kBarBytes = (2 * STAGES + 2 * kSlots) * 8 + 8;   // mbarriers, TMEM address, abort flag
+  static constexpr int kBytes = kBarOff + 1024 + 1024;                  // + barrier area + alignment slack
+  static_assert(kBarBytes <= 1024, "barrier area");
+  static_assert(kBytes <= 232448, "shared memory per CTA");
   static constexpr uint32_t kTmemCols = (kSlots * NX) < 32 ? 32 : (kSlots * NX);
 };
 
@@ -107,6 +113,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();   // global memory only from here on
 
   if (warp == 0) {
     if (lane == 0) {
@@ -124,6 +131,7 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_2d(sX + stage * L::kX, &tmX, &full[stage], kb * BK, 0, pol_x);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
+      griddep_launch_dependents();
       for (int i = 0; ok && i < STAGES; ++i) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) break;
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -135,7 +143,14 @@ __global__ void __launch_bounds__(192, 1)
       int stage = 0, slot = 0;
       uint32_t phase = 0, sphase = 0;
       for (int64_t s = b; s < e; ++s) {
-        if (!mbar_wait(&sempty[slot], sphase ^ 1u, abort_flag, kErrWaitTmemEmpty)) break;
+        const int64_t t = s / p.KB;
+        const bool seg_first = (s == b) || (s - t * p.KB == 0);
+        const bool seg_last = (s + 1 == e) || (s + 1 - t * p.KB == p.KB);
+        // Block mode: one TMEM slot per K block (its scales differ).  Channel
+        // mode: one slot per segment, accumulated across its K blocks.
+        const bool open_slot = BLOCK || seg_first;
+        const bool close_slot = BLOCK || seg_last;
+        if (open_slot && !mbar_wait(&sempty[slot], sphase ^ 1u, abort_flag, kErrWaitTmemEmpty)) break;
         if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + slot * NX;
@@ -143,11 +158,14 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t b0 = smem_u32(sX + stage * L::kX);
 #pragma unroll
         for (int k = 0; k < BK / UMMA_K; ++k)
-          mma_e4m3(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + k * UMMA_K), idesc, k != 0);
+          mma_e4m3(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + k * UMMA_K), idesc,
+                   (!open_slot || k != 0) ? 1u : 0u);
         mma_commit(&empty[stage]);
-        mma_commit(&sfull[slot]);
+        if (close_slot) {
+          mma_commit(&sfull[slot]);
+          if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
+        }
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
       }
     }
   } else {
@@ -162,6 +180,8 @@ __global__ void __launch_bounds__(192, 1)
     for (int64_t s = b; s < e; ++s) {
       const int t = static_cast<int>(s / p.KB);
       const int kb = static_cast<int>(s - static_cast<int64_t>(t) * p.KB);
+      const bool seg_last = (s + 1 == e) || (kb + 1 == p.KB);
+      if (!BLOCK && !seg_last) continue;           // channel mode: one drain per segment
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sfull[slot], sphase, abort_flag, kErrWaitTmemFull))) break;
       tc_fence_after();
       uint32_t r[NX];
@@ -182,9 +202,9 @@ __global__ void __launch_bounds__(192, 1)
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < NX; ++j) acc[j] += __uint_as_float(r[j]);
+        for (int j = 0; j < NX; ++j) acc[j] = __uint_as_float(r[j]);
       }
-      if (s + 1 == e || kb + 1 == p.KB) {        // segment ends: publish it
+      if (seg_last) {                              // segment ends: publish it
         float* dst = p.part + (static_cast<int64_t>(t) + c) * NX * 128 + nl;
 #pragma unroll
         for (int j = 0; j < NX; ++j) {
@@ -209,6 +229,7 @@ __global__ void __launch_bounds__(192, 1)
 template <bool BLOCK>
 __global__ void __launch_bounds__(128) decode_reduce_kernel(const Params p, int nx, __nv_bfloat16* __restrict__ y,
                                                             int64_t ldy) {
+  griddep_wait();
   const int t = blockIdx.x;
   const int m = blockIdx.y;
   const int nl = threadIdx.x;

@@ -63,7 +63,10 @@ struct ChannelLayout {
   static constexpr int kOutOff = STAGES * (kA + kB);             // 4 warps x 2 staging buffers
   static constexpr int kWsOff = kOutOff + 4 * 2 * kOutChunk;     // 4 warps x BN w_scale values
   static constexpr int kBarOff = kWsOff + 4 * BN * 4;
-  static constexpr int kBytes = kBarOff + 256 + 1024;            // + barriers + alignment slack
+  static constexpr int kBarBytes = (2 * STAGES + 4) * 8 + 8;    // mbarriers, TMEM address, abort flag
+  static constexpr int kBytes = kBarOff + 1024 + 1024;           // + barrier area + alignment slack
+  static_assert(kBarBytes <= 1024, "barrier area");
+  static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
 // ------------------------------------------------------------- channel ---
@@ -110,6 +113,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();   // global memory only from here on
 
   if (warp == 0) {
     if (lane == 0) {
@@ -128,6 +132,7 @@ __global__ void __launch_bounds__(192, 1)
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
+      griddep_launch_dependents();
       // Tail: wait until the MMA has released every stage, so that no
       // tcgen05.commit arrival is still in flight when the CTA exits.
       for (int i = 0; ok && i < STAGES; ++i) {
@@ -246,7 +251,10 @@ struct BlockLayout {
   static constexpr int kB = BN * BK;
   static constexpr int kSlots = 4;
   static constexpr int kBarOff = STAGES * (kA + kB);
-  static constexpr int kBytes = kBarOff + 256 + 1024;
+  static constexpr int kBarBytes = (2 * STAGES + 2 * kSlots) * 8 + 8;
+  static constexpr int kBytes = kBarOff + 1024 + 1024;
+  static_assert(kBarBytes <= 1024, "barrier area");
+  static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
 template <int STAGES>
@@ -294,6 +302,7 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();   // global memory only from here on
 
   if (warp == 0) {
     if (lane == 0) {
@@ -312,6 +321,7 @@ __global__ void __launch_bounds__(320, 1)
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
+      griddep_launch_dependents();
       for (int i = 0; ok && i < STAGES; ++i) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) break;
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }

@@ -13,17 +13,20 @@
 
 namespace fp8q {
 
-constexpr uint32_t kAbsMask2 = 0x7FFF7FFFu;
-
-__device__ __forceinline__ uint32_t absmax_bits_vec(const uint4& v, uint32_t acc) {
-  acc = __vmaxu2(acc, v.x & kAbsMask2);
-  acc = __vmaxu2(acc, v.y & kAbsMask2);
-  acc = __vmaxu2(acc, v.z & kAbsMask2);
-  acc = __vmaxu2(acc, v.w & kAbsMask2);
-  return acc;
+// max(|a|, |b|) for each bf16 half (sign bit of the result is not meaningful).
+__device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
-__device__ __forceinline__ uint32_t fold_halves(uint32_t m2) { return max(m2 & 0xFFFFu, m2 >> 16); }
+__device__ __forceinline__ uint32_t absmax_bits_vec(const uint4& v, uint32_t acc) {
+  return absmax2(absmax2(acc, v.x), absmax2(absmax2(v.y, v.z), v.w));
+}
+
+// Largest magnitude of the two halves as a 15-bit pattern.  Non-negative bf16
+// values order exactly like their bit patterns, so an unsigned max is exact.
+__device__ __forceinline__ uint32_t fold_halves(uint32_t m2) { return max(m2 & 0x7FFFu, (m2 >> 16) & 0x7FFFu); }
 
 __device__ __forceinline__ float amax_bits_to_float(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
@@ -54,23 +57,54 @@ __device__ __forceinline__ Divider make_divider(float s) {
   return d;
 }
 
-__device__ __forceinline__ float divide(float x, const Divider& d) {
-  if (d.fast) {
-    const float q = __fmul_rn(x, d.y);
-    const float r = __fmaf_rn(-q, d.s, x);
-    // copysign: for x = -0 the correction step gives +0; the quotient keeps x's sign
-    return copysignf(__fmaf_rn(r, d.y, q), x);
-  }
-  return __fdiv_rn(x, d.s);
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
 }
 
-// 8 bf16 (one uint4) -> 8 codes (one uint2), each x / scale in IEEE fp32.
+// Codes of the two bf16 values packed in w (low half first), divided by s.
+template <bool FAST>
+__device__ __forceinline__ uint32_t encode_pair(uint32_t w, const Divider& d, uint64_t y2, uint64_t ns2) {
+  const float xl = bf16lo(w), xh = bf16hi(w);
+  float ql, qh;
+  if constexpr (FAST) {
+    // packed fp32x2: q = x*y; r = x - q*s (exact); q' = q + r*y
+    const uint64_t x2 = f32x2_pack(xl, xh);
+    const uint64_t q2 = mul_f32x2(x2, y2);
+    const uint64_t r2 = fma_f32x2(q2, ns2, x2);
+    f32x2_unpack(fma_f32x2(r2, y2, q2), ql, qh);
+    // for x = -0 the correction gives +0; the quotient keeps the sign of x
+    ql = copysignf(ql, xl);
+    qh = copysignf(qh, xh);
+  } else {
+    ql = __fdiv_rn(xl, d.s);
+    qh = __fdiv_rn(xh, d.s);
+  }
+  return cvt_e4m3x2(ql, qh);
+}
+
+// 8 bf16 (one uint4) -> 8 codes (one uint2).
+template <bool FAST>
 __device__ __forceinline__ uint2 encode_vec(const uint4& v, const Divider& d) {
+  const uint64_t y2 = f32x2_pack(d.y, d.y);
+  const uint64_t ns2 = f32x2_pack(-d.s, -d.s);
   uint2 o;
-  o.x = cvt_e4m3x2(divide(bf16lo(v.x), d), divide(bf16hi(v.x), d)) |
-        (cvt_e4m3x2(divide(bf16lo(v.y), d), divide(bf16hi(v.y), d)) << 16);
-  o.y = cvt_e4m3x2(divide(bf16lo(v.z), d), divide(bf16hi(v.z), d)) |
-        (cvt_e4m3x2(divide(bf16lo(v.w), d), divide(bf16hi(v.w), d)) << 16);
+  o.x = encode_pair<FAST>(v.x, d, y2, ns2) | (encode_pair<FAST>(v.y, d, y2, ns2) << 16);
+  o.y = encode_pair<FAST>(v.z, d, y2, ns2) | (encode_pair<FAST>(v.w, d, y2, ns2) << 16);
   return o;
 }
 
@@ -86,6 +120,7 @@ __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __rest
                                                          uint8_t* __restrict__ q, int64_t ldq,
                                                          float* __restrict__ s) {
   __shared__ uint32_t red[32];
+  griddep_wait();
   const int64_t r = blockIdx.x;
   const int nvec = K >> 3;
   const int T = blockDim.x;
@@ -112,10 +147,18 @@ __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __rest
   if (threadIdx.x == 0) s[r] = sc;
   const Divider dv = make_divider(sc);
   uint8_t* qr = q + r * ldq;
+  if (dv.fast) {
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int idx = threadIdx.x + i * T;
-    if (idx < nvec) *reinterpret_cast<uint2*>(qr + idx * 8) = encode_vec(v[i], dv);
+    for (int i = 0; i < VPT; ++i) {
+      const int idx = threadIdx.x + i * T;
+      if (idx < nvec) *reinterpret_cast<uint2*>(qr + idx * 8) = encode_vec<true>(v[i], dv);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int idx = threadIdx.x + i * T;
+      if (idx < nvec) *reinterpret_cast<uint2*>(qr + idx * 8) = encode_vec<false>(v[i], dv);
+    }
   }
 }
 
@@ -127,6 +170,7 @@ template <int GPT>
 __global__ void __launch_bounds__(256) quant_groups128_kernel(const uint16_t* __restrict__ x, int64_t M, int G,
                                                              int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
                                                              float* __restrict__ s) {
+  griddep_wait();
   const int64_t total = M * static_cast<int64_t>(G);
   const int sub = threadIdx.x & 15;
   const uint32_t half_mask = 0xFFFFu << (threadIdx.x & 16);
@@ -154,7 +198,9 @@ __global__ void __launch_bounds__(256) quant_groups128_kernel(const uint16_t* __
         const float sc = scale_of(amax_bits_to_float(mm));
         const int64_t m = gi / G, g = gi - m * G;
         if (sub == 0) s[gi] = sc;
-        *reinterpret_cast<uint2*>(q + m * ldq + g * 128 + sub * 8) = encode_vec(v[i], make_divider(sc));
+        const Divider dv = make_divider(sc);
+        *reinterpret_cast<uint2*>(q + m * ldq + g * 128 + sub * 8) =
+            dv.fast ? encode_vec<true>(v[i], dv) : encode_vec<false>(v[i], dv);
       }
     }
   }
@@ -168,6 +214,7 @@ __global__ void __launch_bounds__(256) quant_blocks128_kernel(const uint16_t* __
                                                              int64_t ldw, uint8_t* __restrict__ q, int64_t ldq,
                                                              float* __restrict__ s) {
   __shared__ uint32_t red[8];
+  griddep_wait();
   const int kb = blockIdx.x;
   const int64_t nb = blockIdx.y;
   const int vc = threadIdx.x & 15;
@@ -193,7 +240,9 @@ __global__ void __launch_bounds__(256) quant_blocks128_kernel(const uint16_t* __
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int64_t row = nb * 128 + r0 + 16 * i;
-    if (row < N) *reinterpret_cast<uint2*>(q + row * ldq + kb * 128 + vc * 8) = encode_vec(v[i], dv);
+    if (row < N)
+      *reinterpret_cast<uint2*>(q + row * ldq + kb * 128 + vc * 8) =
+          dv.fast ? encode_vec<true>(v[i], dv) : encode_vec<false>(v[i], dv);
   }
 }
 

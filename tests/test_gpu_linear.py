@@ -200,3 +200,31 @@ def test_tiny_workload_in_full():
     P.assert_codes_equal(wq, rwq, "tiny wq")
     P.assert_scales_equal(ws, rws, "tiny ws")
     P.assert_y_close(y.float().cpu().numpy(), oracle.linear(rxq, rxs, rwq, rws, 0), what="tiny")
+
+
+@pytest.mark.parametrize("M,mode", [(4, fq.CHANNEL_TOKEN), (300, fq.CHANNEL_TOKEN), (16, fq.BLOCK128),
+                                    (256, fq.BLOCK128)])
+def test_cuda_graph_replay_matches_eager(M, mode):
+    N, K = 1024, 1024
+    x = synth.make_x(M, K, seed=M).to(DEV)
+    w = synth.make_w(N, K, seed=M).to(DEV)
+    wq, ws = fq.fp8_quant_weight(w, mode)
+    xq, xs = fq.fp8_quant_act(x, mode)
+    y_eager = fq.fp8_linear(xq, xs, wq, ws, mode)
+    xq2, xs2 = torch.empty_like(xq), torch.empty_like(xs)
+    y2 = torch.empty_like(y_eager)
+    wsp = torch.empty(max(1, fq.fp8_linear_workspace_size(M, N, K, mode)), dtype=torch.uint8, device=DEV)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            fq.fp8_quant_act(x, mode, out=(xq2, xs2))
+            fq.fp8_linear(xq2, xs2, wq, ws, mode, out=y2, workspace=wsp)
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(3):
+        y2.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(xq2, xq) and torch.equal(xs2, xs)
+        assert torch.equal(y2, y_eager)

@@ -5,6 +5,8 @@
 // kernel and launch shape, and maps errors to fp8q_status.
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "../../include/fp8q.h"
@@ -168,6 +170,34 @@ fp8q_status launch_rows(const uint16_t* x, int64_t rows, int K, int64_t ldx, uin
 // ------------------------------------------------------------------ linear ---
 
 constexpr int kPrefillBN = 256;
+constexpr int kPairStages = 5;
+
+// Prefill kernel choice for channel mode: the CTA-pair kernel for M >= 256,
+// else the single-CTA kernel.  FP8Q_PREFILL_KERNEL=single|pair forces one
+// (read once), for comparing them on the same problem.
+int prefill_choice() {
+  static int choice = [] {
+    const char* e = getenv("FP8Q_PREFILL_KERNEL");
+    if (e && strcmp(e, "single") == 0) return 1;
+    if (e && strcmp(e, "pair") == 0) return 2;
+    return 0;
+  }();
+  return choice;
+}
+
+// Whole rounds of `per_round` tiles stay whole; the partial last round is cut
+// along N into two halves when that shortens it.  Returns the split (1 or 2)
+// and the number of whole tiles.
+void tail_split(int num_tiles, int per_round, int* full, int* split) {
+  *full = num_tiles >= per_round ? num_tiles / per_round * per_round : 0;
+  const int rest = num_tiles - *full;
+  *split = 1;
+  if (rest) {
+    const double whole = 1.0 * ((rest + per_round - 1) / per_round);
+    const double halves = 0.5 * ((2 * rest + per_round - 1) / per_round);
+    if (halves < whole - 1e-9) *split = 2;
+  }
+}
 constexpr int kPrefillStages = 4;
 constexpr int kBlockStages = 6;
 template <int NX>
@@ -303,6 +333,46 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     return launch_decode_nx<64>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
   }
 
+  const bool pair = mode == FP8Q_CHANNEL_TOKEN && prefill_choice() != 1 && (M >= 256 || prefill_choice() == 2);
+  if (pair) {
+    using L = fp8q::prefill::PairLayout<kPairStages>;
+    auto k = fp8q::prefill::gemm_channel2_kernel<kPairStages>;
+    if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
+    static int max_pairs[kMaxDevices] = {};
+    if (max_pairs[dev] == 0) {
+      cudaLaunchConfig_t qc = {};
+      qc.gridDim = dim3(2 * sms);
+      qc.blockDim = dim3(64 + 32 * L::kEpiWarps);
+      qc.dynamicSmemBytes = L::kBytes;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, k, &qc) != cudaSuccess || n < 1) n = sms / 2;
+      max_pairs[dev] = n;
+    }
+    fp8q::prefill::Params p;
+    p.xs = x_scale;
+    p.ws = w_scale;
+    p.y = static_cast<__nv_bfloat16*>(Y_bf16);
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.ldy = ldy;
+    p.KB = KB;
+    p.num_m = static_cast<int>((M + 255) / 256);
+    p.num_n = static_cast<int>((N + 255) / 256);
+    p.num_tiles = p.num_m * p.num_n;
+    p.group_m = p.num_m < 8 ? p.num_m : 8;
+    const int pairs = max_pairs[dev];
+    tail_split(p.num_tiles, pairs, &p.full, &p.split);
+    const int items = (p.full ? p.full : 0) + (p.num_tiles - p.full) * p.split;
+    const int used = p.full ? pairs : (items < pairs ? items : pairs);
+    CUtensorMap ta, tb, tb64, ty;
+    if ((st = tmap_u8_sw128(&ta, Xq, M, K, K, 128)) != FP8Q_OK) return st;
+    if ((st = tmap_u8_sw128(&tb, Wq, N, K, K, 128)) != FP8Q_OK) return st;
+    if ((st = tmap_u8_sw128(&tb64, Wq, N, K, K, 64)) != FP8Q_OK) return st;
+    if ((st = tmap_bf16_sw64(&ty, Y_bf16, M, N, ldy, 32)) != FP8Q_OK) return st;
+    return launch(k, dim3(2 * used), dim3(64 + 32 * L::kEpiWarps), L::kBytes, stream, ta, tb, tb64, ty, p);
+  }
+
   fp8q::prefill::Params p;
   p.xs = x_scale;
   p.ws = w_scale;
@@ -317,22 +387,33 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
   p.num_n = static_cast<int>((N + BN - 1) / BN);
   p.num_tiles = p.num_m * p.num_n;
   p.group_m = p.num_m < 16 ? p.num_m : 16;
-  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  p.full = p.num_tiles;
+  p.split = 1;
+  if (mode != FP8Q_BLOCK128) {
+    tail_split(p.num_tiles, sms, &p.full, &p.split);
+    const int items = p.full + (p.num_tiles - p.full) * p.split;
+    grid = p.full ? sms : (items < sms ? items : sms);
+  }
   CUtensorMap ta, tb;
   if ((st = tmap_u8_sw128(&ta, Xq, M, K, K, 128)) != FP8Q_OK) return st;
   if ((st = tmap_u8_sw128(&tb, Wq, N, K, K, static_cast<uint32_t>(BN))) != FP8Q_OK) return st;
   if (mode == FP8Q_BLOCK128) {
     using L = fp8q::prefill::BlockLayout<kBlockStages>;
     auto k = fp8q::prefill::gemm_block_kernel<kBlockStages>;
+    CUtensorMap ty;
+    if ((st = tmap_bf16_sw64(&ty, Y_bf16, M, N, ldy, 32)) != FP8Q_OK) return st;
     if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
-    return launch(k, dim3(grid), dim3(320), L::kBytes, stream, ta, tb, p);
+    return launch(k, dim3(grid), dim3(64 + 32 * L::kEpiWarps), L::kBytes, stream, ta, tb, ty, p);
   }
   using L = fp8q::prefill::ChannelLayout<kPrefillBN, kPrefillStages>;
   auto k = fp8q::prefill::gemm_channel_kernel<kPrefillBN, kPrefillStages>;
-  CUtensorMap ty;
+  CUtensorMap ty, tb128, tb64;
   if ((st = tmap_bf16_sw64(&ty, Y_bf16, M, N, ldy, 32)) != FP8Q_OK) return st;
+  if ((st = tmap_u8_sw128(&tb128, Wq, N, K, K, 128)) != FP8Q_OK) return st;
+  if ((st = tmap_u8_sw128(&tb64, Wq, N, K, K, 64)) != FP8Q_OK) return st;
   if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
-  return launch(k, dim3(grid), dim3(192), L::kBytes, stream, ta, tb, ty, p);
+  return launch(k, dim3(grid), dim3(192), L::kBytes, stream, ta, tb, tb128, tb64, ty, p);
 }
 
 const char* fp8q_status_string(int status) {

@@ -37,6 +37,10 @@ struct Params {
   int64_t ldy;
   int KB;          // ceil(K / 128)
   int num_m, num_n, num_tiles, group_m;
+  // Channel kernel work list: tiles [0, full) are whole (tile t goes to CTA
+  // t % gridDim.x); the remaining tiles are cut along N into `split` pieces
+  // (256 / split columns each) handed out round-robin after them.
+  int full, split;
 };
 
 // Tile order: groups of `group_m` row-blocks, column-blocks within a group,
@@ -49,6 +53,30 @@ __device__ __forceinline__ void tile_coords(const Params& p, int t, int& mb, int
   const int r = t - g * per_group;
   mb = first_m + r % gm;
   nb = r / gm;
+}
+
+// Number of work items of CTA c, and item i of it: tile coordinates, the
+// first column inside the 256-wide tile and the column count.
+__device__ __forceinline__ int items_of(const Params& p, int c) {
+  const int G = gridDim.x;
+  const int tail = (p.num_tiles - p.full) * p.split;
+  return p.full / G + (c < tail ? (tail - 1 - c) / G + 1 : 0);
+}
+
+__device__ __forceinline__ void item_coords(const Params& p, int c, int i, int& mb, int& nb, int& n_off,
+                                            int& n_cols) {
+  const int G = gridDim.x;
+  const int nfull = p.full / G;
+  if (i < nfull) {
+    tile_coords(p, c + i * G, mb, nb);
+    n_off = 0;
+    n_cols = 256;
+  } else {
+    const int j = c + (i - nfull) * G;
+    tile_coords(p, p.full + j / p.split, mb, nb);
+    n_cols = 256 / p.split;
+    n_off = (j % p.split) * n_cols;
+  }
 }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -73,7 +101,9 @@ struct ChannelLayout {
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
     gemm_channel_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmB128, const __grid_constant__ CUtensorMap tmB64,
                         const __grid_constant__ CUtensorMap tmY, const Params p) {
+  static_assert(BN == 256, "the work list assumes 256-column tiles");
   using L = ChannelLayout<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -103,6 +133,8 @@ __global__ void __launch_bounds__(192, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmB128);
+    tma_prefetch_desc(&tmB64);
     tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
@@ -121,14 +153,17 @@ __global__ void __launch_bounds__(192, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
-        int mb, nb;
-        tile_coords(p, t, mb, nb);
+      const int nitems = items_of(p, blockIdx.x);
+      for (int i = 0; ok && i < nitems; ++i) {
+        int mb, nb, n_off, n_cols;
+        item_coords(p, blockIdx.x, i, mb, nb, n_off, n_cols);
+        const CUtensorMap* tb = n_cols == 256 ? &tmB : (n_cols == 128 ? &tmB128 : &tmB64);
+        const uint32_t bytes = static_cast<uint32_t>(L::kA + n_cols * BK);
         for (int kb = 0; kb < p.KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], L::kA + L::kB);
+          mbar_arrive_expect_tx(&full[stage], bytes);
           tma_load_2d(sA + stage * L::kA, &tmA, &full[stage], kb * BK, mb * BM, pol);
-          tma_load_2d(sB + stage * L::kB, &tmB, &full[stage], kb * BK, nb * BN, pol);
+          tma_load_2d(sB + stage * L::kB, tb, &full[stage], kb * BK, nb * BN + n_off, pol);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -142,12 +177,14 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
       int stage = 0;
       uint32_t phase = 0;
-      int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
+      const int nitems = items_of(p, blockIdx.x);
+      for (int it = 0; ok && it < nitems; ++it) {
+        int mb, nb, n_off, n_cols;
+        item_coords(p, blockIdx.x, it, mb, nb, n_off, n_cols);
+        const uint32_t idesc = idesc_e4m3_f32(BM, n_cols);
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, kErrWaitTmemEmpty)) break;
@@ -177,10 +214,11 @@ __global__ void __launch_bounds__(192, 1)
     float* ws_s = reinterpret_cast<float*>(smem + L::kWsOff) + ew * BN;
     uint8_t* out_s = smem + L::kOutOff + ew * 2 * L::kOutChunk;
     const int swz = (lane >> 1) & 3;         // 64-byte swizzle of this thread's staging row
-    int it = 0, buf = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++it) {
-      int mb, nb;
-      tile_coords(p, t, mb, nb);
+    int buf = 0;
+    const int nitems = items_of(p, blockIdx.x);
+    for (int it = 0; it < nitems; ++it) {
+      int mb, nb, n_off, n_cols;
+      item_coords(p, blockIdx.x, it, mb, nb, n_off, n_cols);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       // Scales of this tile, fetched while the main loop still runs.
@@ -189,8 +227,8 @@ __global__ void __launch_bounds__(192, 1)
       float wv[BN / 32];
 #pragma unroll
       for (int i = 0; i < BN / 32; ++i) {
-        const int n = nb * BN + i * 32 + lane;
-        wv[i] = n < p.N ? __ldg(p.ws + n) : 0.0f;
+        const int n = nb * BN + n_off + i * 32 + lane;
+        wv[i] = (i * 32 < n_cols && n < p.N) ? __ldg(p.ws + n) : 0.0f;
       }
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrWaitTmemFull))) break;
       tc_fence_after();
@@ -198,12 +236,12 @@ __global__ void __launch_bounds__(192, 1)
       for (int i = 0; i < BN / 32; ++i) ws_s[i * 32 + lane] = wv[i];
       __syncwarp();
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = 0; c < n_cols; c += 32) {
         uint32_t r[32];
         __syncwarp();
         tmem_ld_32x32b_x32(tmem_base + lane_addr + acc * BN + c, r);
         tmem_ld_wait();
-        if (c + 32 == BN) {              // accumulator fully read: hand it back to the MMA
+        if (c + 32 == n_cols) {          // accumulator fully read: hand it back to the MMA
           tc_fence_before();
           mbar_arrive(&tempty[acc]);
         }
@@ -223,7 +261,7 @@ __global__ void __launch_bounds__(192, 1)
               make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         fence_proxy_async_smem();
         __syncwarp();
-        const int row0 = mb * BM + quarter * 32, col0 = nb * BN + c;
+        const int row0 = mb * BM + quarter * 32, col0 = nb * BN + n_off + c;
         if (lane == 0 && row0 < p.M && col0 < p.N) {   // the store clips the rest of the box
           tma_store_2d(&tmY, sb, col0, row0);
           bulk_commit();
@@ -243,6 +281,255 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// ------------------------------------------------------ channel, CTA pair ---
+// The same GEMM with 256 x 256 tiles computed by a cluster of two CTAs with
+// tcgen05 pair instructions.  CTA r of the pair loads rows [128 r, 128 r + 128)
+// of the A tile and of the B tile (B's N split the same way) into its own
+// shared memory; the leader (r = 0) issues one M=256 MMA over both; each CTA's
+// tensor memory receives its own 128 rows of the accumulator.  Per CTA this
+// moves 32 KB per 128-wide K block instead of 48 KB for the same 128 x 256
+// share of the work, and 6 stages fit.
+//   full[s]    leader only: the leader's producer expects both CTAs' bytes;
+//              both CTAs' TMA loads complete on it.
+//   empty[s]   both CTAs: the leader's commit arrives on both.
+//   tfull[a]   both CTAs: the leader's commit arrives on both.
+//   tempty[a]  leader only: all 256 epilogue threads of the pair arrive.
+template <int STAGES>
+struct PairLayout {
+  static constexpr int kA = 128 * BK;                           // this CTA's 128 rows of A
+  static constexpr int kB = 128 * BK;                           // this CTA's (up to) 128 rows of B
+  static constexpr int kEpiWarps = 8;                           // two per TMEM lane quarter
+  static constexpr int kOutChunk = 32 * 32 * 2;
+  static constexpr int kOutOff = STAGES * (kA + kB);
+  static constexpr int kWsOff = kOutOff + kEpiWarps * 2 * kOutChunk;
+  static constexpr int kBarOff = kWsOff + kEpiWarps * 128 * 4;
+  static constexpr int kBarBytes = (2 * STAGES + 4) * 8 + 8;
+  static constexpr int kBytes = kBarOff + 1024 + 1024;
+  static_assert(kBarBytes <= 1024, "barrier area");
+  static_assert(kBytes <= 232448, "shared memory per CTA");
+};
+
+template <int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
+    gemm_channel2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmB64, const __grid_constant__ CUtensorMap tmY,
+                         const Params p) {
+  using L = PairLayout<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * L::kA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  constexpr uint32_t kTmemCols = 512;                           // 2 accumulators x 256 columns
+  constexpr uint16_t kBoth = 0x3;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * 32 * L::kEpiWarps);             // every epilogue thread of the pair
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmB64);
+    tma_prefetch_desc(&tmY);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();                 // barriers of both CTAs initialised before any remote signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();                 // global memory only from here on
+
+  // Work items are per pair: use the pair index and the number of pairs.
+  const int G2 = gridDim.x >> 1;
+  auto count = [&]() {
+    const int tail = (p.num_tiles - p.full) * p.split;
+    return p.full / G2 + (pair < tail ? (tail - 1 - pair) / G2 + 1 : 0);
+  };
+  auto coords = [&](int i, int& mb, int& nb, int& n_off, int& n_cols) {
+    const int nfull = p.full / G2;
+    if (i < nfull) {
+      tile_coords(p, pair + i * G2, mb, nb);
+      n_off = 0;
+      n_cols = 256;
+    } else {
+      const int j = pair + (i - nfull) * G2;
+      tile_coords(p, p.full + j / p.split, mb, nb);
+      n_cols = 256 / p.split;
+      n_off = (j % p.split) * n_cols;
+    }
+  };
+  const int nitems = count();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int i = 0; ok && i < nitems; ++i) {
+        int mb, nb, n_off, n_cols;
+        coords(i, mb, nb, n_off, n_cols);
+        const int half = n_cols / 2;                            // B rows held by each CTA
+        const CUtensorMap* tb = half == 128 ? &tmB : &tmB64;
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) { ok = false; break; }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * static_cast<uint32_t>(L::kA + half * BK));
+          const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
+          tma_load_2d_pair(sA + stage * L::kA, &tmA, bar0, kb * BK, mb * 256 + static_cast<int>(rank) * 128, pol);
+          tma_load_2d_pair(sB + stage * L::kB, tb, bar0, kb * BK, nb * 256 + n_off + static_cast<int>(rank) * half,
+                           pol);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      griddep_launch_dependents();
+      for (int i = 0; ok && i < STAGES; ++i) {   // every stage released by the leader's commits
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) break;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int it = 0; ok && it < nitems; ++it) {
+        int mb, nb, n_off, n_cols;
+        coords(it, mb, nb, n_off, n_cols);
+        const uint32_t idesc = idesc_e4m3_f32(256, n_cols);
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag, kErrWaitTmemEmpty)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * 256;
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * L::kA);
+          const uint32_t b0 = smem_u32(sB + stage * L::kB);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k)
+            mma_e4m3_pair(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + k * UMMA_K), idesc,
+                          (kb | k) != 0);
+          mma_commit_pair(&empty[stage], kBoth);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) mma_commit_pair(&tfull[acc], kBoth);
+      }
+    }
+  } else {
+    // 8 epilogue warps: warp w reads TMEM lanes 32*(w%4)..+31 (its 32 rows)
+    // and takes one half of the item's columns.  The TMEM load of the next
+    // 32-column chunk is issued before the current chunk is scaled, staged
+    // and stored, so its latency overlaps that work.
+    const int ew = warp - 2;
+    const int quarter = warp & 3;
+    const int half = ew >> 2;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    float* ws_s = reinterpret_cast<float*>(smem + L::kWsOff) + ew * 128;
+    uint8_t* out_s = smem + L::kOutOff + ew * 2 * L::kOutChunk;
+    const int swz = (lane >> 1) & 3;
+    const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    int buf = 0;
+    for (int it = 0; it < nitems; ++it) {
+      int mb, nb, n_off, n_cols;
+      coords(it, mb, nb, n_off, n_cols);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      const int my_cols = n_cols / 2;                           // 128 or 64
+      const int c_begin = half * my_cols;
+      const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quarter * 32;
+      const int m = row0 + lane;
+      const float xsm = m < p.M ? __ldg(p.xs + m) : 0.0f;
+      float wv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int n = nb * 256 + n_off + c_begin + i * 32 + lane;
+        wv[i] = (i * 32 < my_cols && n < p.N) ? __ldg(p.ws + n) : 0.0f;
+      }
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrWaitTmemFull))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ws_s[i * 32 + lane] = wv[i];
+      __syncwarp();
+      const uint32_t tcol = tmem_base + lane_addr + acc * 256 + c_begin;
+      const int nchunks = my_cols / 32;                         // 4 or 2: always even
+      // Scale, stage and store one 32-column chunk held in registers.
+      auto emit = [&](const uint32_t (&cur)[32], int c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float2 w = *reinterpret_cast<const float2*>(ws_s + c + 2 * j);
+          pk[j] = pack_bf16x2(__uint_as_float(cur[2 * j]) * xsm * w.x, __uint_as_float(cur[2 * j + 1]) * xsm * w.y);
+        }
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        uint8_t* sb = out_s + buf * L::kOutChunk;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(sb + lane * 64 + ((q ^ swz) << 4)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        const int col0 = nb * 256 + n_off + c_begin + c;
+        if (lane == 0 && row0 < p.M && col0 < p.N) {
+          tma_store_2d(&tmY, sb, col0, row0);
+          bulk_commit();
+        }
+        buf ^= 1;
+      };
+      uint32_t ra[32], rb[32];
+      __syncwarp();
+      tmem_ld_32x32b_x32(tcol, ra);
+#pragma unroll 1
+      for (int ci = 0; ci < nchunks; ci += 2) {
+        tmem_ld_wait_regs(ra);
+        __syncwarp();
+        tmem_ld_32x32b_x32(tcol + (ci + 1) * 32, rb);
+        emit(ra, ci * 32);
+        tmem_ld_wait_regs(rb);
+        if (ci + 2 < nchunks) {
+          __syncwarp();
+          tmem_ld_32x32b_x32(tcol + (ci + 2) * 32, ra);
+        } else {                        // all of this warp's columns read: release the accumulator
+          tc_fence_before();
+          mbar_arrive_cluster(tempty0 + acc * 8);
+        }
+        emit(rb, (ci + 1) * 32);
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                 // no CTA leaves while its pair may still signal it or read its memory
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 // --------------------------------------------------------------- block ---
 template <int STAGES>
 struct BlockLayout {
@@ -250,7 +537,10 @@ struct BlockLayout {
   static constexpr int kA = BM * BK;
   static constexpr int kB = BN * BK;
   static constexpr int kSlots = 4;
-  static constexpr int kBarOff = STAGES * (kA + kB);
+  static constexpr int kEpiWarps = 16;                          // 4 per TMEM lane quarter, 32 columns each
+  static constexpr int kOutChunk = 32 * 32 * 2;                 // one 32 x 32 bf16 staging tile per warp
+  static constexpr int kOutOff = STAGES * (kA + kB);
+  static constexpr int kBarOff = kOutOff + kEpiWarps * kOutChunk;
   static constexpr int kBarBytes = (2 * STAGES + 2 * kSlots) * 8 + 8;
   static constexpr int kBytes = kBarOff + 1024 + 1024;
   static_assert(kBarBytes <= 1024, "barrier area");
@@ -258,9 +548,9 @@ struct BlockLayout {
 };
 
 template <int STAGES>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(576, 1)
     gemm_block_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const Params p) {
+                      const __grid_constant__ CUtensorMap tmY, const Params p) {
   using L = BlockLayout<STAGES>;
   constexpr int BN = L::BN;
   constexpr int kSlots = L::kSlots;
@@ -278,7 +568,7 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   constexpr uint32_t kTmemCols = kSlots * BN;   // 512
-  constexpr int kEpiThreads = 256;
+  constexpr int kEpiThreads = 32 * L::kEpiWarps;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -293,6 +583,7 @@ __global__ void __launch_bounds__(320, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -352,11 +643,17 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else {
-    // 8 epilogue warps: two per TMEM lane quarter, each owning 64 columns.
+    // 16 epilogue warps: four per TMEM lane quarter, each owning 32 columns.
+    // Each 128-wide K slice is folded in with that slice's scale product
+    // (packed fp32x2 FMAs); the finished 32 x 32 bf16 chunk goes out through
+    // a 64-byte-swizzled staging tile and a TMA store.
+    const int ew = warp - 2;
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int cg = ew >> 2;                                   // column group 0..3
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    uint8_t* out_s = smem + L::kOutOff + ew * L::kOutChunk;
+    const int swz = (lane >> 1) & 3;
     int slot = 0;
     uint32_t sphase = 0;
     bool ok = true;
@@ -367,47 +664,51 @@ __global__ void __launch_bounds__(320, 1)
       const bool row_ok = m < p.M;
       const float* xsrow = p.xs + static_cast<int64_t>(m) * p.KB;
       const float* wsrow = p.ws + static_cast<int64_t>(nb) * p.KB;
-      float acc[64];
+      uint64_t acc[16];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < 16; ++j) acc[j] = 0ull;
       float f_next = row_ok ? __ldg(xsrow) * __ldg(wsrow) : 0.0f;
       for (int kb = 0; kb < p.KB; ++kb) {
         const float f = f_next;
         if (kb + 1 < p.KB) f_next = row_ok ? __ldg(xsrow + kb + 1) * __ldg(wsrow + kb + 1) : 0.0f;
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sfull[slot], sphase, abort_flag, kErrWaitTmemFull))) { ok = false; break; }
         tc_fence_after();
-        uint32_t r0[32], r1[32];
+        uint32_t r[32];
         __syncwarp();
-        const uint32_t a = tmem_base + lane_addr + slot * BN + half * 64;
-        tmem_ld_32x32b_x32(a, r0);
-        tmem_ld_32x32b_x32(a + 32, r1);
+        tmem_ld_32x32b_x32(tmem_base + lane_addr + slot * BN + cg * 32, r);
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&sempty[slot]);
+        const uint64_t f2 = f32x2_pack(f, f);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          acc[j] = fmaf(__uint_as_float(r0[j]), f, acc[j]);
-          acc[32 + j] = fmaf(__uint_as_float(r1[j]), f, acc[32 + j]);
-        }
+        for (int j = 0; j < 16; ++j)
+          acc[j] = fma_f32x2(f32x2_pack(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])), f2, acc[j]);
         if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
       }
       if (!ok) break;
-      if (row_ok) {
-        __nv_bfloat16* yrow = p.y + static_cast<int64_t>(m) * p.ldy;
-        const int n0 = nb * BN + half * 64;
+      uint32_t pk[16];
 #pragma unroll
-        for (int j = 0; j < 64; j += 8) {
-          if (n0 + j < p.N) {
-            uint4 o;
-            o.x = pack_bf16x2(acc[j + 0], acc[j + 1]);
-            o.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
-            o.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
-            o.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
-            *reinterpret_cast<uint4*>(yrow + n0 + j) = o;
-          }
-        }
+      for (int j = 0; j < 16; ++j) {
+        float lo, hi;
+        f32x2_unpack(acc[j], lo, hi);
+        pk[j] = pack_bf16x2(lo, hi);
+      }
+      // The staging tile of the previous tile's store must have been read.
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(out_s + lane * 64 + ((q ^ swz) << 4)) =
+            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int row0 = mb * BM + quarter * 32, col0 = nb * BN + cg * 32;
+      if (lane == 0 && row0 < p.M && col0 < p.N) {   // the store clips the rest of the box
+        tma_store_2d(&tmY, out_s, col0, row0);
+        bulk_commit();
       }
     }
+    if (lane == 0) bulk_wait<0>();
   }
 
   tc_fence_before();

@@ -61,11 +61,27 @@ def check_full(M, N, K, mode, seed=0, ldy_pad=0):
     (65, 16, 16),          # smallest prefill problem: one partial tile everywhere
     (200, 320, 272),       # ragged M, N (BN=256) and K (128-byte blocks)
     (129, 512, 256),
-    (384, 768, 1024),      # several tiles in both dimensions, 8 K blocks
-    (2048, 2560, 256),     # 160 tiles > 148 SMs: persistent loop, both accumulators
+    (384, 768, 1024),      # CTA-pair kernel (M >= 256), several tiles, 8 K blocks
+    (300, 320, 272),       # pair kernel with a second 256-row tile mostly past M
+    (1000, 1040, 400),     # pair kernel, ragged in M, N and K
+    (2048, 2560, 256),     # more tiles than pairs: persistent loop, tail split in N halves
 ])
 def test_prefill_channel(M, N, K):
     check_full(M, N, K, fq.CHANNEL_TOKEN, seed=M)
+
+
+@pytest.mark.parametrize("kernel,M,N,K", [("single", 2048, 2560, 256), ("single", 1024, 4096, 512),
+                                          ("pair", 200, 320, 272), ("pair", 65, 512, 128)])
+def test_prefill_kernel_forced(kernel, M, N, K):
+    # each prefill kernel on shapes the default dispatch would give the other one
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, FP8Q_PREFILL_KERNEL=kernel)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-m", "tests._forced_kernel", str(M), str(N), str(K), "0"],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
 
 
 @pytest.mark.parametrize("M,N,K", [

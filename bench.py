@@ -46,7 +46,7 @@ FP8_OVER_BF16 = 2.0        # nominal dense fp8 / bf16 tensor ratio (4.5 / 2.25 P
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="fp8q", choices=["fp8q", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
@@ -123,56 +123,73 @@ def to_metric(units, seconds, unit):
 
 # ------------------------------------------------------------------ clocks ---
 
+_CLOCK_WORKER = r"""
+import json, select, sys, time
+reasons = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+index, period = int(sys.argv[1]), float(sys.argv[2])
+try:
+    import pynvml
+    pynvml.nvmlInit()
+    h = pynvml.nvmlDeviceGetHandleByIndex(index)
+    mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+except Exception as e:
+    print(json.dumps({"error": "nvml unavailable: %s" % e}), flush=True)
+    sys.exit(0)
+print(json.dumps({"ready": True}), flush=True)
+samples, seen = [], set()
+while True:
+    r, _, _ = select.select([sys.stdin], [], [], period)
+    if r:
+        break
+    try:
+        samples.append(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+        ev = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+        seen.update(name for bit, name in reasons.items() if ev & bit)
+    except Exception as e:
+        print(json.dumps({"error": str(e)}), flush=True)
+        sys.exit(0)
+print(json.dumps({"samples": samples, "reasons": sorted(seen), "max": mx}), flush=True)
+"""
+
+
 class ClockSampler:
-    """Samples SM clock and clock-event reasons with NVML while running."""
-    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
-               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
-               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
-               0x100: "display_clock_setting"}
+    """NVML samples of the SM clock and clock-event reasons, taken by a
+    separate small process (no GIL shared with the launching thread) for as
+    long as the timed region runs."""
 
-    def __init__(self, index: int, period_s: float = 0.002):
-        self.samples, self.reasons, self.err = [], set(), None
-        self.period = period_s
-        self.stop_ev = threading.Event()
-        try:
-            import pynvml
-            pynvml.nvmlInit()
-            self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-        except Exception as e:  # no NVML: report why
-            self.nv, self.err, self.max_mhz = None, f"nvml unavailable: {e}", None
-
-    def _run(self):
-        while not self.stop_ev.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
-            except Exception as e:
-                self.err = str(e)
-                return
-            time.sleep(self.period)
+    def __init__(self, index: int, period_s: float = 0.001):
+        self.index, self.period = index, period_s
+        self.result = {"error": "not run"}
 
     def __enter__(self):
-        if self.nv is not None:
-            self.t = threading.Thread(target=self._run, daemon=True)
-            self.t.start()
+        self.proc = subprocess.Popen([sys.executable, "-c", _CLOCK_WORKER, str(self.index), str(self.period)],
+                                     stdin=subprocess.PIPE, stdout=subprocess.PIPE, text=True)
+        first = json.loads(self.proc.stdout.readline() or '{"error": "sampler exited"}')
+        self.ok = "ready" in first
+        if not self.ok:
+            self.result = first
         return self
 
     def __exit__(self, *a):
-        if self.nv is not None:
-            self.stop_ev.set()
-            self.t.join()
+        try:
+            out, _ = self.proc.communicate(input="stop\n", timeout=60)
+            if self.ok:
+                self.result = json.loads(out.strip().splitlines()[-1])
+        except Exception as e:
+            self.proc.kill()
+            self.result = {"error": f"sampler: {e}"}
 
     def summary(self):
-        if self.nv is None or not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                    "samples": len(self.samples), "error": self.err}
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+        r = self.result
+        if "samples" not in r or not r["samples"]:
+            return {"sm_mhz": None, "sm_max_mhz": r.get("max"), "reasons": r.get("reasons", []),
+                    "samples": 0, "error": r.get("error")}
+        smp = r["samples"]
+        return {"sm_mhz": float(statistics.median(smp)), "sm_max_mhz": r["max"], "sm_mhz_min": float(min(smp)),
+                "reasons": [x for x in r["reasons"] if x != "gpu_idle"], "samples": len(smp),
+                "sampler": "NVML in a separate process, every 1 ms during the timed steps"}
 
 
 # --------------------------------------------------------------- GPU arm ---
@@ -329,6 +346,52 @@ def run_gpu(args):
     op_ms = np.array([[a.elapsed_time(b) for a, b in row] for row in op_ev]).mean(axis=0)
     err = fq.device_error(clear=True)
 
+    # ---- GEMMs that read the same activation, run as one GEMM over their
+    # stacked weights (what serving engines do with q/k/v or gate/up); the
+    # per-channel and 128x128-block scales are row-local, so stacking the
+    # quantized weights and scales is exact.
+    merged = None
+    groups = {}
+    for g in wl.gemms:
+        groups.setdefault((g.x, g.mode), []).append(g)
+    if not args.eager and any(len(v) > 1 for v in groups.values()):
+        mops, mnames = [], []
+        for (xk, mode), gs in groups.items():
+            if len(gs) == 1:
+                g = gs[0]
+                mops.append(lambda g=g: fq.fp8_linear(XQ[g.x][0], XQ[g.x][1], WQ[g.name][0], WQ[g.name][1], g.mode,
+                                                      out=Y[g.name], workspace=WS[g.name]))
+                mnames.append(g.name)
+                continue
+            wq_m = torch.cat([WQ[g.name][0] for g in gs])
+            ws_m = torch.cat([WQ[g.name][1] for g in gs])
+            M, K, Nm = gs[0].M, gs[0].K, sum(g.N for g in gs)
+            y_m = torch.empty((M, Nm), dtype=torch.bfloat16, device=dev)
+            nws = fq.fp8_linear_workspace_size(M, Nm, K, mode)
+            ws_buf = torch.empty(nws, dtype=torch.uint8, device=dev) if nws else None
+            mops.append(lambda xk=xk, mode=mode, wq_m=wq_m, ws_m=ws_m, y_m=y_m, ws_buf=ws_buf:
+                        fq.fp8_linear(XQ[xk][0], XQ[xk][1], wq_m, ws_m, mode, out=y_m, workspace=ws_buf))
+            mnames.append("+".join(g.name for g in gs) + f":{M}x{K}->{Nm}")
+        qops = ops[:len(xs_shapes)]
+        for f in qops + mops:
+            f()
+        torch.cuda.synchronize()
+        mgraph = capture(qops + mops)
+        for _ in range(2):
+            mgraph.replay()
+        mev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda._sleep(2_000_000)
+        for s_ in range(args.steps):
+            flush.zero_()
+            mev[s_][0].record(stream)
+            mgraph.replay()
+            mev[s_][1].record(stream)
+        torch.cuda.synchronize()
+        mt = sum(a.elapsed_time(b) for a, b in mev) / 1e3
+        merged = {"value": round(to_metric(units, mt, unit), 3), "unit": unit,
+                  "ms_per_step": round(mt * 1e3 / args.steps, 4), "gemms": mnames,
+                  "note": "same step, GEMMs sharing an input launched as one GEMM over stacked weights"}
+
     # ---- per-kernel detail and the dominant kernel's roofline
     names = [f"quant_act[{k}]" for k in xs_shapes] + [g.name for g in wl.gemms]
     detail = []
@@ -451,6 +514,7 @@ def run_gpu(args):
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g) for g in wl.gemms)),
             "clocks": clk.summary(), "detail": detail, "weight_quant": weight_quant,
+            "merged_shared_input": merged,
             "device_error": err, "gpu": torch.cuda.get_device_name(dev),
         }
         print(json.dumps(line), flush=True)

@@ -170,7 +170,7 @@ fp8q_status launch_rows(const uint16_t* x, int64_t rows, int K, int64_t ldx, uin
 // ------------------------------------------------------------------ linear ---
 
 constexpr int kPrefillBN = 256;
-constexpr int kPairStages = 5;
+constexpr int kPairStages = 6;
 
 // Prefill kernel choice for channel mode: the CTA-pair kernel for M >= 256,
 // else the single-CTA kernel.  FP8Q_PREFILL_KERNEL=single|pair forces one

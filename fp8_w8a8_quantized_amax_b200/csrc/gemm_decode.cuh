@@ -177,6 +177,21 @@ __global__ void __launch_bounds__(192, 1)
     for (int j = 0; j < NX; ++j) acc[j] = 0.0f;
     int slot = 0;
     uint32_t sphase = 0;
+    // Block mode: the scales of step s are fetched one step ahead (for NX <= 32;
+    // at NX = 64 the extra registers would spill).
+    constexpr bool kPrefetch = BLOCK && NX <= 32;
+    float fx[kPrefetch ? NX : 1];
+    float fw = 0.0f;
+    auto fetch = [&](int64_t s) {
+      if constexpr (kPrefetch) {
+        const int t = static_cast<int>(s / p.KB);
+        const int kb = static_cast<int>(s - static_cast<int64_t>(t) * p.KB);
+        fw = __ldg(p.ws + static_cast<int64_t>(t) * p.KB + kb);
+#pragma unroll
+        for (int j = 0; j < NX; ++j) fx[j] = j < p.M ? __ldg(p.xs + static_cast<int64_t>(j) * p.KB + kb) : 0.0f;
+      }
+    };
+    if (b < e) fetch(b);
     for (int64_t s = b; s < e; ++s) {
       const int t = static_cast<int>(s / p.KB);
       const int kb = static_cast<int>(s - static_cast<int64_t>(t) * p.KB);
@@ -193,7 +208,14 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(&sempty[slot]);
       if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
-      if constexpr (BLOCK) {
+      if constexpr (kPrefetch) {
+        float f[NX];
+#pragma unroll
+        for (int j = 0; j < NX; ++j) f[j] = fx[j] * fw;
+        if (s + 1 < e) fetch(s + 1);
+#pragma unroll
+        for (int j = 0; j < NX; ++j) acc[j] = fmaf(__uint_as_float(r[j]), f[j], acc[j]);
+      } else if constexpr (BLOCK) {
         const float wsf = __ldg(p.ws + static_cast<int64_t>(t) * p.KB + kb);
 #pragma unroll
         for (int j = 0; j < NX; ++j) {

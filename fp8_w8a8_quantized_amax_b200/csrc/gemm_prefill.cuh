@@ -300,12 +300,11 @@ struct PairLayout {
   static constexpr int kB = 128 * BK;                           // this CTA's (up to) 128 rows of B
   static constexpr int kEpiWarps = 8;                           // two per TMEM lane quarter
   static constexpr int kOutChunk = 32 * 32 * 2;
-  static constexpr int kOutOff = STAGES * (kA + kB);
-  static constexpr int kWsOff = kOutOff + kEpiWarps * 2 * kOutChunk;
-  static constexpr int kBarOff = kWsOff + kEpiWarps * 128 * 4;
+  static constexpr int kOutOff = STAGES * (kA + kB);           // 2 staging tiles per epilogue warp
+  static constexpr int kBarOff = kOutOff + kEpiWarps * 2 * kOutChunk;
   static constexpr int kBarBytes = (2 * STAGES + 4) * 8 + 8;
-  static constexpr int kBytes = kBarOff + 1024 + 1024;
-  static_assert(kBarBytes <= 1024, "barrier area");
+  static constexpr int kBytes = kBarOff + 256 + 1024;           // + barrier area + alignment slack
+  static_assert(kBarBytes <= 256, "barrier area");
   static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
@@ -438,14 +437,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     }
   } else {
     // 8 epilogue warps: warp w reads TMEM lanes 32*(w%4)..+31 (its 32 rows)
-    // and takes one half of the item's columns.  The TMEM load of the next
-    // 32-column chunk is issued before the current chunk is scaled, staged
-    // and stored, so its latency overlaps that work.
+    // and takes one half of the item's columns (4 or 2 chunks of 32).  The
+    // TMEM load of the next chunk is issued before the current one is scaled,
+    // staged and stored, so its latency overlaps that work.  w_scale of the
+    // chunk's columns is held one value per lane and broadcast by shuffles.
     const int ew = warp - 2;
     const int quarter = warp & 3;
     const int half = ew >> 2;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    float* ws_s = reinterpret_cast<float*>(smem + L::kWsOff) + ew * 128;
     uint8_t* out_s = smem + L::kOutOff + ew * 2 * L::kOutChunk;
     const int swz = (lane >> 1) & 3;
     const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
@@ -456,6 +455,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       const int my_cols = n_cols / 2;                           // 128 or 64
+      const int nchunks = my_cols / 32;                         // 4 or 2
       const int c_begin = half * my_cols;
       const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quarter * 32;
       const int m = row0 + lane;
@@ -464,24 +464,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int n = nb * 256 + n_off + c_begin + i * 32 + lane;
-        wv[i] = (i * 32 < my_cols && n < p.N) ? __ldg(p.ws + n) : 0.0f;
+        wv[i] = (i < nchunks && n < p.N) ? __ldg(p.ws + n) : 0.0f;
       }
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrWaitTmemFull))) break;
       tc_fence_after();
-#pragma unroll
-      for (int i = 0; i < 4; ++i) ws_s[i * 32 + lane] = wv[i];
-      __syncwarp();
       const uint32_t tcol = tmem_base + lane_addr + acc * 256 + c_begin;
-      const int nchunks = my_cols / 32;                         // 4 or 2: always even
       // Scale, stage and store one 32-column chunk held in registers.
-      auto emit = [&](const uint32_t (&cur)[32], int c) {
+      auto emit = [&](const uint32_t (&cur)[32], float w_lane, int c) {
         uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float2 w = *reinterpret_cast<const float2*>(ws_s + c + 2 * j);
-          pk[j] = pack_bf16x2(__uint_as_float(cur[2 * j]) * xsm * w.x, __uint_as_float(cur[2 * j + 1]) * xsm * w.y);
+          const float w0 = __shfl_sync(0xFFFFFFFFu, w_lane, 2 * j);
+          const float w1 = __shfl_sync(0xFFFFFFFFu, w_lane, 2 * j + 1);
+          pk[j] = pack_bf16x2(__uint_as_float(cur[2 * j]) * xsm * w0, __uint_as_float(cur[2 * j + 1]) * xsm * w1);
         }
-        if (lane == 0) bulk_wait_read<1>();
+        if (lane == 0) bulk_wait_read<1>();   // the tile written two chunks ago has been read
         __syncwarp();
         uint8_t* sb = out_s + buf * L::kOutChunk;
 #pragma unroll
@@ -500,21 +497,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       uint32_t ra[32], rb[32];
       __syncwarp();
       tmem_ld_32x32b_x32(tcol, ra);
-#pragma unroll 1
-      for (int ci = 0; ci < nchunks; ci += 2) {
-        tmem_ld_wait_regs(ra);
-        __syncwarp();
-        tmem_ld_32x32b_x32(tcol + (ci + 1) * 32, rb);
-        emit(ra, ci * 32);
-        tmem_ld_wait_regs(rb);
-        if (ci + 2 < nchunks) {
+#pragma unroll
+      for (int ci = 0; ci < 4; ci += 2) {
+        if (ci < nchunks) {
+          tmem_ld_wait_regs(ra);
           __syncwarp();
-          tmem_ld_32x32b_x32(tcol + (ci + 2) * 32, ra);
-        } else {                        // all of this warp's columns read: release the accumulator
-          tc_fence_before();
-          mbar_arrive_cluster(tempty0 + acc * 8);
+          tmem_ld_32x32b_x32(tcol + (ci + 1) * 32, rb);
+          emit(ra, wv[ci], ci * 32);
+          tmem_ld_wait_regs(rb);
+          if (ci + 2 < nchunks) {
+            __syncwarp();
+            tmem_ld_32x32b_x32(tcol + (ci + 2) * 32, ra);
+          } else {                      // all of this warp's columns read: release the accumulator
+            tc_fence_before();
+            mbar_arrive_cluster(tempty0 + acc * 8);
+          }
+          emit(rb, wv[ci + 1], (ci + 1) * 32);
         }
-        emit(rb, (ci + 1) * 32);
       }
     }
     if (lane == 0) bulk_wait<0>();

@@ -197,6 +197,9 @@ def _check_sampled(g: synth.Gemm, seed=0):
 ALL = synth.workloads()
 FULL = [g for name in ("llama3.2-3b_mlp_m2048", "llama3.1-8b_layer_m8192", "llama3.2-3b_block128",
                        "llama3.1-70b_sweep") for g in ALL[name].gemms]
+# GEMMs sharing an input merged over stacked weights (as bench.py also measures)
+FULL += [synth.Gemm("gate_up_proj", 2048, 3072, 16384), synth.Gemm("qkv_proj", 8192, 4096, 6144),
+         synth.Gemm("gate_up_proj_m16_block", 16, 3072, 16384, synth.BLOCK128)]
 
 
 @pytest.mark.parametrize("g", FULL, ids=[f"{g.name}-{g.M}x{g.K}x{g.N}-m{g.mode}" for g in FULL])

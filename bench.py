@@ -194,14 +194,15 @@ class ClockSampler:
 
 # --------------------------------------------------------------- GPU arm ---
 
-def dist_setup(args):
+def dist_setup(args, backend="nccl"):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
 
 
@@ -210,10 +211,14 @@ def barrier(world):
         torch.distributed.barrier()
 
 
+def _collective_device():
+    return "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+
+
 def max_over_ranks(v, world):
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_collective_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -221,9 +226,20 @@ def max_over_ranks(v, world):
 def sum_over_ranks(v, world):
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_collective_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
     return float(t.item())
+
+
+def x_seed(rank: int, i: int) -> int:
+    """Seed of the i-th activation of rank `rank`: every rank quantizes and
+    multiplies its own batch of tokens (token-parallel, weights replicated)."""
+    return 1000 * rank + i
+
+
+def aggregate(units_local: float, seconds_local: float, world: int):
+    """Whole-job work over the slowest rank's time (weak scaling)."""
+    return sum_over_ranks(units_local, world), max_over_ranks(seconds_local, world)
 
 
 def launches_of(g) -> int:
@@ -250,7 +266,7 @@ def run_gpu(args):
     xs_shapes = {}
     for g in wl.gemms:
         xs_shapes.setdefault(g.x, (g.M, g.K, g.mode))
-    X = {k: synth.make_x_device(M, K, seed=1000 * rank + i, device=dev)
+    X = {k: synth.make_x_device(M, K, seed=x_seed(rank, i), device=dev)
          for i, (k, (M, K, _)) in enumerate(xs_shapes.items())}
     WQ = {g.name: fq.fp8_quant_weight(W[g.name], g.mode) for g in wl.gemms}
     XQ = {k: (torch.empty((M, K), dtype=torch.uint8, device=dev),
@@ -327,10 +343,9 @@ def run_gpu(args):
         torch.cuda.synchronize()
     barrier(world)
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    total_s = sum(step_ms) / 1e3
-    total_s = max_over_ranks(total_s, world)
     units = step_units(wl, unit) * args.steps
-    value = to_metric(sum_over_ranks(units, world), total_s, unit)
+    all_units, total_s = aggregate(units, sum(step_ms) / 1e3, world)
+    value = to_metric(all_units, total_s, unit)
 
     # per-op times: every op timed alone after its own L2 flush
     op_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

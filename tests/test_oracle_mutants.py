@@ -1,0 +1,171 @@
+"""The oracle's pins are strong enough to catch plausible mistakes.
+
+Each case plants one mistake in a copy of oracle/fp8_oracle.c (on the CPU,
+in a temporary directory), builds it, and runs independent checks against
+it: torch's float8 casts, exact rational arithmetic, and the properties the
+quantization scheme fixes.  Every mutant must fail at least one check, and
+the unmodified source must pass them all.
+"""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests import _pins
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "fp8_oracle.c")
+
+MUTANTS = {
+    "exponent bias 8": (r"ldexp\(1\.0 \+ m / 8\.0, e - 7\)", "ldexp(1.0 + m / 8.0, e - 8)"),
+    "ties away from even": (r"c = \(uint8_t\)\(\(lo & 1\) \? hi : lo\);", "c = (uint8_t)((lo & 1) ? lo : hi);"),
+    "no sign on codes": (r"return \(uint8_t\)\(c \| sign\);", "return (uint8_t)c;"),
+    "scale amax/447": (r"return num / 448\.0f;", "return num / 447.0f;"),
+    "scale by multiplication": (r"volatile float q = x / s;", "volatile float q = x * (1.0f / s);"),
+    "min instead of max": (r"if \(a > amax\) amax = a;", "if (a < amax || amax == 0.0f) amax = a;"),
+    "w_scale dropped": (r"return \(float\)\(\(double\)xs\[m\] \* \(double\)ws\[n\]", "return (float)((double)xs[m] * 1.0"),
+    "operand rows swapped": (r"code_dot\(xq \+ m \* ldx, wq \+ n \* ldw, 0, K\)", "code_dot(xq + n * ldx, wq + m * ldw, 0, K)"),
+    "block w_scale row": (r"ws\[\(n / 128\) \* KB \+ kb\]", "ws[(n / 64) * KB + kb]"),
+    "block x_scale column": (r"xs\[m \* KB \+ kb\]", "xs[m * KB]"),
+    "group of 64": (r"for \(int64_t k = g \* 128; k < g \* 128 \+ 128; \+\+k\) \{", "for (int64_t k = g * 128; k < g * 128 + 64; ++k) {"),
+    "amax = 0 gives scale 0": (r"if \(amax == 0\.0f\) return 1\.0f;", "if (amax == 0.0f) return 0.0f;"),
+}
+
+
+def build_variant(src_text, tmp):
+    c = os.path.join(tmp, "o.c")
+    so = os.path.join(tmp, "o.so")
+    open(c, "w").write(src_text)
+    subprocess.check_call(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off",
+                           c, "-o", so, "-lm"])
+    L = ctypes.CDLL(so)
+    P, I = ctypes.c_void_p, ctypes.c_int64
+    L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+    L.orc_e4m3_decode.restype = ctypes.c_double
+    L.orc_e4m3_encode_n.argtypes = [P, I, P]
+    for f in ("orc_quant_rows", "orc_quant_groups128", "orc_quant_blocks128"):
+        getattr(L, f).argtypes = [P, I, I, I, P, I, P]
+    L.orc_linear.argtypes = [P, P, P, P, I, I, I, I, I, ctypes.c_int, P]
+    return L
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def checks(L):
+    """Returns the names of the independent checks this build fails."""
+    failed = []
+    vals = _pins.e4m3_values_torch()
+    dec = np.array([L.orc_e4m3_decode(c) for c in range(256)])
+    if not np.all((np.isnan(dec) & np.isnan(vals)) | (dec == vals)):
+        failed.append("decode vs torch")
+    # encoder vs torch RNE cast on every bf16 pattern below 464
+    bits = torch.arange(65536, dtype=torch.int32).to(torch.int16).view(torch.bfloat16).float()
+    f = bits[torch.isfinite(bits) & (bits.abs() < 464)].numpy().astype(np.float32)
+    out = np.empty(f.size, np.uint8)
+    L.orc_e4m3_encode_n(_p(f), f.size, _p(out))
+    if not np.array_equal(out, torch.from_numpy(f).to(torch.float8_e4m3fn).view(torch.uint8).numpy()):
+        failed.append("encode vs torch")
+    # row quantization: max element -> +-448 code, scale ~ amax/448, codes ~ x/s
+    x = synth.make_x(8, 256, seed=3)
+    xb = x.view(torch.int16).numpy().view(np.uint16).copy()
+    q = np.empty((8, 256), np.uint8)
+    s = np.empty(8, np.float32)
+    L.orc_quant_rows(_p(xb), 8, 256, 256, _p(q), 256, _p(s))
+    xf = x.float().numpy().astype(np.float64)
+    for r in range(8):
+        i = np.abs(xf[r]).argmax()
+        amax = np.abs(xf[r]).max()
+        if (q[r, i] & 0x7F) != 0x7E or abs(float(s[r]) * 448 - amax) > amax * 2 ** -22:
+            failed.append("row amax -> 448")
+            break
+    quot = (x.float().numpy() / s[:, None]).astype(np.float32)
+    if not np.array_equal(q.ravel(), _pins.encode_argmin(quot.ravel())):
+        failed.append("row codes vs argmin of x/s")
+    # IEEE division (not x * (1/s)): every bf16 x <= 1632 against amax 1632
+    allv = torch.arange(0, 0x7F80, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    xs_ = allv[(allv.float() <= 1632.0) & (allv.float() >= 0.05)][:1023]   # includes 0.0747, 0.1494
+    row = torch.cat([torch.tensor([1632.0], dtype=torch.bfloat16), xs_]).reshape(1, -1)
+    rb = row.view(torch.int16).numpy().view(np.uint16).copy()
+    qd = np.empty(rb.shape, np.uint8)
+    sd = np.empty(1, np.float32)
+    L.orc_quant_rows(_p(rb), 1, rb.shape[1], rb.shape[1], _p(qd), rb.shape[1], _p(sd))
+    sref = np.float32(np.float32(1632.0) / np.float32(448.0))
+    want = torch.from_numpy((row.float().numpy() / sref).astype(np.float32)).to(torch.float8_e4m3fn) \
+        .view(torch.uint8).numpy()
+    if not np.array_equal(qd, want):
+        failed.append("IEEE division")
+    z = np.zeros((2, 256), np.uint16)
+    qz = np.empty((2, 256), np.uint8)
+    sz = np.empty(2, np.float32)
+    L.orc_quant_rows(_p(z), 2, 256, 256, _p(qz), 256, _p(sz))
+    if not (np.all(sz == 1.0) and np.all(qz == 0)):
+        failed.append("zero rows")
+    # groups: each group equals a row quantization of that group alone
+    xg = synth.make_x(3, 384, seed=4)
+    xgb = xg.view(torch.int16).numpy().view(np.uint16).copy()
+    qg = np.empty((3, 384), np.uint8)
+    sg = np.empty((3, 3), np.float32)
+    L.orc_quant_groups128(_p(xgb), 3, 384, 384, _p(qg), 384, _p(sg))
+    for g in range(3):
+        sub = np.ascontiguousarray(xgb[:, g * 128:(g + 1) * 128])
+        qs = np.empty((3, 128), np.uint8)
+        ss = np.empty(3, np.float32)
+        L.orc_quant_rows(_p(sub), 3, 128, 128, _p(qs), 128, _p(ss))
+        amax = np.abs(xg.float().numpy()[:, g * 128:(g + 1) * 128]).max(axis=1)
+        if not (np.array_equal(qs, qg[:, g * 128:(g + 1) * 128]) and np.array_equal(ss, sg[:, g])) or \
+                np.any(np.abs(sg[:, g].astype(np.float64) * 448 - amax) > amax * 2 ** -22):
+            failed.append("groups")
+            break
+    # linear vs exact rationals, both modes, non-square
+    rng = np.random.default_rng(5)
+    M, N, K = 3, 130, 256
+    xq = rng.integers(0, 256, (M, K)).astype(np.uint8)
+    wq = rng.integers(0, 256, (N, K)).astype(np.uint8)
+    xq[(xq & 0x7F) == 0x7F] = 0x38
+    wq[(wq & 0x7F) == 0x7F] = 0x38
+    xs = rng.uniform(0.1, 2, M).astype(np.float32)
+    ws = rng.uniform(0.01, 0.1, N).astype(np.float32)
+    y = np.empty((M, N), np.float32)
+    L.orc_linear(_p(xq), _p(xs), _p(wq), _p(ws), M, N, K, K, K, 0, _p(y))
+    for m, n in [(0, 0), (2, 129), (1, 64)]:
+        e = sum(Fraction(float(vals[a])) * Fraction(float(vals[b])) for a, b in zip(xq[m], wq[n]))
+        e = float(e * Fraction(float(xs[m])) * Fraction(float(ws[n])))
+        if abs(float(y[m, n]) - e) > _pins.f32_ulp(e):
+            failed.append("linear channel vs rationals")
+            break
+    xsb = rng.uniform(0.1, 2, (M, K // 128)).astype(np.float32)
+    wsb = rng.uniform(0.01, 0.1, ((N + 127) // 128, K // 128)).astype(np.float32)
+    L.orc_linear(_p(xq), _p(xsb), _p(wq), _p(wsb), M, N, K, K, K, 1, _p(y))
+    for m, n in [(0, 0), (2, 129), (1, 64)]:
+        e = Fraction(0)
+        for k in range(K):
+            e += Fraction(float(vals[xq[m, k]])) * Fraction(float(vals[wq[n, k]])) * \
+                Fraction(float(xsb[m, k // 128])) * Fraction(float(wsb[n // 128, k // 128]))
+        if abs(float(y[m, n]) - float(e)) > _pins.f32_ulp(float(e)) * 2:
+            failed.append("linear block vs rationals")
+            break
+    return failed
+
+
+def test_unmodified_oracle_passes_every_check():
+    with tempfile.TemporaryDirectory() as tmp:
+        assert checks(build_variant(open(SRC).read(), tmp)) == []
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name):
+    pat, rep = MUTANTS[name]
+    src = open(SRC).read()
+    mutated, n = re.subn(pat, rep, src)
+    assert n >= 1, f"mutation '{name}' did not apply"
+    with tempfile.TemporaryDirectory() as tmp:
+        failed = checks(build_variant(mutated, tmp))
+    assert failed, f"planted mistake '{name}' passed every check"

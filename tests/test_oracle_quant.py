@@ -159,3 +159,35 @@ def test_codes_match_independent_encoder_on_synthetic_rows():
     xf = x.to(torch.float32).numpy()
     quot = (xf / s[:, None]).astype(np.float32)   # numpy fp32 IEEE division
     assert np.array_equal(q.ravel(), _pins.encode_argmin(quot.ravel()))
+
+
+def _division_rows(amax):
+    """Rows whose amax is `amax`, holding every bf16 value in [0, amax]."""
+    allv = torch.arange(0, 0x7F80, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    xs = allv[allv.float() <= amax]
+    per = 1023
+    rows = []
+    for i in range(0, xs.numel(), per):
+        chunk = xs[i:i + per]
+        row = torch.zeros(per + 1, dtype=torch.bfloat16)
+        row[0] = amax
+        row[1:1 + chunk.numel()] = chunk
+        rows.append(row)
+    return torch.stack(rows)
+
+
+@pytest.mark.parametrize("amax", [1632.0, 191.0, 66.0, 8224768.0])
+def test_codes_follow_ieee_division(amax):
+    """Reading R3: the code is E4M3 of the IEEE fp32 quotient x / s.  For these
+    amax values some x give a different code under x * (1/s); numpy's fp32
+    division and torch's fp8 cast fix the expected codes independently."""
+    x = _division_rows(amax)
+    q, s = oracle.quant_rows(x)
+    s_ref = np.float32(np.float32(amax) / np.float32(448.0))
+    assert np.all(s == s_ref)
+    xf = x.float().numpy()
+    want = torch.from_numpy((xf / s_ref).astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    recip = torch.from_numpy((xf * np.float32(np.float32(1) / s_ref)).astype(np.float32)) \
+        .to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.any(want != recip)          # the case really separates the two readings
+    assert np.array_equal(q, want)

@@ -192,6 +192,78 @@ class ClockSampler:
                 "sampler": "NVML in a separate process, every 1 ms during the timed steps"}
 
 
+_MONITOR_SRC = r"""
+extern "C" __global__ void clock_monitor(unsigned long long duration_ns, unsigned long long* out, int max_samples) {
+  // One thread: every ~0.5 ms record (clock64, globaltimer) of this SM, for
+  // duration_ns of wall time or max_samples samples, whichever comes first.
+  unsigned long long t0, t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (int i = 0; i < max_samples; ++i) {
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    out[2 * i] = clock64();
+    out[2 * i + 1] = t;
+    if (t - t0 > duration_ns) { out[2 * i + 2] = 0; return; }
+    for (int k = 0; k < 10; ++k) __nanosleep(50000);
+  }
+}
+"""
+
+
+class ClockMonitor:
+    """Measures the SM clock the kernels actually run at: a one-warp kernel
+    on a side stream records this SM's cycle counter against the global
+    nanosecond timer while the timed steps run (NVML's reading lags by tens
+    of milliseconds and misses power capping in short runs)."""
+
+    def __init__(self, duration_s: float, max_samples: int = 4096):
+        self.err, self.samples = None, None
+        try:
+            import tempfile
+            from cuda.bindings import driver as cu
+            self.cu = cu
+            d = tempfile.mkdtemp(prefix="clkmon")
+            src, cub = os.path.join(d, "m.cu"), os.path.join(d, "m.cubin")
+            open(src, "w").write(_MONITOR_SRC)
+            nvcc = "/usr/local/cuda/bin/nvcc" if os.path.exists("/usr/local/cuda/bin/nvcc") else "nvcc"
+            subprocess.check_call([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-cubin", "-o", cub, src],
+                                  stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            err, self.mod = cu.cuModuleLoad(cub.encode())
+            err2, self.fn = cu.cuModuleGetFunction(self.mod, b"clock_monitor")
+            if int(err) or int(err2):
+                raise RuntimeError(f"module load: {err} {err2}")
+            self.max = max_samples
+            self.buf = torch.zeros(2 * max_samples + 2, dtype=torch.int64, device="cuda")
+            self.duration_ns = int(duration_s * 1e9)
+            self.stream = torch.cuda.Stream()
+        except Exception as e:
+            self.err = f"clock monitor unavailable: {e}"
+
+    def start(self):
+        if self.err:
+            return
+        import ctypes
+        self._args = (ctypes.c_ulonglong(self.duration_ns), ctypes.c_void_p(self.buf.data_ptr()),
+                      ctypes.c_int(self.max))
+        self._ptrs = (ctypes.c_void_p * 3)(*[ctypes.addressof(a) for a in self._args])
+        (r,) = self.cu.cuLaunchKernel(self.fn, 1, 1, 1, 1, 1, 1, 0, self.stream.cuda_stream,
+                                      ctypes.addressof(self._ptrs), 0)
+        if int(r):
+            self.err = f"clock monitor launch: {r}"
+
+    def summary(self):
+        if self.err:
+            return {"error": self.err}
+        torch.cuda.synchronize()
+        v = self.buf.cpu().numpy().reshape(-1, 2)
+        v = v[: np.argmax(v[:, 1] == 0)] if np.any(v[:, 1] == 0) else v
+        if len(v) < 3:
+            return {"error": "too few samples"}
+        mhz = np.diff(v[:, 0]) / np.diff(v[:, 1]) * 1e3
+        return {"sm_mhz_median": round(float(np.median(mhz)), 1), "sm_mhz_min": round(float(mhz.min()), 1),
+                "intervals": int(mhz.size),
+                "method": "clock64 / %globaltimer on one SM, ~0.5 ms intervals, during an untimed repeat of the steps"}
+
+
 # --------------------------------------------------------------- GPU arm ---
 
 def dist_setup(args, backend="nccl"):
@@ -331,6 +403,13 @@ def run_gpu(args):
 
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
+    # expected length of the timed loop, for the clock monitor
+    t_est = time.perf_counter()
+    for _ in range(3):
+        flush.zero_()
+        step_runner()
+    torch.cuda.synchronize()
+    loop_s = (time.perf_counter() - t_est) / 3 * args.steps
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
@@ -343,6 +422,15 @@ def run_gpu(args):
         torch.cuda.synchronize()
     barrier(world)
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    # The clock the kernels actually ran at, measured on an untimed repeat of
+    # the same steps (the monitor's warp occupies one SM, so it stays out of
+    # the timed loop).
+    mon = ClockMonitor(duration_s=loop_s + 0.005)
+    mon.start()
+    for _ in range(args.steps):
+        flush.zero_()
+        step_runner()
+    torch.cuda.synchronize()
     units = step_units(wl, unit) * args.steps
     all_units, total_s = aggregate(units, sum(step_ms) / 1e3, world)
     value = to_metric(all_units, total_s, unit)
@@ -528,7 +616,7 @@ def run_gpu(args):
                        "parallelism": "single GPU" if world == 1 else f"token-parallel x{world}, weights replicated"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g) for g in wl.gemms)),
-            "clocks": clk.summary(), "detail": detail, "weight_quant": weight_quant,
+            "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant,
             "merged_shared_input": merged,
             "device_error": err, "gpu": torch.cuda.get_device_name(dev),
         }

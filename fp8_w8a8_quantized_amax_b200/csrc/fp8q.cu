@@ -172,7 +172,7 @@ fp8q_status launch_rows(const uint16_t* x, int64_t rows, int K, int64_t ldx, uin
 constexpr int kPrefillBN = 256;
 constexpr int kPairStages = 6;
 
-// Prefill kernel choice for channel mode: the CTA-pair kernel for M >= 256,
+// Prefill kernel choice (both modes): the CTA-pair kernel for M >= 256,
 // else the single-CTA kernel.  FP8Q_PREFILL_KERNEL=single|pair forces one
 // (read once), for comparing them on the same problem.
 int prefill_choice() {
@@ -333,20 +333,30 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     return launch_decode_nx<64>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
   }
 
-  const bool pair = mode == FP8Q_CHANNEL_TOKEN && prefill_choice() != 1 && (M >= 256 || prefill_choice() == 2);
+  const bool pair = prefill_choice() != 1 && (M >= 256 || prefill_choice() == 2);
   if (pair) {
     using L = fp8q::prefill::PairLayout<kPairStages>;
-    auto k = fp8q::prefill::gemm_channel2_kernel<kPairStages>;
+    const bool block = mode == FP8Q_BLOCK128;
+    auto k = block ? fp8q::prefill::gemm_block2_kernel<kPairStages> : fp8q::prefill::gemm_channel2_kernel<kPairStages>;
+    static_assert(fp8q::prefill::PairLayout<kPairStages, 4>::kBytes == L::kBytes, "one shared-memory size");
+    const int threads = block ? fp8q::prefill::kBlock2Threads : 64 + 32 * L::kEpiWarps;
     if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
-    static int max_pairs[kMaxDevices] = {};
-    if (max_pairs[dev] == 0) {
+    static int max_pairs[2][kMaxDevices] = {};
+    if (max_pairs[block][dev] == 0) {
+      if (block) {
+        // The kernel moves registers between its warpgroups; that is only
+        // safe when it is launched with the register count it was built for.
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return FP8Q_ERR_CUDA;
+        if (fa.numRegs != fp8q::prefill::kBlock2LaunchRegs) return FP8Q_ERR_UNSUPPORTED;
+      }
       cudaLaunchConfig_t qc = {};
       qc.gridDim = dim3(2 * sms);
-      qc.blockDim = dim3(64 + 32 * L::kEpiWarps);
+      qc.blockDim = dim3(threads);
       qc.dynamicSmemBytes = L::kBytes;
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, k, &qc) != cudaSuccess || n < 1) n = sms / 2;
-      max_pairs[dev] = n;
+      max_pairs[block][dev] = n;
     }
     fp8q::prefill::Params p;
     p.xs = x_scale;
@@ -361,7 +371,7 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     p.num_n = static_cast<int>((N + 255) / 256);
     p.num_tiles = p.num_m * p.num_n;
     p.group_m = p.num_m < 8 ? p.num_m : 8;
-    const int pairs = max_pairs[dev];
+    const int pairs = max_pairs[block][dev];
     tail_split(p.num_tiles, pairs, &p.full, &p.split);
     const int items = (p.full ? p.full : 0) + (p.num_tiles - p.full) * p.split;
     const int used = p.full ? pairs : (items < pairs ? items : pairs);
@@ -370,7 +380,7 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     if ((st = tmap_u8_sw128(&tb, Wq, N, K, K, 128)) != FP8Q_OK) return st;
     if ((st = tmap_u8_sw128(&tb64, Wq, N, K, K, 64)) != FP8Q_OK) return st;
     if ((st = tmap_bf16_sw64(&ty, Y_bf16, M, N, ldy, 32)) != FP8Q_OK) return st;
-    return launch(k, dim3(2 * used), dim3(64 + 32 * L::kEpiWarps), L::kBytes, stream, ta, tb, tb64, ty, p);
+    return launch(k, dim3(2 * used), dim3(threads), L::kBytes, stream, ta, tb, tb64, ty, p);
   }
 
   fp8q::prefill::Params p;

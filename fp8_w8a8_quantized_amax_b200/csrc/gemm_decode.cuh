@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < kSlots; ++a) {
       mbar_init(&sfull[a], 1);
-      mbar_init(&sempty[a], 128);
+      mbar_init(&sempty[a], 4);                  // one arrival per epilogue warp
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -206,7 +206,8 @@ __global__ void __launch_bounds__(192, 1)
                                                            *reinterpret_cast<uint32_t(*)[16]>(&r[j]));
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&sempty[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_relaxed(&sempty[slot]);
       if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
       if constexpr (kPrefetch) {
         float f[NX];

@@ -20,6 +20,8 @@
 // warps fold each slot into fp32 registers with that slice's scale product.
 #pragma once
 
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace fp8q {
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 4);                  // one arrival per epilogue warp
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -243,7 +245,8 @@ __global__ void __launch_bounds__(192, 1)
         tmem_ld_wait();
         if (c + 32 == n_cols) {          // accumulator fully read: hand it back to the MMA
           tc_fence_before();
-          mbar_arrive(&tempty[acc]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive_relaxed(&tempty[acc]);
         }
         uint32_t pk[16];
 #pragma unroll
@@ -293,8 +296,8 @@ __global__ void __launch_bounds__(192, 1)
 //              both CTAs' TMA loads complete on it.
 //   empty[s]   both CTAs: the leader's commit arrives on both.
 //   tfull[a]   both CTAs: the leader's commit arrives on both.
-//   tempty[a]  leader only: all 256 epilogue threads of the pair arrive.
-template <int STAGES>
+//   tempty[a]  leader only: lane 0 of each of the pair's 16 epilogue warps arrives.
+template <int STAGES, int NACC = 2>
 struct PairLayout {
   static constexpr int kA = 128 * BK;                           // this CTA's 128 rows of A
   static constexpr int kB = 128 * BK;                           // this CTA's (up to) 128 rows of B
@@ -302,7 +305,7 @@ struct PairLayout {
   static constexpr int kOutChunk = 32 * 32 * 2;
   static constexpr int kOutOff = STAGES * (kA + kB);           // 2 staging tiles per epilogue warp
   static constexpr int kBarOff = kOutOff + kEpiWarps * 2 * kOutChunk;
-  static constexpr int kBarBytes = (2 * STAGES + 4) * 8 + 8;
+  static constexpr int kBarBytes = (2 * STAGES + 2 * NACC) * 8 + 8;   // + TMEM address, abort flag
   static constexpr int kBytes = kBarOff + 256 + 1024;           // + barrier area + alignment slack
   static_assert(kBarBytes <= 256, "barrier area");
   static_assert(kBytes <= 232448, "shared memory per CTA");
@@ -339,7 +342,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 2 * 32 * L::kEpiWarps);             // every epilogue thread of the pair
+      mbar_init(&tempty[a], 2 * L::kEpiWarps);                  // every epilogue warp of the pair
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -510,7 +513,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
             tmem_ld_32x32b_x32(tcol + (ci + 2) * 32, ra);
           } else {                      // all of this warp's columns read: release the accumulator
             tc_fence_before();
-            mbar_arrive_cluster(tempty0 + acc * 8);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + acc * 8);
           }
           emit(rb, wv[ci + 1], (ci + 1) * 32);
         }
@@ -522,6 +526,324 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
   tc_fence_before();
   __syncthreads();
   cluster_sync();                 // no CTA leaves while its pair may still signal it or read its memory
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------- block, CTA pair ---
+// Block-scaled GEMM on 256 x 256 tiles computed by a CTA pair, with the same
+// operand split as the channel pair kernel (32 KB per CTA per 128-wide K
+// block).  Every K block is issued as two M=256, N=128 MMAs: MMA j reads
+// B rows [64 j, 64 j + 64) of each CTA's 128-row B stage, so its 128
+// accumulator columns are [64 j, +64) of the first weight block of the tile
+// (the leader's B rows) followed by [64 j, +64) of the second (the peer's).
+// Each MMA writes a fresh partial product into one of four 128-column TMEM
+// slots, which the epilogue folds into fp32 registers with that K block's
+// scale product x_scale[m, kb] * w_scale[n / 128, kb] and releases.  Four
+// slots let the MMAs run up to two K blocks ahead of the epilogue.
+//   tfull[s]   both CTAs: the leader's commit arrives on both.
+//   tempty[s]  leader only: one arrival per epilogue warp of the pair (16),
+//              by lane 0 once the whole warp has read the slot.
+// A tail item of 128 columns (one weight block) issues only MMA j = 0 over
+// 64 B rows per CTA.
+// Three warpgroups: warp 0 loads, warp 1 issues the MMAs (warps 2-3 idle),
+// warpgroups 1 and 2 are the epilogue.  The epilogue keeps 128 fp32
+// accumulators per thread, so registers are moved from the first warpgroup
+// to the other two: 128 x kCtlRegs + 256 x kEpiRegs = 384 x kLaunchRegs.
+constexpr int kBlock2Threads = 384;
+constexpr int kBlock2LaunchRegs = 168;
+constexpr int kBlock2CtlRegs = 56;
+constexpr int kBlock2EpiRegs = 224;
+static_assert(128 * kBlock2CtlRegs + 256 * kBlock2EpiRegs <= kBlock2Threads * kBlock2LaunchRegs, "register split");
+static_assert(kBlock2CtlRegs + 2 * kBlock2EpiRegs <= 512, "registers of one SM sub-partition");
+
+template <int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
+    gemm_block2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmB64, const __grid_constant__ CUtensorMap tmY,
+                       const Params p) {
+  constexpr int kSlots = 4;
+  using L = PairLayout<STAGES, kSlots>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * L::kA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + kSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + kSlots);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  constexpr uint32_t kTmemCols = kSlots * 128;
+  constexpr uint16_t kBoth = 0x3;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < kSlots; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * L::kEpiWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmB64);
+    tma_prefetch_desc(&tmY);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();
+
+  const int G2 = gridDim.x >> 1;
+  auto count = [&]() {
+    const int tail = (p.num_tiles - p.full) * p.split;
+    return p.full / G2 + (pair < tail ? (tail - 1 - pair) / G2 + 1 : 0);
+  };
+  auto coords = [&](int i, int& mb, int& nb, int& n_off, int& n_cols) {
+    const int nfull = p.full / G2;
+    if (i < nfull) {
+      tile_coords(p, pair + i * G2, mb, nb);
+      n_off = 0;
+      n_cols = 256;
+    } else {
+      const int j = pair + (i - nfull) * G2;
+      tile_coords(p, p.full + j / p.split, mb, nb);
+      n_cols = 256 / p.split;
+      n_off = (j % p.split) * n_cols;
+    }
+  };
+  const int nitems = count();
+
+  if (warp < 4) regs_shrink<kBlock2CtlRegs>();
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int i = 0; ok && i < nitems; ++i) {
+        int mb, nb, n_off, n_cols;
+        coords(i, mb, nb, n_off, n_cols);
+        const int half = n_cols / 2;
+        const CUtensorMap* tb = half == 128 ? &tmB : &tmB64;
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) { ok = false; break; }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * static_cast<uint32_t>(L::kA + half * BK));
+          const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
+          tma_load_2d_pair(sA + stage * L::kA, &tmA, bar0, kb * BK, mb * 256 + static_cast<int>(rank) * 128, pol);
+          tma_load_2d_pair(sB + stage * L::kB, tb, bar0, kb * BK, nb * 256 + n_off + static_cast<int>(rank) * half,
+                           pol);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      griddep_launch_dependents();
+      for (int i = 0; ok && i < STAGES; ++i) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) break;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(256, 128);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t slot_count = 0;
+      bool ok = true;
+      for (int it = 0; ok && it < nitems; ++it) {
+        int mb, nb, n_off, n_cols;
+        coords(it, mb, nb, n_off, n_cols);
+        const int nj = n_cols / 128;                            // 2 for a whole tile, 1 for a tail half
+        for (int kb = 0; ok && kb < p.KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * L::kA);
+          const uint32_t b0 = smem_u32(sB + stage * L::kB);
+          for (int j = 0; j < nj; ++j) {
+            const int slot = static_cast<int>(slot_count & (kSlots - 1));
+            const uint32_t sphase = (slot_count / kSlots) & 1u;
+            if (!mbar_wait_cluster(&tempty[slot], sphase ^ 1u, abort_flag, kErrWaitTmemEmpty)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d = tmem_base + slot * 128;
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k)
+              mma_e4m3_pair(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + j * 64 * BK + k * UMMA_K),
+                            idesc, k != 0);
+            mma_commit_pair(&tfull[slot], kBoth);
+            ++slot_count;
+          }
+          if (!ok) break;
+          mma_commit_pair(&empty[stage], kBoth);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp >= 4) {
+    regs_grow<kBlock2EpiRegs>();
+    // 8 epilogue warps: warp w reads TMEM lanes 32*(w%4)..+31 (its 32 rows)
+    // and columns [64 h, 64 h + 64) of every slot, h = (w - 4) / 4: for a
+    // whole tile, 64 columns of weight block h; for a tail half, columns
+    // [64 h, +64) of its single weight block.  acc[j][c] holds columns
+    // [32 c, +32) of that part for MMA j.
+    // The slot halves of a tile are read as one stream of 32-column loads,
+    // each issued before the previous one is folded in, so the TMEM load
+    // latency overlaps the FMAs; a slot is handed back as soon as both of its
+    // halves are in registers.  The scale products are fetched two K blocks
+    // ahead.
+    const int ew = warp - 4;
+    const int quarter = warp & 3;
+    const int h = ew >> 2;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    uint8_t* out_s = smem + L::kOutOff + ew * 2 * L::kOutChunk;
+    const int swz = (lane >> 1) & 3;
+    const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const int NB = (p.N + 127) / 128;
+    uint32_t slot_count = 0;
+    int buf = 0;
+    bool ok = true;
+
+    auto wait_full = [&](uint32_t u) -> bool {
+      const bool done = __all_sync(0xFFFFFFFFu, mbar_wait(&tfull[u & (kSlots - 1)], (u / kSlots) & 1u, abort_flag,
+                                                          kErrWaitTmemFull));
+      tc_fence_after();
+      return done;
+    };
+    auto load = [&](uint32_t u, int c, uint32_t (&r)[32]) {
+      __syncwarp();
+      tmem_ld_32x32b_x32(tmem_base + lane_addr + (u & (kSlots - 1)) * 128 + h * 64 + c * 32, r);
+    };
+    auto release = [&](uint32_t u) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + (u & (kSlots - 1)) * 8);
+    };
+    auto fold = [&](const uint32_t (&r)[32], uint64_t (&a)[16], uint64_t f2) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        a[i] = fma_f32x2(f32x2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), f2, a[i]);
+    };
+
+    for (int it = 0; ok && it < nitems; ++it) {
+      int mb, nb, n_off, n_cols;
+      coords(it, mb, nb, n_off, n_cols);
+      const int nj = n_cols / 128;
+      const int hb = n_cols / 2;                                // B rows per CTA: 128 or 64
+      const int n_first = nb * 256 + n_off + h * hb;            // first column of this warp's part
+      const int blk = n_first / 128;
+      const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quarter * 32;
+      const int m = row0 + lane;
+      const bool live = m < p.M && blk < NB;
+      const float* xsrow = p.xs + static_cast<int64_t>(live ? m : 0) * p.KB;
+      const float* wsrow = p.ws + static_cast<int64_t>(live ? blk : 0) * p.KB;
+      uint64_t acc[2][2][16];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[j][c][i] = 0ull;
+      float xa = live ? __ldg(xsrow) : 0.0f, wa = live ? __ldg(wsrow) : 0.0f;
+      float xb = live && p.KB > 1 ? __ldg(xsrow + 1) : 0.0f, wb = live && p.KB > 1 ? __ldg(wsrow + 1) : 0.0f;
+
+      uint32_t ra[32], rb[32];
+      uint32_t u = slot_count;                                  // first slot of the current K block
+      if (!wait_full(u)) { ok = false; break; }
+      load(u, 0, ra);
+      tmem_ld_wait_regs(ra);
+      // One K block: the half-slots s = 2 j + c, s < 2 NJ, alternating between
+      // ra (even s) and rb (odd s); the load after the last one is the first
+      // half of the next K block, into ra again.
+      auto kblock = [&](auto NJc, int kb) {
+        constexpr int NJ = decltype(NJc)::value;
+        const uint64_t f2 = f32x2_pack(xa * wa, xa * wa);
+        xa = xb;
+        wa = wb;
+        if (live && kb + 2 < p.KB) {
+          xb = __ldg(xsrow + kb + 2);
+          wb = __ldg(wsrow + kb + 2);
+        }
+#pragma unroll
+        for (int s2 = 0; s2 < 2 * NJ; ++s2) {
+          const int j = s2 >> 1, c = s2 & 1;
+          const bool last = s2 + 1 == 2 * NJ;
+          const bool has_next = !last || kb + 1 < p.KB;
+          const uint32_t u_next = last ? u + NJ : u + ((s2 + 1) >> 1);
+          const int c_next = last ? 0 : ((s2 + 1) & 1);
+          uint32_t (&cur)[32] = (s2 & 1) ? rb : ra;
+          uint32_t (&nxt)[32] = (s2 & 1) ? ra : rb;
+          if (has_next && ok) {
+            if (c_next == 0 && !wait_full(u_next)) ok = false;
+            if (ok) load(u_next, c_next, nxt);
+          }
+          fold(cur, acc[j][c], f2);
+          if (has_next && ok) {
+            tmem_ld_wait_regs(nxt);
+            if (c_next == 1) release(u_next);                   // both halves of slot u + j are in registers
+          }
+        }
+        u += NJ;
+      };
+      if (nj == 2) {
+        for (int kb = 0; ok && kb < p.KB; ++kb) kblock(std::integral_constant<int, 2>(), kb);
+      } else {
+        for (int kb = 0; ok && kb < p.KB; ++kb) kblock(std::integral_constant<int, 1>(), kb);
+      }
+      slot_count = u;
+      if (!ok) break;
+      // Round to bf16 and store: columns [64 j + 32 c, +32) of this warp's part.
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (j < nj) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float lo, hi;
+              f32x2_unpack(acc[j][c][i], lo, hi);
+              pk[i] = pack_bf16x2(lo, hi);
+            }
+            if (lane == 0) bulk_wait_read<1>();   // the staging tile written two chunks ago has been read
+            __syncwarp();
+            uint8_t* sb = out_s + buf * L::kOutChunk;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<uint4*>(sb + lane * 64 + ((q ^ swz) << 4)) =
+                  make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            const int col0 = n_first + 64 * j + 32 * c;
+            if (lane == 0 && row0 < p.M && col0 < p.N) {
+              tma_store_2d(&tmY, sb, col0, row0);
+              bulk_commit();
+            }
+            buf ^= 1;
+          }
+        }
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -567,7 +889,6 @@ __global__ void __launch_bounds__(576, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   constexpr uint32_t kTmemCols = kSlots * BN;   // 512
-  constexpr int kEpiThreads = 32 * L::kEpiWarps;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -576,7 +897,7 @@ __global__ void __launch_bounds__(576, 1)
     }
     for (int a = 0; a < kSlots; ++a) {
       mbar_init(&sfull[a], 1);
-      mbar_init(&sempty[a], kEpiThreads);
+      mbar_init(&sempty[a], L::kEpiWarps);      // one arrival per epilogue warp
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -677,7 +998,8 @@ __global__ void __launch_bounds__(576, 1)
         tmem_ld_32x32b_x32(tmem_base + lane_addr + slot * BN + cg * 32, r);
         tmem_ld_wait();
         tc_fence_before();
-        mbar_arrive(&sempty[slot]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_relaxed(&sempty[slot]);
         const uint64_t f2 = f32x2_pack(f, f);
 #pragma unroll
         for (int j = 0; j < 16; ++j)

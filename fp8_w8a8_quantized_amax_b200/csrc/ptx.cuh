@@ -120,6 +120,18 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// Arrivals that only say "this buffer may be overwritten" (a tensor-memory
+// slot whose loads have completed with tcgen05.wait::ld) hand over no memory,
+// so they are relaxed: a release arrive would first wait for every global load
+// the thread still has in flight (the scale prefetch), about a thousand cycles
+// per arrive.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -162,6 +174,19 @@ __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wa
 // griddep_wait() for this grid to finish).
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Per-warpgroup register split.  Every warp of a warpgroup executes the same
+// instruction; an increase waits until the registers are free, so the sum of
+// the warpgroups' shares must not exceed what the block was launched with
+// (the host checks the kernel's register count before launching).
+template <uint32_t R>
+__device__ __forceinline__ void regs_shrink() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void regs_grow() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
 }
 
 // ------------------------------------------------------------------ TMA ---

@@ -70,16 +70,18 @@ def test_prefill_channel(M, N, K):
     check_full(M, N, K, fq.CHANNEL_TOKEN, seed=M)
 
 
-@pytest.mark.parametrize("kernel,M,N,K", [("single", 2048, 2560, 256), ("single", 1024, 4096, 512),
-                                          ("pair", 200, 320, 272), ("pair", 65, 512, 128)])
-def test_prefill_kernel_forced(kernel, M, N, K):
+@pytest.mark.parametrize("kernel,M,N,K,mode", [("single", 2048, 2560, 256, 0), ("single", 1024, 4096, 512, 0),
+                                               ("pair", 200, 320, 272, 0), ("pair", 65, 512, 128, 0),
+                                               ("single", 1024, 3072, 512, 1), ("pair", 200, 384, 384, 1),
+                                               ("pair", 65, 272, 128, 1)])
+def test_prefill_kernel_forced(kernel, M, N, K, mode):
     # each prefill kernel on shapes the default dispatch would give the other one
     import os
     import subprocess
     import sys
     env = dict(os.environ, FP8Q_PREFILL_KERNEL=kernel)
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    r = subprocess.run([sys.executable, "-m", "tests._forced_kernel", str(M), str(N), str(K), "0"],
+    r = subprocess.run([sys.executable, "-m", "tests._forced_kernel", str(M), str(N), str(K), str(mode)],
                        cwd=root, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr
 
@@ -87,7 +89,12 @@ def test_prefill_kernel_forced(kernel, M, N, K):
 @pytest.mark.parametrize("M,N,K", [
     (200, 384, 384),
     (130, 144, 256),       # a partial 128-row weight block
-    (1024, 3072, 512),     # 192 tiles > 148 SMs
+    (256, 256, 128),       # CTA-pair kernel (M >= 256): one tile, one K block
+    (300, 384, 384),       # pair kernel: second tile half past N (its second weight block absent)
+    (1000, 1040, 512),     # pair kernel, ragged M and a 16-row last weight block
+    (1024, 3072, 512),     # pair kernel, 48 tiles
+    (2048, 2560, 256),     # more tiles than pairs: persistent loop, tail split into 128-column halves
+    (4096, 1024, 1152),    # 9 K blocks: slots wrap over an odd number of K blocks per tile
 ])
 def test_prefill_block(M, N, K):
     check_full(M, N, K, fq.BLOCK128, seed=N)

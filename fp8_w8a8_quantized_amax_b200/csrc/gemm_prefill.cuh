@@ -536,19 +536,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
 // ------------------------------------------------------- block, CTA pair ---
 // Block-scaled GEMM on 256 x 256 tiles computed by a CTA pair, with the same
 // operand split as the channel pair kernel (32 KB per CTA per 128-wide K
-// block).  Every K block is issued as two M=256, N=128 MMAs: MMA j reads
-// B rows [64 j, 64 j + 64) of each CTA's 128-row B stage, so its 128
-// accumulator columns are [64 j, +64) of the first weight block of the tile
-// (the leader's B rows) followed by [64 j, +64) of the second (the peer's).
-// Each MMA writes a fresh partial product into one of four 128-column TMEM
-// slots, which the epilogue folds into fp32 registers with that K block's
-// scale product x_scale[m, kb] * w_scale[n / 128, kb] and releases.  Four
-// slots let the MMAs run up to two K blocks ahead of the epilogue.
+// block) and the same M=256, N=256 MMAs.  The scale x_scale[m, kb] *
+// w_scale[n / 128, kb] changes with every K block, so each K block's MMAs
+// write a fresh partial product into one of two 256-column TMEM slots, which
+// the epilogue folds into fp32 registers and hands back; the MMAs of the next
+// K block run meanwhile in the other slot.  Accumulator columns [0, 128) are
+// the first weight block of the tile (the leader's B rows), [128, 256) the
+// second (the peer's), so each epilogue warp meets one scale per K block.
 //   tfull[s]   both CTAs: the leader's commit arrives on both.
 //   tempty[s]  leader only: one arrival per epilogue warp of the pair (16),
 //              by lane 0 once the whole warp has read the slot.
-// A tail item of 128 columns (one weight block) issues only MMA j = 0 over
-// 64 B rows per CTA.
+// A tail item of 128 columns (one weight block) uses N=128 MMAs over 64 B
+// rows per CTA.
 // Three warpgroups: warp 0 loads, warp 1 issues the MMAs (warps 2-3 idle),
 // warpgroups 1 and 2 are the epilogue.  The epilogue keeps 128 fp32
 // accumulators per thread, so registers are moved from the first warpgroup
@@ -559,13 +558,14 @@ constexpr int kBlock2CtlRegs = 56;
 constexpr int kBlock2EpiRegs = 224;
 static_assert(128 * kBlock2CtlRegs + 256 * kBlock2EpiRegs <= kBlock2Threads * kBlock2LaunchRegs, "register split");
 static_assert(kBlock2CtlRegs + 2 * kBlock2EpiRegs <= 512, "registers of one SM sub-partition");
+static_assert(kBlock2CtlRegs % 8 == 0 && kBlock2EpiRegs % 8 == 0, "setmaxnreg takes multiples of 8");
 
 template <int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
     gemm_block2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmB64, const __grid_constant__ CUtensorMap tmY,
                        const Params p) {
-  constexpr int kSlots = 4;
+  constexpr int kSlots = 2;
   using L = PairLayout<STAGES, kSlots>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -582,7 +582,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1;
-  constexpr uint32_t kTmemCols = kSlots * 128;
+  constexpr uint32_t kTmemCols = kSlots * 256;
   constexpr uint16_t kBoth = 0x3;
 
   if (threadIdx.x == 0) {
@@ -633,35 +633,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
 
   if (warp < 4) regs_shrink<kBlock2CtlRegs>();
   if (warp == 0) {
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int i = 0; ok && i < nitems; ++i) {
-        int mb, nb, n_off, n_cols;
-        coords(i, mb, nb, n_off, n_cols);
-        const int half = n_cols / 2;
-        const CUtensorMap* tb = half == 128 ? &tmB : &tmB64;
-        for (int kb = 0; kb < p.KB; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) { ok = false; break; }
+    // The whole warp runs the loop; one elected lane issues the copies.
+    const uint64_t pol = policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int i = 0; ok && i < nitems; ++i) {
+      int mb, nb, n_off, n_cols;
+      coords(i, mb, nb, n_off, n_cols);
+      const int half = n_cols / 2;
+      const CUtensorMap* tb = half == 128 ? &tmB : &tmB64;
+      for (int kb = 0; kb < p.KB; ++kb) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty))) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * static_cast<uint32_t>(L::kA + half * BK));
           const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
           tma_load_2d_pair(sA + stage * L::kA, &tmA, bar0, kb * BK, mb * 256 + static_cast<int>(rank) * 128, pol);
           tma_load_2d_pair(sB + stage * L::kB, tb, bar0, kb * BK, nb * 256 + n_off + static_cast<int>(rank) * half,
                            pol);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-      }
-      griddep_launch_dependents();
-      for (int i = 0; ok && i < STAGES; ++i) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) break;
+        __syncwarp();
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
     }
+    if (elect_one()) griddep_launch_dependents();
+    __syncwarp();
+    for (int i = 0; ok && i < STAGES; ++i) {
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty))) break;
+      if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+    }
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(256, 128);
+    // The leader's whole warp runs the loop; one elected lane issues the MMAs
+    // and commits (always the same lane: a commit tracks that thread's MMAs).
+    if (rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t slot_count = 0;
@@ -669,27 +676,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
       for (int it = 0; ok && it < nitems; ++it) {
         int mb, nb, n_off, n_cols;
         coords(it, mb, nb, n_off, n_cols);
-        const int nj = n_cols / 128;                            // 2 for a whole tile, 1 for a tail half
+        const uint32_t idesc = idesc_e4m3_f32(256, n_cols);
         for (int kb = 0; ok && kb < p.KB; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) { ok = false; break; }
+          const int slot = static_cast<int>(slot_count & (kSlots - 1));
+          const uint32_t sphase = (slot_count / kSlots) & 1u;
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) ||
+              !__all_sync(0xFFFFFFFFu,
+                          mbar_wait_cluster(&tempty[slot], sphase ^ 1u, abort_flag, kErrWaitTmemEmpty))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * L::kA);
           const uint32_t b0 = smem_u32(sB + stage * L::kB);
-          for (int j = 0; j < nj; ++j) {
-            const int slot = static_cast<int>(slot_count & (kSlots - 1));
-            const uint32_t sphase = (slot_count / kSlots) & 1u;
-            if (!mbar_wait_cluster(&tempty[slot], sphase ^ 1u, abort_flag, kErrWaitTmemEmpty)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t d = tmem_base + slot * 128;
+          const uint32_t d = tmem_base + slot * 256;
+          if (elect_one()) {
 #pragma unroll
             for (int k = 0; k < BK / UMMA_K; ++k)
-              mma_e4m3_pair(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + j * 64 * BK + k * UMMA_K),
-                            idesc, k != 0);
+              mma_e4m3_pair(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + k * UMMA_K), idesc, k != 0);
             mma_commit_pair(&tfull[slot], kBoth);
-            ++slot_count;
+            mma_commit_pair(&empty[stage], kBoth);
           }
-          if (!ok) break;
-          mma_commit_pair(&empty[stage], kBoth);
+          __syncwarp();
+          ++slot_count;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -697,15 +706,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
   } else if (warp >= 4) {
     regs_grow<kBlock2EpiRegs>();
     // 8 epilogue warps: warp w reads TMEM lanes 32*(w%4)..+31 (its 32 rows)
-    // and columns [64 h, 64 h + 64) of every slot, h = (w - 4) / 4: for a
-    // whole tile, 64 columns of weight block h; for a tail half, columns
-    // [64 h, +64) of its single weight block.  acc[j][c] holds columns
-    // [32 c, +32) of that part for MMA j.
-    // The slot halves of a tile are read as one stream of 32-column loads,
-    // each issued before the previous one is folded in, so the TMEM load
-    // latency overlaps the FMAs; a slot is handed back as soon as both of its
-    // halves are in registers.  The scale products are fetched two K blocks
-    // ahead.
+    // and columns [h hb, h hb + hb) of every slot, h = (w - 4) / 4, hb = half
+    // the item's columns (128, or 64 for a tail half): one weight block's
+    // part.  acc[c] holds its columns [32 c, +32).
+    // The slots are read as one stream of 32-column loads, each issued before
+    // the previous one is folded in, so the TMEM load latency overlaps the
+    // FMAs; a slot is handed back once all of its chunks are in registers.
+    // The scale products are fetched two K blocks ahead.
     const int ew = warp - 4;
     const int quarter = warp & 3;
     const int h = ew >> 2;
@@ -724,9 +731,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
       tc_fence_after();
       return done;
     };
-    auto load = [&](uint32_t u, int c, uint32_t (&r)[32]) {
+    auto load = [&](uint32_t u, int col, uint32_t (&r)[32]) {
       __syncwarp();
-      tmem_ld_32x32b_x32(tmem_base + lane_addr + (u & (kSlots - 1)) * 128 + h * 64 + c * 32, r);
+      tmem_ld_32x32b_x32(tmem_base + lane_addr + (u & (kSlots - 1)) * 256 + col, r);
     };
     auto release = [&](uint32_t u) {
       tc_fence_before();
@@ -742,35 +749,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
     for (int it = 0; ok && it < nitems; ++it) {
       int mb, nb, n_off, n_cols;
       coords(it, mb, nb, n_off, n_cols);
-      const int nj = n_cols / 128;
-      const int hb = n_cols / 2;                                // B rows per CTA: 128 or 64
-      const int n_first = nb * 256 + n_off + h * hb;            // first column of this warp's part
+      const int hb = n_cols / 2;                                // columns of this warp: 128 or 64
+      const int col_base = h * hb;                              // first accumulator column of this warp
+      const int n_first = nb * 256 + n_off + col_base;          // its first output column
       const int blk = n_first / 128;
       const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quarter * 32;
       const int m = row0 + lane;
       const bool live = m < p.M && blk < NB;
       const float* xsrow = p.xs + static_cast<int64_t>(live ? m : 0) * p.KB;
       const float* wsrow = p.ws + static_cast<int64_t>(live ? blk : 0) * p.KB;
-      uint64_t acc[2][2][16];
+      uint64_t acc[4][16];
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
+      for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) acc[j][c][i] = 0ull;
+        for (int i = 0; i < 16; ++i) acc[c][i] = 0ull;
       float xa = live ? __ldg(xsrow) : 0.0f, wa = live ? __ldg(wsrow) : 0.0f;
       float xb = live && p.KB > 1 ? __ldg(xsrow + 1) : 0.0f, wb = live && p.KB > 1 ? __ldg(wsrow + 1) : 0.0f;
 
       uint32_t ra[32], rb[32];
-      uint32_t u = slot_count;                                  // first slot of the current K block
+      uint32_t u = slot_count;                                  // slot of the current K block
       if (!wait_full(u)) { ok = false; break; }
-      load(u, 0, ra);
+      load(u, col_base, ra);
       tmem_ld_wait_regs(ra);
-      // One K block: the half-slots s = 2 j + c, s < 2 NJ, alternating between
-      // ra (even s) and rb (odd s); the load after the last one is the first
-      // half of the next K block, into ra again.
-      auto kblock = [&](auto NJc, int kb) {
-        constexpr int NJ = decltype(NJc)::value;
+      // One K block: chunks c < NC alternate between ra (even c) and rb (odd
+      // c); the load after the last one is the next K block's chunk 0, into
+      // ra again (NC is even).
+      auto kblock = [&](auto NCc, int kb) {
+        constexpr int NC = decltype(NCc)::value;
         const uint64_t f2 = f32x2_pack(xa * wa, xa * wa);
         xa = xb;
         wa = wb;
@@ -779,62 +784,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
           wb = __ldg(wsrow + kb + 2);
         }
 #pragma unroll
-        for (int s2 = 0; s2 < 2 * NJ; ++s2) {
-          const int j = s2 >> 1, c = s2 & 1;
-          const bool last = s2 + 1 == 2 * NJ;
+        for (int c = 0; c < NC; ++c) {
+          const bool last = c + 1 == NC;
           const bool has_next = !last || kb + 1 < p.KB;
-          const uint32_t u_next = last ? u + NJ : u + ((s2 + 1) >> 1);
-          const int c_next = last ? 0 : ((s2 + 1) & 1);
-          uint32_t (&cur)[32] = (s2 & 1) ? rb : ra;
-          uint32_t (&nxt)[32] = (s2 & 1) ? ra : rb;
+          uint32_t (&cur)[32] = (c & 1) ? rb : ra;
+          uint32_t (&nxt)[32] = (c & 1) ? ra : rb;
           if (has_next && ok) {
-            if (c_next == 0 && !wait_full(u_next)) ok = false;
-            if (ok) load(u_next, c_next, nxt);
+            if (last && !wait_full(u + 1)) ok = false;
+            if (ok) load(last ? u + 1 : u, col_base + (last ? 0 : (c + 1) * 32), nxt);
           }
-          fold(cur, acc[j][c], f2);
-          if (has_next && ok) {
-            tmem_ld_wait_regs(nxt);
-            if (c_next == 1) release(u_next);                   // both halves of slot u + j are in registers
-          }
+          fold(cur, acc[c], f2);
+          if (has_next && ok) tmem_ld_wait_regs(nxt);
+          if (c + 2 == NC && ok) release(u);                    // the slot's last chunk is now in registers
         }
-        u += NJ;
+        ++u;
       };
-      if (nj == 2) {
-        for (int kb = 0; ok && kb < p.KB; ++kb) kblock(std::integral_constant<int, 2>(), kb);
+      if (hb == 128) {
+        for (int kb = 0; ok && kb < p.KB; ++kb) kblock(std::integral_constant<int, 4>(), kb);
       } else {
-        for (int kb = 0; ok && kb < p.KB; ++kb) kblock(std::integral_constant<int, 1>(), kb);
+        for (int kb = 0; ok && kb < p.KB; ++kb) kblock(std::integral_constant<int, 2>(), kb);
       }
       slot_count = u;
       if (!ok) break;
-      // Round to bf16 and store: columns [64 j + 32 c, +32) of this warp's part.
+      // Round to bf16 and store: columns [32 c, +32) of this warp's part.
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      for (int c = 0; c < 4; ++c) {
+        if (c * 32 < hb) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          if (j < nj) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float lo, hi;
-              f32x2_unpack(acc[j][c][i], lo, hi);
-              pk[i] = pack_bf16x2(lo, hi);
-            }
-            if (lane == 0) bulk_wait_read<1>();   // the staging tile written two chunks ago has been read
-            __syncwarp();
-            uint8_t* sb = out_s + buf * L::kOutChunk;
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              *reinterpret_cast<uint4*>(sb + lane * 64 + ((q ^ swz) << 4)) =
-                  make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            const int col0 = n_first + 64 * j + 32 * c;
-            if (lane == 0 && row0 < p.M && col0 < p.N) {
-              tma_store_2d(&tmY, sb, col0, row0);
-              bulk_commit();
-            }
-            buf ^= 1;
+          for (int i = 0; i < 16; ++i) {
+            float lo, hi;
+            f32x2_unpack(acc[c][i], lo, hi);
+            pk[i] = pack_bf16x2(lo, hi);
           }
+          if (lane == 0) bulk_wait_read<1>();     // the staging tile written two chunks ago has been read
+          __syncwarp();
+          uint8_t* sb = out_s + buf * L::kOutChunk;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(sb + lane * 64 + ((q ^ swz) << 4)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          const int col0 = n_first + 32 * c;
+          if (lane == 0 && row0 < p.M && col0 < p.N) {
+            tma_store_2d(&tmY, sb, col0, row0);
+            bulk_commit();
+          }
+          buf ^= 1;
         }
       }
     }

@@ -38,6 +38,20 @@ __device__ __forceinline__ uint64_t globaltimer() {
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 
+// True in exactly one lane of a converged warp.  Single-thread instructions
+// (tcgen05.mma, tcgen05.commit, TMA issue) are issued under it while the whole
+// warp runs the loop around them, so that descriptors, coordinates and loop
+// state stay warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xFFFFFFFF;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(p));
+  return p != 0;
+}
+
 // ------------------------------------------------------------- mbarrier ---
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -73,13 +87,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of a phase (no suspension): the cheap first check for
+// waits that are usually already satisfied.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with parity `parity` of `bar` has completed.  Gives up
 // (returns false) when `*abort` becomes nonzero or after kWaitLimitNs, in
 // which case it records `site` in the device error word and raises *abort so
 // that the other roles of the CTA stop too.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int site) {
   const uint32_t b = smem_u32(bar);
-  if (mbar_try_wait(b, parity)) return true;
+  if (mbar_test_wait(b, parity)) return true;
   const uint64_t t0 = globaltimer();
   uint32_t it = 0;
   while (!mbar_try_wait(b, parity)) {
@@ -147,7 +186,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 // mbar_wait for barriers that other CTAs of the cluster arrive on.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort, int site) {
   const uint32_t b = smem_u32(bar);
-  if (mbar_try_wait_cluster(b, parity)) return true;
+  if (mbar_test_wait_cluster(b, parity)) return true;
   const uint64_t t0 = globaltimer();
   uint32_t it = 0;
   while (!mbar_try_wait_cluster(b, parity)) {

@@ -709,9 +709,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
     // and columns [h hb, h hb + hb) of every slot, h = (w - 4) / 4, hb = half
     // the item's columns (128, or 64 for a tail half): one weight block's
     // part.  acc[c] holds its columns [32 c, +32).
-    // The slots are read as one stream of 32-column loads, each issued before
-    // the previous one is folded in, so the TMEM load latency overlaps the
-    // FMAs; a slot is handed back once all of its chunks are in registers.
+    // Each slot is read in 64-column loads (few, large loads: the per-load
+    // cost of tcgen05.ld dominates smaller ones); a slot is handed back once
+    // all of its columns are in registers.
     // The scale products are fetched two K blocks ahead.
     const int ew = warp - 4;
     const int quarter = warp & 3;
@@ -731,19 +731,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
       tc_fence_after();
       return done;
     };
-    auto load = [&](uint32_t u, int col, uint32_t (&r)[32]) {
-      __syncwarp();
-      tmem_ld_32x32b_x32(tmem_base + lane_addr + (u & (kSlots - 1)) * 256 + col, r);
-    };
     auto release = [&](uint32_t u) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + (u & (kSlots - 1)) * 8);
-    };
-    auto fold = [&](const uint32_t (&r)[32], uint64_t (&a)[16], uint64_t f2) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        a[i] = fma_f32x2(f32x2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), f2, a[i]);
     };
 
     for (int it = 0; ok && it < nitems; ++it) {
@@ -766,16 +757,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
       float xa = live ? __ldg(xsrow) : 0.0f, wa = live ? __ldg(wsrow) : 0.0f;
       float xb = live && p.KB > 1 ? __ldg(xsrow + 1) : 0.0f, wb = live && p.KB > 1 ? __ldg(wsrow + 1) : 0.0f;
 
-      uint32_t ra[32], rb[32];
+      uint32_t r[64];
       uint32_t u = slot_count;                                  // slot of the current K block
-      if (!wait_full(u)) { ok = false; break; }
-      load(u, col_base, ra);
-      tmem_ld_wait_regs(ra);
-      // One K block: chunks c < NC alternate between ra (even c) and rb (odd
-      // c); the load after the last one is the next K block's chunk 0, into
-      // ra again (NC is even).
-      auto kblock = [&](auto NCc, int kb) {
-        constexpr int NC = decltype(NCc)::value;
+      const int nh = hb / 64;                                   // 64-column loads: 2, or 1 for a tail half
+      // Per K block: nh loads of 64 columns, each waited for and folded in;
+      // the slot is handed back after its last load.
+      for (int kb = 0; kb < p.KB; ++kb) {
         const uint64_t f2 = f32x2_pack(xa * wa, xa * wa);
         xa = xb;
         wa = wb;
@@ -783,26 +770,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
           xb = __ldg(xsrow + kb + 2);
           wb = __ldg(wsrow + kb + 2);
         }
+        if (!wait_full(u)) {
+          ok = false;
+          break;
+        }
 #pragma unroll
-        for (int c = 0; c < NC; ++c) {
-          const bool last = c + 1 == NC;
-          const bool has_next = !last || kb + 1 < p.KB;
-          uint32_t (&cur)[32] = (c & 1) ? rb : ra;
-          uint32_t (&nxt)[32] = (c & 1) ? ra : rb;
-          if (has_next && ok) {
-            if (last && !wait_full(u + 1)) ok = false;
-            if (ok) load(last ? u + 1 : u, col_base + (last ? 0 : (c + 1) * 32), nxt);
+        for (int c = 0; c < 2; ++c) {
+          if (c < nh) {
+            __syncwarp();
+            tmem_ld_32x32b_x64(tmem_base + lane_addr + (u & (kSlots - 1)) * 256 + col_base + c * 64, r);
+            tmem_ld_wait_regs64(r);
+            if (c + 1 == nh) release(u);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              acc[2 * c + (i >> 4)][i & 15] =
+                  fma_f32x2(f32x2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), f2,
+                            acc[2 * c + (i >> 4)][i & 15]);
           }
-          fold(cur, acc[c], f2);
-          if (has_next && ok) tmem_ld_wait_regs(nxt);
-          if (c + 2 == NC && ok) release(u);                    // the slot's last chunk is now in registers
         }
         ++u;
-      };
-      if (hb == 128) {
-        for (int kb = 0; ok && kb < p.KB; ++kb) kblock(std::integral_constant<int, 4>(), kb);
-      } else {
-        for (int kb = 0; ok && kb < p.KB; ++kb) kblock(std::integral_constant<int, 2>(), kb);
       }
       slot_count = u;
       if (!ok) break;

@@ -709,9 +709,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
     // and columns [h hb, h hb + hb) of every slot, h = (w - 4) / 4, hb = half
     // the item's columns (128, or 64 for a tail half): one weight block's
     // part.  acc[c] holds its columns [32 c, +32).
-    // Each slot is read in 64-column loads (few, large loads: the per-load
-    // cost of tcgen05.ld dominates smaller ones); a slot is handed back once
-    // all of its columns are in registers.
+    // Each slot is read 64 columns at a time as four 16-column loads in
+    // flight; a slot is handed back once all of its columns are in registers.
     // The scale products are fetched two K blocks ahead.
     const int ew = warp - 4;
     const int quarter = warp & 3;
@@ -778,7 +777,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
         for (int c = 0; c < 2; ++c) {
           if (c < nh) {
             __syncwarp();
-            tmem_ld_32x32b_x64(tmem_base + lane_addr + (u & (kSlots - 1)) * 256 + col_base + c * 64, r);
+            tmem_ld_32x32b_x16x4(tmem_base + lane_addr + (u & (kSlots - 1)) * 256 + col_base + c * 64, r);
             tmem_ld_wait_regs64(r);
             if (c + 1 == nh) release(u);
 #pragma unroll

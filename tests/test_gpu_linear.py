@@ -129,6 +129,32 @@ def test_decode_output_stride():
     check_full(3, 512, 512, fq.CHANNEL_TOKEN, ldy_pad=32)
 
 
+@pytest.mark.parametrize("M,N,K,mode", [
+    (1, 128, 65536, fq.CHANNEL_TOKEN),   # one weight tile, 512 K blocks over every SM: ~148 segments to add
+    (3, 256, 8192, fq.CHANNEL_TOKEN),    # 128 steps < SMs: one step per CTA, 64 segments per tile
+    (2, 128, 32768, fq.BLOCK128),        # block mode, one tile split over every SM
+])
+def test_decode_many_segments_per_tile(M, N, K, mode):
+    check_full(M, N, K, mode, seed=K)
+
+
+def test_decode_workspace_reused_across_shapes():
+    # One scratch buffer serves calls of different shapes and modes in a row
+    # (its contents are scratch: nothing carries over between calls).
+    size = max(fq.fp8_linear_workspace_size(M, N, K, mode)
+               for M, N, K, mode in [(1, 4096, 4096, 0), (16, 1024, 2048, 1), (64, 512, 8192, 0)])
+    wsp = torch.full((size,), 0xA5, dtype=torch.uint8, device=DEV)
+    for M, N, K, mode in [(1, 4096, 4096, 0), (16, 1024, 2048, 1), (64, 512, 8192, 0), (1, 4096, 4096, 0)]:
+        x = synth.make_x(M, K, seed=N)
+        w = synth.make_w(N, K, seed=N)
+        wq, ws = fq.fp8_quant_weight(w.to(DEV), mode)
+        xq, xs = fq.fp8_quant_act(x.to(DEV), mode)
+        y = fq.fp8_linear(xq, xs, wq, ws, mode, workspace=wsp).float().cpu().numpy()
+        rxq, rxs = oracle.quant_act(x, mode)
+        rwq, rws = oracle.quant_weight(w, mode)
+        P.assert_y_close(y, oracle.linear(rxq, rxs, rwq, rws, mode), what=f"reused workspace {M}x{N}x{K} m{mode}")
+
+
 def test_zero_activations_give_zero():
     x = torch.zeros(70, 256, dtype=torch.bfloat16)
     w = synth.make_w(128, 256)

@@ -315,7 +315,7 @@ def aggregate(units_local: float, seconds_local: float, world: int):
 
 
 def launches_of(g) -> int:
-    return 2 if g.M <= 64 else 1          # decode: GEMM + reduction kernel
+    return 1                              # one kernel per GEMM (decode reduces inside its kernel)
 
 
 def run_gpu(args):
@@ -345,7 +345,7 @@ def run_gpu(args):
               torch.empty(fq.scale_shape_act(M, K, mode), dtype=torch.float32, device=dev))
           for k, (M, K, mode) in xs_shapes.items()}
     Y = {g.name: torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev) for g in wl.gemms}
-    WS = {g.name: (torch.empty(fq.fp8_linear_workspace_size(g.M, g.N, g.K, g.mode), dtype=torch.uint8,
+    WS = {g.name: (torch.zeros(fq.fp8_linear_workspace_size(g.M, g.N, g.K, g.mode), dtype=torch.uint8,
                                device=dev) if g.M <= 64 else None) for g in wl.gemms}
     flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -471,7 +471,7 @@ def run_gpu(args):
             M, K, Nm = gs[0].M, gs[0].K, sum(g.N for g in gs)
             y_m = torch.empty((M, Nm), dtype=torch.bfloat16, device=dev)
             nws = fq.fp8_linear_workspace_size(M, Nm, K, mode)
-            ws_buf = torch.empty(nws, dtype=torch.uint8, device=dev) if nws else None
+            ws_buf = torch.zeros(nws, dtype=torch.uint8, device=dev) if nws else None
             mops.append(lambda xk=xk, mode=mode, wq_m=wq_m, ws_m=ws_m, y_m=y_m, ws_buf=ws_buf:
                         fq.fp8_linear(XQ[xk][0], XQ[xk][1], wq_m, ws_m, mode, out=y_m, workspace=ws_buf))
             mnames.append("+".join(g.name for g in gs) + f":{M}x{K}->{Nm}")
@@ -506,7 +506,7 @@ def run_gpu(args):
                        "frac_hbm": round(b / (op_ms[i] / 1e3) / 1e9 / pk["hbm_gbs"], 3)})
     for j, g in enumerate(wl.gemms):
         t = op_ms[len(xs_shapes) + j] / 1e3
-        kern = ("gemm_decode+reduce" if g.M <= 64 else
+        kern = ("gemm_decode" if g.M <= 64 else
                 ("gemm_block" if g.mode == synth.BLOCK128 else "gemm_channel"))
         detail.append({"op": g.name, "kernel": kern, "M": g.M, "N": g.N, "K": g.K, "mode": g.mode,
                        "ms": round(float(op_ms[len(xs_shapes) + j]), 5),

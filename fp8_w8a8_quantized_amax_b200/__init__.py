@@ -147,7 +147,8 @@ def fp8_linear(Xq: torch.Tensor, x_scale: torch.Tensor, Wq: torch.Tensor, w_scal
                mode: int = CHANNEL_TOKEN, out: Optional[torch.Tensor] = None,
                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Y bf16 [M, N] = dequant(Xq) . dequant(Wq)^T.  Workspace (small-M path) is
-    taken from torch's caching allocator unless given."""
+    taken from torch's caching allocator, zero-filled, unless given; a given one
+    must have been zero-filled before its first use (every call leaves it all zero)."""
     _require_cuda(Xq, "Xq", torch.uint8)
     _require_cuda(Wq, "Wq", torch.uint8)
     M, K = Xq.shape
@@ -160,7 +161,7 @@ def fp8_linear(Xq: torch.Tensor, x_scale: torch.Tensor, Wq: torch.Tensor, w_scal
         out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
     need = fp8_linear_workspace_size(M, N, K, mode)
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=Xq.device)
+        workspace = torch.zeros(need, dtype=torch.uint8, device=Xq.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().fp8_linear(_ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), M, N, K, int(mode),
                           _ptr(out), out.stride(0), _ptr(workspace), wbytes, _stream(Xq))

@@ -214,8 +214,19 @@ void decode_shape(int64_t M, int64_t N, int64_t K, int sms, int* n_tiles, int64_
   *nx = decode_nx(M);
 }
 
+// Decode workspace: [n_tiles][4] arrival counters, padded to 16 bytes, then
+// [(n_tiles + G - 1)][nx][128] fp32 partial sums.  All zero between calls.
+size_t decode_counter_bytes(int n_tiles) { return (static_cast<size_t>(n_tiles) * 4 * sizeof(unsigned) + 15) & ~size_t(15); }
+
 size_t decode_workspace_bytes(int n_tiles, int G, int nx) {
-  return static_cast<size_t>(n_tiles + G - 1) * nx * 128 * sizeof(float);
+  return decode_counter_bytes(n_tiles) + static_cast<size_t>(n_tiles + G - 1) * nx * 128 * sizeof(float);
+}
+
+void decode_bind_workspace(Params& p, void* ws, void* Y, int64_t ldy) {
+  p.count = static_cast<unsigned*>(ws);
+  p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + decode_counter_bytes(p.n_tiles));
+  p.y = static_cast<__nv_bfloat16*>(Y);
+  p.ldy = ldy;
 }
 
 fp8q_status check_linear_args(const uint8_t* Xq, const float* xs, const uint8_t* Wq, const float* ws, int64_t M,
@@ -233,24 +244,36 @@ fp8q_status check_linear_args(const uint8_t* Xq, const float* xs, const uint8_t*
   return FP8Q_OK;
 }
 
+// Whether the decode kernel sums split weight tiles itself (else a reduction
+// kernel follows it).  Measured on the Llama-3.1-70B and -3.2-3B decode shapes:
+// in channel mode with up to 16 tokens the in-kernel sums are cheap enough to
+// win everywhere; with 32 or 64 tokens only when every CTA streams at least a
+// tile's worth of steps after them; in block mode the per-K-block epilogue
+// leaves no room, and the separate kernel is faster.
+bool decode_fused(const Params& p, int mode, int nx) {
+  if (mode == FP8Q_BLOCK128) return false;
+  return nx == 16 || p.total >= static_cast<int64_t>(p.KB) * p.G;
+}
+
 template <int NX>
 fp8q_status launch_decode_nx(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p, int mode, int dev,
-                             void* Y, int64_t ldy, void* stream) {
+                             void* stream) {
   constexpr int kDecodeStages = decode_stages<NX>();
   using L = fp8q::decode::Layout<NX, kDecodeStages>;
   fp8q_status st;
-  if (mode == FP8Q_BLOCK128) {
-    auto k = fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, true>;
+  const bool block = mode == FP8Q_BLOCK128;
+  if (decode_fused(p, mode, NX)) {
+    auto k = block ? fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, true, true>
+                   : fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, false, true>;
     if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
-    if ((st = launch(k, dim3(p.G), dim3(192), L::kBytes, stream, tw, tx, p)) != FP8Q_OK) return st;
-    return launch(fp8q::decode::decode_reduce_kernel<true>, dim3(p.n_tiles, p.M), dim3(128), 0, stream, p, NX,
-                  static_cast<__nv_bfloat16*>(Y), ldy);
+    return launch(k, dim3(p.G), dim3(192), L::kBytes, stream, tw, tx, p);
   }
-  auto k = fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, false>;
+  auto k = block ? fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, true, false>
+                 : fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, false, false>;
   if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
   if ((st = launch(k, dim3(p.G), dim3(192), L::kBytes, stream, tw, tx, p)) != FP8Q_OK) return st;
-  return launch(fp8q::decode::decode_reduce_kernel<false>, dim3(p.n_tiles, p.M), dim3(128), 0, stream, p, NX,
-                static_cast<__nv_bfloat16*>(Y), ldy);
+  auto r = block ? fp8q::decode::decode_reduce_kernel<true> : fp8q::decode::decode_reduce_kernel<false>;
+  return launch(r, dim3(p.n_tiles, p.M), dim3(128), 0, stream, p, NX);
 }
 
 }  // namespace
@@ -320,7 +343,6 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     Params p;
     p.xs = x_scale;
     p.ws = w_scale;
-    p.part = static_cast<float*>(workspace);
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(N);
     p.K = static_cast<int>(K);
@@ -328,9 +350,10 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     p.n_tiles = n_tiles;
     p.total = total;
     p.G = G;
-    if (nx == 16) return launch_decode_nx<16>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
-    if (nx == 32) return launch_decode_nx<32>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
-    return launch_decode_nx<64>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
+    decode_bind_workspace(p, workspace, Y_bf16, ldy);
+    if (nx == 16) return launch_decode_nx<16>(tw, tx, p, mode, dev, stream);
+    if (nx == 32) return launch_decode_nx<32>(tw, tx, p, mode, dev, stream);
+    return launch_decode_nx<64>(tw, tx, p, mode, dev, stream);
   }
 
   const bool pair = prefill_choice() != 1 && (M >= 256 || prefill_choice() == 2);
@@ -507,7 +530,6 @@ fp8q_status fp8_linear_noalloc(const uint8_t* Xq, const float* x_scale, const ui
   Params p;
   p.xs = x_scale;
   p.ws = w_scale;
-  p.part = static_cast<float*>(scratch);
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
@@ -515,9 +537,10 @@ fp8q_status fp8_linear_noalloc(const uint8_t* Xq, const float* x_scale, const ui
   p.n_tiles = n_tiles;
   p.total = total;
   p.G = G;
-  if (nx == 16) return launch_decode_nx<16>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
-  if (nx == 32) return launch_decode_nx<32>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
-  return launch_decode_nx<64>(tw, tx, p, mode, dev, Y_bf16, ldy, stream);
+  decode_bind_workspace(p, scratch, Y_bf16, ldy);
+  if (nx == 16) return launch_decode_nx<16>(tw, tx, p, mode, dev, stream);
+  if (nx == 32) return launch_decode_nx<32>(tw, tx, p, mode, dev, stream);
+  return launch_decode_nx<64>(tw, tx, p, mode, dev, stream);
 }
 
 }  // extern "C"

@@ -7,14 +7,25 @@
 //
 // Stream-K: the (weight tile t, K block kb) pairs, t-major, form one list of
 // T = n_tiles * KB steps that is cut into G equal contiguous ranges, one per
-// CTA (G <= #SMs, every range non-empty).  A CTA walks its range; each run of
-// steps inside one weight tile is a "segment", whose fp32 partial
-// D[n, m] (already multiplied by the block scales in block mode) goes to
-// workspace slot (t + c) -- slots are unique because a CTA's tiles increase
-// with c.  The reduction kernel adds the segments of each tile in CTA order
-// (deterministic), applies the channel scales in channel mode, and writes
-// bf16.  Partial traffic is (n_tiles + G) * NX * 512 bytes, small next to the
-// N * K weight bytes.
+// CTA (G <= #SMs, every range non-empty).  Each run of a CTA's steps inside
+// one weight tile is a "segment".  A segment that is a whole tile is scaled
+// and written as bf16 at once.  A partial segment's fp32 sums D[n, m]
+// (already multiplied by the block scales in block mode) go to workspace
+// slot (t + c) -- unique because a CTA's tiles increase with c -- and each
+// epilogue warp counts its 32 channels in with an atomic on a per-(tile,
+// warp) counter.  The warp that arrives last adds the tile's segments for its
+// channels in CTA order (deterministic: the same sum whichever CTA finishes
+// last), applies the channel scales in channel mode, writes bf16, and sets
+// the counter and the partial sums it read back to zero: the workspace is all
+// zero between calls, whatever their shapes.  Nothing waits on another CTA.
+// A CTA takes its steps in the order: the partial segment at the end of its
+// range (the start of a tile it shares with the next CTA), the segment at the
+// start of its range, then the whole tiles between them, so that the
+// reductions happen under the rest of the weight stream.  Where that does
+// not pay (FUSED = false; the host decides per shape) the partial segments
+// are summed by decode_reduce_kernel after the GEMM kernel, which clears them
+// likewise.  Partial traffic is at most (n_tiles + G) * NX * 512 bytes, small
+// next to the N * K weight bytes.
 //
 // Roles: warp 0 TMA (W tile 128 x 128 B evict-first + X tile NX x 128 B),
 // warp 1 TMEM allocation + MMA issue, warps 2..5 drain TMEM and write
@@ -36,11 +47,14 @@ constexpr int kSlots = 4;
 struct Params {
   const float* xs;
   const float* ws;
-  float* part;        // workspace: [(n_tiles + G - 1)][NX][128] fp32
+  unsigned int* count;  // workspace: [n_tiles][4] arrival counters
+  float* part;          // workspace: [(n_tiles + G - 1)][NX][128] fp32 partial sums
+  __nv_bfloat16* y;
+  int64_t ldy;
   int M, N, K, KB;
   int n_tiles;
-  int64_t total;      // n_tiles * KB
-  int G;              // CTAs
+  int64_t total;        // n_tiles * KB
+  int G;                // CTAs
 };
 
 __host__ __device__ __forceinline__ int64_t range_begin(int64_t c, int64_t total, int64_t G) {
@@ -51,6 +65,48 @@ __host__ __device__ __forceinline__ int64_t range_begin(int64_t c, int64_t total
 __host__ __device__ __forceinline__ int cta_of_step(int64_t x, int64_t total, int64_t G) {
   return static_cast<int>(((x + 1) * G - 1) / total);
 }
+
+// Walks the steps [b, e) of a CTA's range in the order: the partial segment
+// that ends the range ([last_begin, e), empty when e ends a tile), then the
+// segment that starts it ([b, first_end)), then the whole tiles between them
+// ([first_end, last_begin)).  The tile t and K block kb are kept
+// incrementally: 64-bit divisions only where a run starts.
+struct StepIter {
+  int64_t first_end, last_begin, b0, e0;
+  int64_t s, cur_b, cur_e;   // the current run [cur_b, cur_e)
+  int run, t, kb, KB;
+  __device__ StepIter(int64_t b, int64_t e, int kblocks) : b0(b), e0(e), KB(kblocks) {
+    first_end = min(e, (b / KB + 1) * KB);
+    last_begin = (e % KB == 0) ? e : max(first_end, ((e - 1) / KB) * KB);
+    run = -1;
+    next_run();
+  }
+  __device__ void next_run() {
+    for (;;) {
+      ++run;
+      if (run == 0) { cur_b = last_begin; cur_e = e0; }
+      else if (run == 1) { cur_b = b0; cur_e = first_end; }
+      else if (run == 2) { cur_b = first_end; cur_e = last_begin; }
+      else return;
+      if (cur_b < cur_e) break;
+    }
+    s = cur_b;
+    t = static_cast<int>(s / KB);
+    kb = static_cast<int>(s - static_cast<int64_t>(t) * KB);
+  }
+  __device__ bool valid() const { return run < 3; }
+  // Whether this step starts / ends a segment (a run of steps in one tile).
+  __device__ bool seg_first() const { return s == cur_b || kb == 0; }
+  __device__ bool seg_last() const { return s + 1 == cur_e || kb + 1 == KB; }
+  __device__ void next() {
+    if (++s == cur_e) {
+      next_run();
+    } else if (++kb == KB) {
+      kb = 0;
+      ++t;
+    }
+  }
+};
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -68,7 +124,7 @@ struct Layout {
   static constexpr uint32_t kTmemCols = (kSlots * NX) < 32 ? 32 : (kSlots * NX);
 };
 
-template <int NX, int STAGES, bool BLOCK>
+template <int NX, int STAGES, bool BLOCK, bool FUSED>
 __global__ void __launch_bounds__(192, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const Params p) {
@@ -122,9 +178,8 @@ __global__ void __launch_bounds__(192, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int64_t s = b; s < e; ++s) {
-        const int t = static_cast<int>(s / p.KB);
-        const int kb = static_cast<int>(s - static_cast<int64_t>(t) * p.KB);
+      for (StepIter it(b, e, p.KB); it.valid(); it.next()) {
+        const int t = it.t, kb = it.kb;
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) { ok = false; break; }
         mbar_arrive_expect_tx(&full[stage], L::kW + L::kX);
         tma_load_2d(sW + stage * L::kW, &tmW, &full[stage], kb * BK, t * 128, pol_w);
@@ -142,10 +197,9 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t idesc = idesc_e4m3_f32(128, NX);
       int stage = 0, slot = 0;
       uint32_t phase = 0, sphase = 0;
-      for (int64_t s = b; s < e; ++s) {
-        const int64_t t = s / p.KB;
-        const bool seg_first = (s == b) || (s - t * p.KB == 0);
-        const bool seg_last = (s + 1 == e) || (s + 1 - t * p.KB == p.KB);
+      for (StepIter it(b, e, p.KB); it.valid(); it.next()) {
+        const bool seg_first = it.seg_first();
+        const bool seg_last = it.seg_last();
         // Block mode: one TMEM slot per K block (its scales differ).  Channel
         // mode: one slot per segment, accumulated across its K blocks.
         const bool open_slot = BLOCK || seg_first;
@@ -171,6 +225,13 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     const int quarter = warp & 3;
     const int nl = quarter * 32 + lane;          // output channel within the tile
+    // Channel mode: this warp's copy of x_scale in shared memory, read by the
+    // output loop (global loads there would queue behind the output stores).
+    __shared__ float s_xs[4][NX];
+    if constexpr (!BLOCK) {
+      for (int j = lane; j < NX; j += 32) s_xs[quarter][j] = j < p.M ? __ldg(p.xs + j) : 0.0f;
+      __syncwarp();
+    }
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     float acc[NX];
 #pragma unroll
@@ -182,20 +243,20 @@ __global__ void __launch_bounds__(192, 1)
     constexpr bool kPrefetch = BLOCK && NX <= 32;
     float fx[kPrefetch ? NX : 1];
     float fw = 0.0f;
-    auto fetch = [&](int64_t s) {
+    auto fetch = [&](int t, int kb) {
       if constexpr (kPrefetch) {
-        const int t = static_cast<int>(s / p.KB);
-        const int kb = static_cast<int>(s - static_cast<int64_t>(t) * p.KB);
         fw = __ldg(p.ws + static_cast<int64_t>(t) * p.KB + kb);
 #pragma unroll
         for (int j = 0; j < NX; ++j) fx[j] = j < p.M ? __ldg(p.xs + static_cast<int64_t>(j) * p.KB + kb) : 0.0f;
       }
     };
-    if (b < e) fetch(b);
-    for (int64_t s = b; s < e; ++s) {
-      const int t = static_cast<int>(s / p.KB);
-      const int kb = static_cast<int>(s - static_cast<int64_t>(t) * p.KB);
-      const bool seg_last = (s + 1 == e) || (kb + 1 == p.KB);
+    StepIter it(b, e, p.KB);
+    if (it.valid()) fetch(it.t, it.kb);
+    int seg_len = 0;
+    for (; it.valid(); it.next()) {
+      const int t = it.t, kb = it.kb;
+      seg_len = it.seg_first() ? 1 : seg_len + 1;
+      const bool seg_last = it.seg_last();
       if (!BLOCK && !seg_last) continue;           // channel mode: one drain per segment
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sfull[slot], sphase, abort_flag, kErrWaitTmemFull))) break;
       tc_fence_after();
@@ -213,7 +274,9 @@ __global__ void __launch_bounds__(192, 1)
         float f[NX];
 #pragma unroll
         for (int j = 0; j < NX; ++j) f[j] = fx[j] * fw;
-        if (s + 1 < e) fetch(s + 1);
+        StepIter nx = it;
+        nx.next();
+        if (nx.valid()) fetch(nx.t, nx.kb);
 #pragma unroll
         for (int j = 0; j < NX; ++j) acc[j] = fmaf(__uint_as_float(r[j]), f[j], acc[j]);
       } else if constexpr (BLOCK) {
@@ -227,13 +290,64 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int j = 0; j < NX; ++j) acc[j] = __uint_as_float(r[j]);
       }
-      if (seg_last) {                              // segment ends: publish it
-        float* dst = p.part + (static_cast<int64_t>(t) + c) * NX * 128 + nl;
+      if (seg_last) {                              // segment ends
+        const int64_t tile_first = static_cast<int64_t>(t) * p.KB;
+        const int n = t * 128 + nl;
+        // bf16 output of channel n for the token sums v[j]
+        auto emit = [&](const float (&v)[NX]) {
+          if (n < p.N) {
+            const float wn = BLOCK ? 1.0f : __ldg(p.ws + n);
 #pragma unroll
-        for (int j = 0; j < NX; ++j) {
-          if (j < p.M) dst[j * 128] = acc[j];
-          acc[j] = 0.0f;
+            for (int j = 0; j < NX; ++j) {
+              if (j < p.M) {
+                const float o = BLOCK ? v[j] : v[j] * s_xs[quarter][j] * wn;
+                p.y[static_cast<int64_t>(j) * p.ldy + n] = __float2bfloat16_rn(o);
+              }
+            }
+          }
+        };
+        if (seg_len == p.KB) {                     // the whole tile: no partial sums
+          emit(acc);
+        } else {
+          float* dst = p.part + (static_cast<int64_t>(t) + c) * NX * 128 + nl;
+#pragma unroll
+          for (int j = 0; j < NX; ++j)
+            if (j < p.M) dst[j * 128] = acc[j];
+          if constexpr (!FUSED) {
+#pragma unroll
+            for (int j = 0; j < NX; ++j) acc[j] = 0.0f;
+            continue;                              // summed by decode_reduce_kernel
+          }
+          __threadfence();
+          __syncwarp();
+          const int c0 = cta_of_step(tile_first, p.total, p.G);
+          const int c1 = cta_of_step(tile_first + p.KB - 1, p.total, p.G);
+          unsigned int prev = 0;
+          if (lane == 0) prev = atomicAdd(p.count + t * 4 + quarter, 1u);
+          prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+          if (prev == static_cast<unsigned int>(c1 - c0)) {   // every other segment is in
+            __threadfence();
+            // acc is published; it now collects the tile's sum in CTA order
+#pragma unroll
+            for (int j = 0; j < NX; ++j) acc[j] = 0.0f;
+            for (int cc = c0; cc <= c1; ++cc) {
+              const float* src = p.part + (static_cast<int64_t>(t) + cc) * NX * 128 + nl;
+#pragma unroll
+              for (int j = 0; j < NX; ++j)
+                if (j < p.M) acc[j] += __ldcg(src + j * 128);
+            }
+            for (int cc = c0; cc <= c1; ++cc) {   // the workspace is left all zero
+              float* src = p.part + (static_cast<int64_t>(t) + cc) * NX * 128 + nl;
+#pragma unroll
+              for (int j = 0; j < NX; ++j)
+                if (j < p.M) src[j * 128] = 0.0f;
+            }
+            emit(acc);
+            if (lane == 0) p.count[t * 4 + quarter] = 0u;
+          }
         }
+#pragma unroll
+        for (int j = 0; j < NX; ++j) acc[j] = 0.0f;
       }
     }
   }
@@ -247,11 +361,12 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-// Sum the segments of every weight tile in CTA order and write bf16 output.
+// Sum the partial segments of every weight tile that more than one CTA
+// worked on, in CTA order, write bf16 output and clear the partial sums read.
 // grid (n_tiles, M), 128 threads: thread = output channel within the tile.
+// Tiles one CTA covered whole were written by the GEMM kernel.
 template <bool BLOCK>
-__global__ void __launch_bounds__(128) decode_reduce_kernel(const Params p, int nx, __nv_bfloat16* __restrict__ y,
-                                                            int64_t ldy) {
+__global__ void __launch_bounds__(128) decode_reduce_kernel(const Params p, int nx) {
   griddep_wait();
   const int t = blockIdx.x;
   const int m = blockIdx.y;
@@ -259,11 +374,13 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const Params p, int 
   const int n = t * 128 + nl;
   const int c0 = cta_of_step(static_cast<int64_t>(t) * p.KB, p.total, p.G);
   const int c1 = cta_of_step(static_cast<int64_t>(t + 1) * p.KB - 1, p.total, p.G);
+  if (c0 == c1) return;
   float sum = 0.0f;
-  for (int c = c0; c <= c1; ++c) sum += p.part[((static_cast<int64_t>(t) + c) * nx + m) * 128 + nl];
+  for (int c = c0; c <= c1; ++c) sum += __ldcg(p.part + ((static_cast<int64_t>(t) + c) * nx + m) * 128 + nl);
+  for (int c = c0; c <= c1; ++c) p.part[((static_cast<int64_t>(t) + c) * nx + m) * 128 + nl] = 0.0f;
   if (n < p.N) {
     const float v = BLOCK ? sum : sum * __ldg(p.xs + m) * __ldg(p.ws + n);
-    y[static_cast<int64_t>(m) * ldy + n] = __float2bfloat16_rn(v);
+    p.y[static_cast<int64_t>(m) * p.ldy + n] = __float2bfloat16_rn(v);
   }
 }
 

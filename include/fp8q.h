@@ -108,15 +108,21 @@ FP8Q_API fp8q_status fp8_quant_act(const void* X_bf16, int64_t M, int64_t K, int
  *   Y_bf16    [M, ldy] bf16, written.  ldy >= N, (ldy * 2) % 16 == 0, 16-byte aligned.
  *   workspace device scratch of at least fp8_linear_workspace_size(M, N, K, mode)
  *             bytes, 256-byte aligned (may be NULL when that size is 0).  It holds
- *             fp32 split-K partial sums of the small-M (decode) path; its contents
- *             need no initialisation and are garbage afterwards.  Two calls that
- *             run concurrently must not share one workspace.
+ *             the split-K arrival counters and fp32 partial sums of the small-M
+ *             (decode) path.  It must be zero-filled before its first use; every
+ *             completed call leaves it all zero again, so one zeroed buffer
+ *             serves any sequence of calls (of any shape) on one stream.  After
+ *             a call that failed on the device (fp8q_device_error nonzero), zero
+ *             it again.  Two calls that run concurrently must not share one
+ *             workspace.
  *   Requirements: M >= 0 (M == 0 is a no-op), N > 0, K > 0, K % 16 == 0,
  *   N % 16 == 0; K % 128 == 0 in block mode.  The mode must be the one both
  *   operands were quantized with.
  *   Dispatch: M <= 64 takes the decode kernel (weights streamed once, swap-AB,
- *   stream-K split over all SMs, then a reduction kernel); larger M takes the
- *   persistent warp-specialised prefill kernel (no workspace).
+ *   stream-K split over all SMs; the last warp to finish a weight tile's
+ *   channels adds its partial sums in a fixed order, so results are
+ *   deterministic); larger M takes the persistent warp-specialised prefill
+ *   kernels (no workspace).
  */
 FP8Q_API fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq,
                        const float* w_scale, int64_t M, int64_t N, int64_t K, int mode,
@@ -157,8 +163,8 @@ FP8Q_API int fp8q_device_error(int clear);
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.
  *   - Every call on a device shares the one array, which keeps whatever the last
- *     call left in it.  Nothing in it needs to start at zero: each call writes
- *     every partial sum it later reads.  Calls whose kernels overlap on the GPU
+ *     call left in it: zero-filled when the library is loaded, and every
+ *     completed call leaves it all zero again.  Calls whose kernels overlap on the GPU
  *     (different streams, or different host threads) race on the array and give
  *     wrong results; serialise them.
  */

@@ -138,12 +138,13 @@ def test_decode_many_segments_per_tile(M, N, K, mode):
     check_full(M, N, K, mode, seed=K)
 
 
-def test_decode_workspace_reused_across_shapes():
-    # One scratch buffer serves calls of different shapes and modes in a row
-    # (its contents are scratch: nothing carries over between calls).
+def test_decode_workspace_left_reusable():
+    # The workspace is all zero again after every call, so one zero-filled
+    # buffer serves calls of different shapes and modes in a row (a later call
+    # may put its arrival counters where an earlier one kept partial sums).
     size = max(fq.fp8_linear_workspace_size(M, N, K, mode)
                for M, N, K, mode in [(1, 4096, 4096, 0), (16, 1024, 2048, 1), (64, 512, 8192, 0)])
-    wsp = torch.full((size,), 0xA5, dtype=torch.uint8, device=DEV)
+    wsp = torch.zeros(size, dtype=torch.uint8, device=DEV)
     for M, N, K, mode in [(1, 4096, 4096, 0), (16, 1024, 2048, 1), (64, 512, 8192, 0), (1, 4096, 4096, 0)]:
         x = synth.make_x(M, K, seed=N)
         w = synth.make_w(N, K, seed=N)
@@ -153,6 +154,7 @@ def test_decode_workspace_reused_across_shapes():
         rxq, rxs = oracle.quant_act(x, mode)
         rwq, rws = oracle.quant_weight(w, mode)
         P.assert_y_close(y, oracle.linear(rxq, rxs, rwq, rws, mode), what=f"reused workspace {M}x{N}x{K} m{mode}")
+        assert torch.count_nonzero(wsp).item() == 0, "workspace not left zero"
 
 
 def test_zero_activations_give_zero():
@@ -265,7 +267,7 @@ def test_cuda_graph_replay_matches_eager(M, mode):
     y_eager = fq.fp8_linear(xq, xs, wq, ws, mode)
     xq2, xs2 = torch.empty_like(xq), torch.empty_like(xs)
     y2 = torch.empty_like(y_eager)
-    wsp = torch.empty(max(1, fq.fp8_linear_workspace_size(M, N, K, mode)), dtype=torch.uint8, device=DEV)
+    wsp = torch.zeros(max(1, fq.fp8_linear_workspace_size(M, N, K, mode)), dtype=torch.uint8, device=DEV)
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     g = torch.cuda.CUDAGraph()

@@ -26,6 +26,7 @@ def _built():
 
 
 @pytest.mark.parametrize("M,K", [(1, 16), (3, 48), (17, 256), (129, 384), (64, 3072), (5, 4096),
+                                 (2051, 3072), (1000, 1040), (301, 4096),
                                  (2, 14336), (3, 28672), (2, 65536 + 16), (1, 131072)])
 def test_rows_bit_exact(M, K):
     x = synth.make_x(M, K, seed=M + K)

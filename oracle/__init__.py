@@ -59,6 +59,10 @@ def lib() -> ctypes.CDLL:
         _lib.orc_linear.restype = None
         _lib.orc_linear_at.argtypes = [P, P, P, P, I, I, I, ctypes.c_int, P, P, I, P]
         _lib.orc_linear_at.restype = None
+        _lib.orc_rmsnorm_rstd.argtypes = [P, I, I, I, ctypes.c_float, P]
+        _lib.orc_rmsnorm_rstd.restype = None
+        _lib.orc_rmsnorm_quant_rows.argtypes = [P, P, P, I, I, I, P, I, P, P]
+        _lib.orc_rmsnorm_quant_rows.restype = None
     return _lib
 
 
@@ -103,6 +107,31 @@ def quant_rows(x):
     s = np.empty((R,), np.float32)
     lib().orc_quant_rows(_p(xb), R, K, K, _p(q), K, _p(s))
     return q, s
+
+
+def rmsnorm_rstd(x, eps: float = 1e-5) -> np.ndarray:
+    """Per-row 1 / sqrt(mean(x^2) + eps) in fp32 (exact mean, rounded once)."""
+    xb = _bits(x)
+    R, K = xb.shape
+    r = np.empty((R,), np.float32)
+    lib().orc_rmsnorm_rstd(_p(xb), R, K, K, float(eps), _p(r))
+    return r
+
+
+def rmsnorm_quant_rows(x, gamma, rstd=None, eps: float = 1e-5):
+    """RMSNorm of every row (with the given per-row rstd, else the oracle's),
+    then one amax/448 scale per row.
+    -> (codes u8 [R, K], scales f32 [R], normalised rows bf16 bits u16 [R, K], rstd f32 [R])."""
+    xb = _bits(x)
+    gb = _bits(gamma).ravel()
+    R, K = xb.shape
+    assert gb.size == K
+    r = rmsnorm_rstd(xb, eps) if rstd is None else np.ascontiguousarray(rstd, dtype=np.float32)
+    q = np.empty((R, K), np.uint8)
+    s = np.empty((R,), np.float32)
+    y = np.empty((R, K), np.uint16)
+    lib().orc_rmsnorm_quant_rows(_p(xb), _p(gb), _p(r), R, K, K, _p(q), K, _p(s), _p(y))
+    return q, s, y, r
 
 
 def quant_groups128(x):

@@ -152,6 +152,69 @@ ORC_EXPORT void orc_quant_rows(const uint16_t* x, int64_t rows, int64_t K, int64
     }
 }
 
+/* ------------------------------------------------- RMSNorm, then per token */
+/*
+ * [P1] section 1.3 (编码器细节：RMSNorm 与 SwiGLU 的实现差异): Llama 3 normalises
+ * with RMSNorm before attention and before the MLP, eps = 1e-5; section 5
+ * (the fine-tuning notes) keeps RMSNorm in BF16.  So the input of the q/k/v and
+ * gate/up projections is y = RMSNorm(x) in bf16, and its per-token
+ * quantization is the activation quantization above applied to y.
+ * Readings (the pages print no formula): with x in bf16 and gamma the bf16
+ * weight,
+ *   ms   = mean over the row of x^2, rounded once to fp32
+ *   rstd = 1 / sqrt(fl32(ms + eps)), rounded once to fp32
+ *   h    = bf16(fl32(x * rstd)),  y = bf16(fl32(gamma * h))
+ * (normalise in fp32, return to bf16, then scale by the bf16 weight).
+ */
+
+/* Round to the nearest bf16, ties to even (finite inputs). */
+static uint16_t float_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    uint32_t upper = u >> 16, lower = u & 0xFFFFu;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;
+    return (uint16_t)upper;
+}
+
+/* Reciprocal RMS of every row.  The sum of squares is accumulated without
+ * error (each square of a bf16 value is exact in double; pairs of doubles
+ * carry the rounding error of every addition), so ms is the exact mean
+ * rounded to fp32 (one double rounding of the quotient first). */
+ORC_EXPORT void orc_rmsnorm_rstd(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, float eps, float* rstd) {
+    for (int64_t r = 0; r < rows; ++r) {
+        double hi = 0.0, lo = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double v = (double)bf16_to_float(x[r * ld + k]);
+            double sq = v * v;
+            double t = hi + sq;                        /* two-sum: t + err == hi + sq exactly */
+            double bb = t - hi;
+            double err = (hi - (t - bb)) + (sq - bb);
+            hi = t;
+            lo += err;
+        }
+        volatile float ms = (float)((hi + lo) / (double)K);
+        volatile float d = ms + eps;                   /* fp32 addition */
+        rstd[r] = (float)(1.0 / sqrt((double)d));
+    }
+}
+
+/* Normalise each row with the given rstd, then quantize it per token.
+ * gamma: bf16 bits [K].  q/s as orc_quant_rows; y (bf16 bits [rows, K])
+ * receives the normalised rows. */
+ORC_EXPORT void orc_rmsnorm_quant_rows(const uint16_t* x, const uint16_t* gamma, const float* rstd, int64_t rows,
+                                       int64_t K, int64_t ld, uint8_t* q, int64_t ldq, float* s, uint16_t* y) {
+    for (int64_t r = 0; r < rows; ++r) {
+        uint16_t* yr = y + r * K;
+        for (int64_t k = 0; k < K; ++k) {
+            volatile float t = bf16_to_float(x[r * ld + k]) * rstd[r];
+            uint16_t h = float_to_bf16(t);
+            volatile float g = bf16_to_float(gamma[k]) * bf16_to_float(h);
+            yr[k] = float_to_bf16(g);
+        }
+        orc_quant_rows(yr, 1, K, K, q + r * ldq, ldq, s + r);
+    }
+}
+
 /* One scale per 128 consecutive input features of each token [P5].
  * K must be a multiple of 128.  s: [M, K/128] row-major. */
 ORC_EXPORT void orc_quant_groups128(const uint16_t* x, int64_t M, int64_t K, int64_t ld,

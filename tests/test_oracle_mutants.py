@@ -35,6 +35,12 @@ MUTANTS = {
     "block x_scale column": (r"xs\[m \* KB \+ kb\]", "xs[m * KB]"),
     "group of 64": (r"for \(int64_t k = g \* 128; k < g \* 128 \+ 128; \+\+k\) \{", "for (int64_t k = g * 128; k < g * 128 + 64; ++k) {"),
     "amax = 0 gives scale 0": (r"if \(amax == 0\.0f\) return 1\.0f;", "if (amax == 0.0f) return 0.0f;"),
+    "rms without the square root": (r"rstd\[r\] = \(float\)\(1\.0 / sqrt\(\(double\)d\)\);",
+                                    "rstd[r] = (float)(1.0 / (double)d);"),
+    "rms mean over K - 1": (r"\(hi \+ lo\) / \(double\)K\)", "(hi + lo) / (double)(K - 1))"),
+    "rms eps ignored": (r"volatile float d = ms \+ eps;", "volatile float d = ms;"),
+    "rms gamma dropped": (r"volatile float g = bf16_to_float\(gamma\[k\]\) \* bf16_to_float\(h\);",
+                          "volatile float g = bf16_to_float(h);"),
 }
 
 
@@ -52,6 +58,8 @@ def build_variant(src_text, tmp):
     for f in ("orc_quant_rows", "orc_quant_groups128", "orc_quant_blocks128"):
         getattr(L, f).argtypes = [P, I, I, I, P, I, P]
     L.orc_linear.argtypes = [P, P, P, P, I, I, I, I, I, ctypes.c_int, P]
+    L.orc_rmsnorm_rstd.argtypes = [P, I, I, I, ctypes.c_float, P]
+    L.orc_rmsnorm_quant_rows.argtypes = [P, P, P, I, I, I, P, I, P, P]
     return L
 
 
@@ -152,6 +160,27 @@ def checks(L):
         if abs(float(y[m, n]) - float(e)) > _pins.f32_ulp(float(e)) * 2:
             failed.append("linear block vs rationals")
             break
+    # RMSNorm: rstd against the float64 mean of squares (1 ulp), normalised
+    # rows against torch's float64 rms_norm (two bf16 roundings)
+    Kr = 512
+    xr = synth.make_x(4, Kr, seed=6)
+    xrb = xr.view(torch.int16).numpy().view(np.uint16).copy()
+    gr = (1.0 + 0.1 * torch.randn(Kr, generator=torch.Generator().manual_seed(6))).to(torch.bfloat16)
+    grb = gr.view(torch.int16).numpy().view(np.uint16).copy()
+    rs = np.empty(4, np.float32)
+    L.orc_rmsnorm_rstd(_p(xrb), 4, Kr, Kr, ctypes.c_float(1e-5), _p(rs))
+    ms = (xr.double() ** 2).mean(dim=1).float()
+    rref = (1.0 / torch.sqrt((ms + torch.tensor(1e-5, dtype=torch.float32)).double())).float().numpy()
+    if np.abs(rs.view(np.int32).astype(np.int64) - rref.view(np.int32).astype(np.int64)).max() > 1:
+        failed.append("rmsnorm rstd")
+    qr = np.empty((4, Kr), np.uint8)
+    sr = np.empty(4, np.float32)
+    yr = np.empty((4, Kr), np.uint16)
+    L.orc_rmsnorm_quant_rows(_p(xrb), _p(grb), _p(rref.copy()), 4, Kr, Kr, _p(qr), Kr, _p(sr), _p(yr))
+    yref = torch.nn.functional.rms_norm(xr.double(), (Kr,), weight=gr.double(), eps=1e-5)
+    yt = torch.from_numpy(yr.astype(np.int16)).view(torch.bfloat16).double()
+    if not torch.all((yt - yref).abs() <= 2.0 ** -7 * yref.abs() * 1.001 + 1e-30):
+        failed.append("rmsnorm rows")
     return failed
 
 

@@ -556,6 +556,47 @@ def run_gpu(args):
                     "GB/s": round(wqb / (min(wq_ms) / 1e3) / 1e9, 1),
                     "frac_hbm": round(wqb / (min(wq_ms) / 1e3) / 1e9 / pk["hbm_gbs"], 3)}
 
+    # ---- RMSNorm + per-token quantization fused (the activations that follow
+    # an RMSNorm in Llama: the inputs of q/k/v and of gate/up), timed alone,
+    # next to the unfused pair (torch's bf16 rms_norm, then fp8_quant_act)
+    rms = []
+    for k, (M, K, mode) in xs_shapes.items():
+        if mode != synth.CHANNEL_TOKEN or not (k.startswith("attn_in") or k.startswith("mlp_in")):
+            continue
+        gmm = (1.0 + 0.1 * torch.randn(K, generator=torch.Generator().manual_seed(K))).to(torch.bfloat16).to(dev)
+        xq_f, xs_f = torch.empty_like(XQ[k][0]), torch.empty_like(XQ[k][1])
+        y_n = torch.empty_like(X[k])
+
+        def fused(k=k, gmm=gmm, xq_f=xq_f, xs_f=xs_f):
+            fq.fp8_rmsnorm_quant_act(X[k], gmm, 1e-5, out=(xq_f, xs_f))
+
+        def unfused(k=k, gmm=gmm, xq_f=xq_f, xs_f=xs_f, y_n=y_n, K=K):
+            y_n.copy_(torch.nn.functional.rms_norm(X[k], (K,), weight=gmm, eps=1e-5))
+            fq.fp8_quant_act(y_n, synth.CHANNEL_TOKEN, out=(xq_f, xs_f))
+
+        times = []
+        for fn in (fused, unfused):
+            fn()
+            torch.cuda.synchronize()
+            gr = capture([fn]) if not args.eager else None
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            torch.cuda._sleep(2_000_000)
+            for s_ in range(args.steps):
+                flush.zero_()
+                ev[s_][0].record(stream)
+                gr.replay() if gr is not None else fn()
+                ev[s_][1].record(stream)
+            torch.cuda.synchronize()
+            times.append(float(np.median([a.elapsed_time(b) for a, b in ev])))
+        rb = 2 * M * K + 2 * K + M * K + 4 * M
+        rms.append({"act": k, "M": M, "K": K, "ms": round(times[0], 5),
+                    "GB/s": round(rb / (times[0] / 1e3) / 1e9, 1),
+                    "frac_hbm": round(rb / (times[0] / 1e3) / 1e9 / pk["hbm_gbs"], 3),
+                    "unfused_ms": round(times[1], 5),
+                    "bytes": "2*M*K (x) + 2*K (gamma) + M*K (codes) + 4*M (scales)"})
+    assert fq.device_error(clear=True) == 0
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -616,7 +657,7 @@ def run_gpu(args):
                        "parallelism": "single GPU" if world == 1 else f"token-parallel x{world}, weights replicated"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g) for g in wl.gemms)),
-            "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant,
+            "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant, "rmsnorm_quant": rms,
             "merged_shared_input": merged,
             "device_error": err, "gpu": torch.cuda.get_device_name(dev),
         }

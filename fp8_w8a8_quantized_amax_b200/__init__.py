@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.fp8_quant_weight.restype = ctypes.c_int
         L.fp8_quant_act.argtypes = [P, I, I, I, ctypes.c_int, P, I, P, P]
         L.fp8_quant_act.restype = ctypes.c_int
+        L.fp8_rmsnorm_quant_act.argtypes = [P, P, I, I, I, ctypes.c_float, P, I, P, P, P]
+        L.fp8_rmsnorm_quant_act.restype = ctypes.c_int
         L.fp8_linear.argtypes = [P, P, P, P, I, I, I, ctypes.c_int, P, I, P, S, P]
         L.fp8_linear.restype = ctypes.c_int
         L.fp8_linear_workspace_size.argtypes = [I, I, I, ctypes.c_int]
@@ -137,6 +139,26 @@ def fp8_quant_act(X: torch.Tensor, mode: int = CHANNEL_TOKEN,
                              _ptr(xs), _stream(X))
     _check(st, "fp8_quant_act")
     return Xq, xs
+
+
+def fp8_rmsnorm_quant_act(X: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-5,
+                          out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None, return_rstd: bool = False):
+    """RMSNorm(X) * gamma in bf16, quantized per token, in one pass.
+    X bf16 [M, K], gamma bf16 [K] -> (Xq uint8 [M, K], x_scale fp32 [M][, rstd fp32 [M]])."""
+    _require_cuda(X, "X", torch.bfloat16)
+    M, K = X.shape
+    if not gamma.is_cuda or gamma.dtype != torch.bfloat16 or gamma.numel() != K or not gamma.is_contiguous():
+        raise ValueError("gamma must be a contiguous bf16 CUDA tensor of K elements")
+    if out is None:
+        Xq = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+        xs = torch.empty((M,), dtype=torch.float32, device=X.device)
+    else:
+        Xq, xs = out
+    rstd = torch.empty((M,), dtype=torch.float32, device=X.device) if return_rstd else None
+    st = lib().fp8_rmsnorm_quant_act(_ptr(X), _ptr(gamma), M, K, X.stride(0), float(eps), _ptr(Xq), Xq.stride(0),
+                                     _ptr(xs), _ptr(rstd), _stream(X))
+    _check(st, "fp8_rmsnorm_quant_act")
+    return (Xq, xs, rstd) if return_rstd else (Xq, xs)
 
 
 def fp8_linear_workspace_size(M: int, N: int, K: int, mode: int = CHANNEL_TOKEN) -> int:

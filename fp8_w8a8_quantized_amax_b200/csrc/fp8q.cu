@@ -167,6 +167,26 @@ fp8q_status launch_rows(const uint16_t* x, int64_t rows, int K, int64_t ldx, uin
   return FP8Q_ERR_UNSUPPORTED;   // K > 131072
 }
 
+fp8q_status launch_rmsnorm_rows(const uint16_t* x, const uint16_t* gamma, int64_t rows, int K, int64_t ldx,
+                                float eps, uint8_t* q, int64_t ldq, float* s, float* rstd, void* stream) {
+  const int nvec = K / 8;
+  int T = 32 * ((nvec + 32 * 8 - 1) / (32 * 8));
+  if (T > 512) T = 512;
+  const int need = (nvec + T - 1) / T;
+  const dim3 grid(static_cast<unsigned>(rows));
+  const dim3 block(T);
+#define FP8Q_RMS(V)                                                                                             \
+  return launch(fp8q::rmsnorm_quant_rows_kernel<V>, grid, block, 0, stream, x, gamma, K, ldx, eps, q, ldq, s, \
+                rstd)
+  if (need <= 1) FP8Q_RMS(1);
+  if (need <= 2) FP8Q_RMS(2);
+  if (need <= 4) FP8Q_RMS(4);
+  if (need <= 8) FP8Q_RMS(8);
+  if (need <= 16) FP8Q_RMS(16);
+#undef FP8Q_RMS
+  return FP8Q_ERR_UNSUPPORTED;   // K > 65536
+}
+
 // ------------------------------------------------------------------ linear ---
 
 constexpr int kPrefillBN = 256;
@@ -309,6 +329,20 @@ fp8q_status fp8_quant_act(const void* X_bf16, int64_t M, int64_t K, int64_t ldx,
   if (grid > static_cast<int64_t>(sms) * 16) grid = static_cast<int64_t>(sms) * 16;
   return launch(fp8q::quant_groups128_kernel<GPT>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream, x, M,
                 G, ldx, Xq, ldxq, x_scale);
+}
+
+fp8q_status fp8_rmsnorm_quant_act(const void* X_bf16, const void* gamma_bf16, int64_t M, int64_t K, int64_t ldx,
+                                  float eps, uint8_t* Xq, int64_t ldxq, float* x_scale, float* rstd, void* stream) {
+  fp8q_status st = check_quant_args(X_bf16, M, K, ldx, FP8Q_CHANNEL_TOKEN, Xq, ldxq, x_scale);
+  if (st != FP8Q_OK) return st;
+  if (!(eps >= 0.0f) || !(eps < 3.0e38f)) return FP8Q_ERR_INVALID_ARG;   // also rejects NaN
+  if (M == 0) return FP8Q_OK;
+  if (!gamma_bf16) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(gamma_bf16, 16) || (rstd && !aligned(rstd, 4))) return FP8Q_ERR_MISALIGNED;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
+  return launch_rmsnorm_rows(static_cast<const uint16_t*>(X_bf16), static_cast<const uint16_t*>(gamma_bf16), M,
+                             static_cast<int>(K), ldx, eps, Xq, ldxq, x_scale, rstd, stream);
 }
 
 size_t fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int mode) {

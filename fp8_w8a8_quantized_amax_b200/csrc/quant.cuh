@@ -143,6 +143,127 @@ __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __rest
   }
 }
 
+// ----------------------------------------------------- RMSNorm, then rows ---
+// The input of the q/k/v and gate/up projections is RMSNorm(x) in bf16
+// (Llama 3: RMSNorm before attention and MLP, eps 1e-5, kept in BF16).  One
+// CTA per token normalises its row in registers and quantizes it per token,
+// without writing the normalised bf16 row to memory:
+//   ms = fl32(sum x^2) / K, rstd = rsqrt_rn(ms + eps) (both IEEE),
+//   y = bf16(fl32(gamma * bf16(fl32(x * rstd)))), then y as quant_rows.
+// The sum of squares is an fp32 sum in this kernel's order; rstd is written
+// out (when rstd != nullptr) so that a caller can reproduce y exactly.
+
+// y for the 8 bf16 values of v (x) with the matching 8 of g (gamma), two at a
+// time: h = bf16(fl32(x * rstd)) by a packed fp32 multiply and one bf16x2
+// rounding; y = bf16(gamma * h) by one bf16x2 multiply.  The product of two
+// bf16 values is exact in fp32, so rounding it once to bf16 (mul.rn.bf16x2)
+// is the same as rounding the fp32 product.
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint4 rmsnorm_vec(const uint4& v, const uint4& g, uint64_t rs2) {
+  auto one = [&](uint32_t xw, uint32_t gw) -> uint32_t {
+    float pl, ph;
+    f32x2_unpack(mul_f32x2(f32x2_pack(bf16lo(xw), bf16hi(xw)), rs2), pl, ph);
+    return mul_bf16x2(gw, pack_bf16x2(pl, ph));
+  };
+  return make_uint4(one(v.x, g.x), one(v.y, g.y), one(v.z, g.z), one(v.w, g.w));
+}
+
+// Sum of squares of the 8 values of v into two fp32 chains.
+__device__ __forceinline__ uint64_t sumsq_vec(const uint4& v, uint64_t acc2) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint64_t x2 = f32x2_pack(bf16lo(w[i]), bf16hi(w[i]));
+    acc2 = fma_f32x2(x2, x2, acc2);
+  }
+  return acc2;
+}
+
+template <int VPT>
+__global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t* __restrict__ x,
+                                                                 const uint16_t* __restrict__ gamma, int K,
+                                                                 int64_t ldx, float eps, uint8_t* __restrict__ q,
+                                                                 int64_t ldq, float* __restrict__ s,
+                                                                 float* __restrict__ rstd) {
+  __shared__ float red_sum[32];
+  __shared__ uint32_t red_max[32];
+  griddep_wait();
+  const int64_t r = blockIdx.x;
+  const int nvec = K >> 3;
+  const int T = blockDim.x;
+  const int warp = threadIdx.x >> 5, nw = T >> 5;
+  const uint16_t* xr = x + r * ldx;
+  // gamma is loaded with the row (not after the reduction) when it fits in registers
+  constexpr bool kGammaAhead = VPT <= 8;
+  uint4 v[VPT], gv[kGammaAhead ? VPT : 1];
+  uint64_t ss2 = f32x2_pack(0.0f, 0.0f);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = threadIdx.x + i * T;
+    if (idx < nvec) {
+      v[i] = ld_stream16(xr + idx * 8);
+      if constexpr (kGammaAhead) gv[i] = __ldg(reinterpret_cast<const uint4*>(gamma) + idx);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < VPT; ++i)
+    if (threadIdx.x + i * T < nvec) ss2 = sumsq_vec(v[i], ss2);
+  float ss_lo, ss_hi;
+  f32x2_unpack(ss2, ss_lo, ss_hi);
+  float ss = ss_lo + ss_hi;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+  if (T > 32) {
+    if (lane_id() == 0) red_sum[warp] = ss;
+    __syncthreads();
+    ss = lane_id() < nw ? red_sum[lane_id()] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+  }
+  const float rs = __frsqrt_rn(__fadd_rn(__fdiv_rn(ss, static_cast<float>(K)), eps));
+  if (threadIdx.x == 0 && rstd != nullptr) rstd[r] = rs;
+  const uint64_t rs2 = f32x2_pack(rs, rs);
+  uint32_t m2 = 0;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = threadIdx.x + i * T;
+    if (idx < nvec) {
+      if constexpr (kGammaAhead) v[i] = rmsnorm_vec(v[i], gv[i], rs2);
+      else v[i] = rmsnorm_vec(v[i], __ldg(reinterpret_cast<const uint4*>(gamma) + idx), rs2);
+      m2 = absmax_bits_vec(v[i], m2);
+    }
+  }
+  uint32_t m = __reduce_max_sync(0xFFFFFFFFu, fold_halves(m2));
+  if (T > 32) {
+    if (lane_id() == 0) red_max[warp] = m;
+    __syncthreads();
+    m = lane_id() < nw ? red_max[lane_id()] : 0u;
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+  }
+  const float sc = scale_of(amax_bits_to_float(m));
+  if (threadIdx.x == 0) s[r] = sc;
+  const Divider dv = make_divider(sc);
+  uint8_t* qr = q + r * ldq;
+  if (dv.fast) {
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int idx = threadIdx.x + i * T;
+      if (idx < nvec) *reinterpret_cast<uint2*>(qr + idx * 8) = encode_vec<true>(v[i], dv);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int idx = threadIdx.x + i * T;
+      if (idx < nvec) *reinterpret_cast<uint2*>(qr + idx * 8) = encode_vec<false>(v[i], dv);
+    }
+  }
+}
+
 // ----------------------------------------------------------- groups 128 ---
 // Groups of 128 features: 16 consecutive lanes (a half warp) own one group,
 // one 16-byte vector each.  Each half warp walks GPT groups, strided by the

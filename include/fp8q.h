@@ -99,6 +99,33 @@ FP8Q_API fp8q_status fp8_quant_act(const void* X_bf16, int64_t M, int64_t K, int
                           uint8_t* Xq, int64_t ldxq, float* x_scale, void* stream);
 
 /*
+ * fp8_rmsnorm_quant_act -- RMSNorm of bf16 activations, then per-token E4M3
+ * quantization of the result, in one pass (the normalised bf16 rows are not
+ * written).  Llama 3 normalises with RMSNorm (eps 1e-5) before attention and
+ * before the MLP and keeps it in BF16 ("Llama 3 精读实录", sections 1.3 and 5),
+ * so this produces exactly the codes and scales that fp8_quant_act in
+ * FP8Q_CHANNEL_TOKEN mode gives for the bf16 RMSNorm output.
+ *
+ *   X_bf16     [M, ldx] bf16 hidden states, read-only (rules as fp8_quant_act).
+ *   gamma_bf16 [K] bf16 RMSNorm weight, 16-byte aligned.
+ *   eps        >= 0, finite (1e-5 for Llama 3).
+ *   Xq, x_scale as fp8_quant_act in FP8Q_CHANNEL_TOKEN mode ([M] scales).
+ *   rstd       [M] fp32, written when not NULL: the row's 1 / sqrt(ms + eps).
+ *   Per row:  ms   = (sum over the row of x^2 in fp32) / K    (IEEE division)
+ *             rstd = 1 / sqrt(ms + eps), correctly rounded fp32
+ *             y    = bf16(gamma * bf16(x * rstd))           (fp32 products)
+ *             codes and scale of y as fp8_quant_act.
+ *   The fp32 sum of squares is taken in this kernel's order.  Everything
+ *   after it is exact, so rstd determines y and the codes.  Rows whose sum of
+ *   squares overflows fp32 are outside the contract.
+ *   Requirements: M >= 0 (M == 0 is a no-op), K > 0, K % 16 == 0, and
+ *   K <= 65536 (FP8Q_ERR_UNSUPPORTED above).
+ */
+FP8Q_API fp8q_status fp8_rmsnorm_quant_act(const void* X_bf16, const void* gamma_bf16, int64_t M, int64_t K,
+                                           int64_t ldx, float eps, uint8_t* Xq, int64_t ldxq, float* x_scale,
+                                           float* rstd, void* stream);
+
+/*
  * fp8_linear -- Y[M, N] = dequant(Xq) . dequant(Wq)^T in bf16, on tcgen05 tensor cores.
  *
  *   Xq        [M, K] uint8 codes, contiguous (row stride K), 16-byte aligned.

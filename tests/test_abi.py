@@ -99,6 +99,30 @@ def test_quant_act_argument_checks(L, kw, want):
     assert q_act(L, **kw) == want
 
 
+def rms_q(L, x=P, g=P, M=4, K=256, ldx=256, eps=1e-5, q=P, ldq=256, s=P, r=None):
+    return L.fp8_rmsnorm_quant_act(x, g, M, K, ldx, eps, q, ldq, s, r, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(K=0), fq.ERR_INVALID_ARG),
+    (dict(K=24, ldx=24, ldq=32), fq.ERR_INVALID_ARG),        # K % 16
+    (dict(M=-1), fq.ERR_INVALID_ARG),
+    (dict(ldx=128), fq.ERR_INVALID_ARG),
+    (dict(g=None), fq.ERR_INVALID_ARG),
+    (dict(x=None), fq.ERR_INVALID_ARG),
+    (dict(s=None), fq.ERR_INVALID_ARG),
+    (dict(eps=-1.0), fq.ERR_INVALID_ARG),
+    (dict(eps=float("nan")), fq.ERR_INVALID_ARG),
+    (dict(eps=float("inf")), fq.ERR_INVALID_ARG),
+    (dict(g=BAD), fq.ERR_MISALIGNED),
+    (dict(x=BAD), fq.ERR_MISALIGNED),
+    (dict(r=P + 2), fq.ERR_MISALIGNED),
+    (dict(M=0, x=None, g=None, q=None, s=None), fq.OK),      # empty input is a no-op
+])
+def test_rmsnorm_quant_argument_checks(L, kw, want):
+    assert rms_q(L, **kw) == want
+
+
 @pytest.mark.parametrize("kw,want", [
     (dict(mode=3), fq.ERR_INVALID_ARG),
     (dict(N=-2), fq.ERR_INVALID_ARG),
@@ -141,6 +165,7 @@ def test_valid_arguments_without_a_gpu_report_cuda_error(L):
     assert q_act(L) == fq.ERR_CUDA
     assert q_w(L) == fq.ERR_CUDA
     assert lin(L) == fq.ERR_CUDA
+    assert rms_q(L) == fq.ERR_CUDA
 
 
 def test_binding_refuses_cpu_tensors(L):

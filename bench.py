@@ -597,6 +597,32 @@ def run_gpu(args):
                     "bytes": "2*M*K (x) + 2*K (gamma) + M*K (codes) + 4*M (scales)"})
     assert fq.device_error(clear=True) == 0
 
+    # ---- FP8 KV cache: the k_proj / v_proj outputs quantized per (token, head)
+    kvq = []
+    for g in wl.gemms:
+        if g.name not in ("k_proj", "v_proj") or g.N % 128:
+            continue
+        kv = Y[g.name].view(g.M, g.N // 128, 128)
+        kq = torch.empty(kv.shape, dtype=torch.uint8, device=dev)
+        ks = torch.empty((g.M, g.N // 128), dtype=torch.float32, device=dev)
+        fn = (lambda kv=kv, kq=kq, ks=ks: fq.fp8_quant_kv(kv, out=(kq, ks)))
+        fn()
+        torch.cuda.synchronize()
+        gr = capture([fn]) if not args.eager else None
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda._sleep(2_000_000)
+        for s_ in range(args.steps):
+            flush.zero_()
+            ev[s_][0].record(stream)
+            gr.replay() if gr is not None else fn()
+            ev[s_][1].record(stream)
+        torch.cuda.synchronize()
+        t = float(np.median([a.elapsed_time(b) for a, b in ev]))
+        kb = 3 * g.M * g.N + 4 * g.M * (g.N // 128)
+        kvq.append({"kv": g.name, "tokens": g.M, "heads": g.N // 128, "ms": round(t, 5),
+                    "GB/s": round(kb / (t / 1e3) / 1e9, 1), "frac_hbm": round(kb / (t / 1e3) / 1e9 / pk["hbm_gbs"], 3)})
+    assert fq.device_error(clear=True) == 0
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -657,7 +683,7 @@ def run_gpu(args):
                        "parallelism": "single GPU" if world == 1 else f"token-parallel x{world}, weights replicated"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g) for g in wl.gemms)),
-            "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant, "rmsnorm_quant": rms,
+            "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant, "rmsnorm_quant": rms, "kv_quant": kvq,
             "merged_shared_input": merged,
             "device_error": err, "gpu": torch.cuda.get_device_name(dev),
         }

@@ -161,6 +161,23 @@ def fp8_rmsnorm_quant_act(X: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-
     return (Xq, xs, rstd) if return_rstd else (Xq, xs)
 
 
+def fp8_quant_kv(kv: torch.Tensor, out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
+    """FP8 KV cache: one amax/448 scale per (token, head) of a K or V tensor.
+    kv bf16 [T, H, 128] (head_dim 128, contiguous) -> (codes uint8 [T, H, 128], scales fp32 [T, H]).
+    A head's 128 values are one 128-group of the [T, H*128] rows, so this is
+    fp8_quant_act in BLOCK128 mode on that view."""
+    if kv.dim() != 3 or kv.shape[2] != 128 or not kv.is_contiguous():
+        raise ValueError("kv must be a contiguous [tokens, heads, 128] tensor")
+    T, H, D = kv.shape
+    if out is None:
+        q = torch.empty((T, H, D), dtype=torch.uint8, device=kv.device)
+        s = torch.empty((T, H), dtype=torch.float32, device=kv.device)
+    else:
+        q, s = out
+    fp8_quant_act(kv.view(T, H * D), BLOCK128, out=(q.view(T, H * D), s.view(T, H)))
+    return q, s
+
+
 def fp8_linear_workspace_size(M: int, N: int, K: int, mode: int = CHANNEL_TOKEN) -> int:
     return int(lib().fp8_linear_workspace_size(M, N, K, int(mode)))
 

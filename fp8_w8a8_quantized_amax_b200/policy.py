@@ -42,3 +42,13 @@ def llama_linear_names(num_layers: int, tie_head: bool = False) -> list:
     if not tie_head:
         names.append("lm_head")
     return names
+
+
+def kv_cache_bytes(context: int, layers: int, kv_heads: int, head_dim: int, element_bytes: float,
+                   scale_bytes_per_head: int = 0) -> int:
+    """Bytes of a K+V cache: context x layers x KV heads x head_dim x 2 (K and V)
+    x bytes per element (the size model of the Llama-3.2-3B FP8-Block explainer,
+    FAQ Q2), plus, for an FP8 cache with one scale per (token, head), that scale
+    for each of K and V."""
+    n = context * layers * kv_heads * 2
+    return int(n * head_dim * element_bytes + n * scale_bytes_per_head)

@@ -173,3 +173,15 @@ def test_every_bf16_pair_matches_ieee_division():
             r, c = bad.nonzero()[0].tolist()
             raise AssertionError(f"amax {float(a[r])}: x {float(x[r, c])} gives {int(q[r, c]):#04x}, "
                                  f"IEEE division {int(q_ref[r, c]):#04x} ({int(bad.sum())} differ in this chunk)")
+
+
+@pytest.mark.parametrize("T,H", [(1, 8), (37, 8), (8192, 8), (513, 2)])
+def test_kv_cache_per_token_per_head(T, H):
+    # one scale per (token, head) of a [T, H, 128] K or V tensor: each head is a
+    # 128-group of the [T, H*128] rows
+    kv = synth.make_x(T, H * 128, seed=T + H)
+    q, s = fq.fp8_quant_kv(kv.view(T, H, 128).to(DEV))
+    rq, rs = oracle.quant_groups128(kv)
+    assert tuple(q.shape) == (T, H, 128) and tuple(s.shape) == (T, H)
+    P.assert_codes_equal(q.view(T, H * 128), rq, f"kv {T}x{H}")
+    P.assert_scales_equal(s, rs, f"kv {T}x{H}")

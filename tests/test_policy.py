@@ -70,3 +70,13 @@ def test_other_readings_do_not_match_the_page():
     # fp32 scales or an FP8 lm_head would not give the 72.67 GB the page prints
     assert round(_llama70b_bytes(scale_bytes=4)[1] / 1e9, 2) != 72.67
     assert round(_llama70b_bytes(scale_bytes=2, quantize_head=True)[1] / 1e9, 2) != 72.67
+
+
+def test_kv_cache_size_model():
+    # Llama-3.2-3B at its 128K context: 28 layers, 8 KV heads of 128 (FP8-Block explainer, FAQ Q2)
+    from fp8_w8a8_quantized_amax_b200.policy import kv_cache_bytes
+    bf16 = kv_cache_bytes(131072, 28, 8, 128, 2)
+    assert bf16 == 131072 * 28 * 8 * 128 * 2 * 2 == 15032385536            # 15.0 GB
+    fp8 = kv_cache_bytes(131072, 28, 8, 128, 1, scale_bytes_per_head=4)
+    assert fp8 == bf16 // 2 + 131072 * 28 * 8 * 2 * 4                       # half, plus fp32 scales
+    assert abs(fp8 / bf16 - (0.5 + 4 / (128 * 2))) < 1e-12                 # 1.6% of the bf16 size in scales

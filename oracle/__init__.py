@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         _lib.orc_linear.restype = None
         _lib.orc_linear_at.argtypes = [P, P, P, P, I, I, I, ctypes.c_int, P, P, I, P]
         _lib.orc_linear_at.restype = None
+        _lib.orc_linear_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, P]
+        _lib.orc_linear_swiglu.restype = None
         _lib.orc_rmsnorm_rstd.argtypes = [P, I, I, I, ctypes.c_float, P]
         _lib.orc_rmsnorm_rstd.restype = None
         _lib.orc_rmsnorm_quant_rows.argtypes = [P, P, P, I, I, I, P, I, P, P]
@@ -107,6 +109,23 @@ def quant_rows(x):
     s = np.empty((R,), np.float32)
     lib().orc_quant_rows(_p(xb), R, K, K, _p(q), K, _p(s))
     return q, s
+
+
+def linear_swiglu(xq, xs, wq_gate, ws_gate, wq_up, ws_up) -> np.ndarray:
+    """bf16(bf16(silu(g)) * u) of the exact gate and up linears (channel/token
+    scales), g and u rounded to bf16 first.  -> bf16 bits uint16 [M, N]."""
+    xq = np.ascontiguousarray(xq, np.uint8)
+    wg = np.ascontiguousarray(wq_gate, np.uint8)
+    wu = np.ascontiguousarray(wq_up, np.uint8)
+    xs = np.ascontiguousarray(xs, np.float32)
+    sg = np.ascontiguousarray(ws_gate, np.float32)
+    su = np.ascontiguousarray(ws_up, np.float32)
+    M, K = xq.shape
+    N = wg.shape[0]
+    assert wg.shape == (N, K) and wu.shape == (N, K)
+    act = np.empty((M, N), np.uint16)
+    lib().orc_linear_swiglu(_p(xq), _p(xs), _p(wg), _p(sg), _p(wu), _p(su), M, N, K, _p(act))
+    return act
 
 
 def rmsnorm_rstd(x, eps: float = 1e-5) -> np.ndarray:

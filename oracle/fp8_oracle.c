@@ -317,6 +317,33 @@ ORC_EXPORT void orc_linear(const uint8_t* xq, const float* xs, const uint8_t* wq
                 : linear_block_one(xq, xs, wq, ws, K, ldx, ldw, m, n);
 }
 
+/* ------------------------------------------------- gate/up with SiLU * up */
+/*
+ * [P1] section 1.3 (编码器细节：RMSNorm 与 SwiGLU 的实现差异): the Llama MLP
+ * computes gate and up separately and multiplies SiLU(gate) by up (SwiGLU);
+ * the product is down_proj's input.  Reading (the pages print no formula):
+ * with g and u the bf16 outputs of the gate and up linears,
+ *   act = bf16( bf16(silu(g)) * u ),  silu(v) = v / (1 + e^-v),
+ * silu evaluated exactly (double) and rounded once to bf16, the product of
+ * two bf16 values exact in fp32 and rounded once to bf16.
+ * act: bf16 bits [M, N] (row-major, stride N).  Channel/token scales. */
+ORC_EXPORT void orc_linear_swiglu(const uint8_t* xq, const float* xs, const uint8_t* wq_gate,
+                                  const float* ws_gate, const uint8_t* wq_up, const float* ws_up,
+                                  int64_t M, int64_t N, int64_t K, uint16_t* act) {
+    build_ik_table();
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            float g = linear_channel_one(xq, xs, wq_gate, ws_gate, K, K, K, m, n);
+            float u = linear_channel_one(xq, xs, wq_up, ws_up, K, K, K, m, n);
+            double gb = (double)bf16_to_float(float_to_bf16(g));
+            double ub = (double)bf16_to_float(float_to_bf16(u));
+            uint16_t sb = float_to_bf16((float)(gb / (1.0 + exp(-gb))));
+            volatile float p = bf16_to_float(sb) * (float)ub;
+            act[m * N + n] = float_to_bf16(p);
+        }
+}
+
 /* Selected outputs y[i] = Y[ms[i], ns[i]], for spot checks at full size. */
 ORC_EXPORT void orc_linear_at(const uint8_t* xq, const float* xs, const uint8_t* wq,
                               const float* ws, int64_t K, int64_t ldx, int64_t ldw, int mode,

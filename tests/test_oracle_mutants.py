@@ -41,6 +41,11 @@ MUTANTS = {
     "rms eps ignored": (r"volatile float d = ms \+ eps;", "volatile float d = ms;"),
     "rms gamma dropped": (r"volatile float g = bf16_to_float\(gamma\[k\]\) \* bf16_to_float\(h\);",
                           "volatile float g = bf16_to_float(h);"),
+    "swiglu without the sigmoid": (r"float_to_bf16\(\(float\)\(gb / \(1\.0 \+ exp\(-gb\)\)\)\)",
+                                   "float_to_bf16((float)gb)"),
+    "swiglu sigmoid sign": (r"exp\(-gb\)", "exp(gb)"),
+    "swiglu up dropped": (r"volatile float p = bf16_to_float\(sb\) \* \(float\)ub;",
+                          "volatile float p = bf16_to_float(sb);"),
 }
 
 
@@ -60,6 +65,7 @@ def build_variant(src_text, tmp):
     L.orc_linear.argtypes = [P, P, P, P, I, I, I, I, I, ctypes.c_int, P]
     L.orc_rmsnorm_rstd.argtypes = [P, I, I, I, ctypes.c_float, P]
     L.orc_rmsnorm_quant_rows.argtypes = [P, P, P, I, I, I, P, I, P, P]
+    L.orc_linear_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, P]
     return L
 
 
@@ -181,6 +187,22 @@ def checks(L):
     yt = torch.from_numpy(yr.astype(np.int16)).view(torch.bfloat16).double()
     if not torch.all((yt - yref).abs() <= 2.0 ** -7 * yref.abs() * 1.001 + 1e-30):
         failed.append("rmsnorm rows")
+    # SwiGLU: bf16(bf16(silu(g)) * u) against torch's float64 silu on the
+    # (separately checked) linear outputs rounded to bf16 by torch
+    wu = rng.integers(0, 256, (N, K)).astype(np.uint8)
+    wu[(wu & 0x7F) == 0x7F] = 0x38
+    wsu = rng.uniform(0.01, 0.1, N).astype(np.float32)
+    act = np.empty((M, N), np.uint16)
+    L.orc_linear_swiglu(_p(xq), _p(xs), _p(wq), _p(ws), _p(wu), _p(wsu), M, N, K, _p(act))
+    gE = np.empty((M, N), np.float32)
+    uE = np.empty((M, N), np.float32)
+    L.orc_linear(_p(xq), _p(xs), _p(wq), _p(ws), M, N, K, K, K, 0, _p(gE))
+    L.orc_linear(_p(xq), _p(xs), _p(wu), _p(wsu), M, N, K, K, K, 0, _p(uE))
+    gb = torch.from_numpy(gE).to(torch.bfloat16)
+    ub = torch.from_numpy(uE).to(torch.bfloat16)
+    aref = (torch.nn.functional.silu(gb.double()).to(torch.bfloat16) * ub).view(torch.int16).numpy().view(np.uint16)
+    if not np.array_equal(act, aref):
+        failed.append("swiglu")
     return failed
 
 

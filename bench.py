@@ -597,6 +597,55 @@ def run_gpu(args):
                     "bytes": "2*M*K (x) + 2*K (gamma) + M*K (codes) + 4*M (scales)"})
     assert fq.device_error(clear=True) == 0
 
+    # ---- gate/up with the SiLU * up epilogue (one kernel, only the activation
+    # written) next to the separate path: both GEMMs, then torch's silu * up
+    swiglu = []
+    gmap = {g.name.replace("gate_proj", "").replace("up_proj", ""): [] for g in wl.gemms}
+    for g in wl.gemms:
+        if g.mode == synth.CHANNEL_TOKEN and (g.name.startswith("gate_proj") or g.name.startswith("up_proj")):
+            gmap[g.name.replace("gate_proj", "").replace("up_proj", "")].append(g)
+    for suffix, gs in gmap.items():
+        gg = [g for g in gs if g.name.startswith("gate_proj")]
+        gu = [g for g in gs if g.name.startswith("up_proj")]
+        if len(gg) != 1 or len(gu) != 1:
+            continue
+        gg, gu = gg[0], gu[0]
+        act = torch.empty((gg.M, gg.N), dtype=torch.bfloat16, device=dev)
+
+        def fused(gg=gg, gu=gu, act=act):
+            fq.fp8_linear_swiglu(XQ[gg.x][0], XQ[gg.x][1], WQ[gg.name][0], WQ[gg.name][1], WQ[gu.name][0],
+                                 WQ[gu.name][1], out=act)
+
+        def separate(gg=gg, gu=gu, act=act):
+            for g in (gg, gu):
+                fq.fp8_linear(XQ[g.x][0], XQ[g.x][1], WQ[g.name][0], WQ[g.name][1], g.mode, out=Y[g.name],
+                              workspace=WS[g.name])
+            torch.mul(torch.nn.functional.silu(Y[gg.name]), Y[gu.name], out=act)
+
+        times = []
+        for fn in (fused, separate):
+            fn()
+            torch.cuda.synchronize()
+            gr = capture([fn]) if not args.eager else None
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            torch.cuda._sleep(2_000_000)
+            for s_ in range(args.steps):
+                flush.zero_()
+                ev[s_][0].record(stream)
+                gr.replay() if gr is not None else fn()
+                ev[s_][1].record(stream)
+            torch.cuda.synchronize()
+            times.append(float(np.median([a.elapsed_time(b) for a, b in ev])))
+        fl = 2 * gg.flops
+        swiglu.append({"gemms": f"{gg.name}+{gu.name}:{gg.M}x{gg.K}->{gg.N}", "ms": round(times[0], 5),
+                       "TFLOP/s": round(fl / (times[0] / 1e3) / 1e12, 1),
+                       "frac_fp8_peak": round(fl / (times[0] / 1e3) / 1e12 / fp8_peak, 3),
+                       "separate_ms": round(times[1], 5),
+                       "note": "fused: one kernel writes bf16(bf16(silu(gate)) * up); separate: two GEMMs "
+                               "writing gate and up, then torch silu and mul"})
+    assert fq.device_error(clear=True) == 0
+
     # ---- FP8 KV cache: the k_proj / v_proj outputs quantized per (token, head)
     kvq = []
     for g in wl.gemms:
@@ -683,7 +732,7 @@ def run_gpu(args):
                        "parallelism": "single GPU" if world == 1 else f"token-parallel x{world}, weights replicated"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g) for g in wl.gemms)),
-            "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant, "rmsnorm_quant": rms, "kv_quant": kvq,
+            "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant, "rmsnorm_quant": rms, "kv_quant": kvq, "swiglu": swiglu,
             "merged_shared_input": merged,
             "device_error": err, "gpu": torch.cuda.get_device_name(dev),
         }

@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
         L.fp8_quant_act.restype = ctypes.c_int
         L.fp8_rmsnorm_quant_act.argtypes = [P, P, I, I, I, ctypes.c_float, P, I, P, P, P]
         L.fp8_rmsnorm_quant_act.restype = ctypes.c_int
+        L.fp8_linear_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, P, I, P]
+        L.fp8_linear_swiglu.restype = ctypes.c_int
         L.fp8_linear.argtypes = [P, P, P, P, I, I, I, ctypes.c_int, P, I, P, S, P]
         L.fp8_linear.restype = ctypes.c_int
         L.fp8_linear_workspace_size.argtypes = [I, I, I, ctypes.c_int]
@@ -159,6 +161,28 @@ def fp8_rmsnorm_quant_act(X: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-
                                      _ptr(xs), _ptr(rstd), _stream(X))
     _check(st, "fp8_rmsnorm_quant_act")
     return (Xq, xs, rstd) if return_rstd else (Xq, xs)
+
+
+def fp8_linear_swiglu(Xq: torch.Tensor, x_scale: torch.Tensor, Wq_gate: torch.Tensor, w_scale_gate: torch.Tensor,
+                      Wq_up: torch.Tensor, w_scale_up: torch.Tensor,
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """bf16(bf16(silu(g)) * u) of the gate and up projections (channel/token
+    scales), g and u never written.  -> Y bf16 [M, N]."""
+    _require_cuda(Xq, "Xq", torch.uint8)
+    _require_cuda(Wq_gate, "Wq_gate", torch.uint8)
+    _require_cuda(Wq_up, "Wq_up", torch.uint8)
+    M, K = Xq.shape
+    N = Wq_gate.shape[0]
+    if Wq_gate.shape != (N, K) or Wq_up.shape != (N, K):
+        raise ValueError("Wq_gate and Wq_up must both be [N, K] with Xq's K")
+    if not (Xq.is_contiguous() and Wq_gate.is_contiguous() and Wq_up.is_contiguous()):
+        raise ValueError("Xq, Wq_gate and Wq_up must be contiguous")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    st = lib().fp8_linear_swiglu(_ptr(Xq), _ptr(x_scale), _ptr(Wq_gate), _ptr(w_scale_gate), _ptr(Wq_up),
+                                 _ptr(w_scale_up), M, N, K, _ptr(out), out.stride(0), _stream(Xq))
+    _check(st, "fp8_linear_swiglu")
+    return out
 
 
 def fp8_quant_kv(kv: torch.Tensor, out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):

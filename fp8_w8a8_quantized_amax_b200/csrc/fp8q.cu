@@ -483,6 +483,56 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
   return launch(k, dim3(grid), dim3(192), L::kBytes, stream, ta, tb, tb128, tb64, ty, p);
 }
 
+fp8q_status fp8_linear_swiglu(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq_gate,
+                              const float* w_scale_gate, const uint8_t* Wq_up, const float* w_scale_up, int64_t M,
+                              int64_t N, int64_t K, void* Y_bf16, int64_t ldy, void* stream) {
+  fp8q_status st = check_linear_args(Xq, x_scale, Wq_gate, w_scale_gate, M, N, K, FP8Q_CHANNEL_TOKEN, Y_bf16, ldy);
+  if (st != FP8Q_OK || M == 0) return st;
+  if (!Wq_up || !w_scale_up) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(Wq_up, 16) || !aligned(w_scale_up, 4)) return FP8Q_ERR_MISALIGNED;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
+  using L = fp8q::prefill::PairLayout<kPairStages>;
+  auto k = fp8q::prefill::gemm_swiglu2_kernel<kPairStages>;
+  if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
+  static int max_pairs[kMaxDevices] = {};
+  if (max_pairs[dev] == 0) {
+    cudaLaunchConfig_t qc = {};
+    qc.gridDim = dim3(2 * sms);
+    qc.blockDim = dim3(64 + 32 * L::kEpiWarps);
+    qc.dynamicSmemBytes = L::kBytes;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k, &qc) != cudaSuccess || n < 1) n = sms / 2;
+    max_pairs[dev] = n;
+  }
+  fp8q::prefill::Params p;
+  p.xs = x_scale;
+  p.ws = w_scale_gate;
+  p.y = static_cast<__nv_bfloat16*>(Y_bf16);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.ldy = ldy;
+  p.KB = static_cast<int>((K + 127) / 128);
+  p.num_m = static_cast<int>((M + 255) / 256);
+  p.num_n = static_cast<int>((N + 127) / 128);              // tiles of 128 output channels
+  p.num_tiles = p.num_m * p.num_n;
+  p.group_m = p.num_m < 8 ? p.num_m : 8;
+  const int pairs = max_pairs[dev];
+  tail_split(p.num_tiles, pairs, &p.full, &p.split);
+  const int items = (p.full ? p.full : 0) + (p.num_tiles - p.full) * p.split;
+  const int used = p.full ? pairs : (items < pairs ? items : pairs);
+  CUtensorMap ta, tg, tg64, tu, tu64, ty;
+  if ((st = tmap_u8_sw128(&ta, Xq, M, K, K, 128)) != FP8Q_OK) return st;
+  if ((st = tmap_u8_sw128(&tg, Wq_gate, N, K, K, 128)) != FP8Q_OK) return st;
+  if ((st = tmap_u8_sw128(&tg64, Wq_gate, N, K, K, 64)) != FP8Q_OK) return st;
+  if ((st = tmap_u8_sw128(&tu, Wq_up, N, K, K, 128)) != FP8Q_OK) return st;
+  if ((st = tmap_u8_sw128(&tu64, Wq_up, N, K, K, 64)) != FP8Q_OK) return st;
+  if ((st = tmap_bf16_sw64(&ty, Y_bf16, M, N, ldy, 32)) != FP8Q_OK) return st;
+  return launch(k, dim3(2 * used), dim3(64 + 32 * L::kEpiWarps), L::kBytes, stream, ta, tg, tg64, tu, tu64, ty, p,
+                w_scale_up);
+}
+
 const char* fp8q_status_string(int status) {
   switch (status) {
     case FP8Q_OK: return "FP8Q_OK";

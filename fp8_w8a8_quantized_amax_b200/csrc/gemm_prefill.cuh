@@ -533,6 +533,244 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
   }
 }
 
+// --------------------------------------------- gate/up with SiLU*up, pair ---
+// The Llama MLP's gate and up projections share their input and are combined
+// as silu(gate) * up.  Here one CTA pair computes, for 256 tokens and 128
+// output channels, both linears in one M=256, N=256 MMA per K step: the
+// leader loads the 128 gate rows and its peer the same 128 up rows as their B
+// halves, so TMEM columns [0, 128) hold gate and [128, 256) hold up for the
+// same channels.  The epilogue scales both (x_scale * w_scale, channel mode),
+// rounds them to bf16 as the separate linears would, and writes only
+//   act = bf16( bf16(silu(gate)) * up ),
+// half the output of the two linears and no separate SiLU * up pass.  Tail
+// items of 64 channels use N=128 MMAs.  Schedule, barriers and pipeline are
+// those of gemm_channel2_kernel.
+template <int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
+    gemm_swiglu2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
+                        const __grid_constant__ CUtensorMap tmG64, const __grid_constant__ CUtensorMap tmU,
+                        const __grid_constant__ CUtensorMap tmU64, const __grid_constant__ CUtensorMap tmY,
+                        const Params p, const float* __restrict__ ws_up) {
+  using L = PairLayout<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * L::kA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  constexpr uint32_t kTmemCols = 512;
+  constexpr uint16_t kBoth = 0x3;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * L::kEpiWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(rank == 0 ? &tmG : &tmU);
+    tma_prefetch_desc(rank == 0 ? &tmG64 : &tmU64);
+    tma_prefetch_desc(&tmY);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();
+
+  const int G2 = gridDim.x >> 1;
+  auto count = [&]() {
+    const int tail = (p.num_tiles - p.full) * p.split;
+    return p.full / G2 + (pair < tail ? (tail - 1 - pair) / G2 + 1 : 0);
+  };
+  // Item i: tile (mb, nb) of 256 tokens x 128 channels, channel offset c_off
+  // inside it and its channel count (128, or 64 for a tail half).
+  auto coords = [&](int i, int& mb, int& nb, int& c_off, int& n_ch) {
+    const int nfull = p.full / G2;
+    if (i < nfull) {
+      tile_coords(p, pair + i * G2, mb, nb);
+      c_off = 0;
+      n_ch = 128;
+    } else {
+      const int j = pair + (i - nfull) * G2;
+      tile_coords(p, p.full + j / p.split, mb, nb);
+      n_ch = 128 / p.split;
+      c_off = (j % p.split) * n_ch;
+    }
+  };
+  const int nitems = count();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int i = 0; ok && i < nitems; ++i) {
+        int mb, nb, c_off, n_ch;
+        coords(i, mb, nb, c_off, n_ch);
+        // B rows of this CTA: gate (leader) or up (peer), the item's channels
+        const CUtensorMap* tb = rank == 0 ? (n_ch == 128 ? &tmG : &tmG64) : (n_ch == 128 ? &tmU : &tmU64);
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) { ok = false; break; }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * static_cast<uint32_t>(L::kA + n_ch * BK));
+          const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
+          tma_load_2d_pair(sA + stage * L::kA, &tmA, bar0, kb * BK, mb * 256 + static_cast<int>(rank) * 128, pol);
+          tma_load_2d_pair(sB + stage * L::kB, tb, bar0, kb * BK, nb * 128 + c_off, pol);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      griddep_launch_dependents();
+      for (int i = 0; ok && i < STAGES; ++i) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) break;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int it = 0; ok && it < nitems; ++it) {
+        int mb, nb, c_off, n_ch;
+        coords(it, mb, nb, c_off, n_ch);
+        const uint32_t idesc = idesc_e4m3_f32(256, 2 * n_ch);   // gate and up columns
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag, kErrWaitTmemEmpty)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * 256;
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * L::kA);
+          const uint32_t b0 = smem_u32(sB + stage * L::kB);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k)
+            mma_e4m3_pair(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + k * UMMA_K), idesc,
+                          (kb | k) != 0);
+          mma_commit_pair(&empty[stage], kBoth);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) mma_commit_pair(&tfull[acc], kBoth);
+      }
+    }
+  } else {
+    // 8 epilogue warps: warp w reads TMEM lanes 32*(w%4)..+31 (its 32 rows)
+    // and half of the item's channels, h = (w - 2) / 4: gate
+    // columns [h wc, +wc) and the matching up columns [n_ch + h wc, +wc),
+    // wc = n_ch / 2, in chunks of 32.
+    const int ew = warp - 2;
+    const int quarter = warp & 3;
+    const int h = ew >> 2;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    uint8_t* out_s = smem + L::kOutOff + ew * 2 * L::kOutChunk;
+    const int swz = (lane >> 1) & 3;
+    const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const int N = p.N;                                       // output channels (intermediate size)
+    int buf = 0;
+    for (int it = 0; it < nitems; ++it) {
+      int mb, nb, c_off, n_ch;
+      coords(it, mb, nb, c_off, n_ch);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      const int wc = n_ch / 2;                               // this warp's channels: 64 or 32
+      const int nchunks = wc / 32;
+      const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quarter * 32;
+      const int m = row0 + lane;
+      const float xsm = m < p.M ? __ldg(p.xs + m) : 0.0f;
+      const int ch0 = nb * 128 + c_off + h * wc;             // first output channel of this warp
+      float wg[2], wu[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int n = ch0 + i * 32 + lane;
+        const bool live = i < nchunks && n < N;
+        wg[i] = live ? __ldg(p.ws + n) : 0.0f;
+        wu[i] = live ? __ldg(ws_up + n) : 0.0f;
+      }
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrWaitTmemFull))) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + lane_addr + acc * 256;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (c < nchunks) {
+          uint32_t rg[32], ru[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(tbase + h * wc + c * 32, rg);
+          tmem_ld_32x32b_x32(tbase + n_ch + h * wc + c * 32, ru);
+          tmem_ld_wait_regs(rg);
+          tmem_ld_wait_regs(ru);
+          if (c + 1 == nchunks) {                           // all of this warp's columns read
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + acc * 8);
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float a[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int col = 2 * j + e;
+              const float gsc = __shfl_sync(0xFFFFFFFFu, wg[c], col);
+              const float usc = __shfl_sync(0xFFFFFFFFu, wu[c], col);
+              // the two linears' bf16 outputs
+              const float g = __bfloat162float(__float2bfloat16_rn(__uint_as_float(rg[col]) * xsm * gsc));
+              const float u = __bfloat162float(__float2bfloat16_rn(__uint_as_float(ru[col]) * xsm * usc));
+              const float sl = __bfloat162float(__float2bfloat16_rn(g / (1.0f + __expf(-g))));
+              a[e] = sl * u;                                 // exact in fp32; rounded once below
+            }
+            pk[j] = pack_bf16x2(a[0], a[1]);
+          }
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          uint8_t* sb = out_s + buf * L::kOutChunk;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(sb + lane * 64 + ((q ^ swz) << 4)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          const int col0 = ch0 + c * 32;
+          if (lane == 0 && row0 < p.M && col0 < N) {
+            tma_store_2d(&tmY, sb, col0, row0);
+            bulk_commit();
+          }
+          buf ^= 1;
+        }
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 // ------------------------------------------------------- block, CTA pair ---
 // Block-scaled GEMM on 256 x 256 tiles computed by a CTA pair, with the same
 // operand split as the channel pair kernel (32 KB per CTA per 128-wide K

@@ -156,6 +156,25 @@ FP8Q_API fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const u
                        void* Y_bf16, int64_t ldy, void* workspace, size_t workspace_bytes,
                        void* stream);
 
+/*
+ * fp8_linear_swiglu -- the Llama MLP's gate and up projections and their
+ * SwiGLU combination in one kernel ("Llama 3 精读实录" section 1.3: gate and up
+ * computed separately, then silu(gate) * up):
+ *   g = bf16(Xq . Wq_gate^T scaled),  u = bf16(Xq . Wq_up^T scaled)   (as fp8_linear)
+ *   Y = bf16( bf16(silu(g)) * u ),   silu(v) = v / (1 + e^-v)
+ * Only Y ([M, N], the down projection's input) is written.
+ *   Xq, x_scale      as fp8_linear, FP8Q_CHANNEL_TOKEN scales ([M]).
+ *   Wq_gate, Wq_up   [N, K] codes of the two weights (contiguous, 16-byte aligned);
+ *   w_scale_gate/up  [N] fp32 per-channel scales.
+ *   Y_bf16           [M, ldy] bf16, written (rules as fp8_linear).
+ * Requirements as fp8_linear in channel mode.  Any M >= 1 runs the CTA-pair
+ * prefill schedule (256 tokens x 128 channels per pair).  silu uses the fast
+ * exponential; g and u match fp8_linear's outputs.  No workspace.
+ */
+FP8Q_API fp8q_status fp8_linear_swiglu(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq_gate,
+                                       const float* w_scale_gate, const uint8_t* Wq_up, const float* w_scale_up,
+                                       int64_t M, int64_t N, int64_t K, void* Y_bf16, int64_t ldy, void* stream);
+
 /* Bytes of workspace fp8_linear needs for this problem on the current device
  * (0 for the prefill path).  Returns 0 for invalid arguments as well. */
 FP8Q_API size_t fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int mode);

@@ -99,6 +99,25 @@ def test_quant_act_argument_checks(L, kw, want):
     assert q_act(L, **kw) == want
 
 
+def swi(L, M=4, N=64, K=256, y=P, ldy=64, xq=P, xs=P, wg=P, sg=P, wu=P, su=P):
+    return L.fp8_linear_swiglu(xq, xs, wg, sg, wu, su, M, N, K, y, ldy, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(wu=None), fq.ERR_INVALID_ARG),
+    (dict(su=None), fq.ERR_INVALID_ARG),
+    (dict(wg=None), fq.ERR_INVALID_ARG),
+    (dict(K=24), fq.ERR_INVALID_ARG),
+    (dict(N=24, ldy=24), fq.ERR_INVALID_ARG),
+    (dict(ldy=32), fq.ERR_INVALID_ARG),
+    (dict(wu=BAD), fq.ERR_MISALIGNED),
+    (dict(su=P + 2), fq.ERR_MISALIGNED),
+    (dict(M=0, xq=None, xs=None, wg=None, sg=None, wu=None, su=None, y=None), fq.OK),
+])
+def test_swiglu_argument_checks(L, kw, want):
+    assert swi(L, **kw) == want
+
+
 def rms_q(L, x=P, g=P, M=4, K=256, ldx=256, eps=1e-5, q=P, ldq=256, s=P, r=None):
     return L.fp8_rmsnorm_quant_act(x, g, M, K, ldx, eps, q, ldq, s, r, None)
 
@@ -166,6 +185,7 @@ def test_valid_arguments_without_a_gpu_report_cuda_error(L):
     assert q_w(L) == fq.ERR_CUDA
     assert lin(L) == fq.ERR_CUDA
     assert rms_q(L) == fq.ERR_CUDA
+    assert swi(L) == fq.ERR_CUDA
 
 
 def test_binding_refuses_cpu_tensors(L):

@@ -52,7 +52,8 @@ def lib() -> ctypes.CDLL:
         _lib.orc_e4m3_encode.restype = ctypes.c_uint8
         _lib.orc_e4m3_encode_n.argtypes = [P, I, P]
         _lib.orc_e4m3_encode_n.restype = None
-        for f in ("orc_quant_rows", "orc_quant_groups128", "orc_quant_blocks128"):
+        for f in ("orc_quant_rows", "orc_quant_groups128", "orc_quant_blocks128",
+                  "orc_quant_rows_s16", "orc_quant_groups128_s16", "orc_quant_blocks128_s16"):
             getattr(_lib, f).argtypes = [P, I, I, I, P, I, P]
             getattr(_lib, f).restype = None
         _lib.orc_linear.argtypes = [P, P, P, P, I, I, I, I, I, ctypes.c_int, P]
@@ -101,13 +102,14 @@ def e4m3_encode_array(v: np.ndarray) -> np.ndarray:
     return out
 
 
-def quant_rows(x):
-    """One amax/448 scale per row.  x: bf16 [R, K] -> (codes u8 [R, K], scales f32 [R])."""
+def quant_rows(x, scale_bf16: bool = False):
+    """One amax/448 scale per row.  x: bf16 [R, K] -> (codes u8 [R, K], scales f32 [R]).
+    scale_bf16: round each scale to bf16 before computing the codes."""
     xb = _bits(x)
     R, K = xb.shape
     q = np.empty((R, K), np.uint8)
     s = np.empty((R,), np.float32)
-    lib().orc_quant_rows(_p(xb), R, K, K, _p(q), K, _p(s))
+    (lib().orc_quant_rows_s16 if scale_bf16 else lib().orc_quant_rows)(_p(xb), R, K, K, _p(q), K, _p(s))
     return q, s
 
 
@@ -153,34 +155,34 @@ def rmsnorm_quant_rows(x, gamma, rstd=None, eps: float = 1e-5):
     return q, s, y, r
 
 
-def quant_groups128(x):
+def quant_groups128(x, scale_bf16: bool = False):
     """One scale per 128-group of each row.  -> (codes [M, K], scales [M, K/128])."""
     xb = _bits(x)
     M, K = xb.shape
     assert K % 128 == 0
     q = np.empty((M, K), np.uint8)
     s = np.empty((M, K // 128), np.float32)
-    lib().orc_quant_groups128(_p(xb), M, K, K, _p(q), K, _p(s))
+    (lib().orc_quant_groups128_s16 if scale_bf16 else lib().orc_quant_groups128)(_p(xb), M, K, K, _p(q), K, _p(s))
     return q, s
 
 
-def quant_blocks128(w):
+def quant_blocks128(w, scale_bf16: bool = False):
     """One scale per 128x128 tile.  -> (codes [N, K], scales [ceil(N/128), K/128])."""
     wb = _bits(w)
     N, K = wb.shape
     assert K % 128 == 0
     q = np.empty((N, K), np.uint8)
     s = np.empty(((N + 127) // 128, K // 128), np.float32)
-    lib().orc_quant_blocks128(_p(wb), N, K, K, _p(q), K, _p(s))
+    (lib().orc_quant_blocks128_s16 if scale_bf16 else lib().orc_quant_blocks128)(_p(wb), N, K, K, _p(q), K, _p(s))
     return q, s
 
 
-def quant_weight(w, mode: int):
-    return quant_rows(w) if mode == CHANNEL_TOKEN else quant_blocks128(w)
+def quant_weight(w, mode: int, scale_bf16: bool = False):
+    return quant_rows(w, scale_bf16) if mode == CHANNEL_TOKEN else quant_blocks128(w, scale_bf16)
 
 
-def quant_act(x, mode: int):
-    return quant_rows(x) if mode == CHANNEL_TOKEN else quant_groups128(x)
+def quant_act(x, mode: int, scale_bf16: bool = False):
+    return quant_rows(x, scale_bf16) if mode == CHANNEL_TOKEN else quant_groups128(x, scale_bf16)
 
 
 def linear(xq, xs, wq, ws, mode: int) -> np.ndarray:

@@ -130,6 +130,18 @@ static float scale_from_amax(float amax) {
     return num / 448.0f;
 }
 
+static uint16_t float_to_bf16(float f);
+
+/* The scale rounded to bf16, the dtype the FP8 checkpoints store scales in
+ * (reading: the 72.67 GB of [P4] section 二 matches bf16 scales), before the
+ * codes are computed, so that the codes are those a bf16-scale checkpoint
+ * holds.  A scale that rounds to zero (amax below 448 * 2^-134) becomes 1,
+ * like amax = 0: every code of such a unit is zero either way. */
+static float scale_to_bf16(float s) {
+    float r = bf16_to_float(float_to_bf16(s));
+    return r == 0.0f ? 1.0f : r;
+}
+
 static inline uint8_t code_of(float x, float s) {
     volatile float q = x / s;             /* fp32 quotient, RNE */
     return orc_e4m3_encode(q);
@@ -138,8 +150,8 @@ static inline uint8_t code_of(float x, float s) {
 /* One scale per row: per-token activations [P2, P4] and per-output-channel
  * weights [P2] are the same operation on X[M,K] and on W[N,K].
  * x: bf16 bits [rows, ld], q: [rows, ldq], s: [rows]. */
-ORC_EXPORT void orc_quant_rows(const uint16_t* x, int64_t rows, int64_t K, int64_t ld,
-                               uint8_t* q, int64_t ldq, float* s) {
+static void quant_rows_impl(const uint16_t* x, int64_t rows, int64_t K, int64_t ld,
+                            uint8_t* q, int64_t ldq, float* s, int scale_bf16) {
     for (int64_t r = 0; r < rows; ++r) {
         float amax = 0.0f;
         for (int64_t k = 0; k < K; ++k) {
@@ -147,6 +159,7 @@ ORC_EXPORT void orc_quant_rows(const uint16_t* x, int64_t rows, int64_t K, int64
             if (a > amax) amax = a;
         }
         float sr = scale_from_amax(amax);
+        if (scale_bf16) sr = scale_to_bf16(sr);
         s[r] = sr;
         for (int64_t k = 0; k < K; ++k) q[r * ldq + k] = code_of(bf16_to_float(x[r * ld + k]), sr);
     }
@@ -217,8 +230,8 @@ ORC_EXPORT void orc_rmsnorm_quant_rows(const uint16_t* x, const uint16_t* gamma,
 
 /* One scale per 128 consecutive input features of each token [P5].
  * K must be a multiple of 128.  s: [M, K/128] row-major. */
-ORC_EXPORT void orc_quant_groups128(const uint16_t* x, int64_t M, int64_t K, int64_t ld,
-                                    uint8_t* q, int64_t ldq, float* s) {
+static void quant_groups128_impl(const uint16_t* x, int64_t M, int64_t K, int64_t ld,
+                                 uint8_t* q, int64_t ldq, float* s, int scale_bf16) {
     int64_t G = K / 128;
     for (int64_t m = 0; m < M; ++m) {
         for (int64_t g = 0; g < G; ++g) {
@@ -228,6 +241,7 @@ ORC_EXPORT void orc_quant_groups128(const uint16_t* x, int64_t M, int64_t K, int
                 if (a > amax) amax = a;
             }
             float sg = scale_from_amax(amax);
+            if (scale_bf16) sg = scale_to_bf16(sg);
             s[m * G + g] = sg;
             for (int64_t k = g * 128; k < g * 128 + 128; ++k)
                 q[m * ldq + k] = code_of(bf16_to_float(x[m * ld + k]), sg);
@@ -238,8 +252,8 @@ ORC_EXPORT void orc_quant_groups128(const uint16_t* x, int64_t M, int64_t K, int
 /* One scale per 128 x 128 tile of W[N,K] [P5, block_structure [128, 128]].
  * K must be a multiple of 128; the last row-tile may be shorter than 128
  * (amax over the rows that exist).  s: [ceil(N/128), K/128] row-major. */
-ORC_EXPORT void orc_quant_blocks128(const uint16_t* w, int64_t N, int64_t K, int64_t ld,
-                                    uint8_t* q, int64_t ldq, float* s) {
+static void quant_blocks128_impl(const uint16_t* w, int64_t N, int64_t K, int64_t ld,
+                                 uint8_t* q, int64_t ldq, float* s, int scale_bf16) {
     int64_t NB = (N + 127) / 128, KB = K / 128;
     for (int64_t nb = 0; nb < NB; ++nb) {
         int64_t n1 = (nb + 1) * 128 < N ? (nb + 1) * 128 : N;
@@ -251,12 +265,39 @@ ORC_EXPORT void orc_quant_blocks128(const uint16_t* w, int64_t N, int64_t K, int
                     if (a > amax) amax = a;
                 }
             float sb = scale_from_amax(amax);
+            if (scale_bf16) sb = scale_to_bf16(sb);
             s[nb * KB + kb] = sb;
             for (int64_t n = nb * 128; n < n1; ++n)
                 for (int64_t k = kb * 128; k < kb * 128 + 128; ++k)
                     q[n * ldq + k] = code_of(bf16_to_float(w[n * ld + k]), sb);
         }
     }
+}
+
+/* Exported forms: fp32 scales, and scales rounded to bf16 first ("_s16"). */
+ORC_EXPORT void orc_quant_rows(const uint16_t* x, int64_t rows, int64_t K, int64_t ld,
+                               uint8_t* q, int64_t ldq, float* s) {
+    quant_rows_impl(x, rows, K, ld, q, ldq, s, 0);
+}
+ORC_EXPORT void orc_quant_groups128(const uint16_t* x, int64_t M, int64_t K, int64_t ld,
+                                    uint8_t* q, int64_t ldq, float* s) {
+    quant_groups128_impl(x, M, K, ld, q, ldq, s, 0);
+}
+ORC_EXPORT void orc_quant_blocks128(const uint16_t* w, int64_t N, int64_t K, int64_t ld,
+                                    uint8_t* q, int64_t ldq, float* s) {
+    quant_blocks128_impl(w, N, K, ld, q, ldq, s, 0);
+}
+ORC_EXPORT void orc_quant_rows_s16(const uint16_t* x, int64_t rows, int64_t K, int64_t ld,
+                                   uint8_t* q, int64_t ldq, float* s) {
+    quant_rows_impl(x, rows, K, ld, q, ldq, s, 1);
+}
+ORC_EXPORT void orc_quant_groups128_s16(const uint16_t* x, int64_t M, int64_t K, int64_t ld,
+                                        uint8_t* q, int64_t ldq, float* s) {
+    quant_groups128_impl(x, M, K, ld, q, ldq, s, 1);
+}
+ORC_EXPORT void orc_quant_blocks128_s16(const uint16_t* w, int64_t N, int64_t K, int64_t ld,
+                                        uint8_t* q, int64_t ldq, float* s) {
+    quant_blocks128_impl(w, N, K, ld, q, ldq, s, 1);
 }
 
 /* ----------------------------------------------------------------- linear */

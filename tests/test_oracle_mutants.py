@@ -46,6 +46,7 @@ MUTANTS = {
     "swiglu sigmoid sign": (r"exp\(-gb\)", "exp(gb)"),
     "swiglu up dropped": (r"volatile float p = bf16_to_float\(sb\) \* \(float\)ub;",
                           "volatile float p = bf16_to_float(sb);"),
+    "bf16 scale not rounded": (r"float r = bf16_to_float\(float_to_bf16\(s\)\);", "float r = s;"),
 }
 
 
@@ -60,7 +61,7 @@ def build_variant(src_text, tmp):
     L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
     L.orc_e4m3_decode.restype = ctypes.c_double
     L.orc_e4m3_encode_n.argtypes = [P, I, P]
-    for f in ("orc_quant_rows", "orc_quant_groups128", "orc_quant_blocks128"):
+    for f in ("orc_quant_rows", "orc_quant_groups128", "orc_quant_blocks128", "orc_quant_rows_s16"):
         getattr(L, f).argtypes = [P, I, I, I, P, I, P]
     L.orc_linear.argtypes = [P, P, P, P, I, I, I, I, I, ctypes.c_int, P]
     L.orc_rmsnorm_rstd.argtypes = [P, I, I, I, ctypes.c_float, P]
@@ -116,6 +117,13 @@ def checks(L):
         .view(torch.uint8).numpy()
     if not np.array_equal(qd, want):
         failed.append("IEEE division")
+    # scales rounded to bf16 before the codes: the rounded fp32 scales, codes by argmin
+    q16 = np.empty((8, 256), np.uint8)
+    s16 = np.empty(8, np.float32)
+    L.orc_quant_rows_s16(_p(xb), 8, 256, 256, _p(q16), 256, _p(s16))
+    if not np.array_equal(s16, torch.from_numpy(s.copy()).to(torch.bfloat16).float().numpy()) or \
+            not np.array_equal(q16.ravel(), _pins.encode_argmin((x.float().numpy() / s16[:, None]).astype(np.float32).ravel())):
+        failed.append("bf16 scales")
     z = np.zeros((2, 256), np.uint16)
     qz = np.empty((2, 256), np.uint8)
     sz = np.empty(2, np.float32)

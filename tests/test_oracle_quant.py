@@ -191,3 +191,49 @@ def test_codes_follow_ieee_division(amax):
         .to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     assert np.any(want != recip)          # the case really separates the two readings
     assert np.array_equal(q, want)
+
+
+# ------------------------------------------------- scales rounded to bf16
+# The FP8 checkpoints store bf16 scales (the 70B byte count pins it, see
+# test_policy.py); with scale_bf16 the scale is rounded to bf16 before the
+# codes are computed, so the codes are those of a bf16-scale checkpoint.
+
+def _bf16_round(a: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).float().numpy()
+
+
+@pytest.mark.parametrize("kind", ["rows", "groups", "blocks"])
+def test_bf16_scales_are_the_rounded_fp32_scales(kind):
+    x = synth.make_x(300, 512, seed=21)
+    f = {"rows": oracle.quant_rows, "groups": oracle.quant_groups128, "blocks": oracle.quant_blocks128}[kind]
+    _, s32 = f(x)
+    q16, s16 = f(x, scale_bf16=True)
+    assert np.array_equal(s16, _bf16_round(s32))
+    # codes: the nearest E4M3 value of fl32(x / s16), by the independent argmin encoder
+    xf = x.float().numpy()
+    if kind == "rows":
+        sx = np.repeat(s16[:, None], 512, axis=1)
+    elif kind == "groups":
+        sx = np.repeat(s16, 128, axis=1)
+    else:
+        sx = np.repeat(np.repeat(s16, 128, axis=0)[:300], 128, axis=1)
+    quot = (xf / sx).astype(np.float32)
+    assert np.array_equal(q16.ravel(), _pins.encode_argmin(quot.ravel()))
+
+
+def test_bf16_scale_rounding_down_saturates_the_max_element():
+    # amax = 1632: 1632/448 = 3.642857 rounds to bf16 3.640625 (down), so
+    # amax / s = 448.28 > 448 and the max element saturates to 0x7E
+    x = torch.zeros(1, 16, dtype=torch.bfloat16)
+    x[0, 0] = 1632.0
+    x[0, 1] = -1632.0
+    q, s = oracle.quant_rows(x, scale_bf16=True)
+    assert s[0] == np.float32(3.640625)
+    assert q[0, 0] == 0x7E and q[0, 1] == 0xFE
+
+
+def test_bf16_scale_of_zero_and_tiny_units_is_one():
+    x = torch.zeros(2, 16, dtype=torch.bfloat16)
+    x[1, 3] = 2.0 ** -133                        # amax/448 rounds to zero in bf16
+    q, s = oracle.quant_rows(x, scale_bf16=True)
+    assert np.all(s == 1.0) and np.all(q == 0)

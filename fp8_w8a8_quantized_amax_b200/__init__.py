@@ -26,6 +26,7 @@ from .policy import DEFAULT_IGNORE, should_quantize  # noqa: F401
 
 CHANNEL_TOKEN = 0
 BLOCK128 = 1
+SCALE_BF16 = 0x10      # option OR'ed into a quantizer's mode: scales rounded to bf16 before the codes
 
 OK = 0
 ERR_INVALID_ARG = 1
@@ -104,11 +105,11 @@ def _require_cuda(t: torch.Tensor, name: str, dtype) -> None:
 
 
 def scale_shape_weight(N: int, K: int, mode: int) -> Tuple[int, ...]:
-    return (N,) if mode == CHANNEL_TOKEN else ((N + 127) // 128, K // 128)
+    return (N,) if (mode & ~SCALE_BF16) == CHANNEL_TOKEN else ((N + 127) // 128, K // 128)
 
 
 def scale_shape_act(M: int, K: int, mode: int) -> Tuple[int, ...]:
-    return (M,) if mode == CHANNEL_TOKEN else (M, K // 128)
+    return (M,) if (mode & ~SCALE_BF16) == CHANNEL_TOKEN else (M, K // 128)
 
 
 def fp8_quant_weight(W: torch.Tensor, mode: int = CHANNEL_TOKEN,

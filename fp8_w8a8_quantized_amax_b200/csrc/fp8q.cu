@@ -137,9 +137,16 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 // ------------------------------------------------------------ quantization ---
 
+// A mode is FP8Q_CHANNEL_TOKEN or FP8Q_BLOCK128, optionally OR'ed with FP8Q_SCALE_BF16.
+bool valid_mode(int mode) {
+  const int base = mode & ~FP8Q_SCALE_BF16;
+  return base == FP8Q_CHANNEL_TOKEN || base == FP8Q_BLOCK128;
+}
+
 fp8q_status check_quant_args(const void* src, int64_t rows, int64_t K, int64_t ld, int mode, const uint8_t* q,
                              int64_t ldq, const float* s) {
-  if (mode != FP8Q_CHANNEL_TOKEN && mode != FP8Q_BLOCK128) return FP8Q_ERR_INVALID_ARG;
+  if (!valid_mode(mode)) return FP8Q_ERR_INVALID_ARG;
+  mode &= ~FP8Q_SCALE_BF16;
   if (rows < 0 || K <= 0 || ld < K || ldq < K) return FP8Q_ERR_INVALID_ARG;
   if (K % 16 != 0) return FP8Q_ERR_INVALID_ARG;
   if (mode == FP8Q_BLOCK128 && K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
@@ -152,18 +159,18 @@ fp8q_status check_quant_args(const void* src, int64_t rows, int64_t K, int64_t l
 }
 
 fp8q_status launch_rows(const uint16_t* x, int64_t rows, int K, int64_t ldx, uint8_t* q, int64_t ldq, float* s,
-                        void* stream) {
+                        bool s16, void* stream) {
   const int nvec = K / 8;
   int T = 32 * ((nvec + 32 * 8 - 1) / (32 * 8));
   if (T > 1024) T = 1024;
   const int need = (nvec + T - 1) / T;
   const dim3 grid(static_cast<unsigned>(rows));
   const dim3 block(T);
-  if (need <= 1) return launch(fp8q::quant_rows_kernel<1>, grid, block, 0, stream, x, K, ldx, q, ldq, s);
-  if (need <= 2) return launch(fp8q::quant_rows_kernel<2>, grid, block, 0, stream, x, K, ldx, q, ldq, s);
-  if (need <= 4) return launch(fp8q::quant_rows_kernel<4>, grid, block, 0, stream, x, K, ldx, q, ldq, s);
-  if (need <= 8) return launch(fp8q::quant_rows_kernel<8>, grid, block, 0, stream, x, K, ldx, q, ldq, s);
-  if (need <= 16) return launch(fp8q::quant_rows_kernel<16>, grid, block, 0, stream, x, K, ldx, q, ldq, s);
+  if (need <= 1) return launch(fp8q::quant_rows_kernel<1>, grid, block, 0, stream, x, K, ldx, q, ldq, s, s16);
+  if (need <= 2) return launch(fp8q::quant_rows_kernel<2>, grid, block, 0, stream, x, K, ldx, q, ldq, s, s16);
+  if (need <= 4) return launch(fp8q::quant_rows_kernel<4>, grid, block, 0, stream, x, K, ldx, q, ldq, s, s16);
+  if (need <= 8) return launch(fp8q::quant_rows_kernel<8>, grid, block, 0, stream, x, K, ldx, q, ldq, s, s16);
+  if (need <= 16) return launch(fp8q::quant_rows_kernel<16>, grid, block, 0, stream, x, K, ldx, q, ldq, s, s16);
   return FP8Q_ERR_UNSUPPORTED;   // K > 131072
 }
 
@@ -251,7 +258,8 @@ void decode_bind_workspace(Params& p, void* ws, void* Y, int64_t ldy) {
 
 fp8q_status check_linear_args(const uint8_t* Xq, const float* xs, const uint8_t* Wq, const float* ws, int64_t M,
                               int64_t N, int64_t K, int mode, const void* Y, int64_t ldy) {
-  if (mode != FP8Q_CHANNEL_TOKEN && mode != FP8Q_BLOCK128) return FP8Q_ERR_INVALID_ARG;
+  if (!valid_mode(mode)) return FP8Q_ERR_INVALID_ARG;
+  mode &= ~FP8Q_SCALE_BF16;
   if (M < 0 || N <= 0 || K <= 0 || ldy < N) return FP8Q_ERR_INVALID_ARG;
   if (K % 16 != 0 || N % 16 != 0) return FP8Q_ERR_INVALID_ARG;
   if (mode == FP8Q_BLOCK128 && K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
@@ -307,11 +315,14 @@ fp8q_status fp8_quant_weight(const void* W_bf16, int64_t N, int64_t K, int64_t l
   int dev, sms;
   if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
   const uint16_t* w = static_cast<const uint16_t*>(W_bf16);
-  if (mode == FP8Q_CHANNEL_TOKEN) return launch_rows(w, N, static_cast<int>(K), ldw, Wq, ldwq, w_scale, stream);
+  const bool s16 = (mode & FP8Q_SCALE_BF16) != 0;
+  mode &= ~FP8Q_SCALE_BF16;
+  if (mode == FP8Q_CHANNEL_TOKEN)
+    return launch_rows(w, N, static_cast<int>(K), ldw, Wq, ldwq, w_scale, s16, stream);
   const int64_t NB = (N + 127) / 128;
   if (NB > 65535) return FP8Q_ERR_UNSUPPORTED;
   return launch(fp8q::quant_blocks128_kernel, dim3(static_cast<unsigned>(K / 128), static_cast<unsigned>(NB)),
-                dim3(256), 0, stream, w, N, static_cast<int>(K / 128), ldw, Wq, ldwq, w_scale);
+                dim3(256), 0, stream, w, N, static_cast<int>(K / 128), ldw, Wq, ldwq, w_scale, s16);
 }
 
 fp8q_status fp8_quant_act(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, int mode, uint8_t* Xq,
@@ -321,14 +332,17 @@ fp8q_status fp8_quant_act(const void* X_bf16, int64_t M, int64_t K, int64_t ldx,
   int dev, sms;
   if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
   const uint16_t* x = static_cast<const uint16_t*>(X_bf16);
-  if (mode == FP8Q_CHANNEL_TOKEN) return launch_rows(x, M, static_cast<int>(K), ldx, Xq, ldxq, x_scale, stream);
+  const bool s16 = (mode & FP8Q_SCALE_BF16) != 0;
+  mode &= ~FP8Q_SCALE_BF16;
+  if (mode == FP8Q_CHANNEL_TOKEN)
+    return launch_rows(x, M, static_cast<int>(K), ldx, Xq, ldxq, x_scale, s16, stream);
   constexpr int GPT = 4;
   const int G = static_cast<int>(K / 128);
   const int64_t total = M * G;
   int64_t grid = (total + 16 * GPT - 1) / (16 * GPT);
   if (grid > static_cast<int64_t>(sms) * 16) grid = static_cast<int64_t>(sms) * 16;
   return launch(fp8q::quant_groups128_kernel<GPT>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream, x, M,
-                G, ldx, Xq, ldxq, x_scale);
+                G, ldx, Xq, ldxq, x_scale, s16);
 }
 
 fp8q_status fp8_rmsnorm_quant_act(const void* X_bf16, const void* gamma_bf16, int64_t M, int64_t K, int64_t ldx,
@@ -346,7 +360,8 @@ fp8q_status fp8_rmsnorm_quant_act(const void* X_bf16, const void* gamma_bf16, in
 }
 
 size_t fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int mode) {
-  if (mode != FP8Q_CHANNEL_TOKEN && mode != FP8Q_BLOCK128) return 0;
+  if (!valid_mode(mode)) return 0;
+  mode &= ~FP8Q_SCALE_BF16;
   if (M <= 0 || M > kDecodeMaxM || N <= 0 || K <= 0) return 0;
   int dev, sms;
   if (current_device(&dev, &sms) != FP8Q_OK) return 0;
@@ -361,6 +376,7 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
                        size_t workspace_bytes, void* stream) {
   fp8q_status st = check_linear_args(Xq, x_scale, Wq, w_scale, M, N, K, mode, Y_bf16, ldy);
   if (st != FP8Q_OK || M == 0) return st;
+  mode &= ~FP8Q_SCALE_BF16;                     // the scale option concerns quantization only
   int dev, sms;
   if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
   const int KB = static_cast<int>((K + 127) / 128);
@@ -599,6 +615,7 @@ fp8q_status fp8_linear_noalloc(const uint8_t* Xq, const float* x_scale, const ui
                                void* stream) {
   fp8q_status st = check_linear_args(Xq, x_scale, Wq, w_scale, M, N, K, mode, Y_bf16, ldy);
   if (st != FP8Q_OK || M == 0) return st;
+  mode &= ~FP8Q_SCALE_BF16;                     // the scale option concerns quantization only
   if (M > kDecodeMaxM) return FP8Q_ERR_UNSUPPORTED;    // the M > 64 path of fp8_linear needs no scratch
   int dev, sms;
   if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;

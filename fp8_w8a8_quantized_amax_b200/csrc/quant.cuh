@@ -32,6 +32,13 @@ __device__ __forceinline__ float amax_bits_to_float(uint32_t bits16) { return __
 
 __device__ __forceinline__ float scale_of(float amax) { return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f); }
 
+// The scale rounded to bf16 (the checkpoints' scale dtype) before the codes are
+// computed; a scale that rounds to zero becomes 1 (all codes of its unit are 0).
+__device__ __forceinline__ float scale_bf16(float s) {
+  const float r = __bfloat162float(__float2bfloat16_rn(s));
+  return r == 0.0f ? 1.0f : r;
+}
+
 // x / s, correctly rounded (identical to __fdiv_rn), for many x and one s.
 // With y = RN(1/s) and q = RN(x * y) within one ulp of x / s, Markstein's
 // correction step q' = RN(q + RN(x - q*s) * y) -- the residual x - q*s being
@@ -99,7 +106,7 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
 template <int VPT>
 __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __restrict__ x, int K, int64_t ldx,
                                                          uint8_t* __restrict__ q, int64_t ldq,
-                                                         float* __restrict__ s) {
+                                                         float* __restrict__ s, bool s16) {
   __shared__ uint32_t red[32];
   griddep_wait();
   const int64_t r = blockIdx.x;
@@ -124,7 +131,8 @@ __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __rest
     m = lane_id() < nw ? red[lane_id()] : 0u;
     m = __reduce_max_sync(0xFFFFFFFFu, m);
   }
-  const float sc = scale_of(amax_bits_to_float(m));
+  float sc = scale_of(amax_bits_to_float(m));
+  if (s16) sc = scale_bf16(sc);
   if (threadIdx.x == 0) s[r] = sc;
   const Divider dv = make_divider(sc);
   uint8_t* qr = q + r * ldq;
@@ -271,7 +279,7 @@ __global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t*
 template <int GPT>
 __global__ void __launch_bounds__(256) quant_groups128_kernel(const uint16_t* __restrict__ x, int64_t M, int G,
                                                              int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
-                                                             float* __restrict__ s) {
+                                                             float* __restrict__ s, bool s16) {
   griddep_wait();
   const int64_t total = M * static_cast<int64_t>(G);
   const int sub = threadIdx.x & 15;
@@ -297,7 +305,8 @@ __global__ void __launch_bounds__(256) quant_groups128_kernel(const uint16_t* __
         mm = max(mm, __shfl_xor_sync(half_mask, mm, 4, 16));
         mm = max(mm, __shfl_xor_sync(half_mask, mm, 2, 16));
         mm = max(mm, __shfl_xor_sync(half_mask, mm, 1, 16));
-        const float sc = scale_of(amax_bits_to_float(mm));
+        float sc = scale_of(amax_bits_to_float(mm));
+        if (s16) sc = scale_bf16(sc);
         const int64_t m = gi / G, g = gi - m * G;
         if (sub == 0) s[gi] = sc;
         const Divider dv = make_divider(sc);
@@ -314,7 +323,7 @@ __global__ void __launch_bounds__(256) quant_groups128_kernel(const uint16_t* __
 // (the last row-block may be short) and take no part in the amax.
 __global__ void __launch_bounds__(256) quant_blocks128_kernel(const uint16_t* __restrict__ w, int64_t N, int KB,
                                                              int64_t ldw, uint8_t* __restrict__ q, int64_t ldq,
-                                                             float* __restrict__ s) {
+                                                             float* __restrict__ s, bool s16) {
   __shared__ uint32_t red[8];
   griddep_wait();
   const int kb = blockIdx.x;
@@ -336,7 +345,8 @@ __global__ void __launch_bounds__(256) quant_blocks128_kernel(const uint16_t* __
   __syncthreads();
   m = lane_id() < 8 ? red[lane_id()] : 0u;
   m = __reduce_max_sync(0xFFFFFFFFu, m);
-  const float sc = scale_of(amax_bits_to_float(m));
+  float sc = scale_of(amax_bits_to_float(m));
+  if (s16) sc = scale_bf16(sc);
   if (threadIdx.x == 0) s[nb * KB + kb] = sc;
   const Divider dv = make_divider(sc);
 #pragma unroll

@@ -68,7 +68,12 @@ typedef enum {
 
 typedef enum {
     FP8Q_CHANNEL_TOKEN = 0,       /* W: one scale per output channel; X: one per token  */
-    FP8Q_BLOCK128 = 1             /* W: one per 128x128 block;  X: one per 128-group     */
+    FP8Q_BLOCK128 = 1,            /* W: one per 128x128 block;  X: one per 128-group     */
+    /* Option, OR'ed into the mode of fp8_quant_weight / fp8_quant_act: round
+     * every scale to bf16 before the codes are computed (the FP8 checkpoints
+     * store bf16 scales), so the codes are those a bf16-scale checkpoint holds.
+     * A scale that rounds to zero becomes 1.  fp8_linear accepts and ignores it. */
+    FP8Q_SCALE_BF16 = 0x10
 } fp8q_mode;
 
 /*

@@ -94,6 +94,10 @@ def lin(L, M=4, N=64, K=256, mode=0, y=P, ldy=64, xq=P, xs=P, wq=P, ws=P, wsp=P,
     (dict(ldq=264), fq.ERR_MISALIGNED),
     (dict(mode=1, K=192, ldx=192, ldq=192), fq.ERR_INVALID_ARG),   # block mode needs K % 128
     (dict(M=0, x=None, q=None, s=None), fq.OK),              # empty input is a no-op
+    (dict(mode=0x12), fq.ERR_INVALID_ARG),                   # the bf16-scale option on an unknown mode
+    (dict(mode=0x20), fq.ERR_INVALID_ARG),                   # an unknown option
+    (dict(mode=0x11, K=192, ldx=192, ldq=192), fq.ERR_INVALID_ARG),   # block mode with the option: K % 128
+    (dict(mode=0x10, M=0, x=None, q=None, s=None), fq.OK),
 ])
 def test_quant_act_argument_checks(L, kw, want):
     assert q_act(L, **kw) == want

@@ -185,3 +185,36 @@ def test_kv_cache_per_token_per_head(T, H):
     assert tuple(q.shape) == (T, H, 128) and tuple(s.shape) == (T, H)
     P.assert_codes_equal(q.view(T, H * 128), rq, f"kv {T}x{H}")
     P.assert_scales_equal(s, rs, f"kv {T}x{H}")
+
+
+@pytest.mark.parametrize("mode", [fq.CHANNEL_TOKEN, fq.BLOCK128])
+def test_bf16_scale_option_bit_exact(mode):
+    # scales rounded to bf16 before the codes (the checkpoints' scale dtype)
+    x = synth.make_x(300, 1024, seed=31)
+    w = synth.make_w(528, 1024, seed=31)     # N % 128 = 16: a partial last weight block
+    q, s = fq.fp8_quant_act(x.to(DEV), mode | fq.SCALE_BF16)
+    rq, rs = oracle.quant_act(x, mode, scale_bf16=True)
+    P.assert_codes_equal(q, rq, f"act bf16 scales mode {mode}")
+    P.assert_scales_equal(s, rs, f"act bf16 scales mode {mode}")
+    qw, sw = fq.fp8_quant_weight(w.to(DEV), mode | fq.SCALE_BF16)
+    rqw, rsw = oracle.quant_weight(w, mode, scale_bf16=True)
+    P.assert_codes_equal(qw, rqw, f"weight bf16 scales mode {mode}")
+    P.assert_scales_equal(sw, rsw, f"weight bf16 scales mode {mode}")
+    # the linear accepts the option and ignores it
+    y1 = fq.fp8_linear(q, s, qw, sw, mode | fq.SCALE_BF16)
+    y0 = fq.fp8_linear(q, s, qw, sw, mode)
+    assert torch.equal(y0, y1)
+    P.assert_y_close(y1.float().cpu().numpy(), oracle.linear(rq, rs, rqw, rsw, mode), what="linear, bf16 scales")
+
+
+def test_bf16_scale_option_special_values():
+    x = torch.zeros(4, 256, dtype=torch.bfloat16)
+    x[1, 0] = 1632.0                             # scale rounds down: the max element saturates
+    x[1, 5] = -1632.0
+    x[2, 3] = 2.0 ** -133                        # scale rounds to zero: becomes 1
+    x[3] = synth.make_x(1, 256, seed=4)[0]
+    for mode in (fq.CHANNEL_TOKEN, fq.BLOCK128):
+        q, s = fq.fp8_quant_act(x.to(DEV), mode | fq.SCALE_BF16)
+        rq, rs = oracle.quant_act(x, mode, scale_bf16=True)
+        P.assert_codes_equal(q, rq, f"special bf16 scales mode {mode}")
+        P.assert_scales_equal(s, rs, f"special bf16 scales mode {mode}")

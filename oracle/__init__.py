@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         _lib.orc_linear.restype = None
         _lib.orc_linear_at.argtypes = [P, P, P, P, I, I, I, ctypes.c_int, P, P, I, P]
         _lib.orc_linear_at.restype = None
+        _lib.orc_quant_static.argtypes = [P, I, I, I, ctypes.c_float, P, I]
+        _lib.orc_quant_static.restype = None
         _lib.orc_linear_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, P]
         _lib.orc_linear_swiglu.restype = None
         _lib.orc_rmsnorm_rstd.argtypes = [P, I, I, I, ctypes.c_float, P]
@@ -153,6 +155,29 @@ def rmsnorm_quant_rows(x, gamma, rstd=None, eps: float = 1e-5):
     y = np.empty((R, K), np.uint16)
     lib().orc_rmsnorm_quant_rows(_p(xb), _p(gb), _p(r), R, K, K, _p(q), K, _p(s), _p(y))
     return q, s, y, r
+
+
+def quant_static(x, scale: float) -> np.ndarray:
+    """Codes of every element with one fixed scale (no amax).  -> codes u8 [R, K]."""
+    xb = _bits(x)
+    R, K = xb.shape
+    q = np.empty((R, K), np.uint8)
+    lib().orc_quant_static(_p(xb), R, K, K, float(scale), _p(q), K)
+    return q
+
+
+def percentile_scale(x, lo: float = 0.001, hi: float = 0.999) -> float:
+    """Static scale from a calibration tensor: the larger magnitude of its lo and
+    hi quantiles (linear interpolation between order statistics), / 448, in
+    fp32.  1.0 when that range is zero."""
+    f = np.sort(((_bits(x).astype(np.uint32) << 16).view(np.float32)).astype(np.float64), axis=None)
+    def q(p):
+        pos = p * (f.size - 1)
+        i = int(np.floor(pos))
+        j = min(i + 1, f.size - 1)
+        return f[i] + (f[j] - f[i]) * (pos - i)
+    amax = max(abs(q(lo)), abs(q(hi)))
+    return float(np.float32(np.float32(amax) / np.float32(448.0))) if amax > 0 else 1.0
 
 
 def quant_groups128(x, scale_bf16: bool = False):

@@ -274,6 +274,17 @@ static void quant_blocks128_impl(const uint16_t* w, int64_t N, int64_t K, int64_
     }
 }
 
+/* Static scale: [P1] section 2 (FP8 量化实操) calibrates each tensor offline
+ * from percentiles of a calibration set (the 99.9% and 0.1% quantiles as its
+ * range, not min/max) instead of the runtime amax; at run time every element
+ * is coded with that fixed scale, saturating beyond it.  x: bf16 [rows, ld];
+ * q: [rows, ldq]. */
+ORC_EXPORT void orc_quant_static(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, float s,
+                                 uint8_t* q, int64_t ldq) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k) q[r * ldq + k] = code_of(bf16_to_float(x[r * ld + k]), s);
+}
+
 /* Exported forms: fp32 scales, and scales rounded to bf16 first ("_s16"). */
 ORC_EXPORT void orc_quant_rows(const uint16_t* x, int64_t rows, int64_t K, int64_t ld,
                                uint8_t* q, int64_t ldq, float* s) {

@@ -47,6 +47,8 @@ MUTANTS = {
     "swiglu up dropped": (r"volatile float p = bf16_to_float\(sb\) \* \(float\)ub;",
                           "volatile float p = bf16_to_float(sb);"),
     "bf16 scale not rounded": (r"float r = bf16_to_float\(float_to_bf16\(s\)\);", "float r = s;"),
+    "static scale ignored": (r"q\[r \* ldq \+ k\] = code_of\(bf16_to_float\(x\[r \* ld \+ k\]\), s\);",
+                             "q[r * ldq + k] = code_of(bf16_to_float(x[r * ld + k]), 1.0f);"),
 }
 
 
@@ -67,6 +69,7 @@ def build_variant(src_text, tmp):
     L.orc_rmsnorm_rstd.argtypes = [P, I, I, I, ctypes.c_float, P]
     L.orc_rmsnorm_quant_rows.argtypes = [P, P, P, I, I, I, P, I, P, P]
     L.orc_linear_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, P]
+    L.orc_quant_static.argtypes = [P, I, I, I, ctypes.c_float, P, I]
     return L
 
 
@@ -124,6 +127,11 @@ def checks(L):
     if not np.array_equal(s16, torch.from_numpy(s.copy()).to(torch.bfloat16).float().numpy()) or \
             not np.array_equal(q16.ravel(), _pins.encode_argmin((x.float().numpy() / s16[:, None]).astype(np.float32).ravel())):
         failed.append("bf16 scales")
+    # static scale: codes of x / s for a fixed s
+    qs_ = np.empty((8, 256), np.uint8)
+    L.orc_quant_static(_p(xb), 8, 256, 256, ctypes.c_float(0.05), _p(qs_), 256)
+    if not np.array_equal(qs_.ravel(), _pins.encode_argmin((x.float().numpy() / np.float32(0.05)).astype(np.float32).ravel())):
+        failed.append("static scale")
     z = np.zeros((2, 256), np.uint16)
     qz = np.empty((2, 256), np.uint8)
     sz = np.empty(2, np.float32)

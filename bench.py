@@ -646,6 +646,31 @@ def run_gpu(args):
                                "writing gate and up, then torch silu and mul"})
     assert fq.device_error(clear=True) == 0
 
+    # ---- static-scale quantization (offline-calibrated scale, no amax pass)
+    qstatic = []
+    for k, (M, K, mode) in xs_shapes.items():
+        if mode != synth.CHANNEL_TOKEN:
+            continue
+        sc = fq.calibrate_static_scale(X[k][: min(M, 256)])
+        xq_s, xs_s = torch.empty_like(XQ[k][0]), torch.empty_like(XQ[k][1])
+        fn = (lambda k=k, sc=sc, xq_s=xq_s, xs_s=xs_s: fq.fp8_quant_act_static(X[k], sc, out=(xq_s, xs_s)))
+        fn()
+        torch.cuda.synchronize()
+        gr = capture([fn]) if not args.eager else None
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda._sleep(2_000_000)
+        for s_ in range(args.steps):
+            flush.zero_()
+            ev[s_][0].record(stream)
+            gr.replay() if gr is not None else fn()
+            ev[s_][1].record(stream)
+        torch.cuda.synchronize()
+        t = float(np.median([a.elapsed_time(b) for a, b in ev]))
+        qb = 3 * M * K + 4 * M
+        qstatic.append({"act": k, "M": M, "K": K, "ms": round(t, 5), "GB/s": round(qb / (t / 1e3) / 1e9, 1),
+                        "frac_hbm": round(qb / (t / 1e3) / 1e9 / pk["hbm_gbs"], 3)})
+    assert fq.device_error(clear=True) == 0
+
     # ---- FP8 KV cache: the k_proj / v_proj outputs quantized per (token, head)
     kvq = []
     for g in wl.gemms:
@@ -732,7 +757,7 @@ def run_gpu(args):
                        "parallelism": "single GPU" if world == 1 else f"token-parallel x{world}, weights replicated"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g) for g in wl.gemms)),
-            "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant, "rmsnorm_quant": rms, "kv_quant": kvq, "swiglu": swiglu,
+            "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant, "rmsnorm_quant": rms, "kv_quant": kvq, "swiglu": swiglu, "quant_static": qstatic,
             "merged_shared_input": merged,
             "device_error": err, "gpu": torch.cuda.get_device_name(dev),
         }

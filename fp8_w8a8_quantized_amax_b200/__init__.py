@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.fp8_quant_act.restype = ctypes.c_int
         L.fp8_rmsnorm_quant_act.argtypes = [P, P, I, I, I, ctypes.c_float, P, I, P, P, P]
         L.fp8_rmsnorm_quant_act.restype = ctypes.c_int
+        L.fp8_quant_act_static.argtypes = [P, I, I, I, ctypes.c_float, P, I, P, P]
+        L.fp8_quant_act_static.restype = ctypes.c_int
         L.fp8_linear_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, P, I, P]
         L.fp8_linear_swiglu.restype = ctypes.c_int
         L.fp8_linear.argtypes = [P, P, P, P, I, I, I, ctypes.c_int, P, I, P, S, P]
@@ -162,6 +164,43 @@ def fp8_rmsnorm_quant_act(X: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-
                                      _ptr(xs), _ptr(rstd), _stream(X))
     _check(st, "fp8_rmsnorm_quant_act")
     return (Xq, xs, rstd) if return_rstd else (Xq, xs)
+
+
+def fp8_quant_act_static(X: torch.Tensor, scale: float, out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
+    """X bf16 [M, K] coded with one fixed scale -> (Xq uint8 [M, K], x_scale fp32 [M] filled with scale)."""
+    _require_cuda(X, "X", torch.bfloat16)
+    M, K = X.shape
+    if out is None:
+        Xq = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+        xs = torch.empty((M,), dtype=torch.float32, device=X.device)
+    else:
+        Xq, xs = out
+    st = lib().fp8_quant_act_static(_ptr(X), M, K, X.stride(0), float(scale), _ptr(Xq), Xq.stride(0), _ptr(xs),
+                                    _stream(X))
+    _check(st, "fp8_quant_act_static")
+    return Xq, xs
+
+
+def calibrate_static_scale(X: torch.Tensor, lo: float = 0.001, hi: float = 0.999) -> float:
+    """Offline calibration (not part of the per-forward path): the larger
+    magnitude of X's lo and hi quantiles (linear interpolation between order
+    statistics), / 448, rounded to fp32; 1.0 for an all-zero range."""
+    f = X.detach().reshape(-1).double()
+    n = f.numel()
+
+    def q(p):
+        pos = p * (n - 1)
+        i = int(pos // 1)
+        j = min(i + 1, n - 1)
+        a = torch.kthvalue(f, i + 1).values.item()
+        b = torch.kthvalue(f, j + 1).values.item()
+        return a + (b - a) * (pos - i)
+
+    amax = max(abs(q(lo)), abs(q(hi)))
+    if amax == 0.0:
+        return 1.0
+    import numpy as np
+    return float(np.float32(np.float32(amax) / np.float32(448.0)))
 
 
 def fp8_linear_swiglu(Xq: torch.Tensor, x_scale: torch.Tensor, Wq_gate: torch.Tensor, w_scale_gate: torch.Tensor,

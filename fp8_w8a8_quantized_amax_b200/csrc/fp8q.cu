@@ -359,6 +359,25 @@ fp8q_status fp8_rmsnorm_quant_act(const void* X_bf16, const void* gamma_bf16, in
                              static_cast<int>(K), ldx, eps, Xq, ldxq, x_scale, rstd, stream);
 }
 
+fp8q_status fp8_quant_act_static(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, float scale, uint8_t* Xq,
+                                 int64_t ldxq, float* x_scale, void* stream) {
+  if (!(scale > 0.0f) || !(scale < 3.0e38f)) return FP8Q_ERR_INVALID_ARG;   // also rejects NaN
+  if (M < 0 || K <= 0 || ldx < K || ldxq < K || K % 16 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (M == 0) return FP8Q_OK;
+  if (!X_bf16 || !Xq) return FP8Q_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || ldxq % 16 != 0) return FP8Q_ERR_MISALIGNED;
+  if (!aligned(X_bf16, 16) || !aligned(Xq, 16) || (x_scale && !aligned(x_scale, 4))) return FP8Q_ERR_MISALIGNED;
+  if (M > kInt32Max || K > kInt32Max) return FP8Q_ERR_UNSUPPORTED;
+  fp8q_status st;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
+  const int64_t vecs = M * (K / 8);
+  int64_t grid = (vecs + 255) / 256;
+  if (grid > static_cast<int64_t>(sms) * 16) grid = static_cast<int64_t>(sms) * 16;
+  return launch(fp8q::quant_static_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream,
+                static_cast<const uint16_t*>(X_bf16), M, static_cast<int>(K), ldx, scale, Xq, ldxq, x_scale);
+}
+
 size_t fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int mode) {
   if (!valid_mode(mode)) return 0;
   mode &= ~FP8Q_SCALE_BF16;

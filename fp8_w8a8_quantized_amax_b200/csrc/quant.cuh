@@ -272,6 +272,28 @@ __global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t*
   }
 }
 
+// --------------------------------------------------------- static scale ---
+// Every element coded with one fixed, offline-calibrated scale (no amax),
+// saturating beyond it; x_scale (when not null) is filled with that scale so
+// that fp8_linear consumes the codes unchanged.  Grid-stride over the 16-byte
+// vectors of all rows.
+__global__ void __launch_bounds__(256) quant_static_kernel(const uint16_t* __restrict__ x, int64_t M, int K,
+                                                          int64_t ldx, float sc, uint8_t* __restrict__ q,
+                                                          int64_t ldq, float* __restrict__ s) {
+  griddep_wait();
+  const int nvec = K >> 3;
+  const int64_t total = M * nvec;
+  const Divider dv = make_divider(sc);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const int64_t m = i / nvec;
+    const int vi = static_cast<int>(i - m * nvec);
+    const uint4 v = ld_stream16(x + m * ldx + vi * 8);
+    *reinterpret_cast<uint2*>(q + m * ldq + vi * 8) = dv.fast ? encode_vec<true>(v, dv) : encode_vec<false>(v, dv);
+    if (s != nullptr && vi == 0) s[m] = sc;
+  }
+}
+
 // ----------------------------------------------------------- groups 128 ---
 // Groups of 128 features: 16 consecutive lanes (a half warp) own one group,
 // one 16-byte vector each.  Each half warp walks GPT groups, strided by the

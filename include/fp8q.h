@@ -104,6 +104,22 @@ FP8Q_API fp8q_status fp8_quant_act(const void* X_bf16, int64_t M, int64_t K, int
                           uint8_t* Xq, int64_t ldxq, float* x_scale, void* stream);
 
 /*
+ * fp8_quant_act_static -- quantize bf16 activations with one fixed scale.
+ *
+ * The static alternative to the dynamic per-token scheme: "Llama 3 精读实录"
+ * section 2 calibrates each tensor offline from percentiles of a calibration
+ * set (its 0.1% and 99.9% quantiles as the range, not min/max).  Every element
+ * is coded as E4M3(fl32(x / scale)), saturating beyond the range.
+ *   X_bf16, Xq  as fp8_quant_act.
+ *   scale       > 0, finite: the calibrated scale (range / 448).
+ *   x_scale     [M] fp32, written with `scale` when not NULL, so that
+ *               fp8_linear in FP8Q_CHANNEL_TOKEN mode consumes Xq unchanged.
+ *   Requirements: M >= 0 (M == 0 is a no-op), K > 0, K % 16 == 0.
+ */
+FP8Q_API fp8q_status fp8_quant_act_static(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, float scale,
+                                          uint8_t* Xq, int64_t ldxq, float* x_scale, void* stream);
+
+/*
  * fp8_rmsnorm_quant_act -- RMSNorm of bf16 activations, then per-token E4M3
  * quantization of the result, in one pass (the normalised bf16 rows are not
  * written).  Llama 3 normalises with RMSNorm (eps 1e-5) before attention and

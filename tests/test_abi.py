@@ -103,6 +103,27 @@ def test_quant_act_argument_checks(L, kw, want):
     assert q_act(L, **kw) == want
 
 
+def q_static(L, x=P, M=4, K=256, ldx=256, scale=0.05, q=P, ldq=256, s=P):
+    return L.fp8_quant_act_static(x, M, K, ldx, scale, q, ldq, s, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(scale=0.0), fq.ERR_INVALID_ARG),
+    (dict(scale=-1.0), fq.ERR_INVALID_ARG),
+    (dict(scale=float("nan")), fq.ERR_INVALID_ARG),
+    (dict(scale=float("inf")), fq.ERR_INVALID_ARG),
+    (dict(K=24, ldx=24, ldq=32), fq.ERR_INVALID_ARG),
+    (dict(M=-1), fq.ERR_INVALID_ARG),
+    (dict(x=None), fq.ERR_INVALID_ARG),
+    (dict(q=None), fq.ERR_INVALID_ARG),
+    (dict(x=BAD), fq.ERR_MISALIGNED),
+    (dict(s=P + 2), fq.ERR_MISALIGNED),
+    (dict(M=0, x=None, q=None, s=None), fq.OK),
+])
+def test_quant_static_argument_checks(L, kw, want):
+    assert q_static(L, **kw) == want
+
+
 def swi(L, M=4, N=64, K=256, y=P, ldy=64, xq=P, xs=P, wg=P, sg=P, wu=P, su=P):
     return L.fp8_linear_swiglu(xq, xs, wg, sg, wu, su, M, N, K, y, ldy, None)
 
@@ -190,6 +211,8 @@ def test_valid_arguments_without_a_gpu_report_cuda_error(L):
     assert lin(L) == fq.ERR_CUDA
     assert rms_q(L) == fq.ERR_CUDA
     assert swi(L) == fq.ERR_CUDA
+    assert q_static(L) == fq.ERR_CUDA
+    assert q_static(L, s=None) == fq.ERR_CUDA           # x_scale is optional
 
 
 def test_binding_refuses_cpu_tensors(L):

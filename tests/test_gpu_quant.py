@@ -218,3 +218,30 @@ def test_bf16_scale_option_special_values():
         rq, rs = oracle.quant_act(x, mode, scale_bf16=True)
         P.assert_codes_equal(q, rq, f"special bf16 scales mode {mode}")
         P.assert_scales_equal(s, rs, f"special bf16 scales mode {mode}")
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (37, 4096), (2048, 3072), (300, 1040)])
+def test_static_scale_bit_exact(M, K):
+    x = synth.make_x(M, K, seed=M * 3 + K)
+    scale = oracle.percentile_scale(x)
+    xd = x.to(DEV)
+    assert fq.calibrate_static_scale(xd) == scale
+    q, s = fq.fp8_quant_act_static(xd, scale)
+    P.assert_codes_equal(q, oracle.quant_static(x, scale), f"static {M}x{K}")
+    assert torch.all(s == scale)
+    # the codes and the filled per-token scales go straight into the linear
+    w = synth.make_w(256, K, seed=K)
+    wq, ws = fq.fp8_quant_weight(w.to(DEV))
+    y = fq.fp8_linear(q, s, wq, ws).float().cpu().numpy()
+    rwq, rws = oracle.quant_rows(w)
+    rq = oracle.quant_static(x, scale)
+    P.assert_y_close(y, oracle.linear(rq, np.full(M, scale, np.float32), rwq, rws, 0), what=f"static linear {M}x{K}")
+
+
+def test_static_scale_saturates_outliers():
+    x = synth.make_x(64, 512, seed=5)            # outlier columns far above the P99.9 range
+    scale = oracle.percentile_scale(x)
+    q, _ = fq.fp8_quant_act_static(x.to(DEV), scale)
+    ref = oracle.quant_static(x, scale)
+    P.assert_codes_equal(q, ref, "static outliers")
+    assert ((ref & 0x7F) == 0x7E).sum() > 0       # some elements saturate

@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         _lib.orc_linear.restype = None
         _lib.orc_linear_at.argtypes = [P, P, P, P, I, I, I, ctypes.c_int, P, P, I, P]
         _lib.orc_linear_at.restype = None
+        _lib.orc_linear_w8a16.argtypes = [P, P, P, I, I, I, P]
+        _lib.orc_linear_w8a16.restype = None
         _lib.orc_quant_static.argtypes = [P, I, I, I, ctypes.c_float, P, I]
         _lib.orc_quant_static.restype = None
         _lib.orc_linear_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, P]
@@ -113,6 +115,19 @@ def quant_rows(x, scale_bf16: bool = False):
     s = np.empty((R,), np.float32)
     (lib().orc_quant_rows_s16 if scale_bf16 else lib().orc_quant_rows)(_p(xb), R, K, K, _p(q), K, _p(s))
     return q, s
+
+
+def linear_w8a16(x, wq, ws) -> np.ndarray:
+    """Weight-only FP8: bf16 activations x [M, K] times dequantized codes wq [N, K]
+    with per-channel scales ws [N].  -> fp32 [M, N]."""
+    xb = _bits(x)
+    wq = np.ascontiguousarray(wq, np.uint8)
+    ws = np.ascontiguousarray(ws, np.float32)
+    M, K = xb.shape
+    N = wq.shape[0]
+    y = np.empty((M, N), np.float32)
+    lib().orc_linear_w8a16(_p(xb), _p(wq), _p(ws), M, N, K, _p(y))
+    return y
 
 
 def linear_swiglu(xq, xs, wq_gate, ws_gate, wq_up, ws_up) -> np.ndarray:

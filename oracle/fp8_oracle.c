@@ -369,6 +369,27 @@ ORC_EXPORT void orc_linear(const uint8_t* xq, const float* xs, const uint8_t* wq
                 : linear_block_one(xq, xs, wq, ws, K, ldx, ldw, m, n);
 }
 
+/* --------------------------------------------- weight-only FP8 (W8A16) */
+/*
+ * [P4] hardware section and FAQ Q1: without FP8 tensor cores (A100) the FP8
+ * weights are dequantized when the layer runs and multiplied with bf16
+ * activations.  y[m,n] = ws[n] * sum_k x[m,k] * E4M3value(wq[n,k]), x the
+ * bf16 activations (not quantized); the sum is taken in double (each product
+ * is exact in double) and the result rounded once to fp32.  y: [M, N].
+ */
+ORC_EXPORT void orc_linear_w8a16(const uint16_t* x, const uint8_t* wq, const float* ws,
+                                 int64_t M, int64_t N, int64_t K, float* y) {
+    build_mag_table();
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += (double)bf16_to_float(x[m * K + k]) * orc_e4m3_decode(wq[n * K + k]);
+            y[m * N + n] = (float)(acc * (double)ws[n]);
+        }
+}
+
 /* ------------------------------------------------- gate/up with SiLU * up */
 /*
  * [P1] section 1.3 (编码器细节：RMSNorm 与 SwiGLU 的实现差异): the Llama MLP

@@ -47,6 +47,9 @@ MUTANTS = {
     "swiglu up dropped": (r"volatile float p = bf16_to_float\(sb\) \* \(float\)ub;",
                           "volatile float p = bf16_to_float(sb);"),
     "bf16 scale not rounded": (r"float r = bf16_to_float\(float_to_bf16\(s\)\);", "float r = s;"),
+    "w8a16 w_scale dropped": (r"y\[m \* N \+ n\] = \(float\)\(acc \* \(double\)ws\[n\]\);",
+                              "y[m * N + n] = (float)acc;"),
+    "w8a16 weight transposed": (r"orc_e4m3_decode\(wq\[n \* K \+ k\]\)", "orc_e4m3_decode(wq[k * N + n])"),
     "static scale ignored": (r"q\[r \* ldq \+ k\] = code_of\(bf16_to_float\(x\[r \* ld \+ k\]\), s\);",
                              "q[r * ldq + k] = code_of(bf16_to_float(x[r * ld + k]), 1.0f);"),
 }
@@ -70,6 +73,7 @@ def build_variant(src_text, tmp):
     L.orc_rmsnorm_quant_rows.argtypes = [P, P, P, I, I, I, P, I, P, P]
     L.orc_linear_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, P]
     L.orc_quant_static.argtypes = [P, I, I, I, ctypes.c_float, P, I]
+    L.orc_linear_w8a16.argtypes = [P, P, P, I, I, I, P]
     return L
 
 
@@ -219,6 +223,18 @@ def checks(L):
     aref = (torch.nn.functional.silu(gb.double()).to(torch.bfloat16) * ub).view(torch.int16).numpy().view(np.uint16)
     if not np.array_equal(act, aref):
         failed.append("swiglu")
+    # weight-only FP8: bf16 activations times dequantized codes, vs rationals
+    xw = synth.make_x(2, K, seed=7)
+    xwb = xw.view(torch.int16).numpy().view(np.uint16).copy()
+    yw = np.empty((2, N), np.float32)
+    L.orc_linear_w8a16(_p(xwb), _p(wq), _p(ws), 2, N, K, _p(yw))
+    xwf = xw.float().numpy()
+    for m, n in [(0, 0), (1, 129), (1, 64)]:
+        e = sum(Fraction(float(a)) * Fraction(float(vals[b])) for a, b in zip(xwf[m], wq[n]))
+        e = float(e * Fraction(float(ws[n])))
+        if abs(float(yw[m, n]) - e) > _pins.f32_ulp(e):
+            failed.append("w8a16 vs rationals")
+            break
     return failed
 
 

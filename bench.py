@@ -697,6 +697,41 @@ def run_gpu(args):
                     "GB/s": round(kb / (t / 1e3) / 1e9, 1), "frac_hbm": round(kb / (t / 1e3) / 1e9 / pk["hbm_gbs"], 3)})
     assert fq.device_error(clear=True) == 0
 
+    # ---- weight-only FP8 (bf16 activations, codes widened in the kernel):
+    # the decode GEMMs (M <= 64, channel scales), next to the W8A8 path
+    # (activation quantization + FP8 linear) on the same layer
+    def time_graph(fn):
+        fn()
+        torch.cuda.synchronize()
+        gr = capture([fn]) if not args.eager else None
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda._sleep(2_000_000)
+        for s_ in range(args.steps):
+            flush.zero_()
+            ev[s_][0].record(stream)
+            gr.replay() if gr is not None else fn()
+            ev[s_][1].record(stream)
+        torch.cuda.synchronize()
+        return float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+    w8a16 = []
+    for g in wl.gemms:
+        if g.mode != synth.CHANNEL_TOKEN or g.M > 64:
+            continue
+        y16 = torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev)
+        xq_w, xs_w = torch.empty_like(XQ[g.x][0]), torch.empty_like(XQ[g.x][1])
+        wk16 = torch.zeros(max(16, fq.fp8_linear_w8a16_workspace_size(g.M, g.N, g.K)), dtype=torch.uint8, device=dev)
+        t16 = time_graph(lambda g=g, y16=y16, wk16=wk16: fq.fp8_linear_w8a16(X[g.x], WQ[g.name][0], WQ[g.name][1],
+                                                                           out=y16, workspace=wk16))
+        t8 = time_graph(lambda g=g, y16=y16, xq_w=xq_w, xs_w=xs_w: (
+            fq.fp8_quant_act(X[g.x], g.mode, out=(xq_w, xs_w)),
+            fq.fp8_linear(xq_w, xs_w, WQ[g.name][0], WQ[g.name][1], g.mode, out=y16, workspace=WS[g.name])))
+        wb = g.N * g.K + 2 * g.M * g.K + 4 * g.N + 2 * g.M * g.N
+        w8a16.append({"gemm": g.name, "M": g.M, "N": g.N, "K": g.K, "ms": round(t16, 5),
+                      "GB/s": round(wb / (t16 / 1e3) / 1e9, 1), "frac_hbm": round(wb / (t16 / 1e3) / 1e9 / pk["hbm_gbs"], 3),
+                      "w8a8_ms": round(t8, 5), "kernel": "cuda cores" if g.M == 1 else "tcgen05 bf16 (widened tiles)"})
+    assert fq.device_error(clear=True) == 0
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -757,7 +792,7 @@ def run_gpu(args):
                        "parallelism": "single GPU" if world == 1 else f"token-parallel x{world}, weights replicated"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g) for g in wl.gemms)),
-            "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant, "rmsnorm_quant": rms, "kv_quant": kvq, "swiglu": swiglu, "quant_static": qstatic,
+            "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant, "rmsnorm_quant": rms, "kv_quant": kvq, "swiglu": swiglu, "quant_static": qstatic, "w8a16": w8a16,
             "merged_shared_input": merged,
             "device_error": err, "gpu": torch.cuda.get_device_name(dev),
         }

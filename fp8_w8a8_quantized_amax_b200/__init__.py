@@ -66,6 +66,10 @@ def lib() -> ctypes.CDLL:
         L.fp8_quant_act_static.restype = ctypes.c_int
         L.fp8_linear_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, P, I, P]
         L.fp8_linear_swiglu.restype = ctypes.c_int
+        L.fp8_linear_w8a16.argtypes = [P, I, P, P, I, I, I, P, I, P, S, P]
+        L.fp8_linear_w8a16.restype = ctypes.c_int
+        L.fp8_linear_w8a16_workspace_size.argtypes = [I, I, I]
+        L.fp8_linear_w8a16_workspace_size.restype = S
         L.fp8_linear.argtypes = [P, P, P, P, I, I, I, ctypes.c_int, P, I, P, S, P]
         L.fp8_linear.restype = ctypes.c_int
         L.fp8_linear_workspace_size.argtypes = [I, I, I, ctypes.c_int]
@@ -222,6 +226,36 @@ def fp8_linear_swiglu(Xq: torch.Tensor, x_scale: torch.Tensor, Wq_gate: torch.Te
     st = lib().fp8_linear_swiglu(_ptr(Xq), _ptr(x_scale), _ptr(Wq_gate), _ptr(w_scale_gate), _ptr(Wq_up),
                                  _ptr(w_scale_up), M, N, K, _ptr(out), out.stride(0), _stream(Xq))
     _check(st, "fp8_linear_swiglu")
+    return out
+
+
+def fp8_linear_w8a16_workspace_size(M: int, N: int, K: int) -> int:
+    return int(lib().fp8_linear_w8a16_workspace_size(M, N, K))
+
+
+def fp8_linear_w8a16(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                     out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Weight-only FP8 for small M (<= 64): bf16 activations X [M, K] times the
+    dequantized codes Wq [N, K] with per-channel scales w_scale [N], fp32 sums.
+    -> Y bf16 [M, N].  `workspace`: a zero-filled uint8 device buffer of at
+    least fp8_linear_w8a16_workspace_size bytes (allocated here when None)."""
+    _require_cuda(X, "X", torch.bfloat16)
+    _require_cuda(Wq, "Wq", torch.uint8)
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Wq.shape != (N, K) or not Wq.is_contiguous():
+        raise ValueError("Wq must be a contiguous [N, K] tensor with X's K")
+    if X.stride(1) != 1:
+        raise ValueError("X rows must be contiguous")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    wsb = fp8_linear_w8a16_workspace_size(M, N, K) if 0 < M <= 64 else 0
+    if workspace is None and wsb:
+        workspace = torch.zeros(wsb, dtype=torch.uint8, device=X.device)
+    st = lib().fp8_linear_w8a16(_ptr(X), X.stride(0), _ptr(Wq), _ptr(w_scale), M, N, K, _ptr(out), out.stride(0),
+                                _ptr(workspace) if workspace is not None else None,
+                                workspace.numel() if workspace is not None else 0, _stream(X))
+    _check(st, "fp8_linear_w8a16")
     return out
 
 

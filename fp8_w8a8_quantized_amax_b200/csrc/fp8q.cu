@@ -12,6 +12,7 @@
 #include "../../include/fp8q.h"
 #include "gemm_decode.cuh"
 #include "gemm_prefill.cuh"
+#include "gemv_w8a16.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 
@@ -130,6 +131,21 @@ fp8q_status tmap_bf16_sw64(CUtensorMap* m, const void* base, int64_t rows, int64
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+// Row-major bf16 matrix [rows, cols], row stride `ld` elements, tiles of
+// box_rows x 64 values (128 bytes) with the 128-byte swizzle: a tcgen05 operand.
+fp8q_status tmap_bf16_sw128(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                            uint32_t box_rows) {
+  if (get_encode() != FP8Q_OK) return FP8Q_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  cuuint32_t box[2] = {64u, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
@@ -302,6 +318,69 @@ fp8q_status launch_decode_nx(const CUtensorMap& tw, const CUtensorMap& tx, const
   if ((st = launch(k, dim3(p.G), dim3(192), L::kBytes, stream, tw, tx, p)) != FP8Q_OK) return st;
   auto r = block ? fp8q::decode::decode_reduce_kernel<true> : fp8q::decode::decode_reduce_kernel<false>;
   return launch(r, dim3(p.n_tiles, p.M), dim3(128), 0, stream, p, NX);
+}
+
+// Weight-only FP8 on the tensor cores (2 <= M <= 64): the decode schedule
+// with bf16 activations and widened weights.  Stages: 52 / 56 / 64 KB each.
+template <int NX>
+constexpr int w16_stages() { return NX == 64 ? 3 : 4; }
+
+// Widen warps: 8 by default; FP8Q_W16_WIDEN=4 selects four (read once).
+int w16_widen_warps() {
+  static int n = [] {
+    const char* e = getenv("FP8Q_W16_WIDEN");
+    return (e && strcmp(e, "4") == 0) ? 4 : 8;
+  }();
+  return n;
+}
+
+template <int NX, int WIDEN>
+fp8q_status launch_decode_w16_n(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p, int dev,
+                                void* stream) {
+  constexpr int kStages = w16_stages<NX>();
+  using L = fp8q::decode::Layout<NX, kStages, WIDEN>;
+  auto k = fp8q::decode::gemm_decode_kernel<NX, kStages, false, true, WIDEN>;
+  fp8q_status st;
+  if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
+  return launch(k, dim3(p.G), dim3(L::kThreads), L::kBytes, stream, tw, tx, p);
+}
+
+template <int NX>
+fp8q_status launch_decode_w16(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p, int dev, void* stream) {
+  return w16_widen_warps() == 4 ? launch_decode_w16_n<NX, 4>(tw, tx, p, dev, stream)
+                                : launch_decode_w16_n<NX, 8>(tw, tx, p, dev, stream);
+}
+
+// Weight-only kernel choice: the CUDA-core kernel for one token, the tensor
+// cores above.  FP8Q_W8A16_KERNEL=cuda|tc forces one (read once; "cuda"
+// applies up to 16 tokens), for comparing them on the same problem.
+int w8a16_choice() {
+  static int choice = [] {
+    const char* e = getenv("FP8Q_W8A16_KERNEL");
+    if (e && strcmp(e, "cuda") == 0) return 1;
+    if (e && strcmp(e, "tc") == 0) return 2;
+    return 0;
+  }();
+  return choice;
+}
+
+bool w8a16_uses_cuda_cores(int64_t M) {
+  const int c = w8a16_choice();
+  if (c == 1) return M <= fp8q::wonly::kMaxTokens;
+  if (c == 2) return false;
+  return M == 1;
+}
+
+// Weight-only FP8 (small M): MT padded tokens, R channels per CTA, STAGES
+// shared-memory stages, MINB CTAs per SM for the register budget.
+template <int MT, int R, int STAGES, int MINB>
+fp8q_status launch_w8a16(const fp8q::wonly::Params& p, int dev, void* stream) {
+  using L = fp8q::wonly::Layout<R, STAGES>;
+  constexpr int kBytes = L::template bytes<R * MT>();
+  auto k = fp8q::wonly::gemv_w8a16_kernel<MT, R, STAGES, MINB>;
+  fp8q_status st;
+  if ((st = ensure_smem(k, kBytes, dev)) != FP8Q_OK) return st;
+  return launch(k, dim3((p.N + R - 1) / R), dim3(fp8q::wonly::kThreads), kBytes, stream, p);
 }
 
 }  // namespace
@@ -566,6 +645,70 @@ fp8q_status fp8_linear_swiglu(const uint8_t* Xq, const float* x_scale, const uin
   if ((st = tmap_bf16_sw64(&ty, Y_bf16, M, N, ldy, 32)) != FP8Q_OK) return st;
   return launch(k, dim3(2 * used), dim3(64 + 32 * L::kEpiWarps), L::kBytes, stream, ta, tg, tg64, tu, tu64, ty, p,
                 w_scale_up);
+}
+
+size_t fp8_linear_w8a16_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || M > kDecodeMaxM || N <= 0 || K <= 0 || w8a16_uses_cuda_cores(M)) return 0;
+  int dev, sms;
+  if (current_device(&dev, &sms) != FP8Q_OK) return 0;
+  int n_tiles, G, nx;
+  int64_t total;
+  decode_shape(M, N, K, sms, &n_tiles, &total, &G, &nx);
+  return decode_workspace_bytes(n_tiles, G, nx);
+}
+
+fp8q_status fp8_linear_w8a16(const void* X_bf16, int64_t ldx, const uint8_t* Wq, const float* w_scale, int64_t M,
+                             int64_t N, int64_t K, void* Y_bf16, int64_t ldy, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  if (M < 0 || N <= 0 || K <= 0 || K % 16 != 0 || ldx < K || ldy < N) return FP8Q_ERR_INVALID_ARG;
+  if (M == 0) return FP8Q_OK;
+  if (!X_bf16 || !Wq || !w_scale || !Y_bf16) return FP8Q_ERR_INVALID_ARG;
+  if (M > kDecodeMaxM) return FP8Q_ERR_UNSUPPORTED;
+  if (N > kInt32Max || K > kInt32Max) return FP8Q_ERR_UNSUPPORTED;
+  if (ldx % 8 != 0 || !aligned(X_bf16, 16) || !aligned(Wq, 16) || !aligned(Y_bf16, 2) || !aligned(w_scale, 4))
+    return FP8Q_ERR_MISALIGNED;
+  int dev, sms;
+  fp8q_status st;
+  if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
+  if (w8a16_uses_cuda_cores(M)) {
+    fp8q::wonly::Params p;
+    p.x = static_cast<const __nv_bfloat16*>(X_bf16);
+    p.ldx = ldx;
+    p.w = Wq;
+    p.ws = w_scale;
+    p.y = static_cast<__nv_bfloat16*>(Y_bf16);
+    p.ldy = ldy;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    if (M == 1) return launch_w8a16<1, 8, 2, 3>(p, dev, stream);
+    if (M == 2) return launch_w8a16<2, 4, 4, 2>(p, dev, stream);
+    if (M <= 4) return launch_w8a16<4, 4, 4, 2>(p, dev, stream);
+    if (M <= 8) return launch_w8a16<8, 4, 4, 1>(p, dev, stream);
+    return launch_w8a16<16, 1, 8, 1>(p, dev, stream);
+  }
+  int n_tiles, G, nx;
+  int64_t total;
+  decode_shape(M, N, K, sms, &n_tiles, &total, &G, &nx);
+  if (!workspace || workspace_bytes < decode_workspace_bytes(n_tiles, G, nx)) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16)) return FP8Q_ERR_MISALIGNED;
+  CUtensorMap tw, tx;
+  if ((st = tmap_u8_sw128(&tw, Wq, N, K, K, 128)) != FP8Q_OK) return st;
+  if ((st = tmap_bf16_sw128(&tx, X_bf16, M, K, ldx, static_cast<uint32_t>(nx))) != FP8Q_OK) return st;
+  Params p;
+  p.xs = nullptr;
+  p.ws = w_scale;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.KB = static_cast<int>((K + 127) / 128);
+  p.n_tiles = n_tiles;
+  p.total = total;
+  p.G = G;
+  decode_bind_workspace(p, workspace, Y_bf16, ldy);
+  if (nx == 16) return launch_decode_w16<16>(tw, tx, p, dev, stream);
+  if (nx == 32) return launch_decode_w16<32>(tw, tx, p, dev, stream);
+  return launch_decode_w16<64>(tw, tx, p, dev, stream);
 }
 
 const char* fp8q_status_string(int status) {

@@ -112,33 +112,46 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
 }
 
-template <int NX, int STAGES>
+// WIDEN > 0: the weight-only variant (bf16 activations).  Each stage then also
+// holds the bf16 activation tile (NX rows x 128 values, two 128-byte-swizzle
+// atoms of 64 values) and the widened bf16 weight tile (128 rows x 128 values,
+// two atoms of 16 KB), and WIDEN extra warps (4: a thread widens one weight
+// row; 8: half a row) write the latter from the E4M3 tile the TMA brought in.
+template <int NX, int STAGES, int WIDEN = 0>
 struct Layout {
+  static constexpr bool W16 = WIDEN > 0;
   static constexpr int kW = 128 * BK;
-  static constexpr int kX = NX * BK;
-  static constexpr int kBarOff = STAGES * (kW + kX);
-  static constexpr int kBarBytes = (2 * STAGES + 2 * kSlots) * 8 + 8;   // mbarriers, TMEM address, abort flag
+  static constexpr int kX = NX * BK * (W16 ? 2 : 1);
+  static constexpr int kWide = W16 ? 128 * BK * 2 : 0;
+  static constexpr int kBarOff = STAGES * (kW + kX + kWide);
+  static constexpr int kThreads = 192 + 32 * WIDEN;
+  static constexpr int kBarBytes = (2 * STAGES + 2 * kSlots + (W16 ? STAGES : 0)) * 8 + 8;   // mbarriers, TMEM address, abort flag
   static constexpr int kBytes = kBarOff + 1024 + 1024;                  // + barrier area + alignment slack
   static_assert(kBarBytes <= 1024, "barrier area");
   static_assert(kBytes <= 232448, "shared memory per CTA");
   static constexpr uint32_t kTmemCols = (kSlots * NX) < 32 ? 32 : (kSlots * NX);
 };
 
-template <int NX, int STAGES, bool BLOCK, bool FUSED>
-__global__ void __launch_bounds__(192, 1)
+template <int NX, int STAGES, bool BLOCK, bool FUSED, int WIDEN = 0>
+__global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const Params p) {
-  using L = Layout<NX, STAGES>;
+  using L = Layout<NX, STAGES, WIDEN>;
+  constexpr bool W16 = WIDEN > 0;
+  static_assert(WIDEN == 0 || WIDEN == 4 || WIDEN == 8, "widen warps");
   static_assert(NX % 16 == 0 && NX >= 16 && NX <= 64, "token tile");
+  static_assert(!(W16 && (BLOCK || !FUSED)), "the weight-only variant has channel scales and sums its own splits");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sW = smem;
   uint8_t* sX = smem + STAGES * L::kW;
+  uint8_t* sWide = sX + STAGES * L::kX;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* empty = full + STAGES;
   uint64_t* sfull = empty + STAGES;
   uint64_t* sempty = sfull + kSlots;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + kSlots);
+  uint64_t* wfull = sempty + kSlots;                       // W16: widened tile ready (STAGES of them)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wfull + (W16 ? STAGES : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -156,6 +169,8 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&sfull[a], 1);
       mbar_init(&sempty[a], 4);                  // one arrival per epilogue warp
     }
+    if constexpr (W16)
+      for (int s = 0; s < STAGES; ++s) mbar_init(&wfull[s], WIDEN);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmW);
@@ -184,6 +199,8 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive_expect_tx(&full[stage], L::kW + L::kX);
         tma_load_2d(sW + stage * L::kW, &tmW, &full[stage], kb * BK, t * 128, pol_w);
         tma_load_2d(sX + stage * L::kX, &tmX, &full[stage], kb * BK, 0, pol_x);
+        if constexpr (W16)   // bf16 activations: the second 64-value atom of the K block
+          tma_load_2d(sX + stage * L::kX + NX * 128, &tmX, &full[stage], kb * BK + 64, 0, pol_x);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
       griddep_launch_dependents();
@@ -194,7 +211,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(128, NX);
+      constexpr uint32_t idesc = W16 ? idesc_bf16_f32(128, NX) : idesc_e4m3_f32(128, NX);
       int stage = 0, slot = 0;
       uint32_t phase = 0, sphase = 0;
       for (StepIter it(b, e, p.KB); it.valid(); it.next()) {
@@ -206,14 +223,25 @@ __global__ void __launch_bounds__(192, 1)
         const bool close_slot = BLOCK || seg_last;
         if (open_slot && !mbar_wait(&sempty[slot], sphase ^ 1u, abort_flag, kErrWaitTmemEmpty)) break;
         if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) break;
+        if (W16 && !mbar_wait(&wfull[stage], phase, abort_flag, kErrWaitFull)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + slot * NX;
-        const uint32_t a0 = smem_u32(sW + stage * L::kW);
         const uint32_t b0 = smem_u32(sX + stage * L::kX);
+        if constexpr (W16) {
+          // 8 MMAs of K = 16 bf16 values (32 bytes): 4 per 64-value atom
+          const uint32_t a0 = smem_u32(sWide + stage * L::kWide);
 #pragma unroll
-        for (int k = 0; k < BK / UMMA_K; ++k)
-          mma_e4m3(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + k * UMMA_K), idesc,
-                   (!open_slot || k != 0) ? 1u : 0u);
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16(d, umma_desc_sw128(a0 + (k >> 2) * (128 * 128) + (k & 3) * 32),
+                     umma_desc_sw128(b0 + (k >> 2) * (NX * 128) + (k & 3) * 32), idesc,
+                     (!open_slot || k != 0) ? 1u : 0u);
+        } else {
+          const uint32_t a0 = smem_u32(sW + stage * L::kW);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k)
+            mma_e4m3(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + k * UMMA_K), idesc,
+                     (!open_slot || k != 0) ? 1u : 0u);
+        }
         mma_commit(&empty[stage]);
         if (close_slot) {
           mma_commit(&sfull[slot]);
@@ -222,6 +250,37 @@ __global__ void __launch_bounds__(192, 1)
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
     }
+  } else if (W16 && warp >= 6) {
+    // Widen: a thread takes one weight row of the tile (8 warps: half of it).
+    // Its chunks of 16 codes (128-byte swizzle: chunk c sits at c ^ (row & 7))
+    // become chunks of 8 bf16 values in the two 64-value atoms, swizzled the
+    // same way.
+    constexpr int kChunks = WIDEN == 8 ? 4 : 8;
+    const int row = ((warp - 6) & 3) * 32 + lane;
+    const int ch0 = ((warp - 6) >> 2) * kChunks;
+    const int sw = row & 7;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (StepIter it(b, e, p.KB); it.valid(); it.next()) {
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull))) break;
+      const uint8_t* src = sW + stage * L::kW + row * 128;
+      uint8_t* dst = sWide + stage * L::kWide + row * 128;
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const int ch = ch0 + i;
+        const uint4 q = *reinterpret_cast<const uint4*>(src + ((ch ^ sw) << 4));
+        uint4 lo, hi;
+        widen16_bf16(q, lo, hi);
+        uint8_t* atom = dst + (ch >> 2) * (128 * 128);
+        const int c2 = 2 * (ch & 3);
+        *reinterpret_cast<uint4*>(atom + ((c2 ^ sw) << 4)) = lo;
+        *reinterpret_cast<uint4*>(atom + (((c2 + 1) ^ sw) << 4)) = hi;
+      }
+      fence_proxy_async_smem();   // generic-proxy writes, read by the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wfull[stage]);
+      if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+    }
   } else {
     const int quarter = warp & 3;
     const int nl = quarter * 32 + lane;          // output channel within the tile
@@ -229,7 +288,7 @@ __global__ void __launch_bounds__(192, 1)
     // output loop (global loads there would queue behind the output stores).
     __shared__ float s_xs[4][NX];
     if constexpr (!BLOCK) {
-      for (int j = lane; j < NX; j += 32) s_xs[quarter][j] = j < p.M ? __ldg(p.xs + j) : 0.0f;
+      for (int j = lane; j < NX; j += 32) s_xs[quarter][j] = j < p.M ? (W16 ? 1.0f : __ldg(p.xs + j)) : 0.0f;
       __syncwarp();
     }
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;

@@ -342,6 +342,16 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
+// Instruction descriptor: bf16 x bf16 -> fp32 (kind::f16), both operands
+// K-major, tile M x N.  Same fields as above; format code 1 is bf16.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4)                                  // D format: fp32
+         | (1u << 7) | (1u << 10)                   // A, B format: bf16
+         | (0u << 15) | (0u << 16)                  // A, B K-major
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
@@ -353,6 +363,17 @@ __device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint6
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> fp32 (K = 16 per instruction).
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -509,6 +530,39 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Sixteen E4M3 codes (one 16-byte chunk) -> sixteen bf16 values in two
+// 16-byte chunks (codes 0..7, 8..15), exactly: E4M3 -> f16 (every E4M3 value
+// is an f16 value), f16 -> f32, and the upper halves of the fp32 words are the
+// bf16 values (three significant bits; the truncation drops only zeros).
+__device__ __forceinline__ void widen16_bf16(const uint4 q, uint4& lo, uint4& hi) {
+  const uint32_t v[4] = {q.x, q.y, q.z, q.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t f0, f1, f2, f3;
+    asm("{\n\t.reg .b16 c01, c23, h0, h1, h2, h3;\n\t.reg .b32 p01, p23;\n\t.reg .f32 g0, g1, g2, g3;\n\t"
+        "mov.b32 {c01, c23}, %4;\n\t"
+        "cvt.rn.f16x2.e4m3x2 p01, c01;\n\t"
+        "cvt.rn.f16x2.e4m3x2 p23, c23;\n\t"
+        "mov.b32 {h0, h1}, p01;\n\t"
+        "mov.b32 {h2, h3}, p23;\n\t"
+        "cvt.f32.f16 g0, h0;\n\t"
+        "cvt.f32.f16 g1, h1;\n\t"
+        "cvt.f32.f16 g2, h2;\n\t"
+        "cvt.f32.f16 g3, h3;\n\t"
+        "mov.b32 %0, g0;\n\t"
+        "mov.b32 %1, g1;\n\t"
+        "mov.b32 %2, g2;\n\t"
+        "mov.b32 %3, g3;\n\t}"
+        : "=r"(f0), "=r"(f1), "=r"(f2), "=r"(f3)
+        : "r"(v[i]));
+    o[2 * i] = __byte_perm(f0, f1, 0x7632);        // (bf16(f0), bf16(f1))
+    o[2 * i + 1] = __byte_perm(f2, f3, 0x7632);
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -196,6 +196,35 @@ FP8Q_API fp8q_status fp8_linear_swiglu(const uint8_t* Xq, const float* x_scale, 
                                        const float* w_scale_gate, const uint8_t* Wq_up, const float* w_scale_up,
                                        int64_t M, int64_t N, int64_t K, void* Y_bf16, int64_t ldy, void* stream);
 
+/*
+ * fp8_linear_w8a16 -- weight-only FP8: the layer as GPUs without FP8 tensor
+ * cores run these checkpoints ("Llama-3.1-70B-FP8-Dynamic" explainer, section
+ * 三's GPU choice list and FAQ Q1: the FP8 weights are dequantized at compute
+ * time).  The activations stay bf16:
+ *   Y[m, n] = bf16( w_scale[n] * sum_k X[m, k] * E4M3(Wq[n, k]) ),
+ * products and sums in fp32 (any order).
+ *   X_bf16   [M, ldx] bf16 activations, 16-byte aligned, ldx >= K, ldx % 8 == 0.
+ *   Wq       [N, K] uint8 codes, contiguous, 16-byte aligned (fp8_quant_weight,
+ *            FP8Q_CHANNEL_TOKEN).
+ *   w_scale  [N] fp32 per-channel scales.
+ *   Y_bf16   [M, ldy] bf16, written; ldy >= N, 2-byte aligned.
+ *   workspace  device scratch of fp8_linear_w8a16_workspace_size(M, N, K)
+ *            bytes (NULL when that is 0), 16-byte aligned, with fp8_linear's
+ *            contract: zero-filled before its first use, left all zero by
+ *            every completed call; not shared by concurrent calls.
+ * Requirements: 0 <= M <= 64 (M == 0 is a no-op; larger M returns
+ * FP8Q_ERR_UNSUPPORTED: quantize the activations and call fp8_linear),
+ * N > 0, K > 0, K % 16 == 0.
+ * Dispatch: one token runs a CUDA-core kernel that streams the weights through
+ * shared memory (no workspace); 2..64 tokens run the decode kernel's schedule
+ * on the tensor cores with the weight tiles widened to bf16 in shared memory
+ * (exactly: every E4M3 value is a bf16 value) and bf16 MMAs.
+ */
+FP8Q_API size_t fp8_linear_w8a16_workspace_size(int64_t M, int64_t N, int64_t K);
+FP8Q_API fp8q_status fp8_linear_w8a16(const void* X_bf16, int64_t ldx, const uint8_t* Wq, const float* w_scale,
+                                      int64_t M, int64_t N, int64_t K, void* Y_bf16, int64_t ldy,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of workspace fp8_linear needs for this problem on the current device
  * (0 for the prefill path).  Returns 0 for invalid arguments as well. */
 FP8Q_API size_t fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int mode);

@@ -143,6 +143,39 @@ def test_swiglu_argument_checks(L, kw, want):
     assert swi(L, **kw) == want
 
 
+def w16(L, x=P, ldx=256, w=P, ws=P, M=4, N=40, K=256, y=P, ldy=40, wk=P, wkb=1 << 30):
+    return L.fp8_linear_w8a16(x, ldx, w, ws, M, N, K, y, ldy, wk, wkb, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(M=65), fq.ERR_UNSUPPORTED),                       # more than 64 tokens: W8A8 path
+    (dict(M=-1), fq.ERR_INVALID_ARG),
+    (dict(K=24, ldx=24), fq.ERR_INVALID_ARG),               # K % 16
+    (dict(ldx=128), fq.ERR_INVALID_ARG),                    # ldx < K
+    (dict(ldy=39), fq.ERR_INVALID_ARG),                     # ldy < N
+    (dict(N=0), fq.ERR_INVALID_ARG),
+    (dict(w=None), fq.ERR_INVALID_ARG),
+    (dict(ws=None), fq.ERR_INVALID_ARG),
+    (dict(ldx=260), fq.ERR_MISALIGNED),                     # row starts off 16 bytes
+    (dict(x=BAD), fq.ERR_MISALIGNED),
+    (dict(w=P + 8), fq.ERR_MISALIGNED),
+    (dict(y=P + 1), fq.ERR_MISALIGNED),
+    (dict(M=0, x=None, w=None, ws=None, y=None, wk=None, wkb=0), fq.OK),
+])
+def test_w8a16_argument_checks(L, kw, want):
+    assert w16(L, **kw) == want
+
+
+def test_w8a16_workspace_size(L):
+    assert L.fp8_linear_w8a16_workspace_size(1, 8192, 8192) == 0        # one token: CUDA-core kernel, no scratch
+    assert L.fp8_linear_w8a16_workspace_size(65, 8192, 8192) == 0       # not served
+    assert L.fp8_linear_w8a16_workspace_size(0, 8192, 8192) == 0
+    # 2..64 tokens: the same scratch as the FP8 linear of that shape (same
+    # decode schedule; both are 0 on a machine without a CUDA device)
+    for M in (2, 16, 17, 64):
+        assert L.fp8_linear_w8a16_workspace_size(M, 8192, 8192) == L.fp8_linear_workspace_size(M, 8192, 8192, 0)
+
+
 def rms_q(L, x=P, g=P, M=4, K=256, ldx=256, eps=1e-5, q=P, ldq=256, s=P, r=None):
     return L.fp8_rmsnorm_quant_act(x, g, M, K, ldx, eps, q, ldq, s, r, None)
 
@@ -213,6 +246,9 @@ def test_valid_arguments_without_a_gpu_report_cuda_error(L):
     assert swi(L) == fq.ERR_CUDA
     assert q_static(L) == fq.ERR_CUDA
     assert q_static(L, s=None) == fq.ERR_CUDA           # x_scale is optional
+    assert w16(L) == fq.ERR_CUDA
+    assert w16(L, N=41, ldy=41, y=P + 2) == fq.ERR_CUDA    # any N; bf16 output alignment only
+    assert w16(L, M=1, wk=None, wkb=0) == fq.ERR_CUDA      # one token needs no workspace
 
 
 def test_binding_refuses_cpu_tensors(L):

@@ -112,14 +112,14 @@ def test_w8a16_matches_w8a8_layer_loosely():
 
 
 @pytest.mark.parametrize("kernel,M,N,K", [("cuda", 2, 1001, 4112), ("cuda", 8, 520, 8192), ("cuda", 16, 300, 4096),
-                                          ("tc", 1, 1001, 4112), ("widen4", 2, 1001, 4112), ("widen4", 17, 520, 8192),
-                                          ("widen4", 64, 300, 4096)])
+                                          ("tc", 1, 1001, 4112), ("widen8", 2, 1001, 4112), ("widen8", 17, 520, 8192),
+                                          ("widen8", 64, 300, 4096)])
 def test_w8a16_forced_kernel(kernel, M, N, K):
     # both kernels on token counts the default dispatch gives to the other one,
-    # and the tensor-core kernel with four widen warps instead of eight
+    # and the tensor-core kernel with eight widen warps instead of four
     env = dict(os.environ)
-    if kernel == "widen4":
-        env["FP8Q_W16_WIDEN"] = "4"
+    if kernel == "widen8":
+        env["FP8Q_W16_WIDEN"] = "8"
     else:
         env["FP8Q_W8A16_KERNEL"] = kernel
     r = subprocess.run([sys.executable, "-m", "tests._forced_kernel", "w8a16", str(M), str(N), str(K)],

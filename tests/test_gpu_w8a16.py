@@ -84,6 +84,26 @@ def test_w8a16_llama70b_shapes_sampled(M, N, K):
     check(M, N, K, seed=M, rows=rows)
 
 
+def test_w8a16_every_code_widens_exactly():
+    # one-hot activations pick one code per channel: Y[m, n] = bf16(E4M3(n)), no
+    # rounding anywhere, so any inexact widening (a flushed subnormal, a lost
+    # sign) shows; all 254 finite codes, both kernels.  Values are compared
+    # (-0 == +0): the sum for the -0 code starts from +0, as the oracle's does.
+    K = 256
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], np.uint8)
+    N = codes.size
+    wq = np.zeros((N, K), np.uint8)
+    wq[:, 37] = codes
+    ws = np.ones(N, np.float32)
+    vals = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).float()
+    for M in (1, 2, 16):
+        x = torch.zeros(M, K, dtype=torch.bfloat16)
+        x[:, 37] = 1.0
+        y = fq.fp8_linear_w8a16(x.to(DEV), torch.from_numpy(wq).to(DEV), torch.from_numpy(ws).to(DEV))
+        want = vals.to(torch.bfloat16).expand(M, N)
+        assert torch.equal(y.cpu().float(), want.float()), f"M={M}"
+
+
 def test_w8a16_zero_activations_and_codes():
     K, N = 1024, 64
     wq = np.zeros((N, K), np.uint8)
@@ -113,15 +133,22 @@ def test_w8a16_matches_w8a8_layer_loosely():
 
 @pytest.mark.parametrize("kernel,M,N,K", [("cuda", 2, 1001, 4112), ("cuda", 8, 520, 8192), ("cuda", 16, 300, 4096),
                                           ("tc", 1, 1001, 4112), ("widen8", 2, 1001, 4112), ("widen8", 17, 520, 8192),
-                                          ("widen8", 64, 300, 4096)])
+                                          ("widen8", 64, 300, 4096), ("exact-cuda", 2, 0, 0), ("exact-tc", 1, 0, 0)])
 def test_w8a16_forced_kernel(kernel, M, N, K):
     # both kernels on token counts the default dispatch gives to the other one,
     # and the tensor-core kernel with eight widen warps instead of four
+    # ("exact-*": the every-code test under that choice)
     env = dict(os.environ)
     if kernel == "widen8":
         env["FP8Q_W16_WIDEN"] = "8"
     else:
-        env["FP8Q_W8A16_KERNEL"] = kernel
+        env["FP8Q_W8A16_KERNEL"] = kernel.replace("exact-", "")
+    if kernel.startswith("exact-"):
+        r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider",
+                            __file__ + "::test_w8a16_every_code_widens_exactly"],
+                           env=env, capture_output=True, text=True, timeout=600)
+        assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+        return
     r = subprocess.run([sys.executable, "-m", "tests._forced_kernel", "w8a16", str(M), str(N), str(K)],
                        env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]

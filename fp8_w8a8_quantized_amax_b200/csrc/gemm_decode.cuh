@@ -33,6 +33,13 @@
 // whole segment in one slot (drained once per segment); block mode gives
 // every K block its own slot, folded into registers with that block's
 // x_scale * w_scale.
+//
+// Weight-only variant (WIDEN > 0 warps, bf16 activations, channel scales):
+// the same schedule with the activation tile loaded as bf16 (two 64-value
+// atoms per K block), WIDEN extra warps that widen each staged E4M3 weight
+// tile into a bf16 tile in the same swizzled layout (exactly: every E4M3
+// value is a bf16 value), and bf16 MMAs (kind::f16, K = 16) on that tile.
+// No x_scale: the epilogue applies w_scale alone.
 #pragma once
 
 #include "ptx.cuh"

@@ -4,11 +4,13 @@
 // The layer that the "Llama-3.1-70B-FP8-Dynamic" explainer describes for GPUs
 // without FP8 tensor cores (section 三, the GPU choice list; FAQ Q1): the
 // checkpoint's weights stay FP8 in memory and are widened when the layer runs;
-// the activations are not quantized.  For M <= 16 tokens the work is a weight
-// stream (N * K code bytes against 2 * M * N * K flops), so it runs on the CUDA
-// cores: a code is widened exactly (E4M3 -> f16 -> f32; every E4M3 value is an
-// f16 value), multiplied with the bf16 activation widened to f32 and added in
-// fp32 with packed f32x2 FMAs.
+// the activations are not quantized.  For one token (and, on request, up to
+// 16) the work is a weight stream (N * K code bytes against 2 * M * N * K
+// flops), so it runs on the CUDA cores: a code is widened exactly (E4M3 -> f16
+// -> f32; every E4M3 value is an f16 value), multiplied with the bf16
+// activation widened to f32 and added in fp32 with packed f32x2 FMAs.  From two
+// tokens on, the tensor-core variant of the decode kernel is faster (about 7
+// CUDA-core instructions per code at eight tokens).
 //
 // A CTA owns R consecutive output channels and all of K.  One producer warp
 // streams the R weight rows through a ring of shared-memory stages with bulk

@@ -5,6 +5,7 @@
 // kernel and launch shape, and maps errors to fp8q_status.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -513,8 +514,10 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     static_assert(fp8q::prefill::PairLayout<kPairStages, 4>::kBytes == L::kBytes, "one shared-memory size");
     const int threads = block ? fp8q::prefill::kBlock2Threads : 64 + 32 * L::kEpiWarps;
     if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
-    static int max_pairs[2][kMaxDevices] = {};
-    if (max_pairs[block][dev] == 0) {
+    // CTA pairs resident at once, per (kernel, device); computed once (a race
+    // between threads computes the same value twice).
+    static std::atomic<int> max_pairs[2][kMaxDevices];
+    if (max_pairs[block][dev].load(std::memory_order_relaxed) == 0) {
       if (block) {
         // The kernel moves registers between its warpgroups; that is only
         // safe when it is launched with the register count it was built for.
@@ -528,7 +531,7 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
       qc.dynamicSmemBytes = L::kBytes;
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, k, &qc) != cudaSuccess || n < 1) n = sms / 2;
-      max_pairs[block][dev] = n;
+      max_pairs[block][dev].store(n, std::memory_order_relaxed);
     }
     fp8q::prefill::Params p;
     p.xs = x_scale;
@@ -543,7 +546,7 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     p.num_n = static_cast<int>((N + 255) / 256);
     p.num_tiles = p.num_m * p.num_n;
     p.group_m = p.num_m < 8 ? p.num_m : 8;
-    const int pairs = max_pairs[block][dev];
+    const int pairs = max_pairs[block][dev].load(std::memory_order_relaxed);
     tail_split(p.num_tiles, pairs, &p.full, &p.split);
     const int items = (p.full ? p.full : 0) + (p.num_tiles - p.full) * p.split;
     const int used = p.full ? pairs : (items < pairs ? items : pairs);
@@ -610,15 +613,15 @@ fp8q_status fp8_linear_swiglu(const uint8_t* Xq, const float* x_scale, const uin
   using L = fp8q::prefill::PairLayout<kPairStages>;
   auto k = fp8q::prefill::gemm_swiglu2_kernel<kPairStages>;
   if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
-  static int max_pairs[kMaxDevices] = {};
-  if (max_pairs[dev] == 0) {
+  static std::atomic<int> max_pairs[kMaxDevices];
+  if (max_pairs[dev].load(std::memory_order_relaxed) == 0) {
     cudaLaunchConfig_t qc = {};
     qc.gridDim = dim3(2 * sms);
     qc.blockDim = dim3(64 + 32 * L::kEpiWarps);
     qc.dynamicSmemBytes = L::kBytes;
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, k, &qc) != cudaSuccess || n < 1) n = sms / 2;
-    max_pairs[dev] = n;
+    max_pairs[dev].store(n, std::memory_order_relaxed);
   }
   fp8q::prefill::Params p;
   p.xs = x_scale;
@@ -633,7 +636,7 @@ fp8q_status fp8_linear_swiglu(const uint8_t* Xq, const float* x_scale, const uin
   p.num_n = static_cast<int>((N + 127) / 128);              // tiles of 128 output channels
   p.num_tiles = p.num_m * p.num_n;
   p.group_m = p.num_m < 8 ? p.num_m : 8;
-  const int pairs = max_pairs[dev];
+  const int pairs = max_pairs[dev].load(std::memory_order_relaxed);
   tail_split(p.num_tiles, pairs, &p.full, &p.split);
   const int items = (p.full ? p.full : 0) + (p.num_tiles - p.full) * p.split;
   const int used = p.full ? pairs : (items < pairs ? items : pairs);

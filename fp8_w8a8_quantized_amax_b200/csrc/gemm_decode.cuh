@@ -82,13 +82,13 @@ struct StepIter {
   int64_t first_end, last_begin, b0, e0;
   int64_t s, cur_b, cur_e;   // the current run [cur_b, cur_e)
   int run, t, kb, KB;
-  __device__ StepIter(int64_t b, int64_t e, int kblocks) : b0(b), e0(e), KB(kblocks) {
+  __host__ __device__ StepIter(int64_t b, int64_t e, int kblocks) : b0(b), e0(e), KB(kblocks) {
     first_end = min(e, (b / KB + 1) * KB);
     last_begin = (e % KB == 0) ? e : max(first_end, ((e - 1) / KB) * KB);
     run = -1;
     next_run();
   }
-  __device__ void next_run() {
+  __host__ __device__ void next_run() {
     for (;;) {
       ++run;
       if (run == 0) { cur_b = last_begin; cur_e = e0; }
@@ -101,11 +101,11 @@ struct StepIter {
     t = static_cast<int>(s / KB);
     kb = static_cast<int>(s - static_cast<int64_t>(t) * KB);
   }
-  __device__ bool valid() const { return run < 3; }
+  __host__ __device__ bool valid() const { return run < 3; }
   // Whether this step starts / ends a segment (a run of steps in one tile).
-  __device__ bool seg_first() const { return s == cur_b || kb == 0; }
-  __device__ bool seg_last() const { return s + 1 == cur_e || kb + 1 == KB; }
-  __device__ void next() {
+  __host__ __device__ bool seg_first() const { return s == cur_b || kb == 0; }
+  __host__ __device__ bool seg_last() const { return s + 1 == cur_e || kb + 1 == KB; }
+  __host__ __device__ void next() {
     if (++s == cur_e) {
       next_run();
     } else if (++kb == KB) {

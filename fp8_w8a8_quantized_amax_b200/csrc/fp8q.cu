@@ -229,19 +229,6 @@ int prefill_choice() {
   return choice;
 }
 
-// Whole rounds of `per_round` tiles stay whole; the partial last round is cut
-// along N into two halves when that shortens it.  Returns the split (1 or 2)
-// and the number of whole tiles.
-void tail_split(int num_tiles, int per_round, int* full, int* split) {
-  *full = num_tiles >= per_round ? num_tiles / per_round * per_round : 0;
-  const int rest = num_tiles - *full;
-  *split = 1;
-  if (rest) {
-    const double whole = 1.0 * ((rest + per_round - 1) / per_round);
-    const double halves = 0.5 * ((2 * rest + per_round - 1) / per_round);
-    if (halves < whole - 1e-9) *split = 2;
-  }
-}
 constexpr int kPrefillStages = 4;
 constexpr int kBlockStages = 6;
 template <int NX>
@@ -547,7 +534,7 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     p.num_tiles = p.num_m * p.num_n;
     p.group_m = p.num_m < 8 ? p.num_m : 8;
     const int pairs = max_pairs[block][dev].load(std::memory_order_relaxed);
-    tail_split(p.num_tiles, pairs, &p.full, &p.split);
+    fp8q::prefill::tail_split(p.num_tiles, pairs, &p.full, &p.split);
     const int items = (p.full ? p.full : 0) + (p.num_tiles - p.full) * p.split;
     const int used = p.full ? pairs : (items < pairs ? items : pairs);
     CUtensorMap ta, tb, tb64, ty;
@@ -576,7 +563,7 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
   p.full = p.num_tiles;
   p.split = 1;
   if (mode != FP8Q_BLOCK128) {
-    tail_split(p.num_tiles, sms, &p.full, &p.split);
+    fp8q::prefill::tail_split(p.num_tiles, sms, &p.full, &p.split);
     const int items = p.full + (p.num_tiles - p.full) * p.split;
     grid = p.full ? sms : (items < sms ? items : sms);
   }
@@ -637,7 +624,7 @@ fp8q_status fp8_linear_swiglu(const uint8_t* Xq, const float* x_scale, const uin
   p.num_tiles = p.num_m * p.num_n;
   p.group_m = p.num_m < 8 ? p.num_m : 8;
   const int pairs = max_pairs[dev].load(std::memory_order_relaxed);
-  tail_split(p.num_tiles, pairs, &p.full, &p.split);
+  fp8q::prefill::tail_split(p.num_tiles, pairs, &p.full, &p.split);
   const int items = (p.full ? p.full : 0) + (p.num_tiles - p.full) * p.split;
   const int used = p.full ? pairs : (items < pairs ? items : pairs);
   CUtensorMap ta, tg, tg64, tu, tu64, ty;

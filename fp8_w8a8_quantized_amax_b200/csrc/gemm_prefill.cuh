@@ -47,7 +47,7 @@ struct Params {
 
 // Tile order: groups of `group_m` row-blocks, column-blocks within a group,
 // so that the tiles in flight at one time share operands in L2.
-__device__ __forceinline__ void tile_coords(const Params& p, int t, int& mb, int& nb) {
+__host__ __device__ __forceinline__ void tile_coords(const Params& p, int t, int& mb, int& nb) {
   const int per_group = p.group_m * p.num_n;
   const int g = t / per_group;
   const int first_m = g * p.group_m;
@@ -57,27 +57,42 @@ __device__ __forceinline__ void tile_coords(const Params& p, int t, int& mb, int
   nb = r / gm;
 }
 
-// Number of work items of CTA c, and item i of it: tile coordinates, the
-// first column inside the 256-wide tile and the column count.
-__device__ __forceinline__ int items_of(const Params& p, int c) {
-  const int G = gridDim.x;
+// Work list of G persistent workers (CTAs or CTA pairs): tiles [0, full)
+// whole, tile t to worker t % G; then the remaining tiles cut along N into
+// `split` pieces, handed out round-robin.  work_items: the number of items of
+// worker c.  work_item: item i of worker c -- tile coordinates, the first
+// column inside the tile (`tile_cols` wide) and the column count.
+__host__ __device__ __forceinline__ int work_items(const Params& p, int c, int G) {
   const int tail = (p.num_tiles - p.full) * p.split;
   return p.full / G + (c < tail ? (tail - 1 - c) / G + 1 : 0);
 }
 
-__device__ __forceinline__ void item_coords(const Params& p, int c, int i, int& mb, int& nb, int& n_off,
-                                            int& n_cols) {
-  const int G = gridDim.x;
+__host__ __device__ __forceinline__ void work_item(const Params& p, int c, int G, int i, int tile_cols, int& mb,
+                                                   int& nb, int& off, int& cols) {
   const int nfull = p.full / G;
   if (i < nfull) {
     tile_coords(p, c + i * G, mb, nb);
-    n_off = 0;
-    n_cols = 256;
+    off = 0;
+    cols = tile_cols;
   } else {
     const int j = c + (i - nfull) * G;
     tile_coords(p, p.full + j / p.split, mb, nb);
-    n_cols = 256 / p.split;
-    n_off = (j % p.split) * n_cols;
+    cols = tile_cols / p.split;
+    off = (j % p.split) * cols;
+  }
+}
+
+// Whole rounds of `per_round` tiles stay whole; the partial last round is cut
+// along N into two halves when that shortens it.  Returns the split (1 or 2)
+// and the number of whole tiles.
+inline void tail_split(int num_tiles, int per_round, int* full, int* split) {
+  *full = num_tiles >= per_round ? num_tiles / per_round * per_round : 0;
+  const int rest = num_tiles - *full;
+  *split = 1;
+  if (rest) {
+    const double whole = 1.0 * ((rest + per_round - 1) / per_round);
+    const double halves = 0.5 * ((2 * rest + per_round - 1) / per_round);
+    if (halves < whole - 1e-9) *split = 2;
   }
 }
 
@@ -155,10 +170,10 @@ __global__ void __launch_bounds__(192, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      const int nitems = items_of(p, blockIdx.x);
+      const int nitems = work_items(p, blockIdx.x, gridDim.x);
       for (int i = 0; ok && i < nitems; ++i) {
         int mb, nb, n_off, n_cols;
-        item_coords(p, blockIdx.x, i, mb, nb, n_off, n_cols);
+        work_item(p, blockIdx.x, gridDim.x, i, 256, mb, nb, n_off, n_cols);
         const CUtensorMap* tb = n_cols == 256 ? &tmB : (n_cols == 128 ? &tmB128 : &tmB64);
         const uint32_t bytes = static_cast<uint32_t>(L::kA + n_cols * BK);
         for (int kb = 0; kb < p.KB; ++kb) {
@@ -182,10 +197,10 @@ __global__ void __launch_bounds__(192, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      const int nitems = items_of(p, blockIdx.x);
+      const int nitems = work_items(p, blockIdx.x, gridDim.x);
       for (int it = 0; ok && it < nitems; ++it) {
         int mb, nb, n_off, n_cols;
-        item_coords(p, blockIdx.x, it, mb, nb, n_off, n_cols);
+        work_item(p, blockIdx.x, gridDim.x, it, 256, mb, nb, n_off, n_cols);
         const uint32_t idesc = idesc_e4m3_f32(BM, n_cols);
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
@@ -217,10 +232,10 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* out_s = smem + L::kOutOff + ew * 2 * L::kOutChunk;
     const int swz = (lane >> 1) & 3;         // 64-byte swizzle of this thread's staging row
     int buf = 0;
-    const int nitems = items_of(p, blockIdx.x);
+    const int nitems = work_items(p, blockIdx.x, gridDim.x);
     for (int it = 0; it < nitems; ++it) {
       int mb, nb, n_off, n_cols;
-      item_coords(p, blockIdx.x, it, mb, nb, n_off, n_cols);
+      work_item(p, blockIdx.x, gridDim.x, it, 256, mb, nb, n_off, n_cols);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       // Scales of this tile, fetched while the main loop still runs.
@@ -363,24 +378,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
 
   // Work items are per pair: use the pair index and the number of pairs.
   const int G2 = gridDim.x >> 1;
-  auto count = [&]() {
-    const int tail = (p.num_tiles - p.full) * p.split;
-    return p.full / G2 + (pair < tail ? (tail - 1 - pair) / G2 + 1 : 0);
-  };
   auto coords = [&](int i, int& mb, int& nb, int& n_off, int& n_cols) {
-    const int nfull = p.full / G2;
-    if (i < nfull) {
-      tile_coords(p, pair + i * G2, mb, nb);
-      n_off = 0;
-      n_cols = 256;
-    } else {
-      const int j = pair + (i - nfull) * G2;
-      tile_coords(p, p.full + j / p.split, mb, nb);
-      n_cols = 256 / p.split;
-      n_off = (j % p.split) * n_cols;
-    }
+    work_item(p, pair, G2, i, 256, mb, nb, n_off, n_cols);
   };
-  const int nitems = count();
+  const int nitems = work_items(p, pair, G2);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -597,26 +598,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
   griddep_wait();
 
   const int G2 = gridDim.x >> 1;
-  auto count = [&]() {
-    const int tail = (p.num_tiles - p.full) * p.split;
-    return p.full / G2 + (pair < tail ? (tail - 1 - pair) / G2 + 1 : 0);
-  };
   // Item i: tile (mb, nb) of 256 tokens x 128 channels, channel offset c_off
   // inside it and its channel count (128, or 64 for a tail half).
   auto coords = [&](int i, int& mb, int& nb, int& c_off, int& n_ch) {
-    const int nfull = p.full / G2;
-    if (i < nfull) {
-      tile_coords(p, pair + i * G2, mb, nb);
-      c_off = 0;
-      n_ch = 128;
-    } else {
-      const int j = pair + (i - nfull) * G2;
-      tile_coords(p, p.full + j / p.split, mb, nb);
-      n_ch = 128 / p.split;
-      c_off = (j % p.split) * n_ch;
-    }
+    work_item(p, pair, G2, i, 128, mb, nb, c_off, n_ch);
   };
-  const int nitems = count();
+  const int nitems = work_items(p, pair, G2);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -850,24 +837,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBlock2Threads, 1)
   griddep_wait();
 
   const int G2 = gridDim.x >> 1;
-  auto count = [&]() {
-    const int tail = (p.num_tiles - p.full) * p.split;
-    return p.full / G2 + (pair < tail ? (tail - 1 - pair) / G2 + 1 : 0);
-  };
   auto coords = [&](int i, int& mb, int& nb, int& n_off, int& n_cols) {
-    const int nfull = p.full / G2;
-    if (i < nfull) {
-      tile_coords(p, pair + i * G2, mb, nb);
-      n_off = 0;
-      n_cols = 256;
-    } else {
-      const int j = pair + (i - nfull) * G2;
-      tile_coords(p, p.full + j / p.split, mb, nb);
-      n_cols = 256 / p.split;
-      n_off = (j % p.split) * n_cols;
-    }
+    work_item(p, pair, G2, i, 256, mb, nb, n_off, n_cols);
   };
-  const int nitems = count();
+  const int nitems = work_items(p, pair, G2);
 
   if (warp < 4) regs_shrink<kBlock2CtlRegs>();
   if (warp == 0) {

@@ -1,7 +1,8 @@
-// Host-side check of the decode kernel's stream-K schedule (compiled by nvcc
-// for the host only and run by tests/test_schedule.py; no GPU).  For many
-// (tiles, K blocks, CTAs) it checks, with the kernel's own StepIter,
-// range_begin and cta_of_step:
+// Host-side check of the GEMM kernels' work schedules (compiled by nvcc for
+// the host only and run by tests/test_schedule.py; no GPU).
+//
+// Decode (stream-K): for many (tiles, K blocks, CTAs) it checks, with the
+// kernel's own StepIter, range_begin and cta_of_step:
 //   - the CTA ranges partition the T = n_tiles * KB steps, none empty;
 //   - a CTA visits each step of its range exactly once, in the order partial
 //     last segment, first segment, whole tiles, with the right (t, kb) and
@@ -11,12 +12,18 @@
 //     n_tiles + G - 1, the slot count the host allocates;
 //   - for every split tile, CTAs c0..c1 (as the last-arriver sums them) are
 //     exactly the CTAs holding a partial segment of it.
+//
+// Prefill (persistent CTAs or CTA pairs): for many (row blocks, column
+// blocks, workers), with the kernels' own tail_split, work_items, work_item
+// and tile_coords, every column of every tile is computed by exactly one
+// item, for 256- and 128-column tiles.
 #include <cstdio>
 #include <cstdlib>
 #include <set>
 #include <vector>
 
 #include "../fp8_w8a8_quantized_amax_b200/csrc/gemm_decode.cuh"
+#include "../fp8_w8a8_quantized_amax_b200/csrc/gemm_prefill.cuh"
 
 using namespace fp8q::decode;
 
@@ -74,8 +81,51 @@ static int check(int n_tiles, int KB, int G) {
   return 0;
 }
 
+static int check_prefill(int num_m, int num_n, int G, int tile_cols) {
+  fp8q::prefill::Params p{};
+  p.num_m = num_m;
+  p.num_n = num_n;
+  p.num_tiles = num_m * num_n;
+  p.group_m = num_m < 8 ? num_m : 8;
+  fp8q::prefill::tail_split(p.num_tiles, G, &p.full, &p.split);
+  std::vector<int> cov(static_cast<size_t>(p.num_tiles) * tile_cols, 0);
+  for (int c = 0; c < G; ++c) {
+    const int n = fp8q::prefill::work_items(p, c, G);
+    for (int i = 0; i < n; ++i) {
+      int mb, nb, off, cols;
+      fp8q::prefill::work_item(p, c, G, i, tile_cols, mb, nb, off, cols);
+      if (mb < 0 || mb >= num_m || nb < 0 || nb >= num_n || off < 0 || cols <= 0 || off + cols > tile_cols) {
+        std::printf("FAIL prefill item out of range (m=%d n=%d G=%d)\n", num_m, num_n, G);
+        return 1;
+      }
+      for (int x = off; x < off + cols; ++x) ++cov[(static_cast<size_t>(mb) * num_n + nb) * tile_cols + x];
+    }
+  }
+  for (int v : cov)
+    if (v != 1) {
+      std::printf("FAIL prefill coverage (m=%d n=%d G=%d cols=%d)\n", num_m, num_n, G, tile_cols);
+      return 1;
+    }
+  return 0;
+}
+
 int main() {
   int bad = 0, cases = 0;
+  for (int num_m = 1; num_m <= 12; ++num_m)
+    for (int num_n = 1; num_n <= 12; ++num_n)
+      for (int G : {1, 2, 3, 5, 7, 8, 16, 37, 74, 148})
+        for (int cols : {256, 128}) {
+          bad |= check_prefill(num_m, num_n, G, cols);
+          ++cases;
+        }
+  // the Llama prefill shapes on 74 CTA pairs / 148 CTAs
+  const int pshapes[][2] = {{8, 32}, {32, 56}, {32, 16}, {32, 4}, {2, 112}, {2, 40}, {16, 32}, {32, 112}};
+  for (auto& sh : pshapes)
+    for (int G : {74, 148})
+      for (int cols : {256, 128}) {
+        bad |= check_prefill(sh[0], sh[1], G, cols);
+        ++cases;
+      }
   // every small case, then the Llama decode shapes on 148 SMs
   for (int n_tiles = 1; n_tiles <= 24; ++n_tiles)
     for (int KB = 1; KB <= 12; ++KB)

@@ -110,6 +110,39 @@ def _require_cuda(t: torch.Tensor, name: str, dtype) -> None:
         raise ValueError(f"{name} must be 2-D with unit stride in the last dimension")
 
 
+def _numel(shape) -> int:
+    n = 1
+    for d in shape:
+        n *= int(d)
+    return n
+
+
+def _require_like(t: Optional[torch.Tensor], name: str, dtype, min_numel: int, ref: torch.Tensor) -> None:
+    """A scale vector or scratch buffer handed to a kernel: on ref's CUDA device,
+    of `dtype`, contiguous, with at least min_numel elements.  (A host tensor
+    would reach the kernel as a host pointer.)"""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda or t.device != ref.device:
+        raise ValueError(f"{name} must be a CUDA tensor on {ref.device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name} has {t.numel()} elements, needs {min_numel}")
+
+
+def _require_out(t: torch.Tensor, name: str, dtype, shape, ref: torch.Tensor) -> None:
+    """An output matrix: on ref's CUDA device, of `dtype` and `shape`, rows with unit stride."""
+    if not t.is_cuda or t.device != ref.device:
+        raise ValueError(f"{name} must be a CUDA tensor on {ref.device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape) or (t.dim() == 2 and t.stride(1) != 1):
+        raise ValueError(f"{name} must be {tuple(shape)} with unit stride in the last dimension")
+
+
 def scale_shape_weight(N: int, K: int, mode: int) -> Tuple[int, ...]:
     return (N,) if (mode & ~SCALE_BF16) == CHANNEL_TOKEN else ((N + 127) // 128, K // 128)
 
@@ -128,6 +161,8 @@ def fp8_quant_weight(W: torch.Tensor, mode: int = CHANNEL_TOKEN,
         ws = torch.empty(scale_shape_weight(N, K, mode), dtype=torch.float32, device=W.device)
     else:
         Wq, ws = out
+        _require_out(Wq, "Wq", torch.uint8, (N, K), W)
+        _require_like(ws, "w_scale", torch.float32, _numel(scale_shape_weight(N, K, mode)), W)
     st = lib().fp8_quant_weight(_ptr(W), N, K, W.stride(0), int(mode), _ptr(Wq), Wq.stride(0),
                                 _ptr(ws), _stream(W))
     _check(st, "fp8_quant_weight")
@@ -144,6 +179,8 @@ def fp8_quant_act(X: torch.Tensor, mode: int = CHANNEL_TOKEN,
         xs = torch.empty(scale_shape_act(M, K, mode), dtype=torch.float32, device=X.device)
     else:
         Xq, xs = out
+        _require_out(Xq, "Xq", torch.uint8, (M, K), X)
+        _require_like(xs, "x_scale", torch.float32, _numel(scale_shape_act(M, K, mode)), X)
     st = lib().fp8_quant_act(_ptr(X), M, K, X.stride(0), int(mode), _ptr(Xq), Xq.stride(0),
                              _ptr(xs), _stream(X))
     _check(st, "fp8_quant_act")
@@ -156,13 +193,16 @@ def fp8_rmsnorm_quant_act(X: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-
     X bf16 [M, K], gamma bf16 [K] -> (Xq uint8 [M, K], x_scale fp32 [M][, rstd fp32 [M]])."""
     _require_cuda(X, "X", torch.bfloat16)
     M, K = X.shape
-    if not gamma.is_cuda or gamma.dtype != torch.bfloat16 or gamma.numel() != K or not gamma.is_contiguous():
-        raise ValueError("gamma must be a contiguous bf16 CUDA tensor of K elements")
+    if not gamma.is_cuda or gamma.device != X.device or gamma.dtype != torch.bfloat16 or gamma.numel() != K \
+            or not gamma.is_contiguous():
+        raise ValueError("gamma must be a contiguous bf16 CUDA tensor of K elements on X's device")
     if out is None:
         Xq = torch.empty((M, K), dtype=torch.uint8, device=X.device)
         xs = torch.empty((M,), dtype=torch.float32, device=X.device)
     else:
         Xq, xs = out
+        _require_out(Xq, "Xq", torch.uint8, (M, K), X)
+        _require_like(xs, "x_scale", torch.float32, M, X)
     rstd = torch.empty((M,), dtype=torch.float32, device=X.device) if return_rstd else None
     st = lib().fp8_rmsnorm_quant_act(_ptr(X), _ptr(gamma), M, K, X.stride(0), float(eps), _ptr(Xq), Xq.stride(0),
                                      _ptr(xs), _ptr(rstd), _stream(X))
@@ -179,6 +219,9 @@ def fp8_quant_act_static(X: torch.Tensor, scale: float, out: Optional[Tuple[torc
         xs = torch.empty((M,), dtype=torch.float32, device=X.device)
     else:
         Xq, xs = out
+        _require_out(Xq, "Xq", torch.uint8, (M, K), X)
+        if xs is not None:
+            _require_like(xs, "x_scale", torch.float32, M, X)
     st = lib().fp8_quant_act_static(_ptr(X), M, K, X.stride(0), float(scale), _ptr(Xq), Xq.stride(0), _ptr(xs),
                                     _stream(X))
     _check(st, "fp8_quant_act_static")
@@ -221,8 +264,12 @@ def fp8_linear_swiglu(Xq: torch.Tensor, x_scale: torch.Tensor, Wq_gate: torch.Te
         raise ValueError("Wq_gate and Wq_up must both be [N, K] with Xq's K")
     if not (Xq.is_contiguous() and Wq_gate.is_contiguous() and Wq_up.is_contiguous()):
         raise ValueError("Xq, Wq_gate and Wq_up must be contiguous")
+    _require_like(x_scale, "x_scale", torch.float32, M, Xq)
+    _require_like(w_scale_gate, "w_scale_gate", torch.float32, N, Xq)
+    _require_like(w_scale_up, "w_scale_up", torch.float32, N, Xq)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    _require_out(out, "out", torch.bfloat16, (M, N), Xq)
     st = lib().fp8_linear_swiglu(_ptr(Xq), _ptr(x_scale), _ptr(Wq_gate), _ptr(w_scale_gate), _ptr(Wq_up),
                                  _ptr(w_scale_up), M, N, K, _ptr(out), out.stride(0), _stream(Xq))
     _check(st, "fp8_linear_swiglu")
@@ -247,11 +294,15 @@ def fp8_linear_w8a16(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
         raise ValueError("Wq must be a contiguous [N, K] tensor with X's K")
     if X.stride(1) != 1:
         raise ValueError("X rows must be contiguous")
+    _require_like(w_scale, "w_scale", torch.float32, N, X)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _require_out(out, "out", torch.bfloat16, (M, N), X)
     wsb = fp8_linear_w8a16_workspace_size(M, N, K) if 0 < M <= 64 else 0
     if workspace is None and wsb:
         workspace = torch.zeros(wsb, dtype=torch.uint8, device=X.device)
+    if workspace is not None:   # its size is checked by the library (FP8Q_ERR_INVALID_ARG)
+        _require_like(workspace, "workspace", torch.uint8, 0, X)
     st = lib().fp8_linear_w8a16(_ptr(X), X.stride(0), _ptr(Wq), _ptr(w_scale), M, N, K, _ptr(out), out.stride(0),
                                 _ptr(workspace) if workspace is not None else None,
                                 workspace.numel() if workspace is not None else 0, _stream(X))
@@ -294,11 +345,16 @@ def fp8_linear(Xq: torch.Tensor, x_scale: torch.Tensor, Wq: torch.Tensor, w_scal
         raise ValueError("Xq and Wq disagree on K")
     if not (Xq.is_contiguous() and Wq.is_contiguous()):
         raise ValueError("Xq and Wq must be contiguous")
+    _require_like(x_scale, "x_scale", torch.float32, _numel(scale_shape_act(M, K, mode)), Xq)
+    _require_like(w_scale, "w_scale", torch.float32, _numel(scale_shape_weight(N, K, mode)), Xq)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    _require_out(out, "out", torch.bfloat16, (M, N), Xq)
     need = fp8_linear_workspace_size(M, N, K, mode)
     if workspace is None and need > 0:
         workspace = torch.zeros(need, dtype=torch.uint8, device=Xq.device)
+    if workspace is not None:   # its size is checked by the library (FP8Q_ERR_INVALID_ARG)
+        _require_like(workspace, "workspace", torch.uint8, 0, Xq)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().fp8_linear(_ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), M, N, K, int(mode),
                           _ptr(out), out.stride(0), _ptr(workspace), wbytes, _stream(Xq))

@@ -840,16 +840,31 @@ def omp_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(wl, unit, rows, w_cache=None):
-    secs, _ = oracle_sample(wl, rows, w_cache)
-    # linear extrapolation in M of the sampled rows to the whole workload
+def cpu_baseline(wl, unit, rows, w_cache=None, target_s=10.0):
+    """The oracle on the host cores, timed over a bounded sample of the
+    workload: `rows` token rows of every GEMM, grown (up to each GEMM's M)
+    while one pass takes well under target_s, then passes repeated until about
+    target_s of CPU work; extrapolated linearly in M to the whole workload."""
+    secs, w_cache = oracle_sample(wl, rows, w_cache)
+    max_m = max(g.M for g in wl.gemms)
+    while secs < target_s / 3 and rows < max_m:
+        rows = min(max_m, max(2 * rows, int(rows * target_s / 3 / max(secs, 1e-3))))
+        secs, w_cache = oracle_sample(wl, rows, w_cache)
+    total, passes = secs, 1
+    while total < target_s:
+        s_, _ = oracle_sample(wl, rows, w_cache)
+        total += s_
+        passes += 1
+    per_pass = total / passes
     frac = sum(min(rows, g.M) * g.N * g.K for g in wl.gemms) / sum(g.M * g.N * g.K for g in wl.gemms)
-    full_s = secs / frac
+    full_s = per_pass / frac
+    whole = all(rows >= g.M for g in wl.gemms)
     return {"value": round(to_metric(step_units(wl, unit), full_s, unit), 6), "unit": unit,
             "cores": omp_threads(), "kind": "oracle",
-            "sample": f"first {rows} token rows of every GEMM (all N, all K): activation quantization + "
-                      f"exact int64 GEMM, {secs:.2f} s, extrapolated linearly in M (weights quantized "
-                      "before timing, as in the GPU step)"}
+            "sample": (f"{'every' if whole else f'the first {rows}'} token rows of every GEMM (all N, all K): "
+                       f"activation quantization + exact int64 GEMM, {passes} passes, {total:.1f} s of CPU "
+                       f"work{'' if whole else ', extrapolated linearly in M'} (weights quantized before "
+                       "timing, as in the GPU step)")}
 
 
 def run_reference(args):

@@ -132,3 +132,35 @@ def test_tiny_workload_output_close_to_bf16_matmul():
     ref = (x.double() @ w.double().T).numpy()
     rel = np.abs(y - ref).max() / np.abs(ref).max()
     assert rel < 0.05
+
+
+def test_tiny_config_sampled_outputs_equal_exact_rationals():
+    # the tiny 16x256 -> 512 configuration with its synthetic inputs (two
+    # outlier input columns), quantized by the oracle: 96 sampled outputs,
+    # the first and last included, against exact rationals, in both modes
+    M, K, N = 16, 256, 512
+    x = synth.make_x(M, K, seed=0, n_out=2)
+    w = synth.make_w(N, K, seed=0)
+    rng = np.random.default_rng(16)
+    pairs = [(0, 0), (M - 1, N - 1)] + [(int(rng.integers(M)), int(rng.integers(N))) for _ in range(94)]
+    for mode in (oracle.CHANNEL_TOKEN, oracle.BLOCK128):
+        xq, xs = oracle.quant_act(x, mode)
+        wq, ws = oracle.quant_weight(w, mode)
+        y = oracle.linear(xq, xs, wq, ws, mode)
+        sub_m = sorted({m for m, _ in pairs})
+        sub_n = sorted({n for _, n in pairs})
+        if mode == oracle.CHANNEL_TOKEN:
+            ex = _pins.exact_linear_channel(xq[sub_m].tolist(), xs[sub_m], wq[sub_n].tolist(), ws[sub_n])
+            for m, n in pairs:
+                e = float(ex[sub_m.index(m)][sub_n.index(n)])
+                assert abs(float(y[m, n]) - e) <= 0.5 * _pins.f32_ulp(e) * 1.0000001 + 1e-300, (mode, m, n)
+        else:
+            from fractions import Fraction
+            for m, n in pairs:
+                e = Fraction(0)
+                for kb in range(K // 128):
+                    acc = sum(Fraction(float(VALS[xq[m, k]])) * Fraction(float(VALS[wq[n, k]]))
+                              for k in range(128 * kb, 128 * kb + 128))
+                    e += acc * Fraction(float(xs[m, kb])) * Fraction(float(ws[n // 128, kb]))
+                e = float(e)
+                assert abs(float(y[m, n]) - e) <= 2 * _pins.f32_ulp(e) + 1e-300, (mode, m, n)

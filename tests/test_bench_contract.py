@@ -3,6 +3,7 @@ oracle) prints one JSON line with the keys the benchmark line carries, and
 the GPU arm refuses to run without a GPU instead of falling back."""
 import json
 import os
+import socket
 import subprocess
 import sys
 
@@ -39,3 +40,23 @@ def test_gpu_arm_fails_loudly_without_a_gpu():
     r = run_bench("--workload", "tiny_16x256x512", "--steps", "3", "--warmup", "3")
     assert r.returncode != 0
     assert not any(l.strip().startswith("{") for l in r.stdout.splitlines())
+
+
+def _free_port():
+    with socket.socket() as s_:
+        s_.bind(("127.0.0.1", 0))
+        return s_.getsockname()[1]
+
+
+def test_reference_arm_under_torchrun_prints_once_from_rank_0():
+    # the launch the scaling run uses: two ranks; rank 0 alone runs and prints
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                        "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+                        os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny_16x256x512",
+                        "--gpus", "2", "--steps", "3", "--warmup", "3"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2

@@ -24,10 +24,15 @@ CHANNEL_TOKEN = 0
 BLOCK128 = 1
 
 
+# ISO C11 with every warning an error: a compiler that rejects something the
+# source relies on (an implicit declaration, say) fails the build, not the tests.
+WARN_FLAGS = ["-std=c11", "-Wall", "-Wextra", "-Wpedantic", "-Werror"]
+
+
 def build(force: bool = False) -> str:
     """Compile fp8_oracle.c into liboracle.so (gcc, no fast-math, OpenMP)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+        cmd = ["gcc", "-O2"] + WARN_FLAGS + ["-fPIC", "-shared", "-fopenmp",
                "-fno-fast-math", "-ffp-contract=off", "-fvisibility=hidden",
                _SRC, "-o", _LIB + ".tmp", "-lm"]
         subprocess.check_call(cmd)
@@ -68,7 +73,7 @@ def lib() -> ctypes.CDLL:
         _lib.orc_linear_swiglu.restype = None
         _lib.orc_rmsnorm_rstd.argtypes = [P, I, I, I, ctypes.c_float, P]
         _lib.orc_rmsnorm_rstd.restype = None
-        _lib.orc_rmsnorm_quant_rows.argtypes = [P, P, P, I, I, I, P, I, P, P]
+        _lib.orc_rmsnorm_quant_rows.argtypes = [P, P, I, I, I, ctypes.c_float, ctypes.c_int, P, I, P, P, P]
         _lib.orc_rmsnorm_quant_rows.restype = None
     return _lib
 
@@ -156,19 +161,20 @@ def rmsnorm_rstd(x, eps: float = 1e-5) -> np.ndarray:
     return r
 
 
-def rmsnorm_quant_rows(x, gamma, rstd=None, eps: float = 1e-5):
-    """RMSNorm of every row (with the given per-row rstd, else the oracle's),
-    then one amax/448 scale per row.
+def rmsnorm_quant_rows(x, gamma, eps: float = 1e-5, rstd_ulps: int = 0):
+    """RMSNorm of every row with the oracle's own rstd, then one amax/448 scale
+    per row.  rstd_ulps moves that rstd by whole fp32 steps before it is used
+    (0: the definition; the parity tests also use +-1).
     -> (codes u8 [R, K], scales f32 [R], normalised rows bf16 bits u16 [R, K], rstd f32 [R])."""
     xb = _bits(x)
     gb = _bits(gamma).ravel()
     R, K = xb.shape
     assert gb.size == K
-    r = rmsnorm_rstd(xb, eps) if rstd is None else np.ascontiguousarray(rstd, dtype=np.float32)
     q = np.empty((R, K), np.uint8)
     s = np.empty((R,), np.float32)
     y = np.empty((R, K), np.uint16)
-    lib().orc_rmsnorm_quant_rows(_p(xb), _p(gb), _p(r), R, K, K, _p(q), K, _p(s), _p(y))
+    r = np.empty((R,), np.float32)
+    lib().orc_rmsnorm_quant_rows(_p(xb), _p(gb), R, K, K, float(eps), int(rstd_ulps), _p(q), K, _p(s), _p(y), _p(r))
     return q, s, y, r
 
 

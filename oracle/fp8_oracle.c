@@ -130,7 +130,14 @@ static float scale_from_amax(float amax) {
     return num / 448.0f;
 }
 
-static uint16_t float_to_bf16(float f);
+/* Round to the nearest bf16, ties to even (finite inputs). */
+static uint16_t float_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    uint32_t upper = u >> 16, lower = u & 0xFFFFu;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;
+    return (uint16_t)upper;
+}
 
 /* The scale rounded to bf16, the dtype the FP8 checkpoints store scales in
  * (reading: the 72.67 GB of [P4] section 二 matches bf16 scales), before the
@@ -162,69 +169,6 @@ static void quant_rows_impl(const uint16_t* x, int64_t rows, int64_t K, int64_t 
         if (scale_bf16) sr = scale_to_bf16(sr);
         s[r] = sr;
         for (int64_t k = 0; k < K; ++k) q[r * ldq + k] = code_of(bf16_to_float(x[r * ld + k]), sr);
-    }
-}
-
-/* ------------------------------------------------- RMSNorm, then per token */
-/*
- * [P1] section 1.3 (编码器细节：RMSNorm 与 SwiGLU 的实现差异): Llama 3 normalises
- * with RMSNorm before attention and before the MLP, eps = 1e-5; section 5
- * (the fine-tuning notes) keeps RMSNorm in BF16.  So the input of the q/k/v and
- * gate/up projections is y = RMSNorm(x) in bf16, and its per-token
- * quantization is the activation quantization above applied to y.
- * Readings (the pages print no formula): with x in bf16 and gamma the bf16
- * weight,
- *   ms   = mean over the row of x^2, rounded once to fp32
- *   rstd = 1 / sqrt(fl32(ms + eps)), rounded once to fp32
- *   h    = bf16(fl32(x * rstd)),  y = bf16(fl32(gamma * h))
- * (normalise in fp32, return to bf16, then scale by the bf16 weight).
- */
-
-/* Round to the nearest bf16, ties to even (finite inputs). */
-static uint16_t float_to_bf16(float f) {
-    uint32_t u;
-    memcpy(&u, &f, 4);
-    uint32_t upper = u >> 16, lower = u & 0xFFFFu;
-    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;
-    return (uint16_t)upper;
-}
-
-/* Reciprocal RMS of every row.  The sum of squares is accumulated without
- * error (each square of a bf16 value is exact in double; pairs of doubles
- * carry the rounding error of every addition), so ms is the exact mean
- * rounded to fp32 (one double rounding of the quotient first). */
-ORC_EXPORT void orc_rmsnorm_rstd(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, float eps, float* rstd) {
-    for (int64_t r = 0; r < rows; ++r) {
-        double hi = 0.0, lo = 0.0;
-        for (int64_t k = 0; k < K; ++k) {
-            double v = (double)bf16_to_float(x[r * ld + k]);
-            double sq = v * v;
-            double t = hi + sq;                        /* two-sum: t + err == hi + sq exactly */
-            double bb = t - hi;
-            double err = (hi - (t - bb)) + (sq - bb);
-            hi = t;
-            lo += err;
-        }
-        volatile float ms = (float)((hi + lo) / (double)K);
-        volatile float d = ms + eps;                   /* fp32 addition */
-        rstd[r] = (float)(1.0 / sqrt((double)d));
-    }
-}
-
-/* Normalise each row with the given rstd, then quantize it per token.
- * gamma: bf16 bits [K].  q/s as orc_quant_rows; y (bf16 bits [rows, K])
- * receives the normalised rows. */
-ORC_EXPORT void orc_rmsnorm_quant_rows(const uint16_t* x, const uint16_t* gamma, const float* rstd, int64_t rows,
-                                       int64_t K, int64_t ld, uint8_t* q, int64_t ldq, float* s, uint16_t* y) {
-    for (int64_t r = 0; r < rows; ++r) {
-        uint16_t* yr = y + r * K;
-        for (int64_t k = 0; k < K; ++k) {
-            volatile float t = bf16_to_float(x[r * ld + k]) * rstd[r];
-            uint16_t h = float_to_bf16(t);
-            volatile float g = bf16_to_float(gamma[k]) * bf16_to_float(h);
-            yr[k] = float_to_bf16(g);
-        }
-        orc_quant_rows(yr, 1, K, K, q + r * ldq, ldq, s + r);
     }
 }
 
@@ -309,6 +253,176 @@ ORC_EXPORT void orc_quant_groups128_s16(const uint16_t* x, int64_t M, int64_t K,
 ORC_EXPORT void orc_quant_blocks128_s16(const uint16_t* w, int64_t N, int64_t K, int64_t ld,
                                         uint8_t* q, int64_t ldq, float* s) {
     quant_blocks128_impl(w, N, K, ld, q, ldq, s, 1);
+}
+
+/* ------------------------------------------------- RMSNorm, then per token */
+/*
+ * [P1] section 1.3 (编码器细节：RMSNorm 与 SwiGLU 的实现差异): Llama 3 normalises
+ * with RMSNorm before attention and before the MLP, eps = 1e-5; section 5
+ * (the fine-tuning notes) keeps RMSNorm in BF16.  So the input of the q/k/v and
+ * gate/up projections is y = RMSNorm(x) in bf16, and its per-token
+ * quantization is the activation quantization above applied to y.
+ * Readings (the pages print no formula): with x in bf16 and gamma the bf16
+ * weight,
+ *   ms   = the exact mean over the row of x^2, rounded once to fp32
+ *   d    = fl32(ms + eps)
+ *   rstd = 1 / sqrt(d), rounded once to fp32
+ *   h    = bf16(fl32(x * rstd)),  y = bf16(fl32(gamma * h))
+ * (normalise in fp32, return to bf16, then scale by the bf16 weight).
+ * Every rounding above is one IEEE round-to-nearest-even of an exact value,
+ * so the oracle computes each one from the exact value, in integers where a
+ * double would round first.
+ */
+
+/* The exact sum of squares of a row.  A bf16 value is an integer multiple of
+ * 2^-133 (its subnormal step), so its square is an integer multiple of
+ * 2^-266, below 2^256.  The sum is kept as a non-negative integer in units of
+ * 2^-266, in little-endian 64-bit limbs: up to 2^31 squares need 553 bits,
+ * nine limbs hold 576. */
+#define SQ_LIMBS 9
+
+__extension__ typedef unsigned __int128 u128;   /* GCC's 128-bit integer */
+
+static void sq_add(uint64_t* acc, uint16_t b) {
+    int e = (b >> 7) & 0xFF;                 /* |x| = m * 2^(p - 133):                   */
+    uint64_t m = b & 0x7F;                   /*   subnormal (e == 0): m = mantissa, p = 0 */
+    int p = 0;                               /*   normal: m = 128 + mantissa, p = e - 1  */
+    if (e != 0) { m += 128; p = e - 1; }
+    uint64_t sq = m * m;                     /* x^2 = sq * 2^(2p - 266), sq < 2^16      */
+    int bit = 2 * p, li = bit / 64, bo = bit % 64;
+    uint64_t lo = sq << bo, hi = bo ? sq >> (64 - bo) : 0;
+    uint64_t old = acc[li];
+    acc[li] += lo;
+    uint64_t carry = (acc[li] < old) ? 1 : 0;
+    for (int i = li + 1; i < SQ_LIMBS && (hi || carry); ++i) {
+        old = acc[i];
+        acc[i] += hi + carry;                /* hi < 2^16: no double wrap */
+        carry = (acc[i] < old) ? 1 : 0;
+        hi = 0;
+    }
+}
+
+static int sq_bit(const uint64_t* a, int i) { return (int)((a[i / 64] >> (i % 64)) & 1u); }
+
+/* fl32(S * 2^-266 / K) for the integer S in acc: long division by K, then
+ * round to nearest even at 24 significant bits, or at the fixed subnormal
+ * step 2^-149 (bit 117 of the quotient), whichever is coarser. */
+static float sq_mean_f32(const uint64_t* acc, int64_t K) {
+    uint64_t q[SQ_LIMBS];
+    u128 rem = 0;
+    for (int i = SQ_LIMBS - 1; i >= 0; --i) {
+        u128 cur = (rem << 64) | acc[i];
+        q[i] = (uint64_t)(cur / (uint64_t)K);
+        rem = cur % (uint64_t)K;
+    }
+    int top = -1;
+    for (int i = 64 * SQ_LIMBS - 1; i >= 0; --i)
+        if (sq_bit(q, i)) { top = i; break; }
+    if (top < 0) return 0.0f;                /* below 2^-266: rounds to zero */
+    int lsb = top - 23 > 117 ? top - 23 : 117;   /* no bits kept when top < 117 (below 2^-149) */
+    uint32_t mant = 0;
+    for (int i = top; i >= lsb; --i) mant = (mant << 1) | (uint32_t)sq_bit(q, i);
+    int round = sq_bit(q, lsb - 1);
+    int sticky = rem != 0;
+    for (int i = lsb - 2; i >= 0 && !sticky; --i) sticky = sq_bit(q, i);
+    if (round && (sticky || (mant & 1u))) mant += 1u;
+    return ldexpf((float)mant, lsb - 266);
+}
+
+/* x = X * 2^ex with X an integer of at most 24 bits, for a positive finite fp32. */
+static void f32_int_exp(float x, uint64_t* X, int* ex) {
+    int e;
+    float fr = frexpf(x, &e);                /* x = fr * 2^e, fr in [0.5, 1) */
+    *X = (uint64_t)ldexpf(fr, 24);
+    *ex = e - 24;
+}
+
+/* Sign of mid^2 * d - 1, exactly, where mid = (a + b) / 2 for positive fp32
+ * a < b and positive fp32 d. */
+static int mid_sq_d_vs_one(float a, float b, float d) {
+    uint64_t A, B, D;
+    int ea, eb, ed;
+    f32_int_exp(a, &A, &ea);
+    f32_int_exp(b, &B, &eb);
+    f32_int_exp(d, &D, &ed);
+    int e0 = ea < eb ? ea : eb;              /* both on the scale of the smaller exponent */
+    A <<= (ea - e0);
+    B <<= (eb - e0);
+    uint64_t Mid = A + B;                    /* mid = Mid * 2^(e0 - 1), Mid < 2^26 */
+    u128 P = (u128)Mid * Mid * D;   /* < 2^76 */
+    int E = 2 * (e0 - 1) + ed;               /* mid^2 d = P * 2^E */
+    if (E >= 0) return (P == 1 && E == 0) ? 0 : 1;
+    if (-E >= 100) return -1;                /* P < 2^76 < 2^-E */
+    u128 one = (u128)1 << (-E);
+    return P < one ? -1 : (P > one ? 1 : 0);
+}
+
+static int f32_odd(float r) {
+    uint32_t u;
+    memcpy(&u, &r, 4);
+    return (int)(u & 1u);
+}
+
+/* 1 / sqrt(d) rounded to the nearest fp32 (ties to even), for positive finite
+ * d.  A double estimate gives a candidate r; 1/sqrt(d) lies above the
+ * midpoint of r and its upper neighbour exactly when that midpoint squared
+ * times d is below 1, which is decided in integers; r moves until both
+ * midpoints around it bracket 1/sqrt(d). */
+static float rsqrt_f32_rn(float d) {
+    float r = (float)(1.0 / sqrt((double)d));
+    for (;;) {
+        float up = nextafterf(r, INFINITY);
+        int c = mid_sq_d_vs_one(r, up, d);
+        if (c < 0 || (c == 0 && f32_odd(r))) { r = up; continue; }
+        float dn = nextafterf(r, 0.0f);
+        c = mid_sq_d_vs_one(dn, r, d);
+        if (c > 0 || (c == 0 && f32_odd(r))) { r = dn; continue; }
+        return r;
+    }
+}
+
+/* Reciprocal RMS of every row: rstd = RN(1 / sqrt(fl32(ms + eps))) with ms the
+ * exact mean of squares rounded once to fp32.  Rows whose mean of squares
+ * overflows fp32 are outside the definition (rstd 0 is returned for them). */
+ORC_EXPORT void orc_rmsnorm_rstd(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, float eps, float* rstd) {
+    for (int64_t r = 0; r < rows; ++r) {
+        uint64_t acc[SQ_LIMBS] = {0};
+        for (int64_t k = 0; k < K; ++k) sq_add(acc, x[r * ld + k]);
+        float ms = sq_mean_f32(acc, K);
+        volatile float d = ms + eps;                   /* fp32 addition */
+        if (!(d > 0.0f) || isinf(d)) { rstd[r] = d > 0.0f ? 0.0f : INFINITY; continue; }
+        rstd[r] = rsqrt_f32_rn(d);
+    }
+}
+
+/* The fp32 number `ulps` steps away from the positive r (test knob: 0 is r). */
+static float step_ulps(float r, int ulps) {
+    for (; ulps > 0; --ulps) r = nextafterf(r, INFINITY);
+    for (; ulps < 0; ++ulps) r = nextafterf(r, 0.0f);
+    return r;
+}
+
+/* RMSNorm of each row with the oracle's own rstd (moved by `rstd_ulps` fp32
+ * steps: 0 is the definition; the parity tests also take +-1 to accept a
+ * kernel whose rstd is one ulp off), then per-token quantization.
+ * gamma: bf16 bits [K].  q/s as orc_quant_rows; y (bf16 bits [rows, K])
+ * receives the normalised rows and rstd_out [rows] the rstd used. */
+ORC_EXPORT void orc_rmsnorm_quant_rows(const uint16_t* x, const uint16_t* gamma, int64_t rows, int64_t K,
+                                       int64_t ld, float eps, int rstd_ulps, uint8_t* q, int64_t ldq, float* s,
+                                       uint16_t* y, float* rstd_out) {
+    orc_rmsnorm_rstd(x, rows, K, ld, eps, rstd_out);
+    for (int64_t r = 0; r < rows; ++r) {
+        float rs = step_ulps(rstd_out[r], rstd_ulps);
+        rstd_out[r] = rs;
+        uint16_t* yr = y + r * K;
+        for (int64_t k = 0; k < K; ++k) {
+            volatile float t = bf16_to_float(x[r * ld + k]) * rs;
+            uint16_t h = float_to_bf16(t);
+            volatile float g = bf16_to_float(gamma[k]) * bf16_to_float(h);
+            yr[k] = float_to_bf16(g);
+        }
+        orc_quant_rows(yr, 1, K, K, q + r * ldq, ldq, s + r);
+    }
 }
 
 /* ----------------------------------------------------------------- linear */

@@ -103,3 +103,55 @@ def exact_linear_block(xq, xs, wq, ws) -> list:
 def f32_ulp(v: float) -> float:
     v = abs(np.float32(v))
     return float(np.spacing(np.float32(v))) if v > 0 else float(np.spacing(np.float32(0)))
+
+
+def f32_nearest(v: Fraction) -> np.float32:
+    """The fp32 nearest to the exact rational v (ties to even).  Python's
+    Fraction -> float is correctly rounded to double; rounding that double to
+    fp32 again is wrong only when it lands exactly on an fp32 midpoint while v
+    does not, which is then settled by comparing v with that midpoint."""
+    d = float(v)
+    f = np.float32(d)
+    if Fraction(d) != v:
+        lo = np.nextafter(f, np.float32(-np.inf), dtype=np.float32)
+        hi = np.nextafter(f, np.float32(np.inf), dtype=np.float32)
+        for a, b in ((lo, f), (f, hi)):
+            mid = (Fraction(float(a)) + Fraction(float(b))) / 2
+            if Fraction(d) == mid:
+                return b if v > mid else a
+    return f
+
+
+def bf16_bits_sum_of_squares(bits: np.ndarray) -> Fraction:
+    """Exact sum of x^2 over bf16 bit patterns, in Python integers: each bf16
+    value is an integer multiple of 2^-133."""
+    total = 0
+    for b in np.asarray(bits, np.uint16).ravel().tolist():
+        e, m = (b >> 7) & 0xFF, b & 0x7F
+        k = m if e == 0 else (128 + m) << (e - 1)    # |x| = k * 2^-133
+        total += k * k
+    return Fraction(total, 2 ** 266)
+
+
+def rsqrt_f32_mpmath(d: np.float32) -> np.float32:
+    """1 / sqrt(d) rounded to fp32 through mpmath at 200 bits (then to double,
+    then fp32; 1/sqrt of an fp32 value is never an fp32 midpoint, and a
+    200-bit value that rounds to a double midpoint of fp32 is asserted absent)."""
+    import mpmath
+    with mpmath.workprec(200):
+        v = 1 / mpmath.sqrt(mpmath.mpf(float(d)))
+        dv = float(v)
+    f = np.float32(dv)
+    lo = np.nextafter(f, np.float32(0), dtype=np.float32)
+    hi = np.nextafter(f, np.float32(np.inf), dtype=np.float32)
+    for a, b in ((lo, f), (f, hi)):
+        assert Fraction(dv) != (Fraction(float(a)) + Fraction(float(b))) / 2, "double landed on an fp32 midpoint"
+    return f
+
+
+def rmsnorm_rstd_exact(bits_row: np.ndarray, eps: float) -> np.float32:
+    """rstd = RN32(1 / sqrt(RN32(RN32(mean x^2) + eps))) from exact arithmetic."""
+    K = np.asarray(bits_row).size
+    ms = f32_nearest(bf16_bits_sum_of_squares(bits_row) / K)
+    d = np.float32(ms + np.float32(eps))       # one fp32 addition
+    return rsqrt_f32_mpmath(d)

@@ -35,9 +35,11 @@ MUTANTS = {
     "block x_scale column": (r"xs\[m \* KB \+ kb\]", "xs[m * KB]"),
     "group of 64": (r"for \(int64_t k = g \* 128; k < g \* 128 \+ 128; \+\+k\) \{", "for (int64_t k = g * 128; k < g * 128 + 64; ++k) {"),
     "amax = 0 gives scale 0": (r"if \(amax == 0\.0f\) return 1\.0f;", "if (amax == 0.0f) return 0.0f;"),
-    "rms without the square root": (r"rstd\[r\] = \(float\)\(1\.0 / sqrt\(\(double\)d\)\);",
-                                    "rstd[r] = (float)(1.0 / (double)d);"),
-    "rms mean over K - 1": (r"\(hi \+ lo\) / \(double\)K\)", "(hi + lo) / (double)(K - 1))"),
+    "rms without the square root": (r"rstd\[r\] = rsqrt_f32_rn\(d\);", "rstd[r] = 1.0f / d;"),
+    "rms mean over K - 1": (r"float ms = sq_mean_f32\(acc, K\);", "float ms = sq_mean_f32(acc, K - 1);"),
+    "rms sum of |x| not x^2": (r"uint64_t sq = m \* m;", "uint64_t sq = m;"),
+    "rms subnormal exponent": (r"if \(e != 0\) \{ m \+= 128; p = e - 1; \}", "if (e != 0) { m += 128; p = e; }"),
+    "rsqrt rounds up": (r"uint64_t Mid = A \+ B;", "uint64_t Mid = A + A;"),
     "rms eps ignored": (r"volatile float d = ms \+ eps;", "volatile float d = ms;"),
     "rms gamma dropped": (r"volatile float g = bf16_to_float\(gamma\[k\]\) \* bf16_to_float\(h\);",
                           "volatile float g = bf16_to_float(h);"),
@@ -60,7 +62,7 @@ def build_variant(src_text, tmp):
     so = os.path.join(tmp, "o.so")
     open(c, "w").write(src_text)
     subprocess.check_call(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off",
-                           c, "-o", so, "-lm"])
+                           "-Wno-unused-variable", c, "-o", so, "-lm"])
     L = ctypes.CDLL(so)
     P, I = ctypes.c_void_p, ctypes.c_int64
     L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
@@ -70,7 +72,7 @@ def build_variant(src_text, tmp):
         getattr(L, f).argtypes = [P, I, I, I, P, I, P]
     L.orc_linear.argtypes = [P, P, P, P, I, I, I, I, I, ctypes.c_int, P]
     L.orc_rmsnorm_rstd.argtypes = [P, I, I, I, ctypes.c_float, P]
-    L.orc_rmsnorm_quant_rows.argtypes = [P, P, P, I, I, I, P, I, P, P]
+    L.orc_rmsnorm_quant_rows.argtypes = [P, P, I, I, I, ctypes.c_float, ctypes.c_int, P, I, P, P, P]
     L.orc_linear_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, P]
     L.orc_quant_static.argtypes = [P, I, I, I, ctypes.c_float, P, I]
     L.orc_linear_w8a16.argtypes = [P, P, P, I, I, I, P]
@@ -199,10 +201,28 @@ def checks(L):
     rref = (1.0 / torch.sqrt((ms + torch.tensor(1e-5, dtype=torch.float32)).double())).float().numpy()
     if np.abs(rs.view(np.int32).astype(np.int64) - rref.view(np.int32).astype(np.int64)).max() > 1:
         failed.append("rmsnorm rstd")
+    # rstd exactly: rational mean of squares, mpmath reciprocal square root
+    if any(rs[i] != _pins.rmsnorm_rstd_exact(xrb[i], 1e-5) for i in range(4)):
+        failed.append("rmsnorm rstd exact")
+    xe = synth.make_x(24, 64, seed=8)
+    xeb = xe.view(torch.int16).numpy().view(np.uint16).copy()
+    re_ = np.empty(24, np.float32)
+    L.orc_rmsnorm_rstd(_p(xeb), 24, 64, 64, ctypes.c_float(1e-5), _p(re_))
+    if any(re_[i] != _pins.rmsnorm_rstd_exact(xeb[i], 1e-5) for i in range(24)):
+        failed.append("rmsnorm rstd exact, short rows")
+    xt = np.zeros((1, 64), np.uint16)
+    xt[0, 5] = 0x0001                       # the smallest subnormal, with a normal value beside it
+    xt[0, 6] = 0x3F80                       # 1.0
+    rt = np.empty(1, np.float32)
+    L.orc_rmsnorm_rstd(_p(xt), 1, 64, 64, ctypes.c_float(0.0), _p(rt))
+    if rt[0] != _pins.rmsnorm_rstd_exact(xt[0], 0.0):
+        failed.append("rmsnorm rstd subnormal")
     qr = np.empty((4, Kr), np.uint8)
     sr = np.empty(4, np.float32)
     yr = np.empty((4, Kr), np.uint16)
-    L.orc_rmsnorm_quant_rows(_p(xrb), _p(grb), _p(rref.copy()), 4, Kr, Kr, _p(qr), Kr, _p(sr), _p(yr))
+    ro = np.empty(4, np.float32)
+    L.orc_rmsnorm_quant_rows(_p(xrb), _p(grb), 4, Kr, Kr, ctypes.c_float(1e-5), 0, _p(qr), Kr, _p(sr), _p(yr),
+                             _p(ro))
     yref = torch.nn.functional.rms_norm(xr.double(), (Kr,), weight=gr.double(), eps=1e-5)
     yt = torch.from_numpy(yr.astype(np.int16)).view(torch.bfloat16).double()
     if not torch.all((yt - yref).abs() <= 2.0 ** -7 * yref.abs() * 1.001 + 1e-30):

@@ -3,9 +3,12 @@
 Llama 3 normalises with RMSNorm (eps = 1e-5) before attention and the MLP
 ("Llama 3 精读实录", section 1.3) and keeps it in BF16 (section 5), so the
 activations the q/k/v and gate/up projections quantize are RMSNorm outputs.
-The oracle is checked against float64 references computed here by torch (the
-mean of squares, torch.nn.functional.rms_norm) and against properties that
-hold exactly: power-of-two invariance, zero and constant rows, gamma scaling.
+The oracle is checked against exact arithmetic (the mean of squares as a
+Python rational, rounded once to fp32; the reciprocal square root from mpmath
+at 200 bits, rounded once), against float64 references computed here by torch
+(the mean of squares, torch.nn.functional.rms_norm) and against properties
+that hold exactly: power-of-two invariance, zero and constant rows, gamma
+scaling.
 """
 import numpy as np
 import pytest
@@ -35,6 +38,55 @@ def test_rstd_is_the_rounded_reciprocal_rms(M, K, eps):
     ref = (1.0 / torch.sqrt(d.double())).float().numpy()
     ulps = np.abs(r.view(np.int32).astype(np.int64) - ref.view(np.int32).astype(np.int64))
     assert ulps.max() <= 1, f"rstd differs by {ulps.max()} ulp"
+
+
+def _bits(x: torch.Tensor) -> np.ndarray:
+    return x.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("K,eps", [(16, 1e-5), (3072, 1e-5), (4096, 1e-6), (8192, 1e-5), (1040, 0.0),
+                                   (65536, 1e-5)])
+def test_rstd_is_exactly_rounded(K, eps):
+    # ms: the exact rational mean of squares (Python integers) rounded once to
+    # fp32; rstd: 1/sqrt of fl32(ms + eps) from mpmath, rounded once
+    x = synth.make_x(3, K, seed=K + 1)
+    r = oracle.rmsnorm_rstd(x, eps)
+    b = _bits(x)
+    for i in range(3):
+        assert r[i] == _pins.rmsnorm_rstd_exact(b[i], eps), f"row {i}"
+
+
+def test_rstd_exact_on_special_rows():
+    K = 512
+    rows = torch.zeros(7, K, dtype=torch.bfloat16)
+    rows[0] = synth.make_x(1, K, seed=1)[0] * 2.0 ** -70    # squares below fp32's normal range
+    rows[1, 3] = 2.0 ** -133                                 # the smallest bf16 subnormal
+    rows[1, 9] = 1.5 * 2.0 ** -127                           # a bf16 subnormal
+    rows[2] = synth.make_x(1, K, seed=2)[0] * 2.0 ** 40      # large squares
+    rows[3, ::3] = 3.0                                       # a third of the row constant
+    rows[4] = synth.make_x(1, K, seed=4)[0]
+    rows[4, 17] = 2.0 ** 30                                  # one value dominating the sum
+    rows[5] = 1.0                                            # mean of squares exactly 1
+    b = _bits(rows)
+    for eps in (0.0, 1e-5):
+        r = oracle.rmsnorm_rstd(rows, eps)
+        for i in range(7):
+            ms = _pins.f32_nearest(_pins.bf16_bits_sum_of_squares(b[i]) / K)
+            if eps == 0.0 and ms == 0:
+                assert r[i] == np.inf, f"row {i}: mean of squares rounds to 0, rstd = 1/sqrt(0)"
+                continue
+            assert r[i] == _pins.rmsnorm_rstd_exact(b[i], eps), f"row {i} eps {eps}"
+    # mean of squares 1 and eps 0: rstd exactly 1
+    assert oracle.rmsnorm_rstd(rows[5:6], 0.0)[0] == 1.0
+
+
+def test_rstd_ulps_moves_rstd_by_whole_steps():
+    x = synth.make_x(4, 256, seed=5)
+    g = _gamma(256, seed=5)
+    _, _, _, r0 = oracle.rmsnorm_quant_rows(x, g)
+    for u in (-1, 1, 3):
+        _, _, _, ru = oracle.rmsnorm_quant_rows(x, g, rstd_ulps=u)
+        assert np.array_equal(ru.view(np.int32) - r0.view(np.int32), np.full(4, u, np.int32))
 
 
 @pytest.mark.parametrize("M,K", [(6, 3072), (3, 4096), (2, 8192)])

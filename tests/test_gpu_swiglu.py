@@ -44,6 +44,12 @@ def run(M, N, K, seed, rows=None):
     xq, xs = fq.fp8_quant_act(x.to(DEV))
     gq, gs = fq.fp8_quant_weight(wg.to(DEV))
     uq, us = fq.fp8_quant_weight(wu.to(DEV))
+    # the codes and scales the GEMM consumes are first checked against the
+    # oracle's own quantization of the same bf16 tensors
+    for (q, s), t, what in (((xq, xs), x, "x"), ((gq, gs), wg, "w_gate"), ((uq, us), wu, "w_up")):
+        rq, rs = oracle.quant_rows(t)
+        P.assert_codes_equal(q, rq, f"swiglu {what} codes")
+        P.assert_scales_equal(s, rs, f"swiglu {what} scales")
     act = fq.fp8_linear_swiglu(xq, xs, gq, gs, uq, us)
     return act, (xq, xs, gq, gs, uq, us)
 

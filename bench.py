@@ -9,7 +9,10 @@ every GEMM runs.  Weights are quantized once at load time, outside the step
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...     # the CPU oracle, timed on a sample
 
-The L2 cache (126 MB) is flushed by a 256 MiB write before every step; each
+The L2 cache (126 MB) is flushed before every step and before every timed
+op: a 256 MiB buffer is written, then another 256 MiB buffer is read, so the
+timed kernels start with a cold L2 that holds no dirty lines (a write alone
+would leave 126 MB of dirty lines for the timed kernel to write back).  Each
 step and each kernel launch is timed with CUDA events on the launching stream,
 so the flush is not counted.  With N > 1 (torchrun, one rank per GPU) every
 rank runs its own batch of tokens against replicated weights (token-parallel,
@@ -19,6 +22,7 @@ the slowest rank's time.  Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -26,7 +30,6 @@ import subprocess
 import sys
 import threading
 import time
-import zlib
 
 import numpy as np
 import torch
@@ -36,7 +39,7 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
-DEFAULT_WORKLOAD = "llama3.2-3b_mlp_m2048"
+DEFAULT_WORKLOAD = "llama3.1-70b_sweep"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -51,14 +54,17 @@ def parse():
     ap.add_argument("--impl", default="fp8q", choices=["fp8q", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--flush-mib", type=int, default=256)
-    ap.add_argument("--cpu-sample-rows", type=int, default=256,
-                    help="rows of every GEMM the CPU oracle runs for cpu_baseline")
-    ap.add_argument("--ref-sample-rows", type=int, default=32,
+    ap.add_argument("--cpu-sample-rows", type=int, default=16,
+                    help="rows of every GEMM the CPU oracle starts its cpu_baseline sample with")
+    ap.add_argument("--ref-sample-rows", type=int, default=8,
                     help="rows of every GEMM one reference-arm step runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true",
                     help="launch every op from Python each step instead of replaying CUDA graphs")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the next-step sections (RMSNorm, SwiGLU, static scales, KV cache, weight-only, "
+                         "merged GEMMs): for short profiling runs")
     ap.add_argument("--only", default="",
                     help="comma-separated GEMM names: restrict the workload to them (profiling)")
     return ap.parse_args()
@@ -314,8 +320,33 @@ def aggregate(units_local: float, seconds_local: float, world: int):
     return sum_over_ranks(units_local, world), max_over_ranks(seconds_local, world)
 
 
-def launches_of(g) -> int:
-    return 1                              # one kernel per GEMM (decode reduces inside its kernel)
+def decode_reduce_launched(g, sms: int) -> bool:
+    """Whether fp8_linear launches its separate split-sum kernel after the
+    decode GEMM (M <= 64): the library's dispatch rule, restated for counting."""
+    if g.M > 64:
+        return False
+    n_tiles, kb = -(-g.N // 128), -(-g.K // 128)
+    total = n_tiles * kb
+    G = min(total, sms)
+    nx = 16 if g.M <= 16 else (32 if g.M <= 32 else 64)
+    if g.mode == synth.BLOCK128:
+        return True
+    return not (nx == 16 or total >= kb * G)
+
+
+def launches_of(g, sms: int) -> int:
+    return 1 + int(decode_reduce_launched(g, sms))
+
+
+def config_of(wl, world: int, flush_mib: int) -> dict:
+    """The workload description both arms print (the same dict for the same run)."""
+    return {"workload": wl.name,
+            "gemms": [f"{g.name}:{g.M}x{g.K}->{g.N}:{'channel' if g.mode == 0 else 'block128'}" for g in wl.gemms],
+            "weights": sorted({g.weight for g in wl.gemms}),
+            "step": "quantize each activation + every FP8 GEMM; weights quantized at load",
+            "l2": f"GPU arm: L2 flushed before every step and every timed op, outside the timed events: a "
+                  f"{flush_mib} MiB buffer written, then another {flush_mib} MiB read (cold, clean L2)",
+            "parallelism": "single device" if world == 1 else f"token-parallel x{world}, weights replicated"}
 
 
 def run_gpu(args):
@@ -328,26 +359,45 @@ def run_gpu(args):
     wl = select(args)
     metric, unit = metric_for(wl)
     pk = peaks()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
     # ---- load time: weights (replicated), quantized once
     W = {}
     for g in wl.gemms:
-        w = synth.make_w(g.N, g.K, seed=zlib.crc32(g.name.encode()) % 1000).to(dev) if g.N * g.K <= (1 << 26) \
-            else synth.make_w_device(g.N, g.K, seed=zlib.crc32(g.name.encode()) % 1000, device=dev)
-        W[g.name] = w
+        if g.weight in W:
+            continue
+        seed = synth.weight_seed(g.weight)
+        W[g.weight] = synth.make_w(g.N, g.K, seed=seed).to(dev) if g.N * g.K <= (1 << 26) \
+            else synth.make_w_device(g.N, g.K, seed=seed, device=dev)
     xs_shapes = {}
     for g in wl.gemms:
         xs_shapes.setdefault(g.x, (g.M, g.K, g.mode))
     X = {k: synth.make_x_device(M, K, seed=x_seed(rank, i), device=dev)
          for i, (k, (M, K, _)) in enumerate(xs_shapes.items())}
-    WQ = {g.name: fq.fp8_quant_weight(W[g.name], g.mode) for g in wl.gemms}
+    WQ = {}
+    for g in wl.gemms:
+        if g.weight not in WQ:
+            WQ[g.weight] = fq.fp8_quant_weight(W[g.weight], g.mode)
     XQ = {k: (torch.empty((M, K), dtype=torch.uint8, device=dev),
               torch.empty(fq.scale_shape_act(M, K, mode), dtype=torch.float32, device=dev))
           for k, (M, K, mode) in xs_shapes.items()}
     Y = {g.name: torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev) for g in wl.gemms}
     WS = {g.name: (torch.zeros(fq.fp8_linear_workspace_size(g.M, g.N, g.K, g.mode), dtype=torch.uint8,
                                device=dev) if g.M <= 64 else None) for g in wl.gemms}
-    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
+    class _Flush:
+        """Write one buffer larger than L2, then read another: L2 ends up
+        holding only clean lines of the read buffer."""
+
+        def __init__(self, mib):
+            self.w = torch.empty(mib << 20, dtype=torch.uint8, device=dev)
+            self.r = torch.ones(mib << 17, dtype=torch.int64, device=dev)
+            self.sink = torch.empty((), dtype=torch.int64, device=dev)
+
+        def zero_(self):
+            self.w.zero_()
+            torch.amax(self.r, dim=0, out=self.sink)
+
+    flush = _Flush(args.flush_mib)
     stream = torch.cuda.current_stream(dev)
 
     n_ops = len(xs_shapes) + len(wl.gemms)
@@ -359,7 +409,7 @@ def run_gpu(args):
         for g in wl.gemms:
             def op(g=g):
                 xq, xsc = XQ[g.x]
-                wq, wsc = WQ[g.name]
+                wq, wsc = WQ[g.weight]
                 fq.fp8_linear(xq, xsc, wq, wsc, g.mode, out=Y[g.name], workspace=WS[g.name])
             ops.append(op)
         return ops
@@ -457,17 +507,17 @@ def run_gpu(args):
     groups = {}
     for g in wl.gemms:
         groups.setdefault((g.x, g.mode), []).append(g)
-    if not args.eager and any(len(v) > 1 for v in groups.values()):
+    if not args.eager and not args.no_extras and any(len(v) > 1 for v in groups.values()):
         mops, mnames = [], []
         for (xk, mode), gs in groups.items():
             if len(gs) == 1:
                 g = gs[0]
-                mops.append(lambda g=g: fq.fp8_linear(XQ[g.x][0], XQ[g.x][1], WQ[g.name][0], WQ[g.name][1], g.mode,
+                mops.append(lambda g=g: fq.fp8_linear(XQ[g.x][0], XQ[g.x][1], WQ[g.weight][0], WQ[g.weight][1], g.mode,
                                                       out=Y[g.name], workspace=WS[g.name]))
                 mnames.append(g.name)
                 continue
-            wq_m = torch.cat([WQ[g.name][0] for g in gs])
-            ws_m = torch.cat([WQ[g.name][1] for g in gs])
+            wq_m = torch.cat([WQ[g.weight][0] for g in gs])
+            ws_m = torch.cat([WQ[g.weight][1] for g in gs])
             M, K, Nm = gs[0].M, gs[0].K, sum(g.N for g in gs)
             y_m = torch.empty((M, Nm), dtype=torch.bfloat16, device=dev)
             nws = fq.fp8_linear_workspace_size(M, Nm, K, mode)
@@ -495,50 +545,68 @@ def run_gpu(args):
                   "ms_per_step": round(mt * 1e3 / args.steps, 4), "gemms": mnames,
                   "note": "same step, GEMMs sharing an input launched as one GEMM over stacked weights"}
 
-    # ---- per-kernel detail and the dominant kernel's roofline
+    # ---- per-kernel detail and the rooflines: the dominant kernel of the
+    # step, and the dominant prefill GEMM, decode GEMM and quantize launch
     names = [f"quant_act[{k}]" for k in xs_shapes] + [g.name for g in wl.gemms]
     detail = []
     fp8_peak = pk["bf16_tflops"] * FP8_OVER_BF16
     for i, (k, (M, K, mode)) in enumerate(xs_shapes.items()):
         b = quant_bytes(M, K, mode)
-        detail.append({"op": names[i], "kernel": "quant_rows" if mode == 0 else "quant_groups128",
+        detail.append({"op": names[i], "kernel": "quant_rows" if mode == 0 else "quant_groups128", "bound": "hbm",
+                       "M": M, "K": K, "mode": mode,
                        "ms": round(float(op_ms[i]), 5), "GB/s": round(b / (op_ms[i] / 1e3) / 1e9, 1),
                        "frac_hbm": round(b / (op_ms[i] / 1e3) / 1e9 / pk["hbm_gbs"], 3)})
     for j, g in enumerate(wl.gemms):
         t = op_ms[len(xs_shapes) + j] / 1e3
         kern = ("gemm_decode" if g.M <= 64 else
                 ("gemm_block" if g.mode == synth.BLOCK128 else "gemm_channel"))
-        detail.append({"op": g.name, "kernel": kern, "M": g.M, "N": g.N, "K": g.K, "mode": g.mode,
+        detail.append({"op": g.name, "kernel": kern, "bound": "hbm" if g.M <= 64 else "tensor",
+                       "M": g.M, "N": g.N, "K": g.K, "mode": g.mode,
                        "ms": round(float(op_ms[len(xs_shapes) + j]), 5),
                        "TFLOP/s": round(g.flops / t / 1e12, 1),
                        "GB/s": round(gemm_bytes(g) / t / 1e9, 1),
                        "frac_fp8_peak": round(g.flops / t / 1e12 / fp8_peak, 3),
                        "frac_hbm": round(gemm_bytes(g) / t / 1e9 / pk["hbm_gbs"], 3)})
-    gemm_ops = detail[len(xs_shapes):]
-    dom = max(gemm_ops, key=lambda d: d["ms"])
-    gsel = [g for g in wl.gemms if g.name == dom["op"]][0]
-    if unit == "TFLOP/s":
-        roof = {"kernel": dom["kernel"], "bound": "tensor", "achieved": dom["TFLOP/s"],
-                "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
-                "frac": round(dom["TFLOP/s"] / fp8_peak, 3),
-                "peak_basis": f"{pk['source']} bf16 burst {pk['bf16_tflops']} TFLOP/s x {FP8_OVER_BF16} "
-                              "(nominal fp8/bf16 dense ratio)",
-                "algorithmic": f"2*M*N*K = {gsel.flops} flop per launch", "traffic": None}
-    else:
-        roof = {"kernel": dom["kernel"], "bound": "hbm", "achieved": dom["GB/s"], "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": round(dom["GB/s"] / pk["hbm_gbs"], 3),
-                "peak_basis": f"{pk['source']} HBM copy bandwidth",
-                "algorithmic": f"M*K + N*K + 2*M*N + scales = {gemm_bytes(gsel)} bytes per launch",
-                "traffic": None}
+    gemm_by_name = {g.name: g for g in wl.gemms}
+    traffic = {}
     tfile = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tfile):
         try:
-            tr = json.load(open(tfile)).get(f"{args.workload}:{dom['op']}")
-            if tr and tr.get("kernel", "").startswith(dom["kernel"]):
-                roof["traffic"] = tr["bytes"]
-                roof["traffic_source"] = tr["summary"]
+            traffic = json.load(open(tfile))
         except Exception:
-            pass
+            traffic = {}
+
+    def roofline_of(d):
+        if d["bound"] == "tensor":
+            g = gemm_by_name[d["op"]]
+            r = {"op": d["op"], "kernel": d["kernel"], "bound": "tensor", "achieved": d["TFLOP/s"],
+                 "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(d["TFLOP/s"] / fp8_peak, 3),
+                 "peak_basis": f"{pk['source']} bf16 burst {pk['bf16_tflops']} TFLOP/s x {FP8_OVER_BF16} "
+                               "(nominal fp8/bf16 dense ratio), of measured",
+                 "algorithmic": f"2*M*N*K = {g.flops} flop per launch", "traffic": None}
+        else:
+            if d["op"] in gemm_by_name:
+                alg = f"M*K + N*K + 2*M*N + scales = {gemm_bytes(gemm_by_name[d['op']])} bytes per launch"
+            else:
+                alg = f"2*M*K (bf16 in) + M*K (codes) + 4 per scale = {quant_bytes(d['M'], d['K'], d['mode'])} bytes per launch"
+            r = {"op": d["op"], "kernel": d["kernel"], "bound": "hbm", "achieved": d["GB/s"], "peak": pk["hbm_gbs"],
+                 "unit": "GB/s", "frac": round(d["GB/s"] / pk["hbm_gbs"], 3),
+                 "peak_basis": f"{pk['source']} HBM copy bandwidth, of measured", "algorithmic": alg, "traffic": None}
+        tr = traffic.get(f"{wl.name}:{d['op']}")
+        if tr and tr.get("kernel", "").startswith(d["kernel"]):
+            r["traffic"] = tr["bytes"]
+            r["traffic_source"] = tr["summary"]
+        return r
+
+    gemm_ops = detail[len(xs_shapes):]
+    dom = max(gemm_ops, key=lambda d: d["ms"])
+    roof = roofline_of(dom)
+    rooflines = {}
+    for kind, sel in (("prefill", [d for d in gemm_ops if d["bound"] == "tensor"]),
+                      ("decode", [d for d in gemm_ops if d["bound"] == "hbm"]),
+                      ("quantize", detail[:len(xs_shapes)])):
+        if sel:
+            rooflines[kind] = roofline_of(max(sel, key=lambda d: d["ms"]))
 
     # ---- weight quantization (load-time kernel) timed alone
     wq_ms = []
@@ -547,7 +615,7 @@ def run_gpu(args):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        fq.fp8_quant_weight(W[g0.name], g0.mode, out=WQ[g0.name])
+        fq.fp8_quant_weight(W[g0.weight], g0.mode, out=WQ[g0.weight])
         e1.record(stream)
         torch.cuda.synchronize()
         wq_ms.append(e0.elapsed_time(e1))
@@ -560,7 +628,7 @@ def run_gpu(args):
     # an RMSNorm in Llama: the inputs of q/k/v and of gate/up), timed alone,
     # next to the unfused pair (torch's bf16 rms_norm, then fp8_quant_act)
     rms = []
-    for k, (M, K, mode) in xs_shapes.items():
+    for k, (M, K, mode) in ([] if args.no_extras else xs_shapes.items()):
         if mode != synth.CHANNEL_TOKEN or not (k.startswith("attn_in") or k.startswith("mlp_in")):
             continue
         gmm = (1.0 + 0.1 * torch.randn(K, generator=torch.Generator().manual_seed(K))).to(torch.bfloat16).to(dev)
@@ -604,7 +672,7 @@ def run_gpu(args):
     for g in wl.gemms:
         if g.mode == synth.CHANNEL_TOKEN and (g.name.startswith("gate_proj") or g.name.startswith("up_proj")):
             gmap[g.name.replace("gate_proj", "").replace("up_proj", "")].append(g)
-    for suffix, gs in gmap.items():
+    for suffix, gs in ([] if args.no_extras else gmap.items()):
         gg = [g for g in gs if g.name.startswith("gate_proj")]
         gu = [g for g in gs if g.name.startswith("up_proj")]
         if len(gg) != 1 or len(gu) != 1:
@@ -613,12 +681,12 @@ def run_gpu(args):
         act = torch.empty((gg.M, gg.N), dtype=torch.bfloat16, device=dev)
 
         def fused(gg=gg, gu=gu, act=act):
-            fq.fp8_linear_swiglu(XQ[gg.x][0], XQ[gg.x][1], WQ[gg.name][0], WQ[gg.name][1], WQ[gu.name][0],
-                                 WQ[gu.name][1], out=act)
+            fq.fp8_linear_swiglu(XQ[gg.x][0], XQ[gg.x][1], WQ[gg.weight][0], WQ[gg.weight][1], WQ[gu.weight][0],
+                                 WQ[gu.weight][1], out=act)
 
         def separate(gg=gg, gu=gu, act=act):
             for g in (gg, gu):
-                fq.fp8_linear(XQ[g.x][0], XQ[g.x][1], WQ[g.name][0], WQ[g.name][1], g.mode, out=Y[g.name],
+                fq.fp8_linear(XQ[g.x][0], XQ[g.x][1], WQ[g.weight][0], WQ[g.weight][1], g.mode, out=Y[g.name],
                               workspace=WS[g.name])
             torch.mul(torch.nn.functional.silu(Y[gg.name]), Y[gu.name], out=act)
 
@@ -648,7 +716,7 @@ def run_gpu(args):
 
     # ---- static-scale quantization (offline-calibrated scale, no amax pass)
     qstatic = []
-    for k, (M, K, mode) in xs_shapes.items():
+    for k, (M, K, mode) in ([] if args.no_extras else xs_shapes.items()):
         if mode != synth.CHANNEL_TOKEN:
             continue
         sc = fq.calibrate_static_scale(X[k][: min(M, 256)])
@@ -673,7 +741,7 @@ def run_gpu(args):
 
     # ---- FP8 KV cache: the k_proj / v_proj outputs quantized per (token, head)
     kvq = []
-    for g in wl.gemms:
+    for g in ([] if args.no_extras else wl.gemms):
         if g.name not in ("k_proj", "v_proj") or g.N % 128:
             continue
         kv = Y[g.name].view(g.M, g.N // 128, 128)
@@ -715,17 +783,17 @@ def run_gpu(args):
         return float(np.median([a.elapsed_time(b) for a, b in ev]))
 
     w8a16 = []
-    for g in wl.gemms:
+    for g in ([] if args.no_extras else wl.gemms):
         if g.mode != synth.CHANNEL_TOKEN or g.M > 64:
             continue
         y16 = torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev)
         xq_w, xs_w = torch.empty_like(XQ[g.x][0]), torch.empty_like(XQ[g.x][1])
         wk16 = torch.zeros(max(16, fq.fp8_linear_w8a16_workspace_size(g.M, g.N, g.K)), dtype=torch.uint8, device=dev)
-        t16 = time_graph(lambda g=g, y16=y16, wk16=wk16: fq.fp8_linear_w8a16(X[g.x], WQ[g.name][0], WQ[g.name][1],
+        t16 = time_graph(lambda g=g, y16=y16, wk16=wk16: fq.fp8_linear_w8a16(X[g.x], WQ[g.weight][0], WQ[g.weight][1],
                                                                            out=y16, workspace=wk16))
         t8 = time_graph(lambda g=g, y16=y16, xq_w=xq_w, xs_w=xs_w: (
             fq.fp8_quant_act(X[g.x], g.mode, out=(xq_w, xs_w)),
-            fq.fp8_linear(xq_w, xs_w, WQ[g.name][0], WQ[g.name][1], g.mode, out=y16, workspace=WS[g.name])))
+            fq.fp8_linear(xq_w, xs_w, WQ[g.weight][0], WQ[g.weight][1], g.mode, out=y16, workspace=WS[g.name])))
         wb = g.N * g.K + 2 * g.M * g.K + 4 * g.N + 2 * g.M * g.N
         w8a16.append({"gemm": g.name, "M": g.M, "N": g.N, "K": g.K, "ms": round(t16, 5),
                       "GB/s": round(wb / (t16 / 1e3) / 1e9, 1), "frac_hbm": round(wb / (t16 / 1e3) / 1e9 / pk["hbm_gbs"], 3),
@@ -746,7 +814,7 @@ def run_gpu(args):
                 fq.fp8_quant_act(Xd[k], mode, out=XQ[k])
             for g in wl.gemms:
                 xq, xsc = XQ[g.x]
-                wq, wsc = WQ[g.name]
+                wq, wsc = WQ[g.weight]
                 fq.fp8_linear(xq, xsc, wq, wsc, g.mode, out=Y[g.name], workspace=WS[g.name])
                 Yh[g.name].copy_(Y[g.name], non_blocking=True)
 
@@ -782,16 +850,11 @@ def run_gpu(args):
             "ms_per_step": round(total_s * 1e3 / args.steps, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp8_e4m3 (fp32 accumulate, bf16 out)", "data": "synthetic",
-            "config": {"workload": wl.name,
-                       "gemms": [f"{g.name}:{g.M}x{g.K}->{g.N}:{'channel' if g.mode == 0 else 'block128'}"
-                                 for g in wl.gemms],
-                       "step": "quantize each activation + every FP8 GEMM; weights quantized at load",
-                       "l2": f"flushed ({args.flush_mib} MiB write) before every step, outside the timed events",
-                       "launch": "eager" if args.eager else
-                       "step: one CUDA graph replayed per step; per-op detail: each op's own graph, timed alone",
-                       "parallelism": "single GPU" if world == 1 else f"token-parallel x{world}, weights replicated"},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g) for g in wl.gemms)),
+            "config": config_of(wl, world, args.flush_mib),
+            "launch": "eager" if args.eager else
+            "step: one CUDA graph replayed per step; per-op detail: each op's own graph, timed alone",
+            "roofline": roof, "rooflines": rooflines, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g, sms) for g in wl.gemms)),
             "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant, "rmsnorm_quant": rms, "kv_quant": kvq, "swiglu": swiglu, "quant_static": qstatic, "w8a16": w8a16,
             "merged_shared_input": merged,
             "device_error": err, "gpu": torch.cuda.get_device_name(dev),
@@ -804,16 +867,17 @@ def run_gpu(args):
 # ----------------------------------------------------------- CPU oracle ---
 
 def oracle_sample(wl, rows, w_cache=None):
-    """Run the oracle on `rows` rows of every GEMM (all N, all K); returns
-    (seconds, rows used per GEMM, threads)."""
+    """Run the oracle on `rows` rows of every GEMM (all N, all K), after its
+    activation quantization; returns (seconds, weight cache).  Weights are
+    quantized by the oracle once, before timing, as in the GPU step."""
     import oracle
     oracle.build()
     if w_cache is None:
         w_cache = {}
     for g in wl.gemms:
-        if g.name not in w_cache:
-            w = synth.make_w(g.N, g.K, seed=zlib.crc32(g.name.encode()) % 1000)
-            w_cache[g.name] = oracle.quant_weight(w, g.mode)
+        if g.weight not in w_cache:
+            w = synth.make_w(g.N, g.K, seed=synth.weight_seed(g.weight))
+            w_cache[g.weight] = oracle.quant_weight(w, g.mode)
     xs = {}
     for g in wl.gemms:
         if g.x not in xs:
@@ -825,9 +889,14 @@ def oracle_sample(wl, rows, w_cache=None):
             q[g.x] = oracle.quant_act(xs[g.x], g.mode)
     for g in wl.gemms:
         xq, xsc = q[g.x]
-        wq, wsc = w_cache[g.name]
+        wq, wsc = w_cache[g.weight]
         oracle.linear(xq, xsc, wq, wsc, g.mode)
     return time.perf_counter() - t0, w_cache
+
+
+def sample_workload(wl, rows):
+    """The workload with every GEMM cut to its first `rows` token rows."""
+    return synth.Workload(wl.name, [dataclasses.replace(g, M=min(rows, g.M)) for g in wl.gemms])
 
 
 def omp_threads():
@@ -842,9 +911,10 @@ def omp_threads():
 
 def cpu_baseline(wl, unit, rows, w_cache=None, target_s=10.0):
     """The oracle on the host cores, timed over a bounded sample of the
-    workload: `rows` token rows of every GEMM, grown (up to each GEMM's M)
-    while one pass takes well under target_s, then passes repeated until about
-    target_s of CPU work; extrapolated linearly in M to the whole workload."""
+    workload: the first `rows` token rows of every GEMM (all N, all K),
+    grown (up to each GEMM's M) while one pass takes well under target_s,
+    then passes repeated until about target_s of CPU work.  The value is the
+    sample's own work (in the metric's unit) over its own time."""
     secs, w_cache = oracle_sample(wl, rows, w_cache)
     max_m = max(g.M for g in wl.gemms)
     while secs < target_s / 3 and rows < max_m:
@@ -855,40 +925,44 @@ def cpu_baseline(wl, unit, rows, w_cache=None, target_s=10.0):
         s_, _ = oracle_sample(wl, rows, w_cache)
         total += s_
         passes += 1
-    per_pass = total / passes
-    frac = sum(min(rows, g.M) * g.N * g.K for g in wl.gemms) / sum(g.M * g.N * g.K for g in wl.gemms)
-    full_s = per_pass / frac
     whole = all(rows >= g.M for g in wl.gemms)
-    return {"value": round(to_metric(step_units(wl, unit), full_s, unit), 6), "unit": unit,
+    units = step_units(sample_workload(wl, rows), unit) * passes
+    return {"value": round(to_metric(units, total, unit), 6), "unit": unit,
             "cores": omp_threads(), "kind": "oracle",
-            "sample": (f"{'every' if whole else f'the first {rows}'} token rows of every GEMM (all N, all K): "
-                       f"activation quantization + exact int64 GEMM, {passes} passes, {total:.1f} s of CPU "
-                       f"work{'' if whole else ', extrapolated linearly in M'} (weights quantized before "
-                       "timing, as in the GPU step)")}
+            "sample": (f"{'all' if whole else f'the first {rows}'} token rows of every GEMM (all N, all K): "
+                       f"activation quantization + exact int64 GEMM, {passes} passes, {total:.1f} s of CPU work; "
+                       "value = the sample's work over its time (weights quantized before timing, as in the GPU "
+                       "step)")}
 
 
 def run_reference(args):
+    """The reference arm: the CPU oracle, timed step by step.  A step is the
+    oracle on a bounded sample of the workload (the first --ref-sample-rows
+    token rows of every GEMM, all N and all K, with their activation
+    quantization); ms_per_step is that sampled step's measured time and value
+    the sample's work over it."""
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
     wl = select(args)
     metric, unit = metric_for(wl)
     rows = args.ref_sample_rows
     cache = {}
+    oracle_sample(wl, 1, cache)                      # weights quantized once, before timing
     for _ in range(args.warmup):
         oracle_sample(wl, rows, cache)
     secs = [oracle_sample(wl, rows, cache)[0] for _ in range(args.steps)]
-    frac = sum(min(rows, g.M) * g.N * g.K for g in wl.gemms) / sum(g.M * g.N * g.K for g in wl.gemms)
-    full = sum(secs) / frac
-    value = to_metric(step_units(wl, unit) * args.steps, full, unit)
-    sample = (f"first {rows} token rows of every GEMM per step (all N, all K), extrapolated linearly "
-              "in M to the whole workload")
+    units = step_units(sample_workload(wl, rows), unit) * args.steps
+    value = to_metric(units, sum(secs), unit)
+    sample = (f"each step: the first {rows} token rows of every GEMM (all N, all K), activation quantization "
+              "+ exact int64 GEMM on the host cores; value = the sampled steps' work over their measured time")
     line = {"impl": "reference", "metric": metric, "value": round(value, 6), "unit": unit,
-            "n_gpus": int(os.environ.get("WORLD_SIZE", args.gpus)), "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(full * 1e3 / args.steps, 3),
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(sum(secs) * 1e3 / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int64 exact dot products, f64 scaling", "data": "synthetic",
-            "config": {"workload": wl.name, "parallelism": "host cores (oracle)"},
+            "config": config_of(wl, world, args.flush_mib),
             "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": omp_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,

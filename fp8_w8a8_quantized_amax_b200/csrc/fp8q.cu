@@ -24,6 +24,8 @@ using fp8q::decode::Params;
 constexpr int kMaxDevices = 64;
 constexpr int64_t kInt32Max = 2147483647;
 
+fp8q_status noalloc_reset_current_device();
+
 // ------------------------------------------------------------ device info ---
 
 struct DeviceInfo {
@@ -464,6 +466,10 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
   fp8q_status st = check_linear_args(Xq, x_scale, Wq, w_scale, M, N, K, mode, Y_bf16, ldy);
   if (st != FP8Q_OK || M == 0) return st;
   mode &= ~FP8Q_SCALE_BF16;                     // the scale option concerns quantization only
+  if (M <= kDecodeMaxM) {                       // its size needs the device; presence and alignment do not
+    if (!workspace) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return FP8Q_ERR_MISALIGNED;
+  }
   int dev, sms;
   if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
   const int KB = static_cast<int>((K + 127) / 128);
@@ -721,6 +727,10 @@ int fp8q_device_error(int clear) {
   if (clear) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(fp8q::g_device_error, &zero, sizeof(int)) != cudaSuccess) return -1;
+    // A kernel that gave up may have left arrival counters and partial sums in
+    // fp8_linear_noalloc's in-library scratch; clearing the error restores the
+    // all-zero state that entry point relies on.
+    if (v != 0 && noalloc_reset_current_device() != FP8Q_OK) return -1;
   }
   return v;
 }
@@ -747,6 +757,23 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 // variable, not device memory.
 void* g_noalloc_ptr[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
+
+// Zero the allocation-free scratch of the current device, if a call there has
+// looked it up (a device that never ran fp8_linear_noalloc has an untouched,
+// zero-filled array).  cudaMemset allocates nothing.
+fp8q_status noalloc_reset_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FP8Q_ERR_UNSUPPORTED;
+  void* p = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    p = g_noalloc_ptr[dev];
+  }
+  if (p == nullptr) return FP8Q_OK;
+  if (cudaMemset(p, 0, kNoAllocScratchBytes) != cudaSuccess) return FP8Q_ERR_CUDA;
+  return cudaDeviceSynchronize() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
 
 fp8q_status noalloc_scratch(int dev, void** out) {
   std::lock_guard<std::mutex> lk(g_noalloc_mu);

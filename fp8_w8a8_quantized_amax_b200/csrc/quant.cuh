@@ -156,10 +156,12 @@ __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __rest
 // (Llama 3: RMSNorm before attention and MLP, eps 1e-5, kept in BF16).  One
 // CTA per token normalises its row in registers and quantizes it per token,
 // without writing the normalised bf16 row to memory:
-//   ms = fl32(sum x^2) / K, rstd = rsqrt_rn(ms + eps) (both IEEE),
+//   ms = fl32(sum x^2 / K), rstd = rsqrt_rn(fl32(ms + eps)),
 //   y = bf16(fl32(gamma * bf16(fl32(x * rstd)))), then y as quant_rows.
-// The sum of squares is an fp32 sum in this kernel's order; rstd is written
-// out (when rstd != nullptr) so that a caller can reproduce y exactly.
+// The squares are exact in fp64 and summed in fp64 (in this kernel's order),
+// so ms is the exact mean rounded once to fp32 unless that mean lies within a
+// few fp64 roundings of an fp32 rounding boundary; rstd is written out when
+// rstd != nullptr.
 
 // y for the 8 bf16 values of v (x) with the matching 8 of g (gamma), two at a
 // time: h = bf16(fl32(x * rstd)) by a packed fp32 multiply and one bf16x2
@@ -181,15 +183,27 @@ __device__ __forceinline__ uint4 rmsnorm_vec(const uint4& v, const uint4& g, uin
   return make_uint4(one(v.x, g.x), one(v.y, g.y), one(v.z, g.z), one(v.w, g.w));
 }
 
-// Sum of squares of the 8 values of v into two fp32 chains.
-__device__ __forceinline__ uint64_t sumsq_vec(const uint4& v, uint64_t acc2) {
+// |x| of one bf16 value (its low 16 bits of b) as a double, by integer
+// operations: the 15 magnitude bits move into the double's exponent and
+// mantissa fields and the exponent is rebiased by 1023 - 127.  Exact for every
+// normal bf16 value.  A zero or subnormal value becomes a double below 2^-126,
+// whose square (under 2^-252) changes a row's sum of squares by less than
+// 2^-236 in all: far below the sum's own fp64 rounding, and below fp32's
+// smallest subnormal mean.
+__device__ __forceinline__ double bf16_abs_f64(uint32_t b) {
+  return __hiloint2double(static_cast<int>(((b & 0x7FFFu) << 13) + 0x38000000u), 0);
+}
+
+// Squares of the 8 values of v (exact in fp64: 16 significant bits) added
+// into two fp64 chains.
+__device__ __forceinline__ void sumsq_vec(const uint4& v, double& a0, double& a1) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint64_t x2 = f32x2_pack(bf16lo(w[i]), bf16hi(w[i]));
-    acc2 = fma_f32x2(x2, x2, acc2);
+    const double lo = bf16_abs_f64(w[i]), hi = bf16_abs_f64(w[i] >> 16);
+    a0 = fma(lo, lo, a0);
+    a1 = fma(hi, hi, a1);
   }
-  return acc2;
 }
 
 template <int VPT>
@@ -198,7 +212,7 @@ __global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t*
                                                                  int64_t ldx, float eps, uint8_t* __restrict__ q,
                                                                  int64_t ldq, float* __restrict__ s,
                                                                  float* __restrict__ rstd) {
-  __shared__ float red_sum[32];
+  __shared__ double red_sum[32];
   __shared__ uint32_t red_max[32];
   griddep_wait();
   const int64_t r = blockIdx.x;
@@ -209,7 +223,7 @@ __global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t*
   // gamma is loaded with the row (not after the reduction) when it fits in registers
   constexpr bool kGammaAhead = VPT <= 8;
   uint4 v[VPT], gv[kGammaAhead ? VPT : 1];
-  uint64_t ss2 = f32x2_pack(0.0f, 0.0f);
+  double ss0 = 0.0, ss1 = 0.0;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int idx = threadIdx.x + i * T;
@@ -220,20 +234,21 @@ __global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t*
   }
 #pragma unroll
   for (int i = 0; i < VPT; ++i)
-    if (threadIdx.x + i * T < nvec) ss2 = sumsq_vec(v[i], ss2);
-  float ss_lo, ss_hi;
-  f32x2_unpack(ss2, ss_lo, ss_hi);
-  float ss = ss_lo + ss_hi;
+    if (threadIdx.x + i * T < nvec) sumsq_vec(v[i], ss0, ss1);
+  double ss = ss0 + ss1;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
   if (T > 32) {
     if (lane_id() == 0) red_sum[warp] = ss;
     __syncthreads();
-    ss = lane_id() < nw ? red_sum[lane_id()] : 0.0f;
+    ss = lane_id() < nw ? red_sum[lane_id()] : 0.0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
   }
-  const float rs = __frsqrt_rn(__fadd_rn(__fdiv_rn(ss, static_cast<float>(K)), eps));
+  // mean of squares rounded once to fp32 (the double quotient first), then the
+  // correctly rounded reciprocal square root of its IEEE sum with eps
+  const float ms = __double2float_rn(ss / static_cast<double>(K));
+  const float rs = __frsqrt_rn(__fadd_rn(ms, eps));
   if (threadIdx.x == 0 && rstd != nullptr) rstd[r] = rs;
   const uint64_t rs2 = f32x2_pack(rs, rs);
   uint32_t m2 = 0;

@@ -132,13 +132,15 @@ FP8Q_API fp8q_status fp8_quant_act_static(const void* X_bf16, int64_t M, int64_t
  *   eps        >= 0, finite (1e-5 for Llama 3).
  *   Xq, x_scale as fp8_quant_act in FP8Q_CHANNEL_TOKEN mode ([M] scales).
  *   rstd       [M] fp32, written when not NULL: the row's 1 / sqrt(ms + eps).
- *   Per row:  ms   = (sum over the row of x^2 in fp32) / K    (IEEE division)
- *             rstd = 1 / sqrt(ms + eps), correctly rounded fp32
+ *   Per row:  ms   = the mean over the row of x^2, rounded once to fp32
+ *             rstd = 1 / sqrt(fl32(ms + eps)), correctly rounded fp32
  *             y    = bf16(gamma * bf16(x * rstd))           (fp32 products)
  *             codes and scale of y as fp8_quant_act.
- *   The fp32 sum of squares is taken in this kernel's order.  Everything
- *   after it is exact, so rstd determines y and the codes.  Rows whose sum of
- *   squares overflows fp32 are outside the contract.
+ *   The squares are exact in fp64 and summed in fp64, so ms is the exactly
+ *   rounded mean except for a mean within a few fp64 roundings of an fp32
+ *   rounding boundary (then it may be one fp32 step off, and rstd with it).
+ *   Everything after rstd is exact, so rstd determines y and the codes.  Rows
+ *   whose mean of squares overflows fp32 are outside the contract.
  *   Requirements: M >= 0 (M == 0 is a no-op), K > 0, K % 16 == 0, and
  *   K <= 65536 (FP8Q_ERR_UNSUPPORTED above).
  */
@@ -155,7 +157,9 @@ FP8Q_API fp8q_status fp8_rmsnorm_quant_act(const void* X_bf16, const void* gamma
  *   w_scale   [N] or [ceil(N/128), K/128] fp32 (as written by fp8_quant_weight).
  *   Y_bf16    [M, ldy] bf16, written.  ldy >= N, (ldy * 2) % 16 == 0, 16-byte aligned.
  *   workspace device scratch of at least fp8_linear_workspace_size(M, N, K, mode)
- *             bytes, 256-byte aligned (may be NULL when that size is 0).  It holds
+ *             bytes, 16-byte aligned (may be NULL when that size is 0; M > 64
+ *             needs none).  A NULL or misaligned workspace for M <= 64 is
+ *             refused before anything touches the device.  It holds
  *             the split-K arrival counters and fp32 partial sums of the small-M
  *             (decode) path.  It must be zero-filled before its first use; every
  *             completed call leaves it all zero again, so one zeroed buffer
@@ -234,7 +238,9 @@ FP8Q_API const char* fp8q_status_string(int status);
 
 /* Reads the device-side error word of the current device: 0 when no kernel
  * has given up waiting, otherwise a nonzero code naming the wait site.  It
- * synchronizes the device.  clear != 0 resets the word to 0 afterwards. */
+ * synchronizes the device.  clear != 0 resets the word to 0 afterwards and,
+ * when it was nonzero, also zeroes fp8_linear_noalloc's in-library scratch on
+ * this device.  Returns -1 when a CUDA call fails. */
 FP8Q_API int fp8q_device_error(int clear);
 
 /*
@@ -257,12 +263,20 @@ FP8Q_API int fp8q_device_error(int clear);
  *     fp8_linear_workspace_size reports) returns FP8Q_ERR_UNSUPPORTED.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  With CUDA's lazy module loading (the default)
+ *     the array is reserved on a device when the library's device code is
+ *     first loaded there: by that first call, or by any earlier call of this
+ *     library on the device.  A caller whose memory budget is fixed should
+ *     therefore make one call at setup time.
  *   - Every call on a device shares the one array, which keeps whatever the last
  *     call left in it: zero-filled when the library is loaded, and every
  *     completed call leaves it all zero again.  Calls whose kernels overlap on the GPU
  *     (different streams, or different host threads) race on the array and give
  *     wrong results; serialise them.
+ *   - A call whose kernel gave up waiting (fp8q_device_error nonzero) can leave
+ *     counters and partial sums in the array.  fp8q_device_error(1) then zeroes
+ *     the current device's array as well as the error word (cudaMemset, which
+ *     allocates nothing); call it before the next fp8_linear_noalloc.
  */
 FP8Q_API fp8q_status fp8_linear_noalloc(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq,
                                         const float* w_scale, int64_t M, int64_t N, int64_t K, int mode,

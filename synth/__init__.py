@@ -84,10 +84,21 @@ class Gemm:
     N: int
     mode: int = CHANNEL_TOKEN
     x: str = ""          # which activation it reads; GEMMs naming the same one share it
+    w: str = ""          # which weight it multiplies ("" = its own); the M values of one projection share one
 
     @property
     def flops(self) -> int:
         return 2 * self.M * self.N * self.K
+
+    @property
+    def weight(self) -> str:
+        return self.w or self.name
+
+
+def weight_seed(name: str) -> int:
+    """Seed of a workload weight, from its name (stable across runs and processes)."""
+    import zlib
+    return zlib.crc32(name.encode()) % 1000
 
 
 @dataclasses.dataclass(frozen=True)
@@ -112,13 +123,13 @@ def workloads() -> dict:
          Gemm("down_proj", 8192, 14336, 4096, x="mlp_act")])
     w["llama3.2-3b_block128"] = Workload(
         "llama3.2-3b_block128",
-        [Gemm(f"gate_proj_m{m}", m, 3072, 8192, BLOCK128, x=f"mlp_in_m{m}") for m in (1, 16, 4096)])
+        [Gemm(f"gate_proj_m{m}", m, 3072, 8192, BLOCK128, x=f"mlp_in_m{m}", w="gate_proj") for m in (1, 16, 4096)])
     g70 = []
     for m in (1, 8, 64, 512, 8192):
-        g70 += [Gemm(f"gate_proj_m{m}", m, 8192, 28672, x=f"mlp_in_m{m}"),
-                Gemm(f"up_proj_m{m}", m, 8192, 28672, x=f"mlp_in_m{m}"),
-                Gemm(f"down_proj_m{m}", m, 28672, 8192, x=f"mlp_act_m{m}"),
-                Gemm(f"qkv_proj_m{m}", m, 8192, 10240, x=f"attn_in_m{m}")]
+        g70 += [Gemm(f"gate_proj_m{m}", m, 8192, 28672, x=f"mlp_in_m{m}", w="gate_proj"),
+                Gemm(f"up_proj_m{m}", m, 8192, 28672, x=f"mlp_in_m{m}", w="up_proj"),
+                Gemm(f"down_proj_m{m}", m, 28672, 8192, x=f"mlp_act_m{m}", w="down_proj"),
+                Gemm(f"qkv_proj_m{m}", m, 8192, 10240, x=f"attn_in_m{m}", w="qkv_proj")]
     w["llama3.1-70b_sweep"] = Workload("llama3.1-70b_sweep", g70)
     for m in (1, 8, 64, 512, 8192):   # one M of the sweep at a time
         w[f"llama3.1-70b_m{m}"] = Workload(f"llama3.1-70b_m{m}", [g for g in g70 if g.M == m])

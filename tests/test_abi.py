@@ -226,9 +226,32 @@ def test_quant_weight_argument_checks(L, kw, want):
     (dict(xs=None), fq.ERR_INVALID_ARG),
     (dict(M=-3), fq.ERR_INVALID_ARG),
     (dict(M=0, xq=None, xs=None, wq=None, ws=None, y=None), fq.OK),
+    (dict(wsp=None), fq.ERR_INVALID_ARG),                   # M <= 64 needs a workspace
+    (dict(wsp=P + 8), fq.ERR_MISALIGNED),                   # workspace: 16-byte alignment
+    (dict(wsp=P + 4, M=64), fq.ERR_MISALIGNED),
 ])
 def test_linear_argument_checks(L, kw, want):
     assert lin(L, **kw) == want
+
+
+def noalloc(L, M=4, N=64, K=256, mode=0, y=P, ldy=64, xq=P, xs=P, wq=P, ws=P):
+    f = L.fp8_linear_noalloc
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_int64,
+                                                                 ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    return f(xq, xs, wq, ws, M, N, K, mode, y, ldy, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(M=65), fq.ERR_UNSUPPORTED),                       # the M > 64 path needs no scratch: use fp8_linear
+    (dict(mode=5), fq.ERR_INVALID_ARG),
+    (dict(K=40), fq.ERR_INVALID_ARG),
+    (dict(y=BAD), fq.ERR_MISALIGNED),
+    (dict(wq=None), fq.ERR_INVALID_ARG),
+    (dict(M=0, xq=None, xs=None, wq=None, ws=None, y=None), fq.OK),
+])
+def test_noalloc_argument_checks(L, kw, want):
+    assert noalloc(L, **kw) == want
 
 
 def test_workspace_size_is_zero_for_invalid_or_prefill(L):
@@ -242,6 +265,9 @@ def test_valid_arguments_without_a_gpu_report_cuda_error(L):
     assert q_act(L) == fq.ERR_CUDA
     assert q_w(L) == fq.ERR_CUDA
     assert lin(L) == fq.ERR_CUDA
+    assert lin(L, wsp=P + 16) == fq.ERR_CUDA            # 16-byte alignment is enough
+    assert lin(L, M=65, wsp=None, wsb=0) == fq.ERR_CUDA  # the prefill path needs no workspace
+    assert noalloc(L) == fq.ERR_CUDA
     assert rms_q(L) == fq.ERR_CUDA
     assert swi(L) == fq.ERR_CUDA
     assert q_static(L) == fq.ERR_CUDA

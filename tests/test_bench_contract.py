@@ -19,7 +19,10 @@ def run_bench(*args, timeout=300):
 
 
 def test_reference_arm_prints_one_json_line():
+    import time
+    t0 = time.perf_counter()
     r = run_bench("--impl", "reference", "--workload", "tiny_16x256x512", "--steps", "3", "--warmup", "3")
+    wall = time.perf_counter() - t0
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.strip()]
     assert len(lines) == 1
@@ -33,6 +36,13 @@ def test_reference_arm_prints_one_json_line():
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    # the timed steps are measured ones: they fit inside the process's own run
+    assert d["ms_per_step"] * d["steps"] / 1e3 <= wall
+    # the same workload description the GPU arm prints
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    assert d["config"] == bench.config_of(synth.workloads()["tiny_16x256x512"], 1, 256)
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="needs a machine without a CUDA device")

@@ -194,52 +194,10 @@ def test_repeat_calls_are_deterministic():
         assert torch.equal(fq.fp8_linear(xq, xs, wq, ws), y0)
 
 
-# ------------------------------------------------ full workload sizes, sampled ---
-
-def _sample(n, k, seed):
-    rng = np.random.default_rng(seed)
-    return np.array(sorted(set([0, n - 1]) | set(rng.integers(0, n, k).tolist())))
-
-
-def _check_sampled(g: synth.Gemm, seed=0):
-    x = synth.make_x_device(g.M, g.K, seed=seed)
-    w = synth.make_w_device(g.N, g.K, seed=seed)
-    mode = g.mode
-    wq, ws = fq.fp8_quant_weight(w, mode)
-    xq, xs = fq.fp8_quant_act(x, mode)
-    y = fq.fp8_linear(xq, xs, wq, ws, mode)
-    torch.cuda.synchronize()
-    ms = _sample(g.M, 30, seed + 1)
-    nblocks = _sample(g.N // 128, 2, seed + 2)          # whole 128-row weight blocks
-    ns = np.concatenate([np.arange(b * 128, b * 128 + 128) for b in nblocks])
-    xsub = x[torch.as_tensor(ms, device=DEV)].cpu()
-    rxq, rxs = oracle.quant_act(xsub, mode)
-    P.assert_codes_equal(xq[torch.as_tensor(ms, device=DEV)], rxq, f"{g.name} xq")
-    rwq, rws = [], []
-    for b in nblocks:
-        q, s = oracle.quant_weight(w[b * 128:(b + 1) * 128].cpu(), mode)
-        rwq.append(q)
-        rws.append(s)
-    rwq = np.concatenate(rwq)
-    rws = np.concatenate(rws)
-    P.assert_codes_equal(wq[torch.as_tensor(ns, device=DEV)], rwq, f"{g.name} wq")
-    yref = oracle.linear(rxq, rxs, rwq, rws, mode)
-    ygpu = y[torch.as_tensor(ms, device=DEV)][:, torch.as_tensor(ns, device=DEV)].float().cpu().numpy()
-    # the tolerance's first term uses the largest |y| of the sampled outputs
-    P.assert_y_close(ygpu, yref, what=f"{g.name} M={g.M} K={g.K} N={g.N}")
-
+# Every workload at full size (every code and scale, outputs on sampled rows
+# and weight blocks) is in test_gpu_full_size.py.
 
 ALL = synth.workloads()
-FULL = [g for name in ("llama3.2-3b_mlp_m2048", "llama3.1-8b_layer_m8192", "llama3.2-3b_block128",
-                       "llama3.1-70b_sweep") for g in ALL[name].gemms]
-# GEMMs sharing an input merged over stacked weights (as bench.py also measures)
-FULL += [synth.Gemm("gate_up_proj", 2048, 3072, 16384), synth.Gemm("qkv_proj", 8192, 4096, 6144),
-         synth.Gemm("gate_up_proj_m16_block", 16, 3072, 16384, synth.BLOCK128)]
-
-
-@pytest.mark.parametrize("g", FULL, ids=[f"{g.name}-{g.M}x{g.K}x{g.N}-m{g.mode}" for g in FULL])
-def test_full_size_sampled(g):
-    _check_sampled(g)
 
 
 def test_tiny_workload_in_full():

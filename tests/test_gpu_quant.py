@@ -104,45 +104,6 @@ def test_empty_rows():
     assert q.shape == (0, 256) and s.shape == (0,)
 
 
-def _sampled_rows(n, k=24, seed=0):
-    rng = np.random.default_rng(seed)
-    r = set([0, n - 1]) | set(rng.integers(0, n, k).tolist())
-    return np.array(sorted(r))
-
-
-@pytest.mark.parametrize("M,K", [(8192, 4096), (8192, 14336), (8192, 28672), (2048, 3072)])
-def test_full_size_activation_rows(M, K):
-    x = synth.make_x_device(M, K, seed=11)
-    q, s = fq.fp8_quant_act(x, fq.CHANNEL_TOKEN)
-    rows = _sampled_rows(M)
-    rq, rs = P.oracle_rows_for(x.cpu(), rows, fq.CHANNEL_TOKEN)
-    P.assert_codes_equal(q[torch.as_tensor(rows, device=DEV)], rq, f"act {M}x{K}")
-    P.assert_scales_equal(s[torch.as_tensor(rows, device=DEV)], rs, f"act {M}x{K}")
-
-
-@pytest.mark.parametrize("N,K", [(28672, 8192), (8192, 28672), (10240, 8192), (14336, 4096)])
-def test_full_size_weight_rows(N, K):
-    w = synth.make_w_device(N, K, seed=13)
-    q, s = fq.fp8_quant_weight(w, fq.CHANNEL_TOKEN)
-    rows = _sampled_rows(N)
-    rq, rs = oracle.quant_rows(w[torch.as_tensor(rows, device=DEV)].cpu())
-    P.assert_codes_equal(q[torch.as_tensor(rows, device=DEV)], rq, f"weight {N}x{K}")
-    P.assert_scales_equal(s[torch.as_tensor(rows, device=DEV)], rs, f"weight {N}x{K}")
-
-
-def test_full_size_block_weight_and_groups():
-    w = synth.make_w(8192, 3072, seed=0)
-    q, s = fq.fp8_quant_weight(w.to(DEV), fq.BLOCK128)
-    rq, rs = oracle.quant_blocks128(w)
-    P.assert_codes_equal(q, rq, "block weight 8192x3072")
-    P.assert_scales_equal(s, rs, "block weight 8192x3072")
-    x = synth.make_x(4096, 3072, seed=0)
-    q, s = fq.fp8_quant_act(x.to(DEV), fq.BLOCK128)
-    rq, rs = oracle.quant_groups128(x)
-    P.assert_codes_equal(q, rq, "groups 4096x3072")
-    P.assert_scales_equal(s, rs, "groups 4096x3072")
-
-
 def test_every_bf16_pair_matches_ieee_division():
     """The quantizer's division (reciprocal + correction step) against torch's
     IEEE fp32 division and fp8 cast, for every positive finite bf16 amax and

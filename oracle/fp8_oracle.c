@@ -159,6 +159,8 @@ static inline uint8_t code_of(float x, float s) {
  * x: bf16 bits [rows, ld], q: [rows, ldq], s: [rows]. */
 static void quant_rows_impl(const uint16_t* x, int64_t rows, int64_t K, int64_t ld,
                             uint8_t* q, int64_t ldq, float* s, int scale_bf16) {
+    build_mag_table();                    /* before the rows run in parallel (they are independent) */
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
         float amax = 0.0f;
         for (int64_t k = 0; k < K; ++k) {
@@ -177,6 +179,8 @@ static void quant_rows_impl(const uint16_t* x, int64_t rows, int64_t K, int64_t 
 static void quant_groups128_impl(const uint16_t* x, int64_t M, int64_t K, int64_t ld,
                                  uint8_t* q, int64_t ldq, float* s, int scale_bf16) {
     int64_t G = K / 128;
+    build_mag_table();
+#pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m) {
         for (int64_t g = 0; g < G; ++g) {
             float amax = 0.0f;
@@ -199,6 +203,8 @@ static void quant_groups128_impl(const uint16_t* x, int64_t M, int64_t K, int64_
 static void quant_blocks128_impl(const uint16_t* w, int64_t N, int64_t K, int64_t ld,
                                  uint8_t* q, int64_t ldq, float* s, int scale_bf16) {
     int64_t NB = (N + 127) / 128, KB = K / 128;
+    build_mag_table();
+#pragma omp parallel for schedule(static)
     for (int64_t nb = 0; nb < NB; ++nb) {
         int64_t n1 = (nb + 1) * 128 < N ? (nb + 1) * 128 : N;
         for (int64_t kb = 0; kb < KB; ++kb) {
@@ -225,6 +231,8 @@ static void quant_blocks128_impl(const uint16_t* w, int64_t N, int64_t K, int64_
  * q: [rows, ldq]. */
 ORC_EXPORT void orc_quant_static(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, float s,
                                  uint8_t* q, int64_t ldq) {
+    build_mag_table();
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t k = 0; k < K; ++k) q[r * ldq + k] = code_of(bf16_to_float(x[r * ld + k]), s);
 }
@@ -385,6 +393,7 @@ static float rsqrt_f32_rn(float d) {
  * exact mean of squares rounded once to fp32.  Rows whose mean of squares
  * overflows fp32 are outside the definition (rstd 0 is returned for them). */
 ORC_EXPORT void orc_rmsnorm_rstd(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, float eps, float* rstd) {
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
         uint64_t acc[SQ_LIMBS] = {0};
         for (int64_t k = 0; k < K; ++k) sq_add(acc, x[r * ld + k]);
@@ -411,6 +420,8 @@ ORC_EXPORT void orc_rmsnorm_quant_rows(const uint16_t* x, const uint16_t* gamma,
                                        int64_t ld, float eps, int rstd_ulps, uint8_t* q, int64_t ldq, float* s,
                                        uint16_t* y, float* rstd_out) {
     orc_rmsnorm_rstd(x, rows, K, ld, eps, rstd_out);
+    build_mag_table();
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
         float rs = step_ulps(rstd_out[r], rstd_ulps);
         rstd_out[r] = rs;

@@ -485,7 +485,12 @@ def run_gpu(args):
     all_units, total_s = aggregate(units, sum(step_ms) / 1e3, world)
     value = to_metric(all_units, total_s, unit)
 
-    # per-op times: every op timed alone after its own L2 flush
+    # per-op times.  (1) isolated: each op's own graph, one launch after its
+    # own L2 flush -- the launch latency of a lone kernel included.  (2)
+    # back to back: R launches of the op in one graph, over R sets of buffers
+    # (copies of its inputs and outputs) whose footprint together is at least
+    # twice L2, so that every launch reads its inputs from DRAM; per launch =
+    # the graph's time / R, after an L2 flush.  (2) is what "ms" reports.
     op_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(n_ops)] for _ in range(args.steps)]
     torch.cuda._sleep(2_000_000)
@@ -496,7 +501,60 @@ def run_gpu(args):
             r()
             op_ev[s][i][1].record(stream)
     torch.cuda.synchronize()
-    op_ms = np.array([[a.elapsed_time(b) for a, b in row] for row in op_ev]).mean(axis=0)
+    op_ms_isolated = np.array([[a.elapsed_time(b) for a, b in row] for row in op_ev]).mean(axis=0)
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    xs_items = list(xs_shapes.items())
+
+    def rotating(i):
+        """(R, functions): R launches of op i over R buffer sets."""
+        if i < len(xs_items):
+            k, (M, K, mode) = xs_items[i]
+            R = int(min(32, max(2, -(-2 * l2_bytes // quant_bytes(M, K, mode)))))
+            xs_ = [X[k]] + [X[k].clone() for _ in range(R - 1)]
+            outs = [XQ[k]] + [(torch.empty_like(XQ[k][0]), torch.empty_like(XQ[k][1])) for _ in range(R - 1)]
+            return R, [lambda x=x, o=o, mode=mode: fq.fp8_quant_act(x, mode, out=o) for x, o in zip(xs_, outs)]
+        g = wl.gemms[i - len(xs_items)]
+        R = int(min(32, max(2, -(-2 * l2_bytes // gemm_bytes(g)))))
+        xq, xsc = XQ[g.x]
+        wq, wsc = WQ[g.weight]
+        sets = [(xq, xsc, wq, wsc, Y[g.name], WS[g.name])]
+        for _ in range(R - 1):
+            sets.append((xq.clone(), xsc.clone(), wq.clone(), wsc.clone(), torch.empty_like(Y[g.name]),
+                         torch.zeros_like(WS[g.name]) if WS[g.name] is not None else None))
+        return R, [lambda st=st, g=g: fq.fp8_linear(st[0], st[1], st[2], st[3], g.mode, out=st[4], workspace=st[5])
+                   for st in sets]
+
+    LONG_OP_MS = 0.25
+    op_ms = np.zeros(n_ops)
+    op_reps = [1] * n_ops
+    for i in range(n_ops):
+        R, fns = rotating(i)
+        for f in fns:
+            f()
+        torch.cuda.synchronize()
+        gr = capture(fns) if not args.eager else None
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda._sleep(1_000_000)
+        for s_ in range(args.steps):
+            flush.zero_()
+            ev[s_][0].record(stream)
+            if gr is not None:
+                gr.replay()
+            else:
+                for f in fns:
+                    f()
+            ev[s_][1].record(stream)
+        torch.cuda.synchronize()
+        op_ms[i] = float(np.mean([a.elapsed_time(b) for a, b in ev])) / R
+        op_reps[i] = R
+        del gr, fns
+        if op_ms_isolated[i] >= LONG_OP_MS:
+            # a long kernel is reported as timed alone: its launch latency is a
+            # few percent of it, and two back to back already run into the
+            # power cap (its roofline uses the burst peak, measured alone)
+            op_ms[i] = op_ms_isolated[i]
+            op_reps[i] = 1
+    torch.cuda.empty_cache()
     err = fq.device_error(clear=True)
 
     # ---- GEMMs that read the same activation, run as one GEMM over their
@@ -553,7 +611,8 @@ def run_gpu(args):
     for i, (k, (M, K, mode)) in enumerate(xs_shapes.items()):
         b = quant_bytes(M, K, mode)
         detail.append({"op": names[i], "kernel": "quant_rows" if mode == 0 else "quant_groups128", "bound": "hbm",
-                       "M": M, "K": K, "mode": mode,
+                       "M": M, "K": K, "mode": mode, "back_to_back": op_reps[i],
+                       "ms_isolated": round(float(op_ms_isolated[i]), 5),
                        "ms": round(float(op_ms[i]), 5), "GB/s": round(b / (op_ms[i] / 1e3) / 1e9, 1),
                        "frac_hbm": round(b / (op_ms[i] / 1e3) / 1e9 / pk["hbm_gbs"], 3)})
     for j, g in enumerate(wl.gemms):
@@ -561,7 +620,8 @@ def run_gpu(args):
         kern = ("gemm_decode" if g.M <= 64 else
                 ("gemm_block" if g.mode == synth.BLOCK128 else "gemm_channel"))
         detail.append({"op": g.name, "kernel": kern, "bound": "hbm" if g.M <= 64 else "tensor",
-                       "M": g.M, "N": g.N, "K": g.K, "mode": g.mode,
+                       "M": g.M, "N": g.N, "K": g.K, "mode": g.mode, "back_to_back": op_reps[len(xs_shapes) + j],
+                       "ms_isolated": round(float(op_ms_isolated[len(xs_shapes) + j]), 5),
                        "ms": round(float(op_ms[len(xs_shapes) + j]), 5),
                        "TFLOP/s": round(g.flops / t / 1e12, 1),
                        "GB/s": round(gemm_bytes(g) / t / 1e9, 1),
@@ -852,7 +912,10 @@ def run_gpu(args):
             "dtype": "fp8_e4m3 (fp32 accumulate, bf16 out)", "data": "synthetic",
             "config": config_of(wl, world, args.flush_mib),
             "launch": "eager" if args.eager else
-            "step: one CUDA graph replayed per step; per-op detail: each op's own graph, timed alone",
+            "step: one CUDA graph replayed per step; per-op detail (and rooflines): ms = one graph of R "
+            "back-to-back launches of the op over R copies of its buffers (R = back_to_back, footprint >= 2x L2, "
+            "so every launch reads from DRAM) / R, after an L2 flush; ms_isolated = one launch in its own graph "
+            "after an L2 flush, which ms reports (back_to_back = 1) for ops of 0.25 ms or more",
             "roofline": roof, "rooflines": rooflines, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g, sms) for g in wl.gemms)),
             "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant, "rmsnorm_quant": rms, "kv_quant": kvq, "swiglu": swiglu, "quant_static": qstatic, "w8a16": w8a16,

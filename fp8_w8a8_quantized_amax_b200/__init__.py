@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.fp8_rmsnorm_quant_act.restype = ctypes.c_int
         L.fp8_quant_act_static.argtypes = [P, I, I, I, ctypes.c_float, P, I, P, P]
         L.fp8_quant_act_static.restype = ctypes.c_int
+        L.fp8_calibrate_static_scale.argtypes = [P, I, I, I, ctypes.c_double, ctypes.c_double, P, P, P]
+        L.fp8_calibrate_static_scale.restype = ctypes.c_int
         L.fp8_linear_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, P, I, P]
         L.fp8_linear_swiglu.restype = ctypes.c_int
         L.fp8_linear_w8a16.argtypes = [P, I, P, P, I, I, I, P, I, P, S, P]
@@ -228,26 +230,27 @@ def fp8_quant_act_static(X: torch.Tensor, scale: float, out: Optional[Tuple[torc
     return Xq, xs
 
 
-def calibrate_static_scale(X: torch.Tensor, lo: float = 0.001, hi: float = 0.999) -> float:
-    """Offline calibration (not part of the per-forward path): the larger
-    magnitude of X's lo and hi quantiles (linear interpolation between order
-    statistics), / 448, rounded to fp32; 1.0 for an all-zero range."""
-    f = X.detach().reshape(-1).double()
-    n = f.numel()
+CALIB_HIST_BINS = 65536
 
-    def q(p):
-        pos = p * (n - 1)
-        i = int(pos // 1)
-        j = min(i + 1, n - 1)
-        a = torch.kthvalue(f, i + 1).values.item()
-        b = torch.kthvalue(f, j + 1).values.item()
-        return a + (b - a) * (pos - i)
 
-    amax = max(abs(q(lo)), abs(q(hi)))
-    if amax == 0.0:
-        return 1.0
-    import numpy as np
-    return float(np.float32(np.float32(amax) / np.float32(448.0)))
+def calibrate_static_scale(X: torch.Tensor, lo: float = 0.001, hi: float = 0.999,
+                           hist: Optional[torch.Tensor] = None) -> float:
+    """Offline calibration of a static scale (fp8_calibrate_static_scale): the
+    larger magnitude of X's lo and hi quantiles, / 448, in fp32; 1.0 for a
+    zero range.  X bf16 [M, K] on the GPU.  `hist`: a zero-filled int32
+    device buffer of 65536 counts (allocated here when None; left zero)."""
+    _require_cuda(X, "X", torch.bfloat16)
+    if X.dim() != 2:
+        raise ValueError("X must be 2-D [M, K]")
+    M, K = X.shape
+    if hist is None:
+        hist = torch.zeros(CALIB_HIST_BINS, dtype=torch.int32, device=X.device)
+    _require_like(hist, "hist", torch.int32, CALIB_HIST_BINS, X)
+    scale = torch.empty((), dtype=torch.float32, device=X.device)
+    st = lib().fp8_calibrate_static_scale(_ptr(X), M, K, X.stride(0), float(lo), float(hi), _ptr(hist), _ptr(scale),
+                                          _stream(X))
+    _check(st, "fp8_calibrate_static_scale")
+    return float(scale.item())
 
 
 def fp8_linear_swiglu(Xq: torch.Tensor, x_scale: torch.Tensor, Wq_gate: torch.Tensor, w_scale_gate: torch.Tensor,

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "../../include/fp8q.h"
+#include "calib.cuh"
 #include "gemm_decode.cuh"
 #include "gemm_prefill.cuh"
 #include "gemv_w8a16.cuh"
@@ -284,8 +285,20 @@ fp8q_status check_linear_args(const uint8_t* Xq, const float* xs, const uint8_t*
 // win everywhere; with 32 or 64 tokens only when every CTA streams at least a
 // tile's worth of steps after them; in block mode the per-K-block epilogue
 // leaves no room, and the separate kernel is faster.
+// FP8Q_DECODE_BLOCK_SUMS=kernel|separate forces one way in block mode (read
+// once), for comparing them on the same problem.
+int decode_block_sums_choice() {
+  static int choice = [] {
+    const char* e = getenv("FP8Q_DECODE_BLOCK_SUMS");
+    if (e && strcmp(e, "kernel") == 0) return 1;
+    if (e && strcmp(e, "separate") == 0) return 2;
+    return 0;
+  }();
+  return choice;
+}
+
 bool decode_fused(const Params& p, int mode, int nx) {
-  if (mode == FP8Q_BLOCK128) return false;
+  if (mode == FP8Q_BLOCK128) return decode_block_sums_choice() == 1;
   return nx == 16 || p.total >= static_cast<int64_t>(p.KB) * p.G;
 }
 
@@ -448,6 +461,25 @@ fp8q_status fp8_quant_act_static(const void* X_bf16, int64_t M, int64_t K, int64
                 static_cast<const uint16_t*>(X_bf16), M, static_cast<int>(K), ldx, scale, Xq, ldxq, x_scale);
 }
 
+fp8q_status fp8_calibrate_static_scale(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, double lo, double hi,
+                                       uint32_t* hist, float* scale, void* stream) {
+  if (M <= 0 || K <= 0 || ldx < K || K % 8 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (!(lo >= 0.0 && lo <= 1.0) || !(hi >= 0.0 && hi <= 1.0)) return FP8Q_ERR_INVALID_ARG;   // rejects NaN
+  if (!X_bf16 || !hist || !scale) return FP8Q_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || !aligned(X_bf16, 16) || !aligned(hist, 4) || !aligned(scale, 4)) return FP8Q_ERR_MISALIGNED;
+  if (M > kInt32Max || K > kInt32Max || M * K >= (static_cast<int64_t>(1) << 32)) return FP8Q_ERR_UNSUPPORTED;
+  fp8q_status st;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
+  const int64_t vecs = M * (K / 8);
+  int64_t grid = (vecs + 255) / 256;
+  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
+  if ((st = launch(fp8q::calib::hist_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream,
+                   static_cast<const uint16_t*>(X_bf16), M, static_cast<int>(K), ldx, hist)) != FP8Q_OK)
+    return st;
+  return launch(fp8q::calib::select_kernel, dim3(1), dim3(1024), 0, stream, hist, M * K, lo, hi, scale);
+}
+
 size_t fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int mode) {
   if (!valid_mode(mode)) return 0;
   mode &= ~FP8Q_SCALE_BF16;
@@ -491,7 +523,8 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     p.K = static_cast<int>(K);
     p.KB = KB;
     p.n_tiles = n_tiles;
-    p.total = total;
+    if (total > kInt32Max) return FP8Q_ERR_UNSUPPORTED;
+    p.total = static_cast<int>(total);
     p.G = G;
     decode_bind_workspace(p, workspace, Y_bf16, ldy);
     if (nx == 16) return launch_decode_nx<16>(tw, tx, p, mode, dev, stream);
@@ -700,7 +733,8 @@ fp8q_status fp8_linear_w8a16(const void* X_bf16, int64_t ldx, const uint8_t* Wq,
   p.K = static_cast<int>(K);
   p.KB = static_cast<int>((K + 127) / 128);
   p.n_tiles = n_tiles;
-  p.total = total;
+  if (total > kInt32Max) return FP8Q_ERR_UNSUPPORTED;
+  p.total = static_cast<int>(total);
   p.G = G;
   decode_bind_workspace(p, workspace, Y_bf16, ldy);
   if (nx == 16) return launch_decode_w16<16>(tw, tx, p, dev, stream);
@@ -736,6 +770,17 @@ int fp8q_device_error(int clear) {
 }
 
 int fp8q_version(void) { return 100; }
+
+#ifdef FP8Q_TEST_HOOKS
+// Test build only (not declared in fp8q.h, absent from the product library):
+// mode 1 makes the next decode launches withhold one tensor-memory slot
+// release in CTA 0, mode 2 one accumulator commit, so that a wait runs out;
+// 0 turns it off.
+FP8Q_API int fp8q_test_withhold(int mode) {
+  const int v = mode;
+  return cudaMemcpyToSymbol(fp8q::g_test_withhold, &v, sizeof(int)) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 }  // extern "C"
 
@@ -816,7 +861,8 @@ fp8q_status fp8_linear_noalloc(const uint8_t* Xq, const float* x_scale, const ui
   p.K = static_cast<int>(K);
   p.KB = static_cast<int>((K + 127) / 128);
   p.n_tiles = n_tiles;
-  p.total = total;
+  if (total > kInt32Max) return FP8Q_ERR_UNSUPPORTED;
+  p.total = static_cast<int>(total);
   p.G = G;
   decode_bind_workspace(p, scratch, Y_bf16, ldy);
   if (nx == 16) return launch_decode_nx<16>(tw, tx, p, mode, dev, stream);

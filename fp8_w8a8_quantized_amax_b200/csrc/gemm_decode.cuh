@@ -29,10 +29,12 @@
 //
 // Roles: warp 0 TMA (W tile 128 x 128 B evict-first + X tile NX x 128 B),
 // warp 1 TMEM allocation + MMA issue, warps 2..5 drain TMEM and write
-// segments.  TMEM holds 4 slots of NX columns.  Channel mode accumulates a
+// segments.  TMEM holds 8 slots of NX columns.  Channel mode accumulates a
 // whole segment in one slot (drained once per segment); block mode gives
 // every K block its own slot, folded into registers with that block's
-// x_scale * w_scale.
+// x_scale * w_scale.  Block mode's scales reach each epilogue warp through a
+// small shared-memory ring, filled by asynchronous 4-byte copies several
+// steps ahead, so that no scale load sits on the fold's critical path.
 //
 // Weight-only variant (WIDEN > 0 warps, bf16 activations, channel scales):
 // the same schedule with the activation tile loaded as bf16 (two 64-value
@@ -49,7 +51,7 @@ namespace decode {
 
 constexpr int BK = 128;
 constexpr int UMMA_K = 32;
-constexpr int kSlots = 4;
+constexpr int kSlots = 8;
 
 struct Params {
   const float* xs;
@@ -60,29 +62,38 @@ struct Params {
   int64_t ldy;
   int M, N, K, KB;
   int n_tiles;
-  int64_t total;        // n_tiles * KB
+  int total;            // n_tiles * KB (the host refuses 2^31 or more)
   int G;                // CTAs
 };
 
-__host__ __device__ __forceinline__ int64_t range_begin(int64_t c, int64_t total, int64_t G) {
-  return c * total / G;
-}
+// The steps are cut into G contiguous ranges with q = total / G, r = total % G:
+// CTA c takes q + 1 steps when c < r, else q.  32-bit arithmetic throughout
+// (64-bit divisions are long instruction sequences on the critical path of
+// the first load).
+struct Split {
+  int q, r;
+};
 
-// Largest CTA index c whose range starts at or before step x.
-__host__ __device__ __forceinline__ int cta_of_step(int64_t x, int64_t total, int64_t G) {
-  return static_cast<int>(((x + 1) * G - 1) / total);
+__host__ __device__ __forceinline__ Split split_of(int total, int G) { return {total / G, total % G}; }
+
+__host__ __device__ __forceinline__ int range_begin(int c, const Split& sp) { return c * sp.q + min(c, sp.r); }
+
+// The CTA whose range holds step x.
+__host__ __device__ __forceinline__ int cta_of_step(int x, const Split& sp) {
+  const int big = sp.r * (sp.q + 1);
+  return x < big ? x / (sp.q + 1) : sp.r + (x - big) / sp.q;
 }
 
 // Walks the steps [b, e) of a CTA's range in the order: the partial segment
 // that ends the range ([last_begin, e), empty when e ends a tile), then the
 // segment that starts it ([b, first_end)), then the whole tiles between them
 // ([first_end, last_begin)).  The tile t and K block kb are kept
-// incrementally: 64-bit divisions only where a run starts.
+// incrementally: divisions only where a run starts.
 struct StepIter {
-  int64_t first_end, last_begin, b0, e0;
-  int64_t s, cur_b, cur_e;   // the current run [cur_b, cur_e)
+  int first_end, last_begin, b0, e0;
+  int s, cur_b, cur_e;   // the current run [cur_b, cur_e)
   int run, t, kb, KB;
-  __host__ __device__ StepIter(int64_t b, int64_t e, int kblocks) : b0(b), e0(e), KB(kblocks) {
+  __host__ __device__ StepIter(int b, int e, int kblocks) : b0(b), e0(e), KB(kblocks) {
     first_end = min(e, (b / KB + 1) * KB);
     last_begin = (e % KB == 0) ? e : max(first_end, ((e - 1) / KB) * KB);
     run = -1;
@@ -98,8 +109,8 @@ struct StepIter {
       if (cur_b < cur_e) break;
     }
     s = cur_b;
-    t = static_cast<int>(s / KB);
-    kb = static_cast<int>(s - static_cast<int64_t>(t) * KB);
+    t = s / KB;
+    kb = s - t * KB;
   }
   __host__ __device__ bool valid() const { return run < 3; }
   // Whether this step starts / ends a segment (a run of steps in one tile).
@@ -132,7 +143,7 @@ struct Layout {
   static constexpr int kWide = W16 ? 128 * BK * 2 : 0;
   static constexpr int kBarOff = STAGES * (kW + kX + kWide);
   static constexpr int kThreads = 192 + 32 * WIDEN;
-  static constexpr int kBarBytes = (2 * STAGES + 2 * kSlots + (W16 ? STAGES : 0)) * 8 + 8;   // mbarriers, TMEM address, abort flag
+  static constexpr int kBarBytes = (2 * STAGES + 2 * kSlots + (W16 ? STAGES : 0) + 1) * 8 + 8;   // mbarriers, TMEM address, abort flag
   static constexpr int kBytes = kBarOff + 1024 + 1024;                  // + barrier area + alignment slack
   static_assert(kBarBytes <= 1024, "barrier area");
   static_assert(kBytes <= 232448, "shared memory per CTA");
@@ -158,14 +169,16 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
   uint64_t* sfull = empty + STAGES;
   uint64_t* sempty = sfull + kSlots;
   uint64_t* wfull = sempty + kSlots;                       // W16: widened tile ready (STAGES of them)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wfull + (W16 ? STAGES : 0));
+  uint64_t* drain = wfull + (W16 ? STAGES : 0);            // abort path: the MMAs issued have completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int c = blockIdx.x;
-  const int64_t b = range_begin(c, p.total, p.G);
-  const int64_t e = range_begin(c + 1, p.total, p.G);
+  const Split sp = split_of(p.total, p.G);
+  const int b = range_begin(c, sp);
+  const int e = range_begin(c + 1, sp);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -178,6 +191,7 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
     }
     if constexpr (W16)
       for (int s = 0; s < STAGES; ++s) mbar_init(&wfull[s], WIDEN);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmW);
@@ -200,9 +214,11 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      int issued = 0;
       for (StepIter it(b, e, p.KB); it.valid(); it.next()) {
         const int t = it.t, kb = it.kb;
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) { ok = false; break; }
+        ++issued;
         mbar_arrive_expect_tx(&full[stage], L::kW + L::kX);
         tma_load_2d(sW + stage * L::kW, &tmW, &full[stage], kb * BK, t * 128, pol_w);
         tma_load_2d(sX + stage * L::kX, &tmX, &full[stage], kb * BK, 0, pol_x);
@@ -212,8 +228,20 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
       }
       griddep_launch_dependents();
       for (int i = 0; ok && i < STAGES; ++i) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) break;
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) { ok = false; break; }
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) {
+        // Aborted: the last load of each stage may still be in flight.  Each
+        // completes on its own; wait for all of them before the CTA's shared
+        // memory is released.  Walk back from the stage that was not issued.
+        const int n = issued < STAGES ? issued : STAGES;
+        int s = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < n; ++i) {
+          if (--s < 0) { s = STAGES - 1; ph ^= 1u; }
+          mbar_wait_drain(&full[s], ph, kErrWaitDrain);
+        }
       }
     }
   } else if (warp == 1) {
@@ -221,6 +249,10 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
       constexpr uint32_t idesc = W16 ? idesc_bf16_f32(128, NX) : idesc_e4m3_f32(128, NX);
       int stage = 0, slot = 0;
       uint32_t phase = 0, sphase = 0;
+      bool ok = true;
+#ifdef FP8Q_TEST_HOOKS
+      bool withheld = false;
+#endif
       for (StepIter it(b, e, p.KB); it.valid(); it.next()) {
         const bool seg_first = it.seg_first();
         const bool seg_last = it.seg_last();
@@ -228,9 +260,9 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
         // mode: one slot per segment, accumulated across its K blocks.
         const bool open_slot = BLOCK || seg_first;
         const bool close_slot = BLOCK || seg_last;
-        if (open_slot && !mbar_wait(&sempty[slot], sphase ^ 1u, abort_flag, kErrWaitTmemEmpty)) break;
-        if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) break;
-        if (W16 && !mbar_wait(&wfull[stage], phase, abort_flag, kErrWaitFull)) break;
+        if (open_slot && !mbar_wait(&sempty[slot], sphase ^ 1u, abort_flag, kErrWaitTmemEmpty)) { ok = false; break; }
+        if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) { ok = false; break; }
+        if (W16 && !mbar_wait(&wfull[stage], phase, abort_flag, kErrWaitFull)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem_base + slot * NX;
         const uint32_t b0 = smem_u32(sX + stage * L::kX);
@@ -251,11 +283,23 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
         }
         mma_commit(&empty[stage]);
         if (close_slot) {
+#ifdef FP8Q_TEST_HOOKS
+          // Test build, switch 2: CTA 0 withholds its first accumulator commit.
+          const bool withhold = c == 0 && !withheld && g_test_withhold == 2;
+          withheld = withheld || withhold;
+          if (!withhold) mma_commit(&sfull[slot]);
+#else
           mma_commit(&sfull[slot]);
+#endif
           if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
         }
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
+      // Every MMA issued must finish before the tensor memory is released.
+      // Normally the epilogue's waits already imply it; after an abort they
+      // do not, so one more commit tracks all of them, always.
+      mma_commit(drain);
+      if (!mbar_wait_drain(drain, 0, kErrWaitDrain)) ok = false;
     }
   } else if (W16 && warp >= 6) {
     // Widen: a thread takes one weight row of the tile (8 warps: half of it).
@@ -304,23 +348,42 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
     for (int j = 0; j < NX; ++j) acc[j] = 0.0f;
     int slot = 0;
     uint32_t sphase = 0;
-    // Block mode: the scales of step s are fetched one step ahead (for NX <= 32;
-    // at NX = 64 the extra registers would spill).
-    constexpr bool kPrefetch = BLOCK && NX <= 32;
-    float fx[kPrefetch ? NX : 1];
-    float fw = 0.0f;
-    auto fetch = [&](int t, int kb) {
-      if constexpr (kPrefetch) {
-        fw = __ldg(p.ws + static_cast<int64_t>(t) * p.KB + kb);
-#pragma unroll
-        for (int j = 0; j < NX; ++j) fx[j] = j < p.M ? __ldg(p.xs + static_cast<int64_t>(j) * p.KB + kb) : 0.0f;
+    // Block mode: the x_scale column and w_scale of each step go into this
+    // warp's ring slot (step index % kRing) kAhead steps before the step is
+    // folded, by cp.async copies of one float per lane; one commit group per
+    // step, so wait_group<kAhead - 1> means the current step's scales are in.
+    constexpr int kRing = 8, kAhead = 6;
+    __shared__ float s_ring[BLOCK ? 4 : 1][BLOCK ? kRing : 1][NX + 1];
+    float* ring = &s_ring[BLOCK ? quarter : 0][0][0];
+    StepIter pf(b, e, p.KB);                        // the step whose scales are fetched next
+    int pf_i = 0;
+    auto prefetch = [&]() {
+      if constexpr (BLOCK) {
+        if (pf.valid()) {
+          float* dst = ring + (pf_i % kRing) * (NX + 1);
+          for (int j = lane; j < NX; j += 32)
+            if (j < p.M) cp_async_f32(dst + j, p.xs + static_cast<int64_t>(j) * p.KB + pf.kb);
+          if (lane == 0) cp_async_f32(dst + NX, p.ws + static_cast<int64_t>(pf.t) * p.KB + pf.kb);
+          pf.next();
+        }
+        ++pf_i;
+        cp_async_commit();
       }
     };
+    if constexpr (BLOCK) {
+      for (int i = lane; i < kRing * NX; i += 32)   // padded tokens (never copied into) stay 0
+        if (i % NX >= p.M) ring[(i / NX) * (NX + 1) + i % NX] = 0.0f;
+      __syncwarp();
+      for (int i = 0; i < kAhead; ++i) prefetch();
+    }
     StepIter it(b, e, p.KB);
-    if (it.valid()) fetch(it.t, it.kb);
+    int step_i = 0;
     int seg_len = 0;
-    for (; it.valid(); it.next()) {
-      const int t = it.t, kb = it.kb;
+#ifdef FP8Q_TEST_HOOKS
+    bool withheld = false;
+#endif
+    for (; it.valid(); it.next(), ++step_i) {
+      const int t = it.t;
       seg_len = it.seg_first() ? 1 : seg_len + 1;
       const bool seg_last = it.seg_last();
       if (!BLOCK && !seg_last) continue;           // channel mode: one drain per segment
@@ -334,30 +397,30 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
+#ifdef FP8Q_TEST_HOOKS
+      // Test build, switch 1: CTA 0's warp 2 withholds its first slot release.
+      const bool withhold = c == 0 && warp == 2 && !withheld && g_test_withhold == 1;
+      withheld = withheld || withhold;
+      if (lane == 0 && !withhold) mbar_arrive_relaxed(&sempty[slot]);
+#else
       if (lane == 0) mbar_arrive_relaxed(&sempty[slot]);
+#endif
       if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
-      if constexpr (kPrefetch) {
-        float f[NX];
+      if constexpr (BLOCK) {
+        cp_async_wait<kAhead - 1>();               // this step's scales are in the ring
+        __syncwarp();
+        const float* sc = ring + (step_i % kRing) * (NX + 1);
+        const float wsf = sc[NX];
 #pragma unroll
-        for (int j = 0; j < NX; ++j) f[j] = fx[j] * fw;
-        StepIter nx = it;
-        nx.next();
-        if (nx.valid()) fetch(nx.t, nx.kb);
-#pragma unroll
-        for (int j = 0; j < NX; ++j) acc[j] = fmaf(__uint_as_float(r[j]), f[j], acc[j]);
-      } else if constexpr (BLOCK) {
-        const float wsf = __ldg(p.ws + static_cast<int64_t>(t) * p.KB + kb);
-#pragma unroll
-        for (int j = 0; j < NX; ++j) {
-          const float f = j < p.M ? __ldg(p.xs + static_cast<int64_t>(j) * p.KB + kb) * wsf : 0.0f;
-          acc[j] = fmaf(__uint_as_float(r[j]), f, acc[j]);
-        }
+        for (int j = 0; j < NX; ++j) acc[j] = fmaf(__uint_as_float(r[j]), sc[j] * wsf, acc[j]);
+        __syncwarp();                              // every lane has read the slot before it is refilled
+        prefetch();
       } else {
 #pragma unroll
         for (int j = 0; j < NX; ++j) acc[j] = __uint_as_float(r[j]);
       }
       if (seg_last) {                              // segment ends
-        const int64_t tile_first = static_cast<int64_t>(t) * p.KB;
+        const int tile_first = t * p.KB;
         const int n = t * 128 + nl;
         // bf16 output of channel n for the token sums v[j]
         auto emit = [&](const float (&v)[NX]) {
@@ -386,8 +449,8 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
           }
           __threadfence();
           __syncwarp();
-          const int c0 = cta_of_step(tile_first, p.total, p.G);
-          const int c1 = cta_of_step(tile_first + p.KB - 1, p.total, p.G);
+          const int c0 = cta_of_step(tile_first, sp);
+          const int c1 = cta_of_step(tile_first + p.KB - 1, sp);
           unsigned int prev = 0;
           if (lane == 0) prev = atomicAdd(p.count + t * 4 + quarter, 1u);
           prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
@@ -416,6 +479,7 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
         for (int j = 0; j < NX; ++j) acc[j] = 0.0f;
       }
     }
+    if constexpr (BLOCK) cp_async_wait<0>();     // no copy into the ring outlives the CTA
   }
 
   tc_fence_before();
@@ -438,8 +502,9 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const Params p, int 
   const int m = blockIdx.y;
   const int nl = threadIdx.x;
   const int n = t * 128 + nl;
-  const int c0 = cta_of_step(static_cast<int64_t>(t) * p.KB, p.total, p.G);
-  const int c1 = cta_of_step(static_cast<int64_t>(t + 1) * p.KB - 1, p.total, p.G);
+  const Split sp = split_of(p.total, p.G);
+  const int c0 = cta_of_step(t * p.KB, sp);
+  const int c1 = cta_of_step((t + 1) * p.KB - 1, sp);
   if (c0 == c1) return;
   float sum = 0.0f;
   for (int c = c0; c <= c1; ++c) sum += __ldcg(p.part + ((static_cast<int64_t>(t) + c) * nx + m) * 128 + nl);

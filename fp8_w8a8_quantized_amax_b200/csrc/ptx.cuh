@@ -23,8 +23,22 @@ enum : int {
 };
 
 // A wait gives up after this many nanoseconds of %globaltimer.  No healthy
-// run comes near it (the longest single wait is a few microseconds).
-constexpr uint64_t kWaitLimitNs = 4000000000ull;
+// run comes near it (the longest single wait is a few microseconds).  The
+// test build of the library lowers it, so that a test can make a wait run out
+// in milliseconds.
+#ifndef FP8Q_WAIT_LIMIT_NS
+#define FP8Q_WAIT_LIMIT_NS 4000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = FP8Q_WAIT_LIMIT_NS;
+
+#ifdef FP8Q_TEST_HOOKS
+// Test build only (failure-detection tests; the product library has no such
+// switch).  1: the decode kernel's CTA 0 withholds one tensor-memory slot
+// release, so that the MMA warp's wait for that slot runs out.  2: its MMA
+// warp withholds the first accumulator commit, so that the epilogue's wait
+// runs out (and the CTA's split-tile sums are never delivered).
+__device__ int g_test_withhold;
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -137,6 +151,38 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
   }
   return true;
+}
+
+// After an abort: wait for a phase that completes on its own (a TMA load or
+// MMAs already issued), so that nothing is still writing the CTA's shared or
+// tensor memory when it is released.  The abort flag is ignored; the time
+// limit is not (records `site` if it runs out).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int site) {
+  const uint32_t b = smem_u32(bar);
+  const uint64_t t0 = globaltimer();
+  uint32_t it = 0;
+  while (!mbar_try_wait(b, parity)) {
+    if ((++it & 255u) == 0 && globaltimer() - t0 > kWaitLimitNs) {
+      atomicCAS(&g_device_error, 0, site);
+      return false;
+    }
+  }
+  return true;
+}
+
+// ------------------------------------------------- small async copies ---
+
+// One float from global to shared memory, asynchronously (cp.async, cached in
+// L1: scales that every CTA reads).  Completion is tracked per thread by
+// commit groups.
+__device__ __forceinline__ void cp_async_f32(float* dst_smem, const float* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's commit groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // -------------------------------------------------------------- clusters ---

@@ -120,6 +120,26 @@ FP8Q_API fp8q_status fp8_quant_act_static(const void* X_bf16, int64_t M, int64_t
                                           uint8_t* Xq, int64_t ldxq, float* x_scale, void* stream);
 
 /*
+ * fp8_calibrate_static_scale -- the static scale fp8_quant_act_static takes,
+ * from a calibration tensor: "Llama 3 精读实录" section 2 uses its 0.1% and
+ * 99.9% quantiles as the range instead of min / max.  Offline, once per tensor.
+ *   q(p)   = v[i] + (v[j] - v[i]) * (p (n-1) - i),  i = floor(p (n-1)),
+ *            j = min(i + 1, n - 1), v the n = M*K values sorted ascending (double)
+ *   amax   = max(|q(lo)|, |q(hi)|);   scale = fl32(fl32(amax) / 448), 1 when amax == 0
+ * The order statistics are exact: the kernels count the 65536 bf16 bit patterns.
+ *   X_bf16  [M, ldx] bf16, read-only, 16-byte aligned, ldx >= K, ldx % 8 == 0.
+ *   lo, hi  quantile levels in [0, 1] (0.001 and 0.999 for the pages' range).
+ *   hist    device workspace of 65536 uint32 counts (262144 bytes), 4-byte
+ *           aligned, zero-filled before its first use; every completed call
+ *           leaves it all zero.  Not shared by concurrent calls.
+ *   scale   one fp32 in device memory, written.
+ * Requirements: M >= 1, K >= 1, K % 8 == 0, M * K < 2^32 (FP8Q_ERR_UNSUPPORTED
+ * above).  Values must be finite.
+ */
+FP8Q_API fp8q_status fp8_calibrate_static_scale(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, double lo,
+                                                double hi, uint32_t* hist, float* scale, void* stream);
+
+/*
  * fp8_rmsnorm_quant_act -- RMSNorm of bf16 activations, then per-token E4M3
  * quantization of the result, in one pass (the normalised bf16 rows are not
  * written).  Llama 3 normalises with RMSNorm (eps 1e-5) before attention and

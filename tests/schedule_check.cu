@@ -33,21 +33,28 @@ static int fail(const char* what, int n_tiles, int KB, int G) {
 }
 
 static int check(int n_tiles, int KB, int G) {
-  const int64_t total = static_cast<int64_t>(n_tiles) * KB;
+  const int total = n_tiles * KB;
+  const Split sp = split_of(total, G);
   std::vector<int> owner(total, -1), seen(total, 0);
   std::set<int64_t> slots;
   std::vector<std::set<int>> partial_ctas(n_tiles);
+  // sizes: every range q or q + 1 steps
   for (int c = 0; c < G; ++c) {
-    const int64_t b = range_begin(c, total, G), e = range_begin(c + 1, total, G);
+    const int len = range_begin(c + 1, sp) - range_begin(c, sp);
+    if (len != total / G && len != total / G + 1) return fail("range size", n_tiles, KB, G);
+  }
+  if (range_begin(0, sp) != 0 || range_begin(G, sp) != total) return fail("ranges cover", n_tiles, KB, G);
+  for (int c = 0; c < G; ++c) {
+    const int b = range_begin(c, sp), e = range_begin(c + 1, sp);
     if (b >= e) return fail("empty range", n_tiles, KB, G);
-    for (int64_t s = b; s < e; ++s) owner[s] = c;
+    for (int s = b; s < e; ++s) owner[s] = c;
     // expected order
-    const int64_t first_end = std::min(e, (b / KB + 1) * KB);
-    const int64_t last_begin = (e % KB == 0) ? e : std::max(first_end, ((e - 1) / KB) * KB);
-    std::vector<int64_t> want;
-    for (int64_t s = last_begin; s < e; ++s) want.push_back(s);
-    for (int64_t s = b; s < first_end; ++s) want.push_back(s);
-    for (int64_t s = first_end; s < last_begin; ++s) want.push_back(s);
+    const int first_end = std::min(e, (b / KB + 1) * KB);
+    const int last_begin = (e % KB == 0) ? e : std::max(first_end, ((e - 1) / KB) * KB);
+    std::vector<int> want;
+    for (int s = last_begin; s < e; ++s) want.push_back(s);
+    for (int s = b; s < first_end; ++s) want.push_back(s);
+    for (int s = first_end; s < last_begin; ++s) want.push_back(s);
     size_t i = 0;
     int seg_len = 0;
     for (StepIter it(b, e, KB); it.valid(); it.next(), ++i) {
@@ -66,13 +73,13 @@ static int check(int n_tiles, int KB, int G) {
     }
     if (i != want.size()) return fail("steps missing", n_tiles, KB, G);
   }
-  for (int64_t s = 0; s < total; ++s) {
+  for (int s = 0; s < total; ++s) {
     if (seen[s] != 1) return fail("step not visited once", n_tiles, KB, G);
-    if (cta_of_step(s, total, G) != owner[s]) return fail("cta_of_step", n_tiles, KB, G);
+    if (cta_of_step(s, sp) != owner[s]) return fail("cta_of_step", n_tiles, KB, G);
   }
   for (int t = 0; t < n_tiles; ++t) {
-    const int c0 = cta_of_step(static_cast<int64_t>(t) * KB, total, G);
-    const int c1 = cta_of_step(static_cast<int64_t>(t) * KB + KB - 1, total, G);
+    const int c0 = cta_of_step(t * KB, sp);
+    const int c1 = cta_of_step(t * KB + KB - 1, sp);
     std::set<int> want;
     if (c0 != c1)
       for (int c = c0; c <= c1; ++c) want.insert(c);

@@ -254,6 +254,29 @@ def test_noalloc_argument_checks(L, kw, want):
     assert noalloc(L, **kw) == want
 
 
+def calib(L, x=P, M=4, K=256, ldx=256, lo=0.001, hi=0.999, h=P, s=P):
+    return L.fp8_calibrate_static_scale(x, M, K, ldx, lo, hi, h, s, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(M=0), fq.ERR_INVALID_ARG),                         # no values: no quantile
+    (dict(K=12, ldx=12), fq.ERR_INVALID_ARG),                # K % 8
+    (dict(ldx=128), fq.ERR_INVALID_ARG),
+    (dict(lo=-0.1), fq.ERR_INVALID_ARG),
+    (dict(hi=1.5), fq.ERR_INVALID_ARG),
+    (dict(lo=float("nan")), fq.ERR_INVALID_ARG),
+    (dict(x=None), fq.ERR_INVALID_ARG),
+    (dict(h=None), fq.ERR_INVALID_ARG),
+    (dict(s=None), fq.ERR_INVALID_ARG),
+    (dict(x=BAD), fq.ERR_MISALIGNED),
+    (dict(h=P + 2), fq.ERR_MISALIGNED),
+    (dict(ldx=260), fq.ERR_MISALIGNED),
+    (dict(M=1 << 20, K=1 << 12, ldx=1 << 12), fq.ERR_UNSUPPORTED),    # 2^32 values
+])
+def test_calibrate_argument_checks(L, kw, want):
+    assert calib(L, **kw) == want
+
+
 def test_workspace_size_is_zero_for_invalid_or_prefill(L):
     assert L.fp8_linear_workspace_size(0, 64, 256, 0) == 0
     assert L.fp8_linear_workspace_size(128, 64, 256, 0) == 0
@@ -268,6 +291,7 @@ def test_valid_arguments_without_a_gpu_report_cuda_error(L):
     assert lin(L, wsp=P + 16) == fq.ERR_CUDA            # 16-byte alignment is enough
     assert lin(L, M=65, wsp=None, wsb=0) == fq.ERR_CUDA  # the prefill path needs no workspace
     assert noalloc(L) == fq.ERR_CUDA
+    assert calib(L) == fq.ERR_CUDA
     assert rms_q(L) == fq.ERR_CUDA
     assert swi(L) == fq.ERR_CUDA
     assert q_static(L) == fq.ERR_CUDA

@@ -199,6 +199,41 @@ def test_static_scale_bit_exact(M, K):
     P.assert_y_close(y, oracle.linear(rq, np.full(M, scale, np.float32), rwq, rws, 0), what=f"static linear {M}x{K}")
 
 
+def _calib_cases():
+    g = torch.Generator().manual_seed(21)
+    out = {"llama 8b attn_in 8192x4096": synth.make_x(8192, 4096, seed=1),
+           "mostly negative": (-synth.make_x(64, 512, seed=2).float().abs() + 0.01).to(torch.bfloat16),
+           "constant": torch.full((3, 64), -2.5, dtype=torch.bfloat16),
+           "zeros": torch.zeros(4, 16, dtype=torch.bfloat16),
+           "one row of 8": synth.make_x(1, 8, seed=3),
+           "heavy tails": (torch.randn(257, 96, generator=g) ** 3 * 1e3).to(torch.bfloat16)}
+    sub = torch.zeros(8, 64, dtype=torch.bfloat16)
+    sub[:, ::3] = 2.0 ** -130                    # bf16 subnormals
+    sub[0, 1] = -(2.0 ** -133)
+    out["subnormals"] = sub
+    return out
+
+
+@pytest.mark.parametrize("name", list(_calib_cases()))
+@pytest.mark.parametrize("lo,hi", [(0.001, 0.999), (0.0, 1.0), (0.25, 0.5), (0.1, 0.9)])
+def test_calibration_kernel_equals_the_oracle(name, lo, hi):
+    # order statistics from the bit-pattern histogram, interpolated in double:
+    # the same fp32 scale as the oracle's sort, bit for bit; the workspace is
+    # left zero for the next call
+    x = _calib_cases()[name]
+    hist = torch.zeros(fq.CALIB_HIST_BINS, dtype=torch.int32, device=DEV)
+    got = fq.calibrate_static_scale(x.to(DEV), lo, hi, hist=hist)
+    want = oracle.percentile_scale(x, lo, hi)
+    assert np.float32(got) == np.float32(want), f"{name}: {got!r} vs {want!r}"
+    assert int(hist.abs().sum().item()) == 0
+
+
+def test_calibration_of_a_strided_view():
+    big = synth.make_x(300, 1024 + 64, seed=9)
+    xd = big.to(DEV)[:, 32:32 + 1024]
+    assert fq.calibrate_static_scale(xd) == oracle.percentile_scale(big[:, 32:32 + 1024].contiguous())
+
+
 def test_static_scale_saturates_outliers():
     x = synth.make_x(64, 512, seed=5)            # outlier columns far above the P99.9 range
     scale = oracle.percentile_scale(x)

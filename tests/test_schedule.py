@@ -23,3 +23,37 @@ def test_stream_k_schedule_invariants():
         r = subprocess.run([exe], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout[-2000:]
     assert r.stdout.strip().splitlines()[-1].startswith("ok:")
+
+
+MUTANTS = {
+    "range rounding": (r"return c \* sp\.q \+ min\(c, sp\.r\);", "return c * sp.q + min(c, sp.r + 1);"),
+    "owner of a step": (r"return x < big \? x / \(sp\.q \+ 1\) : sp\.r \+ \(x - big\) / sp\.q;",
+                        "return x < big ? x / sp.q : sp.r + (x - big) / sp.q;"),
+    "K-block wrap": (r"\} else if \(\+\+kb == KB\) \{", "} else if (++kb == KB + 1) {"),
+    "first segment end": (r"first_end = min\(e, \(b / KB \+ 1\) \* KB\);", "first_end = min(e, (b / KB + 1) * KB - 1);"),
+}
+
+
+@pytest.mark.skipif(shutil.which("nvcc") is None and not os.path.exists("/usr/local/cuda/bin/nvcc"),
+                    reason="needs nvcc")
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_schedule_check_catches_planted_mistake(name):
+    """A plausible mistake planted in a copy of the decode schedule fails the check."""
+    import re
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    root = os.path.dirname(HERE)
+    pat, rep = MUTANTS[name]
+    with tempfile.TemporaryDirectory() as tmp:
+        shutil.copytree(os.path.join(root, "fp8_w8a8_quantized_amax_b200", "csrc"),
+                        os.path.join(tmp, "fp8_w8a8_quantized_amax_b200", "csrc"))
+        os.makedirs(os.path.join(tmp, "tests"))
+        shutil.copy(os.path.join(HERE, "schedule_check.cu"), os.path.join(tmp, "tests"))
+        hdr = os.path.join(tmp, "fp8_w8a8_quantized_amax_b200", "csrc", "gemm_decode.cuh")
+        src, n = re.subn(pat, rep, open(hdr).read())
+        assert n >= 1, f"mutation '{name}' did not apply"
+        open(hdr, "w").write(src)
+        exe = os.path.join(tmp, "schedule_check")
+        subprocess.check_call([nvcc, "-std=c++17", "-O1", "-gencode", "arch=compute_100a,code=sm_100a", "-x", "cu",
+                               os.path.join(tmp, "tests", "schedule_check.cu"), "-o", exe], timeout=300)
+        r = subprocess.run([exe], capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0 and "FAIL" in r.stdout, f"planted mistake '{name}' passed the schedule check"

@@ -382,8 +382,12 @@ def run_gpu(args):
               torch.empty(fq.scale_shape_act(M, K, mode), dtype=torch.float32, device=dev))
           for k, (M, K, mode) in xs_shapes.items()}
     Y = {g.name: torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev) for g in wl.gemms}
-    WS = {g.name: (torch.zeros(fq.fp8_linear_workspace_size(g.M, g.N, g.K, g.mode), dtype=torch.uint8,
-                               device=dev) if g.M <= 64 else None) for g in wl.gemms}
+    # scratch of the decode path and of the stream-K prefill schedule (where
+    # fp8_linear_workspace_size asks for one), zero-filled once
+    WS = {}
+    for g in wl.gemms:
+        nws = fq.fp8_linear_workspace_size(g.M, g.N, g.K, g.mode)
+        WS[g.name] = torch.zeros(nws, dtype=torch.uint8, device=dev) if nws else None
     class _Flush:
         """Write one buffer larger than L2, then read another: L2 ends up
         holding only clean lines of the read buffer."""
@@ -684,45 +688,77 @@ def run_gpu(args):
                     "GB/s": round(wqb / (min(wq_ms) / 1e3) / 1e9, 1),
                     "frac_hbm": round(wqb / (min(wq_ms) / 1e3) / 1e9 / pk["hbm_gbs"], 3)}
 
+    # ---- the next-step sections: each op timed like the per-op detail (R
+    # back-to-back launches over R copies of its buffers, or alone when long)
+    def timed(run):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda._sleep(1_000_000)
+        for s_ in range(args.steps):
+            flush.zero_()
+            ev[s_][0].record(stream)
+            run()
+            ev[s_][1].record(stream)
+        torch.cuda.synchronize()
+        return float(np.mean([a.elapsed_time(b) for a, b in ev]))
+
+    def as_runner(fns):
+        for f in fns:
+            f()
+        torch.cuda.synchronize()
+        if args.eager:
+            return lambda: [f() for f in fns]
+        gr = capture(fns)
+        return gr.replay
+
+    def time_op(make, footprint):
+        """(ms per launch, R, ms alone) of the op make(0); make(i) for i > 0
+        builds the same op on its own copies of the op's buffers."""
+        f0 = make(0)
+        alone = timed(as_runner([f0]))
+        if alone >= LONG_OP_MS:
+            return alone, 1, alone
+        R = int(min(32, max(2, -(-2 * l2_bytes // max(1, footprint)))))
+        fns = [f0] + [make(i) for i in range(1, R)]
+        t = timed(as_runner(fns)) / R
+        del fns
+        return t, R, alone
+
+    def entry(ms, R, alone, nbytes=None, flops=None):
+        e = {"ms": round(ms, 5), "back_to_back": R, "ms_isolated": round(alone, 5)}
+        if nbytes is not None:
+            e["GB/s"] = round(nbytes / (ms / 1e3) / 1e9, 1)
+            e["frac_hbm"] = round(nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"], 3)
+        if flops is not None:
+            e["TFLOP/s"] = round(flops / (ms / 1e3) / 1e12, 1)
+            e["frac_fp8_peak"] = round(flops / (ms / 1e3) / 1e12 / fp8_peak, 3)
+        return e
+
     # ---- RMSNorm + per-token quantization fused (the activations that follow
-    # an RMSNorm in Llama: the inputs of q/k/v and of gate/up), timed alone,
-    # next to the unfused pair (torch's bf16 rms_norm, then fp8_quant_act)
+    # an RMSNorm in Llama: the inputs of q/k/v and of gate/up), next to the
+    # unfused pair (torch's bf16 rms_norm, then fp8_quant_act)
     rms = []
     for k, (M, K, mode) in ([] if args.no_extras else xs_shapes.items()):
         if mode != synth.CHANNEL_TOKEN or not (k.startswith("attn_in") or k.startswith("mlp_in")):
             continue
         gmm = (1.0 + 0.1 * torch.randn(K, generator=torch.Generator().manual_seed(K))).to(torch.bfloat16).to(dev)
-        xq_f, xs_f = torch.empty_like(XQ[k][0]), torch.empty_like(XQ[k][1])
-        y_n = torch.empty_like(X[k])
 
-        def fused(k=k, gmm=gmm, xq_f=xq_f, xs_f=xs_f):
-            fq.fp8_rmsnorm_quant_act(X[k], gmm, 1e-5, out=(xq_f, xs_f))
+        def make_fused(i, k=k, gmm=gmm):
+            x = X[k] if i == 0 else X[k].clone()
+            o = (torch.empty_like(XQ[k][0]), torch.empty_like(XQ[k][1]))
+            return lambda: fq.fp8_rmsnorm_quant_act(x, gmm, 1e-5, out=o)
 
-        def unfused(k=k, gmm=gmm, xq_f=xq_f, xs_f=xs_f, y_n=y_n, K=K):
-            y_n.copy_(torch.nn.functional.rms_norm(X[k], (K,), weight=gmm, eps=1e-5))
-            fq.fp8_quant_act(y_n, synth.CHANNEL_TOKEN, out=(xq_f, xs_f))
+        def make_unfused(i, k=k, gmm=gmm, K=K):
+            x = X[k] if i == 0 else X[k].clone()
+            y_n = torch.empty_like(X[k])
+            o = (torch.empty_like(XQ[k][0]), torch.empty_like(XQ[k][1]))
+            return lambda: (y_n.copy_(torch.nn.functional.rms_norm(x, (K,), weight=gmm, eps=1e-5)),
+                            fq.fp8_quant_act(y_n, synth.CHANNEL_TOKEN, out=o))
 
-        times = []
-        for fn in (fused, unfused):
-            fn()
-            torch.cuda.synchronize()
-            gr = capture([fn]) if not args.eager else None
-            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
-            torch.cuda._sleep(2_000_000)
-            for s_ in range(args.steps):
-                flush.zero_()
-                ev[s_][0].record(stream)
-                gr.replay() if gr is not None else fn()
-                ev[s_][1].record(stream)
-            torch.cuda.synchronize()
-            times.append(float(np.median([a.elapsed_time(b) for a, b in ev])))
         rb = 2 * M * K + 2 * K + M * K + 4 * M
-        rms.append({"act": k, "M": M, "K": K, "ms": round(times[0], 5),
-                    "GB/s": round(rb / (times[0] / 1e3) / 1e9, 1),
-                    "frac_hbm": round(rb / (times[0] / 1e3) / 1e9 / pk["hbm_gbs"], 3),
-                    "unfused_ms": round(times[1], 5),
-                    "bytes": "2*M*K (x) + 2*K (gamma) + M*K (codes) + 4*M (scales)"})
+        e = entry(*time_op(make_fused, rb), nbytes=rb)
+        e.update({"act": k, "M": M, "K": K, "unfused_ms": round(time_op(make_unfused, rb + 4 * M * K)[0], 5),
+                  "bytes": "2*M*K (x) + 2*K (gamma) + M*K (codes) + 4*M (scales)"})
+        rms.append(e)
     assert fq.device_error(clear=True) == 0
 
     # ---- gate/up with the SiLU * up epilogue (one kernel, only the activation
@@ -738,40 +774,35 @@ def run_gpu(args):
         if len(gg) != 1 or len(gu) != 1:
             continue
         gg, gu = gg[0], gu[0]
-        act = torch.empty((gg.M, gg.N), dtype=torch.bfloat16, device=dev)
 
-        def fused(gg=gg, gu=gu, act=act):
-            fq.fp8_linear_swiglu(XQ[gg.x][0], XQ[gg.x][1], WQ[gg.weight][0], WQ[gg.weight][1], WQ[gu.weight][0],
-                                 WQ[gu.weight][1], out=act)
+        def ops_of(i, gg=gg, gu=gu):
+            c = (lambda t: t) if i == 0 else (lambda t: t.clone())
+            return (c(XQ[gg.x][0]), c(XQ[gg.x][1]), c(WQ[gg.weight][0]), c(WQ[gg.weight][1]), c(WQ[gu.weight][0]),
+                    c(WQ[gu.weight][1]))
 
-        def separate(gg=gg, gu=gu, act=act):
-            for g in (gg, gu):
-                fq.fp8_linear(XQ[g.x][0], XQ[g.x][1], WQ[g.weight][0], WQ[g.weight][1], g.mode, out=Y[g.name],
-                              workspace=WS[g.name])
-            torch.mul(torch.nn.functional.silu(Y[gg.name]), Y[gu.name], out=act)
+        def make_fused(i, gg=gg):
+            o = ops_of(i)
+            act = torch.empty((gg.M, gg.N), dtype=torch.bfloat16, device=dev)
+            return lambda: fq.fp8_linear_swiglu(*o, out=act)
 
-        times = []
-        for fn in (fused, separate):
-            fn()
-            torch.cuda.synchronize()
-            gr = capture([fn]) if not args.eager else None
-            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
-            torch.cuda._sleep(2_000_000)
-            for s_ in range(args.steps):
-                flush.zero_()
-                ev[s_][0].record(stream)
-                gr.replay() if gr is not None else fn()
-                ev[s_][1].record(stream)
-            torch.cuda.synchronize()
-            times.append(float(np.median([a.elapsed_time(b) for a, b in ev])))
+        def make_separate(i, gg=gg, gu=gu):
+            xq, xsc, wg, sg, wu, su = ops_of(i)
+            yg = torch.empty((gg.M, gg.N), dtype=torch.bfloat16, device=dev)
+            yu = torch.empty_like(yg)
+            act = torch.empty_like(yg)
+            wk = {g.name: (torch.zeros_like(WS[g.name]) if WS[g.name] is not None else None) for g in (gg, gu)}
+            return lambda: (fq.fp8_linear(xq, xsc, wg, sg, gg.mode, out=yg, workspace=wk[gg.name]),
+                            fq.fp8_linear(xq, xsc, wu, su, gu.mode, out=yu, workspace=wk[gu.name]),
+                            torch.mul(torch.nn.functional.silu(yg), yu, out=act))
+
         fl = 2 * gg.flops
-        swiglu.append({"gemms": f"{gg.name}+{gu.name}:{gg.M}x{gg.K}->{gg.N}", "ms": round(times[0], 5),
-                       "TFLOP/s": round(fl / (times[0] / 1e3) / 1e12, 1),
-                       "frac_fp8_peak": round(fl / (times[0] / 1e3) / 1e12 / fp8_peak, 3),
-                       "separate_ms": round(times[1], 5),
-                       "note": "fused: one kernel writes bf16(bf16(silu(gate)) * up); separate: two GEMMs "
-                               "writing gate and up, then torch silu and mul"})
+        fb = gg.M * gg.K + 2 * gg.N * gg.K + 2 * gg.M * gg.N
+        e = entry(*time_op(make_fused, fb), flops=fl)
+        e.update({"gemms": f"{gg.name}+{gu.name}:{gg.M}x{gg.K}->{gg.N}",
+                  "separate_ms": round(time_op(make_separate, fb + 4 * gg.M * gg.N)[0], 5),
+                  "note": "fused: one kernel writes bf16(bf16(silu(gate)) * up); separate: two GEMMs "
+                          "writing gate and up, then torch silu and mul"})
+        swiglu.append(e)
     assert fq.device_error(clear=True) == 0
 
     # ---- static-scale quantization (offline-calibrated scale, no amax pass)
@@ -780,23 +811,16 @@ def run_gpu(args):
         if mode != synth.CHANNEL_TOKEN:
             continue
         sc = fq.calibrate_static_scale(X[k][: min(M, 256)])
-        xq_s, xs_s = torch.empty_like(XQ[k][0]), torch.empty_like(XQ[k][1])
-        fn = (lambda k=k, sc=sc, xq_s=xq_s, xs_s=xs_s: fq.fp8_quant_act_static(X[k], sc, out=(xq_s, xs_s)))
-        fn()
-        torch.cuda.synchronize()
-        gr = capture([fn]) if not args.eager else None
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        torch.cuda._sleep(2_000_000)
-        for s_ in range(args.steps):
-            flush.zero_()
-            ev[s_][0].record(stream)
-            gr.replay() if gr is not None else fn()
-            ev[s_][1].record(stream)
-        torch.cuda.synchronize()
-        t = float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+        def make(i, k=k, sc=sc):
+            x = X[k] if i == 0 else X[k].clone()
+            o = (torch.empty_like(XQ[k][0]), torch.empty_like(XQ[k][1]))
+            return lambda: fq.fp8_quant_act_static(x, sc, out=o)
+
         qb = 3 * M * K + 4 * M
-        qstatic.append({"act": k, "M": M, "K": K, "ms": round(t, 5), "GB/s": round(qb / (t / 1e3) / 1e9, 1),
-                        "frac_hbm": round(qb / (t / 1e3) / 1e9 / pk["hbm_gbs"], 3)})
+        e = entry(*time_op(make, qb), nbytes=qb)
+        e.update({"act": k, "M": M, "K": K})
+        qstatic.append(e)
     assert fq.device_error(clear=True) == 0
 
     # ---- FP8 KV cache: the k_proj / v_proj outputs quantized per (token, head)
@@ -804,60 +828,49 @@ def run_gpu(args):
     for g in ([] if args.no_extras else wl.gemms):
         if g.name not in ("k_proj", "v_proj") or g.N % 128:
             continue
-        kv = Y[g.name].view(g.M, g.N // 128, 128)
-        kq = torch.empty(kv.shape, dtype=torch.uint8, device=dev)
-        ks = torch.empty((g.M, g.N // 128), dtype=torch.float32, device=dev)
-        fn = (lambda kv=kv, kq=kq, ks=ks: fq.fp8_quant_kv(kv, out=(kq, ks)))
-        fn()
-        torch.cuda.synchronize()
-        gr = capture([fn]) if not args.eager else None
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        torch.cuda._sleep(2_000_000)
-        for s_ in range(args.steps):
-            flush.zero_()
-            ev[s_][0].record(stream)
-            gr.replay() if gr is not None else fn()
-            ev[s_][1].record(stream)
-        torch.cuda.synchronize()
-        t = float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+        def make(i, g=g):
+            kv = (Y[g.name] if i == 0 else Y[g.name].clone()).view(g.M, g.N // 128, 128)
+            o = (torch.empty(kv.shape, dtype=torch.uint8, device=dev),
+                 torch.empty((g.M, g.N // 128), dtype=torch.float32, device=dev))
+            return lambda: fq.fp8_quant_kv(kv, out=o)
+
         kb = 3 * g.M * g.N + 4 * g.M * (g.N // 128)
-        kvq.append({"kv": g.name, "tokens": g.M, "heads": g.N // 128, "ms": round(t, 5),
-                    "GB/s": round(kb / (t / 1e3) / 1e9, 1), "frac_hbm": round(kb / (t / 1e3) / 1e9 / pk["hbm_gbs"], 3)})
+        e = entry(*time_op(make, kb), nbytes=kb)
+        e.update({"kv": g.name, "tokens": g.M, "heads": g.N // 128})
+        kvq.append(e)
     assert fq.device_error(clear=True) == 0
 
     # ---- weight-only FP8 (bf16 activations, codes widened in the kernel):
     # the decode GEMMs (M <= 64, channel scales), next to the W8A8 path
     # (activation quantization + FP8 linear) on the same layer
-    def time_graph(fn):
-        fn()
-        torch.cuda.synchronize()
-        gr = capture([fn]) if not args.eager else None
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        torch.cuda._sleep(2_000_000)
-        for s_ in range(args.steps):
-            flush.zero_()
-            ev[s_][0].record(stream)
-            gr.replay() if gr is not None else fn()
-            ev[s_][1].record(stream)
-        torch.cuda.synchronize()
-        return float(np.median([a.elapsed_time(b) for a, b in ev]))
-
     w8a16 = []
     for g in ([] if args.no_extras else wl.gemms):
         if g.mode != synth.CHANNEL_TOKEN or g.M > 64:
             continue
-        y16 = torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev)
-        xq_w, xs_w = torch.empty_like(XQ[g.x][0]), torch.empty_like(XQ[g.x][1])
-        wk16 = torch.zeros(max(16, fq.fp8_linear_w8a16_workspace_size(g.M, g.N, g.K)), dtype=torch.uint8, device=dev)
-        t16 = time_graph(lambda g=g, y16=y16, wk16=wk16: fq.fp8_linear_w8a16(X[g.x], WQ[g.weight][0], WQ[g.weight][1],
-                                                                           out=y16, workspace=wk16))
-        t8 = time_graph(lambda g=g, y16=y16, xq_w=xq_w, xs_w=xs_w: (
-            fq.fp8_quant_act(X[g.x], g.mode, out=(xq_w, xs_w)),
-            fq.fp8_linear(xq_w, xs_w, WQ[g.weight][0], WQ[g.weight][1], g.mode, out=y16, workspace=WS[g.name])))
+
+        def make16(i, g=g):
+            x = X[g.x] if i == 0 else X[g.x].clone()
+            wq = WQ[g.weight][0] if i == 0 else WQ[g.weight][0].clone()
+            y16 = torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev)
+            wk16 = torch.zeros(max(16, fq.fp8_linear_w8a16_workspace_size(g.M, g.N, g.K)), dtype=torch.uint8,
+                               device=dev)
+            return lambda: fq.fp8_linear_w8a16(x, wq, WQ[g.weight][1], out=y16, workspace=wk16)
+
+        def make8(i, g=g):
+            x = X[g.x] if i == 0 else X[g.x].clone()
+            wq = WQ[g.weight][0] if i == 0 else WQ[g.weight][0].clone()
+            y16 = torch.empty((g.M, g.N), dtype=torch.bfloat16, device=dev)
+            xq_w, xs_w = torch.empty_like(XQ[g.x][0]), torch.empty_like(XQ[g.x][1])
+            wk = torch.zeros_like(WS[g.name])
+            return lambda: (fq.fp8_quant_act(x, g.mode, out=(xq_w, xs_w)),
+                            fq.fp8_linear(xq_w, xs_w, wq, WQ[g.weight][1], g.mode, out=y16, workspace=wk))
+
         wb = g.N * g.K + 2 * g.M * g.K + 4 * g.N + 2 * g.M * g.N
-        w8a16.append({"gemm": g.name, "M": g.M, "N": g.N, "K": g.K, "ms": round(t16, 5),
-                      "GB/s": round(wb / (t16 / 1e3) / 1e9, 1), "frac_hbm": round(wb / (t16 / 1e3) / 1e9 / pk["hbm_gbs"], 3),
-                      "w8a8_ms": round(t8, 5), "kernel": "cuda cores" if g.M == 1 else "tcgen05 bf16 (widened tiles)"})
+        e = entry(*time_op(make16, wb), nbytes=wb)
+        e.update({"gemm": g.name, "M": g.M, "N": g.N, "K": g.K, "w8a8_ms": round(time_op(make8, wb)[0], 5),
+                  "kernel": "cuda cores" if g.M == 1 else "tcgen05 bf16 (widened tiles)"})
+        w8a16.append(e)
     assert fq.device_error(clear=True) == 0
 
     # ---- end to end through the public API with host buffers

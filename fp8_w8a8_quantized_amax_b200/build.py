@@ -11,7 +11,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp8q.so")
 SOURCES = ["fp8q.cu"]
-DEPS = ["fp8q.cu", "ptx.cuh", "quant.cuh", "gemm_prefill.cuh", "gemm_decode.cuh", "gemv_w8a16.cuh", "calib.cuh"]
+DEPS = ["fp8q.cu", "ptx.cuh", "quant.cuh", "gemm_prefill.cuh", "gemm_decode.cuh", "gemv_w8a16.cuh", "calib.cuh", "sched.cuh"]
 
 
 def nvcc() -> str:

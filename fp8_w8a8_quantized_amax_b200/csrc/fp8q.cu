@@ -387,6 +387,79 @@ fp8q_status launch_w8a16(const fp8q::wonly::Params& p, int dev, void* stream) {
   return launch(k, dim3((p.N + R - 1) / R), dim3(fp8q::wonly::kThreads), kBytes, stream, p);
 }
 
+// CTA pairs resident at once for the pair prefill kernels (block or channel
+// scales), per device; computed once (a race between host threads computes
+// the same value twice).  Also opts the kernels in to their shared memory.
+fp8q_status prefill_pairs(bool block, int dev, int sms, int* out) {
+  using L = fp8q::prefill::PairLayout<kPairStages>;
+  static std::atomic<int> max_pairs[2][kMaxDevices];
+  fp8q_status st;
+  if (block) {
+    auto k = fp8q::prefill::gemm_block2_kernel<kPairStages>;
+    if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
+  } else {
+    if ((st = ensure_smem(fp8q::prefill::gemm_channel2_kernel<kPairStages, false>, L::kBytes, dev)) != FP8Q_OK)
+      return st;
+  }
+  if (max_pairs[block][dev].load(std::memory_order_relaxed) == 0) {
+    cudaLaunchConfig_t qc = {};
+    qc.gridDim = dim3(2 * sms);
+    qc.dynamicSmemBytes = L::kBytes;
+    int n = 0;
+    cudaError_t e;
+    if (block) {
+      // The kernel moves registers between its warpgroups; that is only
+      // safe when it is launched with the register count it was built for.
+      auto k = fp8q::prefill::gemm_block2_kernel<kPairStages>;
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return FP8Q_ERR_CUDA;
+      if (fa.numRegs != fp8q::prefill::kBlock2LaunchRegs) return FP8Q_ERR_UNSUPPORTED;
+      qc.blockDim = dim3(fp8q::prefill::kBlock2Threads);
+      e = cudaOccupancyMaxActiveClusters(&n, k, &qc);
+    } else {
+      qc.blockDim = dim3(64 + 32 * L::kEpiWarps);
+      e = cudaOccupancyMaxActiveClusters(&n, fp8q::prefill::gemm_channel2_kernel<kPairStages, false>, &qc);
+    }
+    if (e != cudaSuccess || n < 1) n = sms / 2;
+    max_pairs[block][dev].store(n, std::memory_order_relaxed);
+  }
+  *out = max_pairs[block][dev].load(std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
+// Stream-K for the channel pair kernel, on request (FP8Q_PREFILL_STREAMK=1,
+// read once): shapes whose 256 x 256 tiles fill the pairs unevenly (the
+// data-parallel schedule, its last round cut into N halves where that helps,
+// keeps under 92% of the pairs busy).  Not the default: measured on the
+// B200 it is slower on every such Llama shape (70B M=512 gate/up 0.67 against
+// 0.74 of the FP8 peak, down 0.66 against 0.83, qkv 0.47 against 0.54; 8B
+// k/v at M=8192 0.51 against 0.71), because pairs working on different K
+// ranges no longer share operand tiles through L2 at the same time, and these
+// shapes are close to the HBM ridge.
+bool prefill_streamk(int num_tiles, int pairs) {
+  static bool on = [] {
+    const char* e = getenv("FP8Q_PREFILL_STREAMK");
+    return e && strcmp(e, "1") == 0;
+  }();
+  if (!on) return false;
+  int full, split;
+  fp8q::prefill::tail_split(num_tiles, pairs, &full, &split);
+  const int rest = num_tiles - full;
+  const double rounds = full / static_cast<double>(pairs) +
+                        (rest ? (split == 2 ? 0.5 * ((2 * rest + pairs - 1) / pairs) : (rest + pairs - 1) / pairs) : 0);
+  return num_tiles / (rounds * pairs) < 0.92;
+}
+
+// Stream-K workspace: [num_tiles][2][8] arrival counters (padded to 256 bytes),
+// then 2 fp32 256 x 256 partial tiles per pair.
+size_t prefill_sk_counter_bytes(int num_tiles) {
+  return (static_cast<size_t>(num_tiles) * 16 * sizeof(unsigned) + 255) & ~size_t(255);
+}
+size_t prefill_sk_bytes(int num_tiles, int pairs) {
+  return prefill_sk_counter_bytes(num_tiles) +
+         static_cast<size_t>(2 * pairs) * fp8q::prefill::kSkSlotFloats * sizeof(float);
+}
+
 }  // namespace
 
 extern "C" {
@@ -422,8 +495,9 @@ fp8q_status fp8_quant_act(const void* X_bf16, int64_t M, int64_t K, int64_t ldx,
   constexpr int GPT = 4;
   const int G = static_cast<int>(K / 128);
   const int64_t total = M * G;
+  if (total >= (static_cast<int64_t>(1) << 31)) return FP8Q_ERR_UNSUPPORTED;   // 32-bit group walk
   int64_t grid = (total + 16 * GPT - 1) / (16 * GPT);
-  if (grid > static_cast<int64_t>(sms) * 16) grid = static_cast<int64_t>(sms) * 16;
+  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
   return launch(fp8q::quant_groups128_kernel<GPT>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream, x, M,
                 G, ldx, Xq, ldxq, x_scale, s16);
 }
@@ -455,8 +529,9 @@ fp8q_status fp8_quant_act_static(const void* X_bf16, int64_t M, int64_t K, int64
   int dev, sms;
   if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
   const int64_t vecs = M * (K / 8);
-  int64_t grid = (vecs + 255) / 256;
-  if (grid > static_cast<int64_t>(sms) * 16) grid = static_cast<int64_t>(sms) * 16;
+  if (vecs >= (static_cast<int64_t>(1) << 31)) return FP8Q_ERR_UNSUPPORTED;   // 32-bit positions
+  int64_t grid = (vecs + 1023) / 1024;
+  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
   return launch(fp8q::quant_static_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream,
                 static_cast<const uint16_t*>(X_bf16), M, static_cast<int>(K), ldx, scale, Xq, ldxq, x_scale);
 }
@@ -483,9 +558,19 @@ fp8q_status fp8_calibrate_static_scale(const void* X_bf16, int64_t M, int64_t K,
 size_t fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int mode) {
   if (!valid_mode(mode)) return 0;
   mode &= ~FP8Q_SCALE_BF16;
-  if (M <= 0 || M > kDecodeMaxM || N <= 0 || K <= 0) return 0;
+  if (M <= 0 || N <= 0 || K <= 0 || M > kInt32Max || N > kInt32Max || K > kInt32Max) return 0;
   int dev, sms;
   if (current_device(&dev, &sms) != FP8Q_OK) return 0;
+  if (M > kDecodeMaxM) {            // prefill: the stream-K schedule's scratch, where it pays
+    const bool pair = prefill_choice() != 1 && (M >= 256 || prefill_choice() == 2);
+    if (!pair || mode == FP8Q_BLOCK128) return 0;
+    int pairs = 0;
+    if (prefill_pairs(false, dev, sms, &pairs) != FP8Q_OK) return 0;
+    const int num_tiles = static_cast<int>(((M + 255) / 256) * ((N + 255) / 256));
+    const int64_t steps = static_cast<int64_t>(num_tiles) * ((K + 127) / 128);
+    if (steps > kInt32Max || !prefill_streamk(num_tiles, pairs)) return 0;
+    return prefill_sk_bytes(num_tiles, pairs);
+  }
   int n_tiles, G, nx;
   int64_t total;
   decode_shape(M, N, K, sms, &n_tiles, &total, &G, &nx);
@@ -536,29 +621,9 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
   if (pair) {
     using L = fp8q::prefill::PairLayout<kPairStages>;
     const bool block = mode == FP8Q_BLOCK128;
-    auto k = block ? fp8q::prefill::gemm_block2_kernel<kPairStages> : fp8q::prefill::gemm_channel2_kernel<kPairStages>;
     static_assert(fp8q::prefill::PairLayout<kPairStages, 4>::kBytes == L::kBytes, "one shared-memory size");
-    const int threads = block ? fp8q::prefill::kBlock2Threads : 64 + 32 * L::kEpiWarps;
-    if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
-    // CTA pairs resident at once, per (kernel, device); computed once (a race
-    // between threads computes the same value twice).
-    static std::atomic<int> max_pairs[2][kMaxDevices];
-    if (max_pairs[block][dev].load(std::memory_order_relaxed) == 0) {
-      if (block) {
-        // The kernel moves registers between its warpgroups; that is only
-        // safe when it is launched with the register count it was built for.
-        cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return FP8Q_ERR_CUDA;
-        if (fa.numRegs != fp8q::prefill::kBlock2LaunchRegs) return FP8Q_ERR_UNSUPPORTED;
-      }
-      cudaLaunchConfig_t qc = {};
-      qc.gridDim = dim3(2 * sms);
-      qc.blockDim = dim3(threads);
-      qc.dynamicSmemBytes = L::kBytes;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, k, &qc) != cudaSuccess || n < 1) n = sms / 2;
-      max_pairs[block][dev].store(n, std::memory_order_relaxed);
-    }
+    int pairs = 0;
+    if ((st = prefill_pairs(block, dev, sms, &pairs)) != FP8Q_OK) return st;
     fp8q::prefill::Params p;
     p.xs = x_scale;
     p.ws = w_scale;
@@ -572,16 +637,34 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     p.num_n = static_cast<int>((N + 255) / 256);
     p.num_tiles = p.num_m * p.num_n;
     p.group_m = p.num_m < 8 ? p.num_m : 8;
-    const int pairs = max_pairs[block][dev].load(std::memory_order_relaxed);
-    fp8q::prefill::tail_split(p.num_tiles, pairs, &p.full, &p.split);
-    const int items = (p.full ? p.full : 0) + (p.num_tiles - p.full) * p.split;
-    const int used = p.full ? pairs : (items < pairs ? items : pairs);
     CUtensorMap ta, tb, tb64, ty;
     if ((st = tmap_u8_sw128(&ta, Xq, M, K, K, 128)) != FP8Q_OK) return st;
     if ((st = tmap_u8_sw128(&tb, Wq, N, K, K, 128)) != FP8Q_OK) return st;
     if ((st = tmap_u8_sw128(&tb64, Wq, N, K, K, 64)) != FP8Q_OK) return st;
     if ((st = tmap_bf16_sw64(&ty, Y_bf16, M, N, ldy, 32)) != FP8Q_OK) return st;
-    return launch(k, dim3(2 * used), dim3(threads), L::kBytes, stream, ta, tb, tb64, ty, p);
+    const int64_t steps = static_cast<int64_t>(p.num_tiles) * KB;
+    if (!block && steps <= kInt32Max && prefill_streamk(p.num_tiles, pairs) && workspace &&
+        workspace_bytes >= prefill_sk_bytes(p.num_tiles, pairs) && aligned(workspace, 16)) {
+      auto k = fp8q::prefill::gemm_channel2_kernel<kPairStages, true>;
+      if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
+      fp8q::prefill::SkParams sk;
+      sk.count = static_cast<unsigned int*>(workspace);
+      sk.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + prefill_sk_counter_bytes(p.num_tiles));
+      p.full = 0;
+      p.split = 1;
+      const int used = steps < pairs ? static_cast<int>(steps) : pairs;
+      return launch(k, dim3(2 * used), dim3(64 + 32 * L::kEpiWarps), L::kBytes, stream, ta, tb, tb64, ty, p, sk);
+    }
+    fp8q::prefill::tail_split(p.num_tiles, pairs, &p.full, &p.split);
+    const int items = (p.full ? p.full : 0) + (p.num_tiles - p.full) * p.split;
+    const int used = p.full ? pairs : (items < pairs ? items : pairs);
+    if (block) {
+      auto k = fp8q::prefill::gemm_block2_kernel<kPairStages>;
+      return launch(k, dim3(2 * used), dim3(fp8q::prefill::kBlock2Threads), L::kBytes, stream, ta, tb, tb64, ty, p);
+    }
+    auto k = fp8q::prefill::gemm_channel2_kernel<kPairStages, false>;
+    return launch(k, dim3(2 * used), dim3(64 + 32 * L::kEpiWarps), L::kBytes, stream, ta, tb, tb64, ty, p,
+                  fp8q::prefill::SkParams{nullptr, nullptr});
   }
 
   fp8q::prefill::Params p;

@@ -23,6 +23,7 @@
 #include <type_traits>
 
 #include "ptx.cuh"
+#include "sched.cuh"
 
 namespace fp8q {
 namespace prefill {
@@ -326,11 +327,30 @@ struct PairLayout {
   static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
-template <int STAGES>
+// Stream-K schedule (SK = true), for problems whose 256 x 256 tiles fill the
+// pairs unevenly (a few tiles more than a whole number of rounds): the
+// (tile, K block) steps are cut into equal contiguous ranges, one per pair
+// (sched.cuh), as the decode kernel does.  A tile cut between pairs is
+// accumulated by each in its own segment; every epilogue warp stores its
+// 32 x 128 fp32 share of a partial segment to a workspace slot, counts itself
+// in on a per-(tile, CTA, warp) counter, and the warp that arrives last adds
+// the tile's slots in pair order (deterministic), applies the scales and
+// writes bf16 through the usual staging path, and sets the counter back to 0.
+// A pair's partial segments can only lie in the first or the last tile of its
+// range: slot 2c holds pair c's share of its first tile, slot 2c + 1 of its
+// last.  Nothing waits on another pair.
+struct SkParams {
+  unsigned int* count;  // [num_tiles][2 CTAs][8 warps] arrival counters, left zero
+  float* part;          // [2 * pairs][2 CTAs][8 warps][128 columns][32 rows] fp32 partial tiles
+};
+
+constexpr int kSkSlotFloats = 256 * 256;
+
+template <int STAGES, bool SK = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     gemm_channel2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmB64, const __grid_constant__ CUtensorMap tmY,
-                         const Params p) {
+                         const Params p, const SkParams sk) {
   using L = PairLayout<STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -381,7 +401,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
   auto coords = [&](int i, int& mb, int& nb, int& n_off, int& n_cols) {
     work_item(p, pair, G2, i, 256, mb, nb, n_off, n_cols);
   };
-  const int nitems = work_items(p, pair, G2);
+  const int nitems = SK ? 0 : work_items(p, pair, G2);
+  // Stream-K: this pair's steps [ub, ue) of the num_tiles * KB list.
+  const sched::Split sp = sched::split_of(SK ? p.num_tiles * p.KB : G2, G2);
+  const int ub = SK ? sched::range_begin(pair, sp) : 0;
+  const int ue = SK ? sched::range_begin(pair + 1, sp) : 0;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -389,19 +413,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int i = 0; ok && i < nitems; ++i) {
-        int mb, nb, n_off, n_cols;
-        coords(i, mb, nb, n_off, n_cols);
-        const int half = n_cols / 2;                            // B rows held by each CTA
+      auto load = [&](int mb, int nb, int n_off, int half, int kb) -> bool {
         const CUtensorMap* tb = half == 128 ? &tmB : &tmB64;
-        for (int kb = 0; kb < p.KB; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) { ok = false; break; }
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * static_cast<uint32_t>(L::kA + half * BK));
-          const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
-          tma_load_2d_pair(sA + stage * L::kA, &tmA, bar0, kb * BK, mb * 256 + static_cast<int>(rank) * 128, pol);
-          tma_load_2d_pair(sB + stage * L::kB, tb, bar0, kb * BK, nb * 256 + n_off + static_cast<int>(rank) * half,
-                           pol);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kErrWaitEmpty)) return false;
+        if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * static_cast<uint32_t>(L::kA + half * BK));
+        const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
+        tma_load_2d_pair(sA + stage * L::kA, &tmA, bar0, kb * BK, mb * 256 + static_cast<int>(rank) * 128, pol);
+        tma_load_2d_pair(sB + stage * L::kB, tb, bar0, kb * BK, nb * 256 + n_off + static_cast<int>(rank) * half,
+                         pol);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        return true;
+      };
+      if constexpr (SK) {
+        for (sched::StepIter it(ub, ue, p.KB); ok && it.valid(); it.next()) {
+          int mb, nb;
+          tile_coords(p, it.t, mb, nb);
+          ok = load(mb, nb, 0, 128, it.kb);
+        }
+      } else {
+        for (int i = 0; ok && i < nitems; ++i) {
+          int mb, nb, n_off, n_cols;
+          coords(i, mb, nb, n_off, n_cols);
+          for (int kb = 0; ok && kb < p.KB; ++kb) ok = load(mb, nb, n_off, n_cols / 2, kb);
         }
       }
       griddep_launch_dependents();
@@ -415,28 +448,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int it = 0; ok && it < nitems; ++it) {
-        int mb, nb, n_off, n_cols;
-        coords(it, mb, nb, n_off, n_cols);
-        const uint32_t idesc = idesc_e4m3_f32(256, n_cols);
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
-        if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag, kErrWaitTmemEmpty)) break;
+      // one K block into accumulator d (accumulate unless it is the first of the segment)
+      auto mma_step = [&](uint32_t d, uint32_t idesc, bool first) -> bool {
+        if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) return false;
         tc_fence_after();
-        const uint32_t d = tmem_base + acc * 256;
-        for (int kb = 0; kb < p.KB; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, kErrWaitFull)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * L::kA);
-          const uint32_t b0 = smem_u32(sB + stage * L::kB);
+        const uint32_t a0 = smem_u32(sA + stage * L::kA);
+        const uint32_t b0 = smem_u32(sB + stage * L::kB);
 #pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k)
-            mma_e4m3_pair(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + k * UMMA_K), idesc,
-                          (kb | k) != 0);
-          mma_commit_pair(&empty[stage], kBoth);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        for (int k = 0; k < BK / UMMA_K; ++k)
+          mma_e4m3_pair(d, umma_desc_sw128(a0 + k * UMMA_K), umma_desc_sw128(b0 + k * UMMA_K), idesc,
+                        (!first || k != 0) ? 1u : 0u);
+        mma_commit_pair(&empty[stage], kBoth);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        return true;
+      };
+      if constexpr (SK) {
+        constexpr uint32_t idesc = idesc_e4m3_f32(256, 256);
+        int seg = 0;
+        for (sched::StepIter it(ub, ue, p.KB); it.valid(); it.next()) {
+          const int acc = seg & 1;
+          if (it.seg_first()) {
+            if (!mbar_wait_cluster(&tempty[acc], ((seg >> 1) & 1) ^ 1u, abort_flag, kErrWaitTmemEmpty)) break;
+            tc_fence_after();
+          }
+          if (!mma_step(tmem_base + acc * 256, idesc, it.seg_first())) break;
+          if (it.seg_last()) {
+            mma_commit_pair(&tfull[acc], kBoth);
+            ++seg;
+          }
         }
-        if (ok) mma_commit_pair(&tfull[acc], kBoth);
+      } else {
+        for (int it = 0; ok && it < nitems; ++it) {
+          int mb, nb, n_off, n_cols;
+          coords(it, mb, nb, n_off, n_cols);
+          const uint32_t idesc = idesc_e4m3_f32(256, n_cols);
+          const int acc = it & 1;
+          const uint32_t acc_phase = (it >> 1) & 1;
+          if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag, kErrWaitTmemEmpty)) break;
+          tc_fence_after();
+          const uint32_t d = tmem_base + acc * 256;
+          for (int kb = 0; ok && kb < p.KB; ++kb) ok = mma_step(d, idesc, kb == 0);
+          if (ok) mma_commit_pair(&tfull[acc], kBoth);
+        }
       }
     }
   } else {
@@ -453,51 +506,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     const int swz = (lane >> 1) & 3;
     const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
     int buf = 0;
-    for (int it = 0; it < nitems; ++it) {
-      int mb, nb, n_off, n_cols;
-      coords(it, mb, nb, n_off, n_cols);
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
+    // One output segment: tile (mb, nb), columns [n_off, n_off + n_cols), in
+    // accumulator `acc`.  This warp takes rows row0.. of its lane quarter and
+    // half of the columns.
+    float xsm = 0.0f, wv[4];
+    int row0 = 0, col_base = 0;
+    auto setup = [&](int mb, int nb, int n_off, int n_cols) {
       const int my_cols = n_cols / 2;                           // 128 or 64
-      const int nchunks = my_cols / 32;                         // 4 or 2
       const int c_begin = half * my_cols;
-      const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quarter * 32;
+      row0 = mb * 256 + static_cast<int>(rank) * 128 + quarter * 32;
       const int m = row0 + lane;
-      const float xsm = m < p.M ? __ldg(p.xs + m) : 0.0f;
-      float wv[4];
+      xsm = m < p.M ? __ldg(p.xs + m) : 0.0f;
+      col_base = nb * 256 + n_off + c_begin;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int n = nb * 256 + n_off + c_begin + i * 32 + lane;
-        wv[i] = (i < nchunks && n < p.N) ? __ldg(p.ws + n) : 0.0f;
+        const int n = col_base + i * 32 + lane;
+        wv[i] = (i < my_cols / 32 && n < p.N) ? __ldg(p.ws + n) : 0.0f;
       }
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrWaitTmemFull))) break;
-      tc_fence_after();
-      const uint32_t tcol = tmem_base + lane_addr + acc * 256 + c_begin;
-      // Scale, stage and store one 32-column chunk held in registers.
-      auto emit = [&](const uint32_t (&cur)[32], float w_lane, int c) {
-        uint32_t pk[16];
+      return c_begin;
+    };
+    // Scale, stage and store one 32-column chunk held in registers.
+    auto emit = [&](const uint32_t (&cur)[32], float w_lane, int c) {
+      uint32_t pk[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float w0 = __shfl_sync(0xFFFFFFFFu, w_lane, 2 * j);
-          const float w1 = __shfl_sync(0xFFFFFFFFu, w_lane, 2 * j + 1);
-          pk[j] = pack_bf16x2(__uint_as_float(cur[2 * j]) * xsm * w0, __uint_as_float(cur[2 * j + 1]) * xsm * w1);
-        }
-        if (lane == 0) bulk_wait_read<1>();   // the tile written two chunks ago has been read
-        __syncwarp();
-        uint8_t* sb = out_s + buf * L::kOutChunk;
+      for (int j = 0; j < 16; ++j) {
+        const float w0 = __shfl_sync(0xFFFFFFFFu, w_lane, 2 * j);
+        const float w1 = __shfl_sync(0xFFFFFFFFu, w_lane, 2 * j + 1);
+        pk[j] = pack_bf16x2(__uint_as_float(cur[2 * j]) * xsm * w0, __uint_as_float(cur[2 * j + 1]) * xsm * w1);
+      }
+      if (lane == 0) bulk_wait_read<1>();   // the tile written two chunks ago has been read
+      __syncwarp();
+      uint8_t* sb = out_s + buf * L::kOutChunk;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          *reinterpret_cast<uint4*>(sb + lane * 64 + ((q ^ swz) << 4)) =
-              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        const int col0 = nb * 256 + n_off + c_begin + c;
-        if (lane == 0 && row0 < p.M && col0 < p.N) {
-          tma_store_2d(&tmY, sb, col0, row0);
-          bulk_commit();
-        }
-        buf ^= 1;
-      };
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(sb + lane * 64 + ((q ^ swz) << 4)) =
+            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int col0 = col_base + c;
+      if (lane == 0 && row0 < p.M && col0 < p.N) {
+        tma_store_2d(&tmY, sb, col0, row0);
+        bulk_commit();
+      }
+      buf ^= 1;
+    };
+    // The whole segment from TMEM: the load of the next chunk is issued before
+    // the current one is scaled, staged and stored, so its latency overlaps
+    // that work; the accumulator is released once all chunks are in registers.
+    auto emit_from_tmem = [&](uint32_t tcol, int nchunks, int acc) {
       uint32_t ra[32], rb[32];
       __syncwarp();
       tmem_ld_32x32b_x32(tcol, ra);
@@ -519,6 +575,85 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
           }
           emit(rb, wv[ci + 1], (ci + 1) * 32);
         }
+      }
+    };
+    if constexpr (SK) {
+      int seg = 0, seg_len = 0;
+      for (sched::StepIter st(ub, ue, p.KB); st.valid(); st.next()) {
+        seg_len = st.seg_first() ? 1 : seg_len + 1;
+        if (!st.seg_last()) continue;
+        const int t = st.t;
+        int mb, nb;
+        tile_coords(p, t, mb, nb);
+        const int acc = seg & 1;
+        const uint32_t acc_phase = (seg >> 1) & 1;
+        ++seg;
+        const int c_begin = setup(mb, nb, 0, 256);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrWaitTmemFull))) break;
+        tc_fence_after();
+        const uint32_t tcol = tmem_base + lane_addr + acc * 256 + c_begin;
+        if (seg_len == p.KB) {          // the whole tile in this pair
+          emit_from_tmem(tcol, 4, acc);
+          continue;
+        }
+        // A part of the tile: this warp's 32 x 128 fp32 share to the pair's
+        // slot (column-major in 32-row strips: each store is 128 contiguous
+        // bytes), then count in.
+        auto share = [&](int c) -> int64_t {
+          const int slot = (sched::range_begin(c, sp) / p.KB == t) ? 2 * c : 2 * c + 1;
+          return (static_cast<int64_t>(slot) * 16 + static_cast<int>(rank) * 8 + ew) * (128 * 32) + lane;
+        };
+        float* dst = sk.part + share(pair);
+        uint32_t ra[32];
+#pragma unroll 1
+        for (int ci = 0; ci < 4; ++ci) {
+          __syncwarp();
+          tmem_ld_32x32b_x32(tcol + ci * 32, ra);
+          tmem_ld_wait_regs(ra);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) dst[(ci * 32 + j) * 32] = __uint_as_float(ra[j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + acc * 8);
+        __threadfence();
+        __syncwarp();
+        const int c0 = sched::cta_of_step(t * p.KB, sp);
+        const int c1 = sched::cta_of_step(t * p.KB + p.KB - 1, sp);
+        unsigned int* cnt = sk.count + (static_cast<int64_t>(t) * 2 + rank) * 8 + ew;
+        unsigned int prev = 0;
+        if (lane == 0) prev = atomicAdd(cnt, 1u);
+        prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+        if (prev != static_cast<unsigned int>(c1 - c0)) continue;
+        // Every other part is in: sum the shares in pair order, then scale and store.
+        __threadfence();
+#pragma unroll 1
+        for (int ci = 0; ci < 4; ++ci) {
+          float sum[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sum[j] = 0.0f;
+          for (int cc = c0; cc <= c1; ++cc) {
+            const float* src = sk.part + share(cc) + ci * 32 * 32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sum[j] += __ldcg(src + j * 32);
+          }
+          uint32_t bits[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) bits[j] = __float_as_uint(sum[j]);
+          emit(bits, wv[ci], ci * 32);
+        }
+        if (lane == 0) *cnt = 0u;
+      }
+    } else {
+      for (int it = 0; it < nitems; ++it) {
+        int mb, nb, n_off, n_cols;
+        coords(it, mb, nb, n_off, n_cols);
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        const int c_begin = setup(mb, nb, n_off, n_cols);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrWaitTmemFull))) break;
+        tc_fence_after();
+        emit_from_tmem(tmem_base + lane_addr + acc * 256 + c_begin, n_cols / 64, acc);
       }
     }
     if (lane == 0) bulk_wait<0>();

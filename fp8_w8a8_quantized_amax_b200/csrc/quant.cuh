@@ -220,8 +220,10 @@ __global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t*
   const int T = blockDim.x;
   const int warp = threadIdx.x >> 5, nw = T >> 5;
   const uint16_t* xr = x + r * ldx;
-  // gamma is loaded with the row (not after the reduction) when it fits in registers
-  constexpr bool kGammaAhead = VPT <= 8;
+  // gamma is read after the reductions (it is L1/L2-resident: every row reads
+  // the same K values); holding it in registers from the start would cost a
+  // third of the registers and so a third of the rows in flight per SM
+  constexpr bool kGammaAhead = false;
   uint4 v[VPT], gv[kGammaAhead ? VPT : 1];
   double ss0 = 0.0, ss1 = 0.0;
 #pragma unroll
@@ -295,59 +297,95 @@ __global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t*
 __global__ void __launch_bounds__(256) quant_static_kernel(const uint16_t* __restrict__ x, int64_t M, int K,
                                                           int64_t ldx, float sc, uint8_t* __restrict__ q,
                                                           int64_t ldq, float* __restrict__ s) {
+  // 4 vectors per thread per round, all loads issued before any store, so
+  // that 64 bytes per thread are in flight; vector u of a round is u * stride
+  // further on (coalesced across the grid).  (row, vector) positions advance
+  // incrementally in 32-bit arithmetic (the host keeps M * K / 8 below 2^31).
+  constexpr int kVec = 4;
   griddep_wait();
-  const int nvec = K >> 3;
-  const int64_t total = M * nvec;
+  const uint32_t nvec = static_cast<uint32_t>(K) >> 3;
+  const uint32_t Mu = static_cast<uint32_t>(M);
+  const uint32_t stride = gridDim.x * blockDim.x;
+  const uint32_t st_m = stride / nvec, st_r = stride - st_m * nvec;
+  const uint32_t i0 = blockIdx.x * blockDim.x + threadIdx.x;
+  uint32_t m = i0 / nvec, r = i0 - m * nvec;
+  auto advance = [&](uint32_t& mm, uint32_t& rr) {
+    mm += st_m;
+    rr += st_r;
+    if (rr >= nvec) { rr -= nvec; ++mm; }
+  };
   const Divider dv = make_divider(sc);
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
-    const int64_t m = i / nvec;
-    const int vi = static_cast<int>(i - m * nvec);
-    const uint4 v = ld_stream16(x + m * ldx + vi * 8);
-    *reinterpret_cast<uint2*>(q + m * ldq + vi * 8) = dv.fast ? encode_vec<true>(v, dv) : encode_vec<false>(v, dv);
-    if (s != nullptr && vi == 0) s[m] = sc;
+  while (m < Mu) {
+    uint4 v[kVec];
+    uint32_t mi[kVec], ri[kVec];
+#pragma unroll
+    for (int u = 0; u < kVec; ++u) {
+      mi[u] = m;
+      ri[u] = r;
+      if (m < Mu) v[u] = ld_stream16(x + static_cast<int64_t>(m) * ldx + r * 8);
+      advance(m, r);
+    }
+#pragma unroll
+    for (int u = 0; u < kVec; ++u) {
+      if (mi[u] < Mu) {
+        *reinterpret_cast<uint2*>(q + static_cast<int64_t>(mi[u]) * ldq + ri[u] * 8) =
+            dv.fast ? encode_vec<true>(v[u], dv) : encode_vec<false>(v[u], dv);
+        if (s != nullptr && ri[u] == 0) s[mi[u]] = sc;
+      }
+    }
   }
 }
 
 // ----------------------------------------------------------- groups 128 ---
 // Groups of 128 features: 16 consecutive lanes (a half warp) own one group,
-// one 16-byte vector each.  Each half warp walks GPT groups, strided by the
-// number of half warps in the grid, with all loads issued before any reduce.
+// one 16-byte vector each.  Half warp h takes the groups h, h + H, h + 2H, ...
+// of the row-major (token, group) list (H half warps in the grid), GPT of them
+// in flight with all loads issued before any reduction.  The (token, group)
+// position of each is advanced incrementally in 32-bit arithmetic: one
+// division per half warp at the start, none in the loop.
 template <int GPT>
 __global__ void __launch_bounds__(256) quant_groups128_kernel(const uint16_t* __restrict__ x, int64_t M, int G,
                                                              int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
                                                              float* __restrict__ s, bool s16) {
   griddep_wait();
-  const int64_t total = M * static_cast<int64_t>(G);
   const int sub = threadIdx.x & 15;
   const uint32_t half_mask = 0xFFFFu << (threadIdx.x & 16);
-  const int64_t nhalf = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 4);
-  const int64_t h = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
-  for (int64_t base = h; base < total; base += nhalf * GPT) {
+  const uint32_t H = (gridDim.x * blockDim.x) >> 4;
+  const uint32_t h = (blockIdx.x * blockDim.x + threadIdx.x) >> 4;
+  const uint32_t Mu = static_cast<uint32_t>(M), Gu = static_cast<uint32_t>(G);
+  const uint32_t step_m = H / Gu, step_g = H - step_m * Gu;   // (token, group) advance of H groups
+  uint32_t m = h / Gu, g = h - m * Gu;                          // the half warp's next group
+  auto advance = [&](uint32_t& mm, uint32_t& gg) {
+    mm += step_m;
+    gg += step_g;
+    if (gg >= Gu) { gg -= Gu; ++mm; }
+  };
+  while (m < Mu) {
     uint4 v[GPT];
+    uint32_t mi[GPT], gi[GPT];
+    uint32_t mm = m, gg = g;
 #pragma unroll
     for (int i = 0; i < GPT; ++i) {
-      const int64_t gi = base + i * nhalf;
-      if (gi < total) {
-        const int64_t m = gi / G, g = gi - m * G;
-        v[i] = ld_stream16(x + m * ldx + g * 128 + sub * 8);
-      }
+      mi[i] = mm;
+      gi[i] = gg;
+      if (mm < Mu) v[i] = ld_stream16(x + static_cast<int64_t>(mm) * ldx + gg * 128 + sub * 8);
+      advance(mm, gg);
     }
+    m = mm;
+    g = gg;
 #pragma unroll
     for (int i = 0; i < GPT; ++i) {
-      const int64_t gi = base + i * nhalf;
-      if (gi < total) {  // uniform across the half warp
-        uint32_t mm = fold_halves(absmax_bits_vec(v[i], 0u));
-        mm = max(mm, __shfl_xor_sync(half_mask, mm, 8, 16));
-        mm = max(mm, __shfl_xor_sync(half_mask, mm, 4, 16));
-        mm = max(mm, __shfl_xor_sync(half_mask, mm, 2, 16));
-        mm = max(mm, __shfl_xor_sync(half_mask, mm, 1, 16));
-        float sc = scale_of(amax_bits_to_float(mm));
+      if (mi[i] < Mu) {  // uniform across the half warp
+        uint32_t am = fold_halves(absmax_bits_vec(v[i], 0u));
+        am = max(am, __shfl_xor_sync(half_mask, am, 8, 16));
+        am = max(am, __shfl_xor_sync(half_mask, am, 4, 16));
+        am = max(am, __shfl_xor_sync(half_mask, am, 2, 16));
+        am = max(am, __shfl_xor_sync(half_mask, am, 1, 16));
+        float sc = scale_of(amax_bits_to_float(am));
         if (s16) sc = scale_bf16(sc);
-        const int64_t m = gi / G, g = gi - m * G;
-        if (sub == 0) s[gi] = sc;
+        if (sub == 0) s[static_cast<int64_t>(mi[i]) * Gu + gi[i]] = sc;
         const Divider dv = make_divider(sc);
-        *reinterpret_cast<uint2*>(q + m * ldq + g * 128 + sub * 8) =
+        *reinterpret_cast<uint2*>(q + static_cast<int64_t>(mi[i]) * ldq + gi[i] * 128 + sub * 8) =
             dv.fast ? encode_vec<true>(v[i], dv) : encode_vec<false>(v[i], dv);
       }
     }

@@ -177,9 +177,14 @@ FP8Q_API fp8q_status fp8_rmsnorm_quant_act(const void* X_bf16, const void* gamma
  *   w_scale   [N] or [ceil(N/128), K/128] fp32 (as written by fp8_quant_weight).
  *   Y_bf16    [M, ldy] bf16, written.  ldy >= N, (ldy * 2) % 16 == 0, 16-byte aligned.
  *   workspace device scratch of at least fp8_linear_workspace_size(M, N, K, mode)
- *             bytes, 16-byte aligned (may be NULL when that size is 0; M > 64
- *             needs none).  A NULL or misaligned workspace for M <= 64 is
- *             refused before anything touches the device.  It holds
+ *             bytes, 16-byte aligned (may be NULL when that size is 0).  For
+ *             M <= 64 it is required: a NULL or misaligned one is refused
+ *             before anything touches the device.  For M > 64 it is optional:
+ *             a nonzero size means the stream-K prefill schedule pays for this
+ *             shape (channel mode, few 256 x 256 tiles per CTA pair) and runs
+ *             when the workspace is given; without it (NULL, or shorter) the
+ *             data-parallel schedule runs, with the same result up to the
+ *             order of the fp32 sums.  It holds
  *             the split-K arrival counters and fp32 partial sums of the small-M
  *             (decode) path.  It must be zero-filled before its first use; every
  *             completed call leaves it all zero again, so one zeroed buffer
@@ -194,7 +199,8 @@ FP8Q_API fp8q_status fp8_rmsnorm_quant_act(const void* X_bf16, const void* gamma
  *   stream-K split over all SMs; the last warp to finish a weight tile's
  *   channels adds its partial sums in a fixed order, so results are
  *   deterministic); larger M takes the persistent warp-specialised prefill
- *   kernels (no workspace).
+ *   kernels, with 256 x 256 tiles per CTA pair, data-parallel or stream-K
+ *   (parts of a tile summed in a fixed order by the last pair to finish it).
  */
 FP8Q_API fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq,
                        const float* w_scale, int64_t M, int64_t N, int64_t K, int mode,

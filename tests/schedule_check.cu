@@ -25,7 +25,7 @@
 #include "../fp8_w8a8_quantized_amax_b200/csrc/gemm_decode.cuh"
 #include "../fp8_w8a8_quantized_amax_b200/csrc/gemm_prefill.cuh"
 
-using namespace fp8q::decode;
+using namespace fp8q::sched;
 
 static int fail(const char* what, int n_tiles, int KB, int G) {
   std::printf("FAIL %s (n_tiles=%d KB=%d G=%d)\n", what, n_tiles, KB, G);

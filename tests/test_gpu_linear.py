@@ -87,6 +87,45 @@ def test_prefill_kernel_forced(kernel, M, N, K, mode):
 
 
 @pytest.mark.parametrize("M,N,K", [
+    (512, 10240, 1024),    # 80 tiles on the pairs: the default schedule is stream-K
+    (8192, 1024, 512),     # 128 tiles (the Llama-3.1-8B k/v_proj shape, shorter K)
+    (300, 2560, 640),      # tiles cut at K blocks that are not tile boundaries, a ragged second row-tile
+    (1000, 1040, 400),     # ragged M, N and K
+])
+def test_prefill_streamk(M, N, K):
+    # the stream-K pair schedule (parts of tiles summed by the last pair to
+    # finish), forced on, against the oracle; repeated with the same workspace:
+    # its counters are left zero
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, FP8Q_PREFILL_STREAMK="1", FP8Q_PREFILL_KERNEL="pair")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-m", "tests._forced_kernel", "streamk", str(M), str(N), str(K)],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
+def test_prefill_needs_no_workspace_by_default():
+    # stream-K is opt-in (FP8Q_PREFILL_STREAMK=1): by default no prefill shape asks for scratch
+    for M, N, K in ((512, 10240, 8192), (8192, 1024, 4096), (8192, 4096, 4096)):
+        assert fq.fp8_linear_workspace_size(M, N, K, fq.CHANNEL_TOKEN) == 0
+        assert fq.fp8_linear_workspace_size(M, N, K, fq.BLOCK128) == 0
+
+
+def test_streamk_falls_back_without_a_workspace():
+    # forced on, but no workspace (or a short one): the data-parallel schedule runs
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, FP8Q_PREFILL_STREAMK="1")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-m", "tests._forced_kernel", "streamk_fallback"],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
+@pytest.mark.parametrize("M,N,K", [
     (200, 384, 384),
     (130, 144, 256),       # a partial 128-row weight block
     (256, 256, 128),       # CTA-pair kernel (M >= 256): one tile, one K block
@@ -98,6 +137,8 @@ def test_prefill_kernel_forced(kernel, M, N, K, mode):
 ])
 def test_prefill_block(M, N, K):
     check_full(M, N, K, fq.BLOCK128, seed=N)
+
+
 
 
 @pytest.mark.parametrize("mode", [0, 1])

@@ -32,23 +32,30 @@ MUTANTS = {
     "K-block wrap": (r"\} else if \(\+\+kb == KB\) \{", "} else if (++kb == KB + 1) {"),
     "first segment end": (r"first_end = min\(e, \(b / KB \+ 1\) \* KB\);", "first_end = min(e, (b / KB + 1) * KB - 1);"),
 }
+PREFILL_MUTANTS = {
+    "piece offset": (r"off = \(j % p\.split\) \* cols;", "off = 0;"),
+    "tile index in group": (r"const int r = t - g \* per_group;", "const int r = t - g * per_group + 1;"),
+    "item count": (r"\(tail - 1 - c\) / G \+ 1 : 0\);", "(tail - 1 - c) / G : 0);"),
+    "last group's height": (r"const int gm = min\(p\.group_m, p\.num_m - first_m\);", "const int gm = p.group_m;"),
+}
 
 
 @pytest.mark.skipif(shutil.which("nvcc") is None and not os.path.exists("/usr/local/cuda/bin/nvcc"),
                     reason="needs nvcc")
-@pytest.mark.parametrize("name", sorted(MUTANTS))
+@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(PREFILL_MUTANTS))
 def test_schedule_check_catches_planted_mistake(name):
-    """A plausible mistake planted in a copy of the decode schedule fails the check."""
+    """A plausible mistake planted in a copy of the decode or prefill schedule fails the check."""
     import re
     nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
     root = os.path.dirname(HERE)
-    pat, rep = MUTANTS[name]
+    pat, rep = MUTANTS[name] if name in MUTANTS else PREFILL_MUTANTS[name]
+    header = "sched.cuh" if name in MUTANTS else "gemm_prefill.cuh"
     with tempfile.TemporaryDirectory() as tmp:
         shutil.copytree(os.path.join(root, "fp8_w8a8_quantized_amax_b200", "csrc"),
                         os.path.join(tmp, "fp8_w8a8_quantized_amax_b200", "csrc"))
         os.makedirs(os.path.join(tmp, "tests"))
         shutil.copy(os.path.join(HERE, "schedule_check.cu"), os.path.join(tmp, "tests"))
-        hdr = os.path.join(tmp, "fp8_w8a8_quantized_amax_b200", "csrc", "gemm_decode.cuh")
+        hdr = os.path.join(tmp, "fp8_w8a8_quantized_amax_b200", "csrc", header)
         src, n = re.subn(pat, rep, open(hdr).read())
         assert n >= 1, f"mutation '{name}' did not apply"
         open(hdr, "w").write(src)

@@ -148,11 +148,19 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
+  // The first weight tiles of this CTA's range into L2 before waiting for the
+  // previous kernel: the weights are not what that kernel writes (and L2 is
+  // coherent if they were), so their DRAM latency overlaps its tail.
+  if (warp == 0 && lane == 0) {
+    int i = 0;
+    for (StepIter it(b, e, p.KB); it.valid() && i < STAGES; it.next(), ++i)
+      tma_prefetch_l2_2d(&tmW, it.kb * BK, it.t * 128);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  griddep_wait();   // global memory only from here on
+  griddep_wait();   // global memory only from here on (reads of the prefetched tiles included)
 
   if (warp == 0) {
     if (lane == 0) {

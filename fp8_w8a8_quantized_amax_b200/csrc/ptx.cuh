@@ -256,9 +256,11 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
 // ------------------------------------------- programmatic dependent launch ---
 // Kernels are launched with programmatic stream serialization: a kernel may
 // start while its predecessor in the stream is still finishing.  Every kernel
-// calls griddep_wait() before its first global-memory access (read or write),
-// which returns once the predecessor grid has completed and its memory is
-// visible; only shared/tensor-memory set-up runs before it.
+// calls griddep_wait() before its first global-memory load or store, which
+// returns once the predecessor grid has completed and its memory is visible;
+// only shared/tensor-memory set-up runs before it, and, in the decode kernel,
+// L2 prefetches of weight tiles (a cache hint: the loads that use the data
+// come after the wait, and L2 is coherent).
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // Lets the next kernel in the stream begin launching (it still waits in
 // griddep_wait() for this grid to finish).
@@ -287,6 +289,14 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
 
 // 2-D tile load global -> shared, completion counted in bytes on `bar`.
 // c0 is the innermost (contiguous) coordinate in elements, c1 the row.
+// Bring one tile of a tensor into L2 (no shared memory, no barrier).  A cache
+// hint only: L2 is the device's coherence point, so a line fetched early is
+// still current when a later load reads it, whatever was written in between.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(m)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t c0,
                                             int32_t c1, uint64_t cache_hint) {
   asm volatile(

@@ -65,22 +65,23 @@ __device__ __forceinline__ Divider make_divider(float s) {
 }
 
 // Codes of the two bf16 values packed in w (low half first), divided by s.
+// The fast form runs on the negated values nx = -x (one xor of the two sign
+// bits): q = nx * (-y) = x * y, r' = q * s - x = -r (exact in the FMA), and
+// q' = q - r' * y = q + r * y: the same roundings as the textbook steps, and
+// the signs come out right for x = +-0 as well (+0 + -0 would lose the sign
+// of -0 in q + r * y; here the last FMA adds two zeros of x's sign).
 template <bool FAST>
-__device__ __forceinline__ uint32_t encode_pair(uint32_t w, const Divider& d, uint64_t y2, uint64_t ns2) {
-  const float xl = bf16lo(w), xh = bf16hi(w);
+__device__ __forceinline__ uint32_t encode_pair(uint32_t w, const Divider& d, uint64_t ny2, uint64_t s2) {
   float ql, qh;
   if constexpr (FAST) {
-    // packed fp32x2: q = x*y; r = x - q*s (exact); q' = q + r*y
-    const uint64_t x2 = f32x2_pack(xl, xh);
-    const uint64_t q2 = mul_f32x2(x2, y2);
-    const uint64_t r2 = fma_f32x2(q2, ns2, x2);
-    f32x2_unpack(fma_f32x2(r2, y2, q2), ql, qh);
-    // for x = -0 the correction gives +0; the quotient keeps the sign of x
-    ql = copysignf(ql, xl);
-    qh = copysignf(qh, xh);
+    const uint32_t wn = w ^ 0x80008000u;
+    const uint64_t nx2 = f32x2_pack(bf16lo(wn), bf16hi(wn));
+    const uint64_t q2 = mul_f32x2(nx2, ny2);
+    const uint64_t rn2 = fma_f32x2(q2, s2, nx2);
+    f32x2_unpack(fma_f32x2(rn2, ny2, q2), ql, qh);
   } else {
-    ql = __fdiv_rn(xl, d.s);
-    qh = __fdiv_rn(xh, d.s);
+    ql = __fdiv_rn(bf16lo(w), d.s);
+    qh = __fdiv_rn(bf16hi(w), d.s);
   }
   return cvt_e4m3x2(ql, qh);
 }
@@ -88,11 +89,11 @@ __device__ __forceinline__ uint32_t encode_pair(uint32_t w, const Divider& d, ui
 // 8 bf16 (one uint4) -> 8 codes (one uint2).
 template <bool FAST>
 __device__ __forceinline__ uint2 encode_vec(const uint4& v, const Divider& d) {
-  const uint64_t y2 = f32x2_pack(d.y, d.y);
-  const uint64_t ns2 = f32x2_pack(-d.s, -d.s);
+  const uint64_t ny2 = f32x2_pack(-d.y, -d.y);
+  const uint64_t s2 = f32x2_pack(d.s, d.s);
   uint2 o;
-  o.x = encode_pair<FAST>(v.x, d, y2, ns2) | (encode_pair<FAST>(v.y, d, y2, ns2) << 16);
-  o.y = encode_pair<FAST>(v.z, d, y2, ns2) | (encode_pair<FAST>(v.w, d, y2, ns2) << 16);
+  o.x = encode_pair<FAST>(v.x, d, ny2, s2) | (encode_pair<FAST>(v.y, d, ny2, s2) << 16);
+  o.y = encode_pair<FAST>(v.z, d, ny2, s2) | (encode_pair<FAST>(v.w, d, ny2, s2) << 16);
   return o;
 }
 
@@ -191,7 +192,12 @@ __device__ __forceinline__ uint4 rmsnorm_vec(const uint4& v, const uint4& g, uin
 // 2^-236 in all: far below the sum's own fp64 rounding, and below fp32's
 // smallest subnormal mean.
 __device__ __forceinline__ double bf16_abs_f64(uint32_t b) {
-  return __hiloint2double(static_cast<int>(((b & 0x7FFFu) << 13) + 0x38000000u), 0);
+  return __hiloint2double(static_cast<int>((b & 0x7FFFu) * 8192u + 0x38000000u), 0);
+}
+// The same for the high half of w, without a separate shift: (w & 0x7FFF0000) >> 3
+// is the high word of the product with 2^29.
+__device__ __forceinline__ double bf16hi_abs_f64(uint32_t w) {
+  return __hiloint2double(static_cast<int>(__umulhi(w & 0x7FFF0000u, 0x20000000u) + 0x38000000u), 0);
 }
 
 // Squares of the 8 values of v (exact in fp64: 16 significant bits) added
@@ -200,7 +206,7 @@ __device__ __forceinline__ void sumsq_vec(const uint4& v, double& a0, double& a1
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const double lo = bf16_abs_f64(w[i]), hi = bf16_abs_f64(w[i] >> 16);
+    const double lo = bf16_abs_f64(w[i]), hi = bf16hi_abs_f64(w[i]);
     a0 = fma(lo, lo, a0);
     a1 = fma(hi, hi, a1);
   }

@@ -34,6 +34,7 @@ __device__ __forceinline__ double key_value(uint32_t key) {
 __global__ void __launch_bounds__(256) hist_kernel(const uint16_t* __restrict__ x, int64_t M, int K, int64_t ldx,
                                                    uint32_t* __restrict__ hist) {
   griddep_wait();
+  griddep_launch_dependents();
   const int nvec = K >> 3;
   const int64_t total = M * nvec;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -59,6 +60,7 @@ __global__ void __launch_bounds__(1024) select_kernel(uint32_t* __restrict__ his
   __shared__ unsigned long long warp_sums[32];
   __shared__ uint32_t found[4];
   griddep_wait();
+  griddep_launch_dependents();
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
   unsigned long long local = 0;

@@ -148,18 +148,20 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
-  // The first weight tiles of this CTA's range into L2 before waiting for the
-  // previous kernel: the weights are not what that kernel writes (and L2 is
-  // coherent if they were), so their DRAM latency overlaps its tail.
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // The producer prefetches the first weight tiles of this CTA's range into L2
+  // before waiting for the previous kernel: the weights are not what that
+  // kernel writes (and L2 is coherent if they were), so their DRAM latency
+  // overlaps its tail.  The first prefetch waits for the tensor map to be
+  // fetched; only the producer waits for it, after the CTA barrier.
   if (warp == 0 && lane == 0) {
     int i = 0;
     for (StepIter it(b, e, p.KB); it.valid() && i < STAGES; it.next(), ++i)
       tma_prefetch_l2_2d(&tmW, it.kb * BK, it.t * 128);
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
   griddep_wait();   // global memory only from here on (reads of the prefetched tiles included)
 
   if (warp == 0) {
@@ -411,14 +413,33 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
           prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
           if (prev == static_cast<unsigned int>(c1 - c0)) {   // every other segment is in
             __threadfence();
-            // acc is published; it now collects the tile's sum in CTA order
+            // acc is published; it now collects the tile's sum in CTA order,
+            // the partial sums of kBatch CTAs loaded at once (one L2 round
+            // trip per batch; the +0 of an absent CTA changes no sum, which
+            // starts at +0 and so is never -0)
+            constexpr int kBatch = NX <= 16 ? 4 : (NX <= 32 ? 2 : 1);
 #pragma unroll
             for (int j = 0; j < NX; ++j) acc[j] = 0.0f;
-            for (int cc = c0; cc <= c1; ++cc) {
-              const float* src = p.part + (static_cast<int64_t>(t) + cc) * NX * 128 + nl;
+            for (int cc0 = c0; cc0 <= c1; cc0 += kBatch) {
+              if constexpr (kBatch == 1) {           // 64 tokens: no registers for a batch
+                const float* src = p.part + (static_cast<int64_t>(t) + cc0) * NX * 128 + nl;
 #pragma unroll
-              for (int j = 0; j < NX; ++j)
-                if (j < p.M) acc[j] += __ldcg(src + j * 128);
+                for (int j = 0; j < NX; ++j)
+                  if (j < p.M) acc[j] += __ldcg(src + j * 128);
+              } else {
+                float v[kBatch][NX];
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                  const float* src = p.part + (static_cast<int64_t>(t) + cc0 + u) * NX * 128 + nl;
+#pragma unroll
+                  for (int j = 0; j < NX; ++j)
+                    v[u][j] = (cc0 + u <= c1 && j < p.M) ? __ldcg(src + j * 128) : 0.0f;
+                }
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+                  for (int j = 0; j < NX; ++j) acc[j] += v[u][j];
+              }
             }
             for (int cc = c0; cc <= c1; ++cc) {   // the workspace is left all zero
               float* src = p.part + (static_cast<int64_t>(t) + cc) * NX * 128 + nl;
@@ -453,6 +474,7 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
 template <bool BLOCK>
 __global__ void __launch_bounds__(128) decode_reduce_kernel(const Params p, int nx) {
   griddep_wait();
+  griddep_launch_dependents();
   const int t = blockIdx.x;
   const int m = blockIdx.y;
   const int nl = threadIdx.x;

@@ -263,7 +263,11 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
 // come after the wait, and L2 is coherent).
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // Lets the next kernel in the stream begin launching (it still waits in
-// griddep_wait() for this grid to finish).
+// griddep_wait() for this grid to finish).  The next grid launches once every
+// CTA of this one has called it or exited, so kernels whose CTAs have nothing
+// to hand over call it right after griddep_wait(): by then all of this grid's
+// CTAs have been placed, and the next grid's CTAs (launch and set-up) take
+// SM room only as this grid's CTAs leave it.
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }

@@ -70,30 +70,33 @@ __device__ __forceinline__ Divider make_divider(float s) {
 // q' = q - r' * y = q + r * y: the same roundings as the textbook steps, and
 // the signs come out right for x = +-0 as well (+0 + -0 would lose the sign
 // of -0 in q + r * y; here the last FMA adds two zeros of x's sign).
-template <bool FAST>
+// NEG: w holds the negated values already (a producer that can negate for
+// free, such as the RMSNorm below, skips the xor).
+template <bool FAST, bool NEG = false>
 __device__ __forceinline__ uint32_t encode_pair(uint32_t w, const Divider& d, uint64_t ny2, uint64_t s2) {
   float ql, qh;
   if constexpr (FAST) {
-    const uint32_t wn = w ^ 0x80008000u;
+    const uint32_t wn = NEG ? w : (w ^ 0x80008000u);
     const uint64_t nx2 = f32x2_pack(bf16lo(wn), bf16hi(wn));
     const uint64_t q2 = mul_f32x2(nx2, ny2);
     const uint64_t rn2 = fma_f32x2(q2, s2, nx2);
     f32x2_unpack(fma_f32x2(rn2, ny2, q2), ql, qh);
   } else {
-    ql = __fdiv_rn(bf16lo(w), d.s);
-    qh = __fdiv_rn(bf16hi(w), d.s);
+    const uint32_t wp = NEG ? (w ^ 0x80008000u) : w;
+    ql = __fdiv_rn(bf16lo(wp), d.s);
+    qh = __fdiv_rn(bf16hi(wp), d.s);
   }
   return cvt_e4m3x2(ql, qh);
 }
 
 // 8 bf16 (one uint4) -> 8 codes (one uint2).
-template <bool FAST>
+template <bool FAST, bool NEG = false>
 __device__ __forceinline__ uint2 encode_vec(const uint4& v, const Divider& d) {
   const uint64_t ny2 = f32x2_pack(-d.y, -d.y);
   const uint64_t s2 = f32x2_pack(d.s, d.s);
   uint2 o;
-  o.x = encode_pair<FAST>(v.x, d, ny2, s2) | (encode_pair<FAST>(v.y, d, ny2, s2) << 16);
-  o.y = encode_pair<FAST>(v.z, d, ny2, s2) | (encode_pair<FAST>(v.w, d, ny2, s2) << 16);
+  o.x = encode_pair<FAST, NEG>(v.x, d, ny2, s2) | (encode_pair<FAST, NEG>(v.y, d, ny2, s2) << 16);
+  o.y = encode_pair<FAST, NEG>(v.z, d, ny2, s2) | (encode_pair<FAST, NEG>(v.w, d, ny2, s2) << 16);
   return o;
 }
 
@@ -110,6 +113,7 @@ __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __rest
                                                          float* __restrict__ s, bool s16) {
   __shared__ uint32_t red[32];
   griddep_wait();
+  griddep_launch_dependents();
   const int64_t r = blockIdx.x;
   const int nvec = K >> 3;
   const int T = blockDim.x;
@@ -164,11 +168,14 @@ __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __rest
 // few fp64 roundings of an fp32 rounding boundary; rstd is written out when
 // rstd != nullptr.
 
-// y for the 8 bf16 values of v (x) with the matching 8 of g (gamma), two at a
-// time: h = bf16(fl32(x * rstd)) by a packed fp32 multiply and one bf16x2
-// rounding; y = bf16(gamma * h) by one bf16x2 multiply.  The product of two
+// -y for the 8 bf16 values of v (x) with the matching 8 of g (gamma), two at
+// a time: -h = bf16(fl32(x * -rstd)) by a packed fp32 multiply and one bf16x2
+// rounding; -y = bf16(gamma * -h) by one bf16x2 multiply.  The product of two
 // bf16 values is exact in fp32, so rounding it once to bf16 (mul.rn.bf16x2)
-// is the same as rounding the fp32 product.
+// is the same as rounding the fp32 product.  Negation is exact and
+// round-to-nearest-even is symmetric, so these are exactly the negated values
+// of the textbook steps, as the encode wants them (encode_vec<..., true>);
+// the amax ignores signs.
 __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
@@ -201,14 +208,15 @@ __device__ __forceinline__ double bf16hi_abs_f64(uint32_t w) {
 }
 
 // Squares of the 8 values of v (exact in fp64: 16 significant bits) added
-// into two fp64 chains.
-__device__ __forceinline__ void sumsq_vec(const uint4& v, double& a0, double& a1) {
+// into four fp64 chains (one per 32-bit word), so that a thread's dependent
+// fp64 additions per row are 2 * VPT long.
+__device__ __forceinline__ void sumsq_vec(const uint4& v, double (&a)[4]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const double lo = bf16_abs_f64(w[i]), hi = bf16hi_abs_f64(w[i]);
-    a0 = fma(lo, lo, a0);
-    a1 = fma(hi, hi, a1);
+    a[i] = fma(lo, lo, a[i]);
+    a[i] = fma(hi, hi, a[i]);
   }
 }
 
@@ -221,6 +229,7 @@ __global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t*
   __shared__ double red_sum[32];
   __shared__ uint32_t red_max[32];
   griddep_wait();
+  griddep_launch_dependents();
   const int64_t r = blockIdx.x;
   const int nvec = K >> 3;
   const int T = blockDim.x;
@@ -231,7 +240,7 @@ __global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t*
   // third of the registers and so a third of the rows in flight per SM
   constexpr bool kGammaAhead = false;
   uint4 v[VPT], gv[kGammaAhead ? VPT : 1];
-  double ss0 = 0.0, ss1 = 0.0;
+  double ssa[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int idx = threadIdx.x + i * T;
@@ -242,8 +251,8 @@ __global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t*
   }
 #pragma unroll
   for (int i = 0; i < VPT; ++i)
-    if (threadIdx.x + i * T < nvec) sumsq_vec(v[i], ss0, ss1);
-  double ss = ss0 + ss1;
+    if (threadIdx.x + i * T < nvec) sumsq_vec(v[i], ssa);
+  double ss = (ssa[0] + ssa[1]) + (ssa[2] + ssa[3]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
   if (T > 32) {
@@ -258,7 +267,7 @@ __global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t*
   const float ms = __double2float_rn(ss / static_cast<double>(K));
   const float rs = __frsqrt_rn(__fadd_rn(ms, eps));
   if (threadIdx.x == 0 && rstd != nullptr) rstd[r] = rs;
-  const uint64_t rs2 = f32x2_pack(rs, rs);
+  const uint64_t rs2 = f32x2_pack(-rs, -rs);   // v becomes -y (see rmsnorm_vec)
   uint32_t m2 = 0;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
@@ -284,13 +293,13 @@ __global__ void __launch_bounds__(512) rmsnorm_quant_rows_kernel(const uint16_t*
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int idx = threadIdx.x + i * T;
-      if (idx < nvec) *reinterpret_cast<uint2*>(qr + idx * 8) = encode_vec<true>(v[i], dv);
+      if (idx < nvec) *reinterpret_cast<uint2*>(qr + idx * 8) = encode_vec<true, true>(v[i], dv);
     }
   } else {
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int idx = threadIdx.x + i * T;
-      if (idx < nvec) *reinterpret_cast<uint2*>(qr + idx * 8) = encode_vec<false>(v[i], dv);
+      if (idx < nvec) *reinterpret_cast<uint2*>(qr + idx * 8) = encode_vec<false, true>(v[i], dv);
     }
   }
 }
@@ -309,6 +318,7 @@ __global__ void __launch_bounds__(256) quant_static_kernel(const uint16_t* __res
   // incrementally in 32-bit arithmetic (the host keeps M * K / 8 below 2^31).
   constexpr int kVec = 4;
   griddep_wait();
+  griddep_launch_dependents();
   const uint32_t nvec = static_cast<uint32_t>(K) >> 3;
   const uint32_t Mu = static_cast<uint32_t>(M);
   const uint32_t stride = gridDim.x * blockDim.x;
@@ -354,6 +364,7 @@ __global__ void __launch_bounds__(256) quant_groups128_kernel(const uint16_t* __
                                                              int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
                                                              float* __restrict__ s, bool s16) {
   griddep_wait();
+  griddep_launch_dependents();
   const int sub = threadIdx.x & 15;
   const uint32_t half_mask = 0xFFFFu << (threadIdx.x & 16);
   const uint32_t H = (gridDim.x * blockDim.x) >> 4;
@@ -407,6 +418,7 @@ __global__ void __launch_bounds__(256) quant_blocks128_kernel(const uint16_t* __
                                                              float* __restrict__ s, bool s16) {
   __shared__ uint32_t red[8];
   griddep_wait();
+  griddep_launch_dependents();
   const int kb = blockIdx.x;
   const int64_t nb = blockIdx.y;
   const int vc = threadIdx.x & 15;

@@ -74,8 +74,11 @@ fp8q_status ensure_smem(K kernel, int bytes, int dev) {
   return FP8Q_OK;
 }
 
+// cluster_x > 0: launched in clusters of cluster_x CTAs (for kernels without
+// a compile-time cluster shape).
 template <typename... KArgs, typename... Args>
-fp8q_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, void* stream, Args... args) {
+fp8q_status launch_clustered(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, void* stream,
+                             int cluster_x, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -84,12 +87,24 @@ fp8q_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
   // Programmatic dependent launch: the kernel may begin while its stream
   // predecessor finishes; every kernel here waits (griddepcontrol.wait)
   // before touching global memory.
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (cluster_x > 0) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
   return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+template <typename... KArgs, typename... Args>
+fp8q_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, void* stream, Args... args) {
+  return launch_clustered(kernel, grid, block, smem, stream, 0, args...);
 }
 
 // ------------------------------------------------------------ tensor maps ---
@@ -279,44 +294,108 @@ fp8q_status check_linear_args(const uint8_t* Xq, const float* xs, const uint8_t*
   return FP8Q_OK;
 }
 
-// Whether the decode kernel sums split weight tiles itself (else a reduction
-// kernel follows it).  Measured on the Llama-3.1-70B and -3.2-3B decode shapes:
-// in channel mode with up to 16 tokens the in-kernel sums are cheap enough to
+// Where the decode kernel's split weight tiles are summed (gemm_decode.cuh).
+// Measured on the Llama-3.1-70B and -3.2-3B decode shapes: in channel mode
+// with up to 16 tokens the in-kernel sums (last arriver) are cheap enough to
 // win everywhere; with 32 or 64 tokens only when every CTA streams at least a
-// tile's worth of steps after them; in block mode the per-K-block epilogue
-// leaves no room, and the separate kernel is faster.
-// FP8Q_DECODE_BLOCK_SUMS=kernel|separate forces one way in block mode (read
-// once), for comparing them on the same problem.
-int decode_block_sums_choice() {
+// tile's worth of steps after them.  In block mode the last arriver's fence,
+// atomic and loads sit at the end of a short kernel, and the reduction kernel
+// pays a grid boundary; cluster split-K (one weight tile per cluster, sums in
+// distributed shared memory) avoids both wherever its clusters fill most
+// SMs at once.  FP8Q_DECODE_SUMS=separate|kernel|cluster forces one (read
+// once; cluster where some cluster size fits, else the default), for
+// comparing them on the same problem.
+int decode_sums_forced() {
   static int choice = [] {
-    const char* e = getenv("FP8Q_DECODE_BLOCK_SUMS");
-    if (e && strcmp(e, "kernel") == 0) return 1;
-    if (e && strcmp(e, "separate") == 0) return 2;
-    return 0;
+    const char* e = getenv("FP8Q_DECODE_SUMS");
+    if (e && strcmp(e, "separate") == 0) return fp8q::decode::kSumsSeparate;
+    if (e && strcmp(e, "kernel") == 0) return fp8q::decode::kSumsKernel;
+    if (e && strcmp(e, "cluster") == 0) return fp8q::decode::kSumsCluster;
+    return -1;
   }();
   return choice;
 }
 
-bool decode_fused(const Params& p, int mode, int nx) {
-  if (mode == FP8Q_BLOCK128) return decode_block_sums_choice() == 1;
-  return nx == 16 || p.total >= static_cast<int64_t>(p.KB) * p.G;
+// Clusters of C decode CTAs (one CTA per SM) that fit on the device at once,
+// per token tile, cluster size and device; 0 where the query fails.
+template <int NX>
+int decode_max_clusters(int C, int dev, int sms) {
+  constexpr int kDecodeStages = decode_stages<NX>();
+  using L = fp8q::decode::Layout<NX, kDecodeStages>;
+  static std::atomic<int> cache[9][kMaxDevices];   // value + 1; 0 = not asked yet
+  int v = cache[C][dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    auto k = fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, true, fp8q::decode::kSumsCluster>;
+    int n = 0;
+    if (ensure_smem(k, L::kBytes, dev) == FP8Q_OK) {
+      cudaLaunchConfig_t qc = {};
+      qc.gridDim = dim3(static_cast<unsigned>(C * sms));
+      qc.blockDim = dim3(L::kThreads);
+      qc.dynamicSmemBytes = L::kBytes;
+      cudaLaunchAttribute a[1];
+      a[0].id = cudaLaunchAttributeClusterDimension;
+      a[0].val.clusterDim.x = static_cast<unsigned>(C);
+      a[0].val.clusterDim.y = 1;
+      a[0].val.clusterDim.z = 1;
+      qc.attrs = a;
+      qc.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, k, &qc) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+    }
+    v = n + 1;
+    cache[C][dev].store(v, std::memory_order_relaxed);
+  }
+  return v - 1;
+}
+
+// Cluster size for cluster split-K, or 0: C in [2, 8], at most KB (every CTA
+// gets a K block) and at most sms / n_tiles, the largest whose n_tiles
+// clusters the device holds at once; by default only where those
+// n_tiles * C CTAs fill at least 3/4 of the SMs.
+template <int NX>
+int decode_cluster_size(const Params& p, int sms, int dev, bool forced) {
+  int C = sms / p.n_tiles;
+  if (C > 8) C = 8;
+  if (C > p.KB) C = p.KB;
+  for (; C >= 2; --C) {
+    if (!forced && 4 * p.n_tiles * C < 3 * sms) return 0;
+    if (decode_max_clusters<NX>(C, dev, sms) >= p.n_tiles) return C;
+  }
+  return 0;
 }
 
 template <int NX>
 fp8q_status launch_decode_nx(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p, int mode, int dev,
-                             void* stream) {
+                             int sms, void* stream) {
+  using namespace fp8q::decode;
   constexpr int kDecodeStages = decode_stages<NX>();
-  using L = fp8q::decode::Layout<NX, kDecodeStages>;
+  using L = Layout<NX, kDecodeStages>;
   fp8q_status st;
   const bool block = mode == FP8Q_BLOCK128;
-  if (decode_fused(p, mode, NX)) {
-    auto k = block ? fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, true, true>
-                   : fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, false, true>;
+  const int forced = decode_sums_forced();
+  if (forced == kSumsCluster || (forced < 0 && block)) {
+    const int C = decode_cluster_size<NX>(p, sms, dev, forced == kSumsCluster);
+    if (C >= 2) {
+      auto k = block ? gemm_decode_kernel<NX, kDecodeStages, true, kSumsCluster>
+                     : gemm_decode_kernel<NX, kDecodeStages, false, kSumsCluster>;
+      if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
+      Params q = p;
+      q.G = p.n_tiles * C;
+      return launch_clustered(k, dim3(q.G), dim3(L::kThreads), L::kBytes, stream, C, tw, tx, q);
+    }
+  }
+  const bool in_kernel = forced == kSumsKernel ||
+                         (forced != kSumsSeparate && !block && (NX == 16 || p.total >= static_cast<int64_t>(p.KB) * p.G));
+  if (in_kernel) {
+    auto k = block ? gemm_decode_kernel<NX, kDecodeStages, true, kSumsKernel>
+                   : gemm_decode_kernel<NX, kDecodeStages, false, kSumsKernel>;
     if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
     return launch(k, dim3(p.G), dim3(192), L::kBytes, stream, tw, tx, p);
   }
-  auto k = block ? fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, true, false>
-                 : fp8q::decode::gemm_decode_kernel<NX, kDecodeStages, false, false>;
+  auto k = block ? gemm_decode_kernel<NX, kDecodeStages, true, kSumsSeparate>
+                 : gemm_decode_kernel<NX, kDecodeStages, false, kSumsSeparate>;
   if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
   if ((st = launch(k, dim3(p.G), dim3(192), L::kBytes, stream, tw, tx, p)) != FP8Q_OK) return st;
   auto r = block ? fp8q::decode::decode_reduce_kernel<true> : fp8q::decode::decode_reduce_kernel<false>;
@@ -343,7 +422,7 @@ fp8q_status launch_decode_w16_n(const CUtensorMap& tw, const CUtensorMap& tx, co
                                 void* stream) {
   constexpr int kStages = w16_stages<NX>();
   using L = fp8q::decode::Layout<NX, kStages, WIDEN>;
-  auto k = fp8q::decode::gemm_decode_kernel<NX, kStages, false, true, WIDEN>;
+  auto k = fp8q::decode::gemm_decode_kernel<NX, kStages, false, fp8q::decode::kSumsKernel, WIDEN>;
   fp8q_status st;
   if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
   return launch(k, dim3(p.G), dim3(L::kThreads), L::kBytes, stream, tw, tx, p);
@@ -612,9 +691,9 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     p.total = static_cast<int>(total);
     p.G = G;
     decode_bind_workspace(p, workspace, Y_bf16, ldy);
-    if (nx == 16) return launch_decode_nx<16>(tw, tx, p, mode, dev, stream);
-    if (nx == 32) return launch_decode_nx<32>(tw, tx, p, mode, dev, stream);
-    return launch_decode_nx<64>(tw, tx, p, mode, dev, stream);
+    if (nx == 16) return launch_decode_nx<16>(tw, tx, p, mode, dev, sms, stream);
+    if (nx == 32) return launch_decode_nx<32>(tw, tx, p, mode, dev, sms, stream);
+    return launch_decode_nx<64>(tw, tx, p, mode, dev, sms, stream);
   }
 
   const bool pair = prefill_choice() != 1 && (M >= 256 || prefill_choice() == 2);
@@ -948,9 +1027,9 @@ fp8q_status fp8_linear_noalloc(const uint8_t* Xq, const float* x_scale, const ui
   p.total = static_cast<int>(total);
   p.G = G;
   decode_bind_workspace(p, scratch, Y_bf16, ldy);
-  if (nx == 16) return launch_decode_nx<16>(tw, tx, p, mode, dev, stream);
-  if (nx == 32) return launch_decode_nx<32>(tw, tx, p, mode, dev, stream);
-  return launch_decode_nx<64>(tw, tx, p, mode, dev, stream);
+  if (nx == 16) return launch_decode_nx<16>(tw, tx, p, mode, dev, sms, stream);
+  if (nx == 32) return launch_decode_nx<32>(tw, tx, p, mode, dev, sms, stream);
+  return launch_decode_nx<64>(tw, tx, p, mode, dev, sms, stream);
 }
 
 }  // extern "C"

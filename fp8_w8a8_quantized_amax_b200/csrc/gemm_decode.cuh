@@ -22,10 +22,18 @@
 // range (the start of a tile it shares with the next CTA), the segment at the
 // start of its range, then the whole tiles between them, so that the
 // reductions happen under the rest of the weight stream.  Where that does
-// not pay (FUSED = false; the host decides per shape) the partial segments
+// not pay (SUMS = kSumsSeparate; the host decides per shape) the partial segments
 // are summed by decode_reduce_kernel after the GEMM kernel, which clears them
 // likewise.  Partial traffic is at most (n_tiles + G) * NX * 512 bytes, small
 // next to the N * K weight bytes.
+//
+// Cluster split-K (SUMS = kSumsCluster; the host picks it for small block-mode
+// problems, n_tiles * C CTAs filling most SMs): CTA rank r of cluster t (C
+// CTAs) takes K blocks [r KB / C, (r + 1) KB / C) of weight tile t, a single
+// partial segment.  Its sums stay in its own shared memory; after a cluster
+// barrier rank 0 adds the C partial tiles in rank order through distributed
+// shared memory and writes the bf16 tile, and a second barrier keeps every
+// CTA resident until then.  No workspace, no atomics, no second kernel.
 //
 // Roles: warp 0 TMA (W tile 128 x 128 B evict-first + X tile NX x 128 B),
 // warp 1 TMEM allocation + MMA issue, warps 2..5 drain TMEM and write
@@ -60,6 +68,11 @@ constexpr int BK = 128;
 constexpr int UMMA_K = 32;
 constexpr int kSlots = 8;
 
+// Where a weight tile's partial segments are added: decode_reduce_kernel after
+// the GEMM kernel, the last CTA to finish one (through the workspace), or rank 0
+// of the tile's cluster (through distributed shared memory).
+constexpr int kSumsSeparate = 0, kSumsKernel = 1, kSumsCluster = 2;
+
 struct Params {
   const float* xs;
   const float* ws;
@@ -70,7 +83,7 @@ struct Params {
   int M, N, K, KB;
   int n_tiles;
   int total;            // n_tiles * KB (the host refuses 2^31 or more)
-  int G;                // CTAs
+  int G;                // CTAs (cluster split-K: n_tiles * cluster size)
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -97,7 +110,7 @@ struct Layout {
   static constexpr uint32_t kTmemCols = (kSlots * NX) < 32 ? 32 : (kSlots * NX);
 };
 
-template <int NX, int STAGES, bool BLOCK, bool FUSED, int WIDEN = 0>
+template <int NX, int STAGES, bool BLOCK, int SUMS, int WIDEN = 0>
 __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const Params p) {
@@ -105,7 +118,9 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
   constexpr bool W16 = WIDEN > 0;
   static_assert(WIDEN == 0 || WIDEN == 4 || WIDEN == 8, "widen warps");
   static_assert(NX % 16 == 0 && NX >= 16 && NX <= 64, "token tile");
-  static_assert(!(W16 && (BLOCK || !FUSED)), "the weight-only variant has channel scales and sums its own splits");
+  static_assert(!(W16 && (BLOCK || SUMS != kSumsKernel)),
+                "the weight-only variant has channel scales and sums its own splits");
+  static_assert(SUMS == kSumsSeparate || SUMS == kSumsKernel || SUMS == kSumsCluster, "sums");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sW = smem;
@@ -124,8 +139,14 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int c = blockIdx.x;
   const Split sp = split_of(p.total, p.G);
-  const int b = range_begin(c, sp);
-  const int e = range_begin(c + 1, sp);
+  int b, e;
+  if constexpr (SUMS == kSumsCluster) {
+    const int C = static_cast<int>(cluster_nctarank());
+    sched::cluster_range(c / C, static_cast<int>(cluster_ctarank()), C, p.KB, &b, &e);
+  } else {
+    b = range_begin(c, sp);
+    e = range_begin(c + 1, sp);
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -152,15 +173,16 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // The producer prefetches the first weight tiles of this CTA's range into L2
-  // before waiting for the previous kernel: the weights are not what that
-  // kernel writes (and L2 is coherent if they were), so their DRAM latency
-  // overlaps its tail.  The first prefetch waits for the tensor map to be
-  // fetched; only the producer waits for it, after the CTA barrier.
-  if (warp == 0 && lane == 0) {
+  // The first weight tiles of this CTA's range are prefetched into L2 before
+  // the wait for the previous kernel: the weights are not what that kernel
+  // writes (and L2 is coherent if they were), so their DRAM latency overlaps
+  // its tail.  The epilogue warps issue them (every fourth step each; they
+  // have nothing to do until the first accumulator is ready), so that the
+  // producer's first load is not queued behind them.
+  if (warp >= 2 && warp < 6 && lane == 0) {
     int i = 0;
     for (StepIter it(b, e, p.KB); it.valid() && i < STAGES; it.next(), ++i)
-      tma_prefetch_l2_2d(&tmW, it.kb * BK, it.t * 128);
+      if ((i & 3) == warp - 2) tma_prefetch_l2_2d(&tmW, it.kb * BK, it.t * 128);
   }
   griddep_wait();   // global memory only from here on (reads of the prefetched tiles included)
 
@@ -394,12 +416,19 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
         };
         if (seg_len == p.KB) {                     // the whole tile: no partial sums
           emit(acc);
+        } else if constexpr (SUMS == kSumsCluster) {
+          // the CTA's one segment: every MMA has completed (this slot was the
+          // last one committed) and every stage has been consumed, so the
+          // stage area holds the partial tile [NX][128] for rank 0 to read
+          float* part_s = reinterpret_cast<float*>(sW);
+#pragma unroll
+          for (int j = 0; j < NX; ++j) part_s[j * 128 + nl] = acc[j];
         } else {
           float* dst = p.part + (static_cast<int64_t>(t) + c) * NX * 128 + nl;
 #pragma unroll
           for (int j = 0; j < NX; ++j)
             if (j < p.M) dst[j * 128] = acc[j];
-          if constexpr (!FUSED) {
+          if constexpr (SUMS == kSumsSeparate) {
 #pragma unroll
             for (int j = 0; j < NX; ++j) acc[j] = 0.0f;
             continue;                              // summed by decode_reduce_kernel
@@ -458,6 +487,36 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
     if constexpr (BLOCK) cp_async_wait<0>();     // no copy into the ring outlives the CTA
   }
 
+  if constexpr (SUMS == kSumsCluster) {
+    cluster_sync();   // every CTA of the cluster has its partial tile in shared memory
+    const int C = static_cast<int>(cluster_nctarank());
+    if (C > 1 && cluster_ctarank() == 0 && warp >= 2 && warp < 6) {
+      // rank 0's epilogue threads: channel nl of the tile, the C partial sums
+      // of each token added in rank order
+      const int nl = (warp & 3) * 32 + lane;
+      const int n = (c / C) * 128 + nl;
+      const uint32_t part_s = smem_u32(sW);
+      float sum[NX];
+#pragma unroll
+      for (int j = 0; j < NX; ++j) sum[j] = 0.0f;
+      for (int r = 0; r < C; ++r) {
+        const uint32_t src = mapa_shared(part_s, static_cast<uint32_t>(r)) + static_cast<uint32_t>(nl) * 4u;
+#pragma unroll
+        for (int j = 0; j < NX; ++j)
+          if (j < p.M) sum[j] += ld_shared_cluster_f32(src + static_cast<uint32_t>(j) * 512u);
+      }
+      if (n < p.N) {
+        const float wn = BLOCK ? 1.0f : __ldg(p.ws + n);
+#pragma unroll
+        for (int j = 0; j < NX; ++j)
+          if (j < p.M) {
+            const float o = BLOCK ? sum[j] : sum[j] * __ldg(p.xs + j) * wn;
+            p.y[static_cast<int64_t>(j) * p.ldy + n] = __float2bfloat16_rn(o);
+          }
+      }
+    }
+    cluster_sync();   // rank 0 has read every partial tile before any CTA leaves
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -71,5 +71,13 @@ struct StepIter {
   }
 };
 
+// Cluster split-K (decode): rank r of the C CTAs that share weight tile t
+// takes its K blocks [r KB / C, (r + 1) KB / C), the steps [b, e) of the
+// list: one segment, non-empty when C <= KB.
+__host__ __device__ __forceinline__ void cluster_range(int t, int r, int C, int KB, int* b, int* e) {
+  *b = t * KB + r * KB / C;
+  *e = t * KB + (r + 1) * KB / C;
+}
+
 }  // namespace sched
 }  // namespace fp8q

@@ -11,6 +11,12 @@ or three calls of the stream-K prefill schedule (FP8Q_PREFILL_STREAMK=1) on one
 workspace, each checked against the oracle and the counters checked zero:
 
     python -m tests._forced_kernel streamk M N K
+
+or three decode calls (M <= 64) with the split-tile sums forced by
+FP8Q_DECODE_SUMS (separate, kernel or cluster) on one workspace, each checked
+against the oracle, bit-equal to each other, the workspace left zero:
+
+    python -m tests._forced_kernel decode M N K mode
 """
 import sys
 
@@ -83,7 +89,32 @@ def streamk_fallback():
     print("ok")
 
 
+def decode():
+    import torch
+    M, N, K, mode = (int(a) for a in sys.argv[2:6])
+    x = synth.make_x(M, K, seed=M + N)
+    w = synth.make_w(N, K, seed=M + N)
+    wq, ws = fq.fp8_quant_weight(w.to("cuda"), mode)
+    xq, xs = fq.fp8_quant_act(x.to("cuda"), mode)
+    wk = torch.zeros(fq.fp8_linear_workspace_size(M, N, K, mode), dtype=torch.uint8, device="cuda")
+    rxq, rxs = oracle.quant_act(x, mode)
+    rwq, rws = oracle.quant_weight(w, mode)
+    yref = oracle.linear(rxq, rxs, rwq, rws, mode)
+    ys = []
+    for _ in range(3):
+        y = fq.fp8_linear(xq, xs, wq, ws, mode, workspace=wk)
+        torch.cuda.synchronize()
+        P.assert_y_close(y.float().cpu().numpy(), yref, what=f"decode {M}x{N}x{K} mode {mode}")
+        assert torch.count_nonzero(wk).item() == 0, "workspace not left zero"
+        ys.append(y)
+    assert all(torch.equal(ys[0], y) for y in ys[1:]), "decode sums are not deterministic"
+    assert fq.device_error(clear=True) == 0
+    print("ok")
+
+
 def main():
+    if sys.argv[1] == "decode":
+        return decode()
     if sys.argv[1] == "w8a16":
         return w8a16()
     if sys.argv[1] == "streamk":

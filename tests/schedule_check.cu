@@ -13,6 +13,11 @@
 //   - for every split tile, CTAs c0..c1 (as the last-arriver sums them) are
 //     exactly the CTAs holding a partial segment of it.
 //
+// Cluster split-K (decode): for every K-block count and cluster size C <= KB,
+// with the kernel's own cluster_range and StepIter, the C ranks' ranges
+// partition the tile's K blocks in rank order, each is one non-empty segment
+// of that tile (first and last step flagged), and none is the whole tile.
+//
 // Prefill (persistent CTAs or CTA pairs): for many (row blocks, column
 // blocks, workers), with the kernels' own tail_split, work_items, work_item
 // and tile_coords, every column of every tile is computed by exactly one
@@ -88,6 +93,27 @@ static int check(int n_tiles, int KB, int G) {
   return 0;
 }
 
+static int check_cluster(int n_tiles, int KB, int C) {
+  for (int t = 0; t < n_tiles; ++t) {
+    int next = t * KB;
+    for (int r = 0; r < C; ++r) {
+      int b, e;
+      cluster_range(t, r, C, KB, &b, &e);
+      if (b != next || e <= b || e > (t + 1) * KB) return fail("cluster ranges", n_tiles, KB, C);
+      next = e;
+      int n = 0;
+      for (StepIter it(b, e, KB); it.valid(); it.next(), ++n) {
+        if (it.s != b + n || it.t != t || it.kb != it.s - t * KB) return fail("cluster steps", n_tiles, KB, C);
+        if (it.seg_first() != (n == 0) || it.seg_last() != (it.s + 1 == e))
+          return fail("cluster segment flags", n_tiles, KB, C);
+      }
+      if (n != e - b || n == KB) return fail("cluster segment length", n_tiles, KB, C);
+    }
+    if (next != (t + 1) * KB) return fail("cluster ranges cover the tile", n_tiles, KB, C);
+  }
+  return 0;
+}
+
 static int check_prefill(int num_m, int num_n, int G, int tile_cols) {
   fp8q::prefill::Params p{};
   p.num_m = num_m;
@@ -144,6 +170,10 @@ int main() {
       bad |= check(sh[0], sh[1], G);
       ++cases;
     }
+  // cluster split-K: every cluster size on small K-block counts and the
+  // FP8-Block decode shapes (K = 3072 and 8192: 24 and 64 K blocks)
+  for (int KB = 2; KB <= 70; ++KB)
+    for (int C = 2; C <= 8 && C <= KB; ++C, ++cases) bad |= check_cluster(3, KB, C);
   std::printf("%s: %d schedules\n", bad ? "FAIL" : "ok", cases);
   return bad;
 }

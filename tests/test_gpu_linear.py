@@ -179,6 +179,31 @@ def test_decode_many_segments_per_tile(M, N, K, mode):
     check_full(M, N, K, mode, seed=K)
 
 
+@pytest.mark.parametrize("sums,M,N,K,mode", [
+    ("cluster", 1, 272, 384, fq.BLOCK128),        # 3 weight tiles of 3 K blocks: clusters of 3, one K block a CTA
+    ("cluster", 16, 1024, 2048, fq.BLOCK128),     # 8 tiles of 16 K blocks: clusters of 8
+    ("cluster", 3, 8192, 3072, fq.BLOCK128),      # the Llama-3.2-3B gate/up_proj shape (the default picks clusters)
+    ("cluster", 33, 3072, 8192, fq.BLOCK128),     # down_proj: 24 tiles, 64 K blocks, 64-token tile
+    ("cluster", 40, 528, 1040, fq.CHANNEL_TOKEN),  # channel scales, ragged N and K
+    ("cluster", 5, 304, 1024, fq.CHANNEL_TOKEN),   # a partial last weight tile
+    ("cluster", 64, 256, 128, fq.BLOCK128),       # one K block: no cluster fits, the default path runs
+    ("kernel", 16, 1024, 2048, fq.BLOCK128),      # block scales, summed by the last CTA to finish
+    ("separate", 8, 1024, 4096, fq.CHANNEL_TOKEN),  # channel scales, summed by the reduction kernel
+    ("separate", 16, 8192, 3072, fq.BLOCK128),
+])
+def test_decode_sums_forced(sums, M, N, K, mode):
+    # each place the split weight tiles can be summed, forced on shapes the
+    # default dispatch may give another; three calls on one workspace
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, FP8Q_DECODE_SUMS=sums)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-m", "tests._forced_kernel", "decode", str(M), str(N), str(K), str(mode)],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
 def test_decode_workspace_left_reusable():
     # The workspace is all zero again after every call, so one zero-filled
     # buffer serves calls of different shapes and modes in a row (a later call

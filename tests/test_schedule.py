@@ -31,6 +31,7 @@ MUTANTS = {
                         "return x < big ? x / sp.q : sp.r + (x - big) / sp.q;"),
     "K-block wrap": (r"\} else if \(\+\+kb == KB\) \{", "} else if (++kb == KB + 1) {"),
     "first segment end": (r"first_end = min\(e, \(b / KB \+ 1\) \* KB\);", "first_end = min(e, (b / KB + 1) * KB - 1);"),
+    "cluster range end": (r"\*e = t \* KB \+ \(r \+ 1\) \* KB / C;", "*e = t * KB + (r + 1) * (KB / C);"),
 }
 PREFILL_MUTANTS = {
     "piece offset": (r"off = \(j % p\.split\) \* cols;", "off = 0;"),

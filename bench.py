@@ -330,12 +330,39 @@ def decode_reduce_launched(g, sms: int) -> bool:
     G = min(total, sms)
     nx = 16 if g.M <= 16 else (32 if g.M <= 32 else 64)
     if g.mode == synth.BLOCK128:
-        return True
+        # cluster split-K (no second kernel) where clusters of C in [2, 8] CTAs,
+        # one weight tile each, fill at least 3/4 of the SMs (assuming the
+        # device holds that many clusters at once, as the library checks)
+        C = min(8, sms // n_tiles, kb)
+        return not (C >= 2 and 4 * n_tiles * C >= 3 * sms)
     return not (nx == 16 or total >= kb * G)
 
 
 def launches_of(g, sms: int) -> int:
     return 1 + int(decode_reduce_launched(g, sms))
+
+
+def graph_kernel_nodes(graph):
+    """Kernel launches in a captured CUDA graph (its kernel nodes), or None
+    where the graph cannot be inspected."""
+    try:
+        from cuda.bindings import runtime as rt
+        h = rt.cudaGraph_t(init_value=graph.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(h, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(h, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        count = 0
+        for node in nodes[:n]:
+            err, kind = rt.cudaGraphNodeGetType(node)
+            if err != rt.cudaError_t.cudaSuccess:
+                return None
+            count += int(kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+        return count
+    except Exception:
+        return None
 
 
 def config_of(wl, world: int, flush_mib: int) -> dict:
@@ -426,8 +453,8 @@ def run_gpu(args):
     torch.cuda.synchronize()
     assert fq.device_error(clear=True) == 0
 
-    def capture(fns):
-        g = torch.cuda.CUDAGraph()
+    def capture(fns, keep=False):
+        g = torch.cuda.CUDAGraph(keep_graph=keep)
         side = torch.cuda.Stream(dev)
         side.wait_stream(stream)
         with torch.cuda.stream(side):
@@ -441,11 +468,17 @@ def run_gpu(args):
     # The step as one CUDA graph (kernels of consecutive ops overlap their
     # launch through programmatic dependent launch); each op also as its own
     # graph, timed alone for the per-kernel figures.
+    launches_per_step = len(xs_shapes) + sum(launches_of(g, sms) for g in wl.gemms)
+    launches_source = "the library's dispatch rule, restated (decode_reduce_launched)"
     if args.eager:
         step_runner = lambda: [op() for op in ops]
         op_runners = ops
     else:
-        step_graph = capture(ops)
+        step_graph = capture(ops, keep=True)    # kept, to count its kernel nodes
+        counted = graph_kernel_nodes(step_graph)
+        if counted is not None:
+            launches_per_step, launches_source = counted, "kernel nodes of the captured step graph"
+        step_graph.instantiate()
         op_graphs = [capture([op]) for op in ops]
         step_runner = step_graph.replay
         op_runners = [g.replay for g in op_graphs]
@@ -930,7 +963,8 @@ def run_gpu(args):
             "so every launch reads from DRAM) / R, after an L2 flush; ms_isolated = one launch in its own graph "
             "after an L2 flush, which ms reports (back_to_back = 1) for ops of 0.25 ms or more",
             "roofline": roof, "rooflines": rooflines, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps * (len(xs_shapes) + sum(launches_of(g, sms) for g in wl.gemms)),
+            "gpu_launches": args.steps * launches_per_step,
+            "gpu_launches_source": launches_source,
             "clocks": dict(clk.summary(), measured=mon.summary()), "detail": detail, "weight_quant": weight_quant, "rmsnorm_quant": rms, "kv_quant": kvq, "swiglu": swiglu, "quant_static": qstatic, "w8a16": w8a16,
             "merged_shared_input": merged,
             "device_error": err, "gpu": torch.cuda.get_device_name(dev),

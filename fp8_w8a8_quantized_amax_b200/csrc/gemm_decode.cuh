@@ -178,8 +178,11 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
   // writes (and L2 is coherent if they were), so their DRAM latency overlaps
   // its tail.  The epilogue warps issue them (every fourth step each; they
   // have nothing to do until the first accumulator is ready), so that the
-  // producer's first load is not queued behind them.
-  if (warp >= 2 && warp < 6 && lane == 0) {
+  // producer's first load is not queued behind them.  Only where the range
+  // is longer than the stages: where the producer issues every load of the
+  // range at once, the doubled requests measured slower (3B FP8-Block shapes,
+  // ~1 us), while longer ranges gain (70B gate/qkv, 0.5-1 us back to back).
+  if (warp >= 2 && warp < 6 && lane == 0 && e - b > STAGES) {
     int i = 0;
     for (StepIter it(b, e, p.KB); it.valid() && i < STAGES; it.next(), ++i)
       if ((i & 3) == warp - 2) tma_prefetch_l2_2d(&tmW, it.kb * BK, it.t * 128);
@@ -433,15 +436,17 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
             for (int j = 0; j < NX; ++j) acc[j] = 0.0f;
             continue;                              // summed by decode_reduce_kernel
           }
-          __threadfence();
+          // publish: the warp's partial stores, then one acquire-release
+          // increment (a release of the stores the __syncwarp ordered before
+          // it, and for the last arriver an acquire of everyone else's)
           __syncwarp();
           const int c0 = cta_of_step(tile_first, sp);
           const int c1 = cta_of_step(tile_first + p.KB - 1, sp);
           unsigned int prev = 0;
-          if (lane == 0) prev = atomicAdd(p.count + t * 4 + quarter, 1u);
+          if (lane == 0) prev = atom_add_acq_rel_gpu(p.count + t * 4 + quarter, 1u);
           prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+          __syncwarp();                            // the other lanes' loads come after the acquire
           if (prev == static_cast<unsigned int>(c1 - c0)) {   // every other segment is in
-            __threadfence();
             // acc is published; it now collects the tile's sum in CTA order,
             // the partial sums of kBatch CTAs loaded at once (one L2 round
             // trip per batch; the +0 of an absent CTA changes no sum, which
@@ -515,7 +520,7 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
           }
       }
     }
-    cluster_sync();   // rank 0 has read every partial tile before any CTA leaves
+    cluster_sync_relaxed();   // rank 0 has read every partial tile before any CTA leaves
   }
   tc_fence_before();
   __syncthreads();

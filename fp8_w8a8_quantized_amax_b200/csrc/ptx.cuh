@@ -203,6 +203,23 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// The same barrier without memory ordering: only that every thread of the
+// cluster has reached it (so every instruction before it has executed: a
+// load whose value was used has completed).  The release form would also wait
+// until the CTA's earlier global stores are visible to the cluster.
+__device__ __forceinline__ void cluster_sync_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// atomicAdd at GPU scope with acquire-release semantics: the caller's earlier
+// writes (and those ordered before them, such as its warp's writes before a
+// __syncwarp) are visible to a thread that observes the new count, and the
+// caller's later reads see what the earlier incrementers published.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 
 // Address, in the cluster shared window, of the variable at `local_addr` in CTA `rank`.
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {

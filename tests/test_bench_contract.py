@@ -70,3 +70,21 @@ def test_reference_arm_under_torchrun_prints_once_from_rank_0():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2
+
+
+def test_launch_count_rule_follows_the_decode_dispatch():
+    # the fallback count of the bench's gpu_launches (used where the step graph
+    # cannot be inspected): the FP8-Block decode shapes of Llama-3.2-3B take
+    # cluster split-K (one kernel); a few-tile block problem, and channel mode
+    # with 64 tokens on few steps per CTA, add the reduction kernel
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    G = lambda M, N, K, mode: synth.Gemm(name="g", M=M, N=N, K=K, mode=mode, x="x", w="w")
+    for M in (1, 16):
+        for N, K in ((8192, 3072), (5120, 3072), (3072, 8192)):
+            assert bench.launches_of(G(M, N, K, synth.BLOCK128), 148) == 1, (M, N, K)
+    assert bench.launches_of(G(16, 1024, 2048, synth.BLOCK128), 148) == 2
+    assert bench.launches_of(G(8, 28672, 8192, synth.CHANNEL_TOKEN), 148) == 1
+    assert bench.launches_of(G(64, 1024, 1024, synth.CHANNEL_TOKEN), 148) == 2
+    assert bench.launches_of(G(512, 28672, 8192, synth.CHANNEL_TOKEN), 148) == 1

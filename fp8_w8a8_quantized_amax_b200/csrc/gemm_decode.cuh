@@ -369,6 +369,46 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
       seg_len = it.seg_first() ? 1 : seg_len + 1;
       const bool seg_last = it.seg_last();
       if (!BLOCK && !seg_last) continue;           // channel mode: one drain per segment
+      // channel mode: the channel's w_scale is loaded before the wait for the
+      // accumulator, so that scaling the output never waits on a DRAM load
+      float wn_pre = 1.0f;
+      if constexpr (!BLOCK) {
+        const int n0 = t * 128 + nl;
+        if (n0 < p.N) wn_pre = __ldg(p.ws + n0);
+      }
+      // In-kernel sums, a partial segment's last step: if every other CTA of
+      // the tile has already published its part (an acquire load of the
+      // counter), this warp is the tile's last contributor for certain.  It
+      // then loads their partial sums now, while its own MMAs finish, and
+      // later adds them to its own in CTA order without publishing anything:
+      // the same sums in the same order as the last arriver's, off the end
+      // of the kernel's critical path.
+      constexpr int kPre = SUMS == kSumsKernel ? (NX == 16 ? 3 : (NX == 32 ? 1 : 0)) : 0;
+      bool known_last = false;
+      float pre[kPre > 0 ? kPre + 1 : 1][NX];      // by position in c0..c0+kPre (own and absent: 0)
+      if constexpr (kPre > 0) {
+        if (seg_last && seg_len != p.KB) {
+          const int c0 = cta_of_step(t * p.KB, sp);
+          const int c1 = cta_of_step(t * p.KB + p.KB - 1, sp);
+          if (c1 - c0 <= kPre) {
+            unsigned int cnt = 0;
+            if (lane == 0) cnt = ld_acquire_gpu(p.count + t * 4 + quarter);
+            cnt = __shfl_sync(0xFFFFFFFFu, cnt, 0);
+            __syncwarp();                          // the other lanes' loads come after the acquire
+            known_last = cnt == static_cast<unsigned int>(c1 - c0);
+            if (known_last) {
+#pragma unroll
+              for (int u = 0; u <= kPre; ++u) {
+                const int cc = c0 + u;
+                const float* src = p.part + (static_cast<int64_t>(t) + cc) * NX * 128 + nl;
+#pragma unroll
+                for (int j = 0; j < NX; ++j)
+                  pre[u][j] = (cc != c && cc <= c1 && j < p.M) ? __ldcg(src + j * 128) : 0.0f;
+              }
+            }
+          }
+        }
+      }
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sfull[slot], sphase, abort_flag, kErrWaitTmemFull))) break;
       tc_fence_after();
       uint32_t r[NX];
@@ -407,7 +447,7 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
         // bf16 output of channel n for the token sums v[j]
         auto emit = [&](const float (&v)[NX]) {
           if (n < p.N) {
-            const float wn = BLOCK ? 1.0f : __ldg(p.ws + n);
+            const float wn = wn_pre;
 #pragma unroll
             for (int j = 0; j < NX; ++j) {
               if (j < p.M) {
@@ -419,6 +459,30 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
         };
         if (seg_len == p.KB) {                     // the whole tile: no partial sums
           emit(acc);
+        } else if (kPre > 0 && known_last) {
+          // every other part is in (loaded above): add the parts in CTA order,
+          // clear what was read, write the tile, reset the counter
+          const int c0 = cta_of_step(tile_first, sp);
+          const int c1 = cta_of_step(tile_first + p.KB - 1, sp);
+          float sum[NX];
+#pragma unroll
+          for (int j = 0; j < NX; ++j) sum[j] = 0.0f;
+#pragma unroll
+          for (int u = 0; u <= kPre; ++u) {            // position u of c0..c1 (the +0 of an absent one changes no sum)
+            const bool own = c0 + u == c;
+#pragma unroll
+            for (int j = 0; j < NX; ++j) sum[j] += own ? acc[j] : pre[u][j];
+          }
+          for (int cc = c0; cc <= c1; ++cc) {
+            if (cc == c) continue;
+            float* src = p.part + (static_cast<int64_t>(t) + cc) * NX * 128 + nl;
+#pragma unroll
+            for (int j = 0; j < NX; ++j)
+              if (j < p.M) src[j * 128] = 0.0f;
+          }
+          emit(sum);
+          __syncwarp();
+          if (lane == 0) p.count[t * 4 + quarter] = 0u;
         } else if constexpr (SUMS == kSumsCluster) {
           // the CTA's one segment: every MMA has completed (this slot was the
           // last one committed) and every stage has been consumed, so the

@@ -211,6 +211,14 @@ __device__ __forceinline__ void cluster_sync_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 
+// A 32-bit load with acquire semantics at GPU scope (pairs with the release
+// of atom_add_acq_rel_gpu).
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // atomicAdd at GPU scope with acquire-release semantics: the caller's earlier
 // writes (and those ordered before them, such as its warp's writes before a
 // __syncwarp) are visible to a thread that observes the new count, and the

@@ -512,9 +512,11 @@ fp8q_status prefill_pairs(bool block, int dev, int sms, int* out) {
 // keeps under 92% of the pairs busy).  Not the default: measured on the
 // B200 it is slower on every such Llama shape (70B M=512 gate/up 0.67 against
 // 0.74 of the FP8 peak, down 0.66 against 0.83, qkv 0.47 against 0.54; 8B
-// k/v at M=8192 0.51 against 0.71), because pairs working on different K
-// ranges no longer share operand tiles through L2 at the same time, and these
-// shapes are close to the HBM ridge.
+// k/v at M=8192 0.51 against 0.71).  Likely costs: pairs working on different
+// K ranges no longer share operand tiles through L2 at the same time, and a
+// tile cut over many pairs is summed by one pair that reads every other pair's
+// 256 x 256 fp32 partial alone (a variant that kept whole rounds data-parallel
+// and cut only the last round's tiles by steps was slower still).
 bool prefill_streamk(int num_tiles, int pairs) {
   static bool on = [] {
     const char* e = getenv("FP8Q_PREFILL_STREAMK");

@@ -393,11 +393,8 @@ __global__ void __launch_bounds__(256) quant_groups128_kernel(const uint16_t* __
 #pragma unroll
     for (int i = 0; i < GPT; ++i) {
       if (mi[i] < Mu) {  // uniform across the half warp
-        uint32_t am = fold_halves(absmax_bits_vec(v[i], 0u));
-        am = max(am, __shfl_xor_sync(half_mask, am, 8, 16));
-        am = max(am, __shfl_xor_sync(half_mask, am, 4, 16));
-        am = max(am, __shfl_xor_sync(half_mask, am, 2, 16));
-        am = max(am, __shfl_xor_sync(half_mask, am, 1, 16));
+        // the half warp's max (each half warp reduces over its own 16 lanes)
+        const uint32_t am = __reduce_max_sync(half_mask, fold_halves(absmax_bits_vec(v[i], 0u)));
         float sc = scale_of(amax_bits_to_float(am));
         if (s16) sc = scale_bf16(sc);
         if (sub == 0) s[static_cast<int64_t>(mi[i]) * Gu + gi[i]] = sc;

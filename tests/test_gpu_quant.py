@@ -136,6 +136,36 @@ def test_every_bf16_pair_matches_ieee_division():
                                  f"IEEE division {int(q_ref[r, c]):#04x} ({int(bad.sum())} differ in this chunk)")
 
 
+def test_groups_every_bf16_pair_matches_ieee_division():
+    """The per-128-group quantizer (scale and reciprocal from tables of the
+    amax's mantissa for amax >= 2^-117, by division below) against torch's IEEE
+    fp32 division and fp8 cast: for every positive finite bf16 amax, groups
+    holding amax first and then every bf16 x with |x| <= amax (127 per group,
+    both signs, zeros and subnormals included)."""
+    allv = torch.arange(65536, dtype=torch.int32).to(torch.int16).view(torch.bfloat16).to(DEV)
+    allv = torch.where(torch.isfinite(allv.float()), allv, torch.zeros_like(allv))
+    amax_bits = torch.arange(1, 0x7F80, dtype=torch.int32, device=DEV)   # +subnormals .. max finite
+    G = -(-65536 // 127)                                                  # groups per amax
+    pad = G * 127 - 65536
+    chunk = 512
+    for lo in range(0, amax_bits.numel(), chunk):
+        a = amax_bits[lo:lo + chunk].to(torch.int16).view(torch.bfloat16)
+        R = a.numel()
+        keep = allv.float().abs()[None, :] <= a.float()[:, None]
+        vals = torch.where(keep, allv[None, :], torch.zeros((), dtype=torch.bfloat16, device=DEV))
+        vals = torch.cat([vals, torch.zeros((R, pad), dtype=torch.bfloat16, device=DEV)], dim=1).view(R, G, 127)
+        x = torch.cat([a.view(R, 1, 1).expand(R, G, 1), vals], dim=2).reshape(R, G * 128)
+        q, s = fq.fp8_quant_act(x, fq.BLOCK128)
+        s_ref = (a.float() / torch.full((R,), 448.0, device=DEV))[:, None].expand(R, G)
+        assert torch.equal(s.view(torch.int32), s_ref.contiguous().view(torch.int32)), f"scales differ in rows {lo}.."
+        q_ref = (x.float().view(R, G, 128) / s_ref[:, :, None]).to(torch.float8_e4m3fn).view(torch.uint8).view(R, -1)
+        bad = q != q_ref
+        if bad.any():
+            r, c = bad.nonzero()[0].tolist()
+            raise AssertionError(f"amax {float(a[r])}: x {float(x[r, c])} gives {int(q[r, c]):#04x}, "
+                                 f"IEEE division {int(q_ref[r, c]):#04x} ({int(bad.sum())} differ in this chunk)")
+
+
 @pytest.mark.parametrize("T,H", [(1, 8), (37, 8), (8192, 8), (513, 2)])
 def test_kv_cache_per_token_per_head(T, H):
     # one scale per (token, head) of a [T, H, 128] K or V tensor: each head is a

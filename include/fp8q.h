@@ -180,7 +180,8 @@ FP8Q_API fp8q_status fp8_rmsnorm_quant_act(const void* X_bf16, const void* gamma
  *             bytes, 16-byte aligned (may be NULL when that size is 0).  For
  *             M <= 64 it is required: a NULL or misaligned one is refused
  *             before anything touches the device.  For M > 64 it is optional:
- *             a nonzero size means the stream-K prefill schedule pays for this
+ *             a nonzero size means the stream-K prefill schedule is switched
+ *             on (environment FP8Q_PREFILL_STREAMK=1; off by default) for this
  *             shape (channel mode, few 256 x 256 tiles per CTA pair) and runs
  *             when the workspace is given; without it (NULL, or shorter) the
  *             data-parallel schedule runs, with the same result up to the
@@ -198,8 +199,11 @@ FP8Q_API fp8q_status fp8_rmsnorm_quant_act(const void* X_bf16, const void* gamma
  *   Dispatch: M <= 64 takes the decode kernel (weights streamed once, swap-AB,
  *   stream-K split over all SMs; the last warp to finish a weight tile's
  *   channels adds its partial sums in a fixed order, so results are
- *   deterministic); larger M takes the persistent warp-specialised prefill
- *   kernels, with 256 x 256 tiles per CTA pair, data-parallel or stream-K
+ *   deterministic; small block-scaled problems split each weight tile's K over
+ *   the CTAs of one thread-block cluster instead, summed in distributed shared
+ *   memory, and leave the workspace untouched); larger M takes the
+ *   persistent warp-specialised prefill kernels, with 256 x 256 tiles per CTA
+ *   pair, data-parallel or stream-K
  *   (parts of a tile summed in a fixed order by the last pair to finish it).
  */
 FP8Q_API fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq,

@@ -366,11 +366,42 @@ int decode_cluster_size(const Params& p, int sms, int dev, bool forced) {
   return 0;
 }
 
+// Half the stages (and at most two CTAs' worth of registers, so the early
+// loads of the last contributor's partners are left out) let two decode CTAs
+// share an SM: the next kernel's CTAs start beside this kernel's last ones
+// (programmatic dependent launch), so their set-up and first loads overlap
+// its tail.  Measured on the Llama-3.1-70B decode shapes back to back, with
+// 16-token tiles: qkv 0.567 -> 0.594 of HBM at M=1, down 0.73 -> 0.75,
+// gate/up unchanged, the 3B FP8-Block M=1/16 0.37 -> 0.38; with 64-token
+// tiles (4 stages, and two CTAs no longer fit in tensor memory) slower: down
+// 0.67 -> 0.50, qkv 0.46 -> 0.35.  So by default 16-token tiles only.
+// FP8Q_DECODE_STAGES=full|half (read once) forces one form for every tile.
+bool decode_half_stages(int nx) {
+  static int choice = [] {
+    const char* e = getenv("FP8Q_DECODE_STAGES");
+    if (e && strcmp(e, "full") == 0) return 1;
+    if (e && strcmp(e, "half") == 0) return 2;
+    return 0;
+  }();
+  return choice == 2 || (choice == 0 && nx == 16);
+}
+
+template <int NX, int kDecodeStages, int MINB>
+fp8q_status launch_decode_nx_s(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p, int mode, int dev,
+                               int sms, void* stream);
+
 template <int NX>
 fp8q_status launch_decode_nx(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p, int mode, int dev,
                              int sms, void* stream) {
+  if (decode_half_stages(NX))
+    return launch_decode_nx_s<NX, decode_stages<NX>() / 2, 2>(tw, tx, p, mode, dev, sms, stream);
+  return launch_decode_nx_s<NX, decode_stages<NX>(), 1>(tw, tx, p, mode, dev, sms, stream);
+}
+
+template <int NX, int kDecodeStages, int MINB>
+fp8q_status launch_decode_nx_s(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p, int mode, int dev,
+                               int sms, void* stream) {
   using namespace fp8q::decode;
-  constexpr int kDecodeStages = decode_stages<NX>();
   using L = Layout<NX, kDecodeStages>;
   fp8q_status st;
   const bool block = mode == FP8Q_BLOCK128;
@@ -378,8 +409,8 @@ fp8q_status launch_decode_nx(const CUtensorMap& tw, const CUtensorMap& tx, const
   if (forced == kSumsCluster || (forced < 0 && block)) {
     const int C = decode_cluster_size<NX>(p, sms, dev, forced == kSumsCluster);
     if (C >= 2) {
-      auto k = block ? gemm_decode_kernel<NX, kDecodeStages, true, kSumsCluster>
-                     : gemm_decode_kernel<NX, kDecodeStages, false, kSumsCluster>;
+      auto k = block ? gemm_decode_kernel<NX, kDecodeStages, true, kSumsCluster, 0, MINB>
+                     : gemm_decode_kernel<NX, kDecodeStages, false, kSumsCluster, 0, MINB>;
       if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
       Params q = p;
       q.G = p.n_tiles * C;
@@ -389,13 +420,13 @@ fp8q_status launch_decode_nx(const CUtensorMap& tw, const CUtensorMap& tx, const
   const bool in_kernel = forced == kSumsKernel ||
                          (forced != kSumsSeparate && !block && (NX == 16 || p.total >= static_cast<int64_t>(p.KB) * p.G));
   if (in_kernel) {
-    auto k = block ? gemm_decode_kernel<NX, kDecodeStages, true, kSumsKernel>
-                   : gemm_decode_kernel<NX, kDecodeStages, false, kSumsKernel>;
+    auto k = block ? gemm_decode_kernel<NX, kDecodeStages, true, kSumsKernel, 0, MINB>
+                   : gemm_decode_kernel<NX, kDecodeStages, false, kSumsKernel, 0, MINB>;
     if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
     return launch(k, dim3(p.G), dim3(192), L::kBytes, stream, tw, tx, p);
   }
-  auto k = block ? gemm_decode_kernel<NX, kDecodeStages, true, kSumsSeparate>
-                 : gemm_decode_kernel<NX, kDecodeStages, false, kSumsSeparate>;
+  auto k = block ? gemm_decode_kernel<NX, kDecodeStages, true, kSumsSeparate, 0, MINB>
+                 : gemm_decode_kernel<NX, kDecodeStages, false, kSumsSeparate, 0, MINB>;
   if ((st = ensure_smem(k, L::kBytes, dev)) != FP8Q_OK) return st;
   if ((st = launch(k, dim3(p.G), dim3(192), L::kBytes, stream, tw, tx, p)) != FP8Q_OK) return st;
   auto r = block ? fp8q::decode::decode_reduce_kernel<true> : fp8q::decode::decode_reduce_kernel<false>;

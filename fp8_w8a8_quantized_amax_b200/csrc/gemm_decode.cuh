@@ -110,8 +110,11 @@ struct Layout {
   static constexpr uint32_t kTmemCols = (kSlots * NX) < 32 ? 32 : (kSlots * NX);
 };
 
-template <int NX, int STAGES, bool BLOCK, int SUMS, int WIDEN = 0>
-__global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
+// MINB = 2: built to fit two CTAs per SM (registers; the caller picks stages
+// that fit two in shared memory), so that the next kernel's CTAs can start
+// beside this one's while it finishes.
+template <int NX, int STAGES, bool BLOCK, int SUMS, int WIDEN = 0, int MINB = 1>
+__global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, MINB)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const Params p) {
   using L = Layout<NX, STAGES, WIDEN>;
@@ -383,7 +386,7 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, 1)
       // later adds them to its own in CTA order without publishing anything:
       // the same sums in the same order as the last arriver's, off the end
       // of the kernel's critical path.
-      constexpr int kPre = SUMS == kSumsKernel ? (NX == 16 ? 3 : (NX == 32 ? 1 : 0)) : 0;
+      constexpr int kPre = (SUMS == kSumsKernel && MINB == 1) ? (NX == 16 ? 3 : (NX == 32 ? 1 : 0)) : 0;
       bool known_last = false;
       float pre[kPre > 0 ? kPre + 1 : 1][NX];      // by position in c0..c0+kPre (own and absent: 0)
       if constexpr (kPre > 0) {

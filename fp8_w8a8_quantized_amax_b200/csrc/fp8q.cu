@@ -294,6 +294,27 @@ fp8q_status check_linear_args(const uint8_t* Xq, const float* xs, const uint8_t*
   return FP8Q_OK;
 }
 
+// In-kernel sums: a warp that finds every other part of its tile already in
+// loads them while its own MMAs finish (gemm_decode.cuh).  Measured on the
+// 70B decode shapes on one box (back to back), it pays where every CTA streams
+// at least a tile's worth of K blocks (gate/up: 0.76 -> 0.78 of HBM) and costs
+// where the ranges are shorter than a tile (qkv 0.59 -> 0.58, down 0.74 ->
+// 0.735): there the counter read sits in front of most segments' drains.
+// FP8Q_DECODE_EARLY=0|1 forces it off or on (read once).
+int decode_early_forced() {
+  static int v = [] {
+    const char* e = getenv("FP8Q_DECODE_EARLY");
+    if (e && strcmp(e, "0") == 0) return 0;
+    if (e && strcmp(e, "1") == 0) return 1;
+    return -1;
+  }();
+  return v;
+}
+bool decode_early(int64_t total, int G, int KB) {
+  const int f = decode_early_forced();
+  return f >= 0 ? f == 1 : total / G >= KB;
+}
+
 // Where the decode kernel's split weight tiles are summed (gemm_decode.cuh).
 // Measured on the Llama-3.1-70B and -3.2-3B decode shapes: in channel mode
 // with up to 16 tokens the in-kernel sums (last arriver) are cheap enough to
@@ -712,7 +733,8 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
     CUtensorMap tw, tx;
     if ((st = tmap_u8_sw128(&tw, Wq, N, K, K, 128)) != FP8Q_OK) return st;
     if ((st = tmap_u8_sw128(&tx, Xq, M, K, K, static_cast<uint32_t>(nx))) != FP8Q_OK) return st;
-    Params p;
+    Params p{};
+    p.early = decode_early(total, G, KB) ? 1 : 0;
     p.xs = x_scale;
     p.ws = w_scale;
     p.M = static_cast<int>(M);
@@ -920,7 +942,8 @@ fp8q_status fp8_linear_w8a16(const void* X_bf16, int64_t ldx, const uint8_t* Wq,
   CUtensorMap tw, tx;
   if ((st = tmap_u8_sw128(&tw, Wq, N, K, K, 128)) != FP8Q_OK) return st;
   if ((st = tmap_bf16_sw128(&tx, X_bf16, M, K, ldx, static_cast<uint32_t>(nx))) != FP8Q_OK) return st;
-  Params p;
+  Params p{};
+  p.early = decode_early(total, G, static_cast<int>((K + 127) / 128)) ? 1 : 0;
   p.xs = nullptr;
   p.ws = w_scale;
   p.M = static_cast<int>(M);
@@ -1048,7 +1071,8 @@ fp8q_status fp8_linear_noalloc(const uint8_t* Xq, const float* x_scale, const ui
   CUtensorMap tw, tx;
   if ((st = tmap_u8_sw128(&tw, Wq, N, K, K, 128)) != FP8Q_OK) return st;
   if ((st = tmap_u8_sw128(&tx, Xq, M, K, K, static_cast<uint32_t>(nx))) != FP8Q_OK) return st;
-  Params p;
+  Params p{};
+  p.early = decode_early(total, G, static_cast<int>((K + 127) / 128)) ? 1 : 0;
   p.xs = x_scale;
   p.ws = w_scale;
   p.M = static_cast<int>(M);

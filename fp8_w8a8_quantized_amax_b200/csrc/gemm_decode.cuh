@@ -84,6 +84,7 @@ struct Params {
   int n_tiles;
   int total;            // n_tiles * KB (the host refuses 2^31 or more)
   int G;                // CTAs (cluster split-K: n_tiles * cluster size)
+  int early;            // in-kernel sums: a known last contributor loads its partners' sums early
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -386,11 +387,15 @@ __global__ void __launch_bounds__(Layout<NX, STAGES, WIDEN>::kThreads, MINB)
       // later adds them to its own in CTA order without publishing anything:
       // the same sums in the same order as the last arriver's, off the end
       // of the kernel's critical path.
-      constexpr int kPre = (SUMS == kSumsKernel && MINB == 1) ? (NX == 16 ? 3 : (NX == 32 ? 1 : 0)) : 0;
+      // (at most 168 registers when built for two CTAs per SM: up to two
+      // partners, channel scales)
+      constexpr int kPre = SUMS != kSumsKernel ? 0
+                           : MINB == 1 ? (NX == 16 ? 3 : (NX == 32 ? 1 : 0))
+                                       : ((NX == 16 && !BLOCK) ? 2 : 0);
       bool known_last = false;
       float pre[kPre > 0 ? kPre + 1 : 1][NX];      // by position in c0..c0+kPre (own and absent: 0)
       if constexpr (kPre > 0) {
-        if (seg_last && seg_len != p.KB) {
+        if (p.early && seg_last && seg_len != p.KB) {
           const int c0 = cta_of_step(t * p.KB, sp);
           const int c1 = cta_of_step(t * p.KB + p.KB - 1, sp);
           if (c1 - c0 <= kPre) {

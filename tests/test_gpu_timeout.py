@@ -133,3 +133,34 @@ def test_undelivered_split_sums_and_recovery(T, noalloc):
         torch.cuda.synchronize()
         assert T.fp8q_device_error(0) == 0
         assert torch.equal(y.view(torch.int16), fq.fp8_linear(*ops2, mode).view(torch.int16)), f"seed {seed}"
+
+
+# Cluster split-K (the Llama-3.2-3B FP8-Block gate/up decode shape: 64 weight
+# tiles, clusters of 2 CTAs, 12 K blocks each): CTA 0, rank 0 of its cluster,
+# withholds its first slot release (its MMA warp comes back to slot 0 at the
+# ninth K block) or its first accumulator commit.  Its partner finishes and
+# waits at the cluster barrier, which CTA 0 reaches after its own bounded
+# waits have run out and its loads and MMAs have drained.
+CLUSTER = (16, 8192, 3072, fq.BLOCK128)
+
+
+@pytest.mark.parametrize("withhold,sites", [(WITHHOLD_RELEASE, RELEASE_SITES), (WITHHOLD_COMMIT, (ERR_WAIT_TMEM_FULL,))],
+                         ids=["release", "commit"])
+def test_cluster_path_wait_runs_out_and_the_next_call_is_correct(T, withhold, sites):
+    M, N, K, mode = CLUSTER
+    ops = _operands(M, N, K, mode)
+    ref = fq.fp8_linear(*ops, mode)
+    nws = T.fp8_linear_workspace_size(M, N, K, mode)
+    assert T.fp8q_test_withhold(withhold) == 0
+    _call(T, ops, mode, N, torch.zeros(nws, dtype=torch.uint8, device=DEV))
+    site = T.fp8q_device_error(0)
+    assert site in sites, hex(site)
+    assert T.fp8q_test_withhold(0) == 0
+    assert T.fp8q_device_error(1) == site
+    for seed in (0, 1):
+        ops2 = ops if seed == 0 else _operands(M, N, K, mode, seed=seed)
+        y = _call(T, ops2, mode, N, torch.zeros(nws, dtype=torch.uint8, device=DEV))
+        torch.cuda.synchronize()
+        assert T.fp8q_device_error(0) == 0
+        want = ref if seed == 0 else fq.fp8_linear(*ops2, mode)
+        assert torch.equal(y.view(torch.int16), want.view(torch.int16)), f"seed {seed}"

@@ -373,8 +373,11 @@ int decode_max_clusters(int C, int dev, int sms) {
 
 // Cluster size for cluster split-K, or 0: C in [2, 8], at most KB (every CTA
 // gets a K block) and at most sms / n_tiles, the largest whose n_tiles
-// clusters the device holds at once; by default only where those
-// n_tiles * C CTAs fill at least 3/4 of the SMs.
+// clusters the device holds at once (asked of the one-CTA-per-SM build, so
+// that every CTA of a cluster gets an SM of its own); by default only where
+// those n_tiles * C CTAs fill at least 3/4 of the SMs.  Clusters twice as
+// large, planned for two CTAs per SM, measured slower on the 3B FP8-Block
+// decode shapes (0.38 -> 0.35 of HBM).
 template <int NX>
 int decode_cluster_size(const Params& p, int sms, int dev, bool forced) {
   int C = sms / p.n_tiles;

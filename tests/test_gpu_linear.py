@@ -204,6 +204,28 @@ def test_decode_sums_forced(sums, M, N, K, mode):
     assert r.returncode == 0, r.stdout + r.stderr
 
 
+@pytest.mark.parametrize("env,M,N,K,mode", [
+    ({"FP8Q_DECODE_STAGES": "full"}, 8, 4096, 4096, fq.CHANNEL_TOKEN),   # 16-token tiles, one CTA per SM
+    ({"FP8Q_DECODE_STAGES": "full"}, 16, 8192, 3072, fq.BLOCK128),       # ... on the cluster path
+    ({"FP8Q_DECODE_STAGES": "half"}, 32, 2048, 4096, fq.CHANNEL_TOKEN),  # 32-token tiles, two CTAs per SM
+    ({"FP8Q_DECODE_STAGES": "half"}, 64, 1024, 8192, fq.CHANNEL_TOKEN),  # 64-token tiles, two CTAs per SM
+    ({"FP8Q_DECODE_EARLY": "1"}, 1, 10240, 8192, fq.CHANNEL_TOKEN),      # early loads where ranges are shorter than a tile
+    ({"FP8Q_DECODE_EARLY": "0"}, 8, 20480, 1024, fq.CHANNEL_TOKEN),      # none where they are longer
+    ({"FP8Q_DECODE_EARLY": "1", "FP8Q_DECODE_STAGES": "full"}, 4, 10240, 8192, fq.CHANNEL_TOKEN),
+])
+def test_decode_builds_forced(env, M, N, K, mode):
+    # the decode kernel's other builds (one or two CTAs per SM, early loads of
+    # a known last contributor on or off), forced on shapes the default
+    # dispatch gives another; three calls on one workspace
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-m", "tests._forced_kernel", "decode", str(M), str(N), str(K), str(mode)],
+                       cwd=root, env=dict(os.environ, **env), capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
 def test_decode_workspace_left_reusable():
     # The workspace is all zero again after every call, so one zero-filled
     # buffer serves calls of different shapes and modes in a row (a later call

@@ -628,14 +628,23 @@ fp8q_status fp8_quant_act(const void* X_bf16, int64_t M, int64_t K, int64_t ldx,
   mode &= ~FP8Q_SCALE_BF16;
   if (mode == FP8Q_CHANNEL_TOKEN)
     return launch_rows(x, M, static_cast<int>(K), ldx, Xq, ldxq, x_scale, s16, stream);
-  constexpr int GPT = 4;
   const int G = static_cast<int>(K / 128);
   const int64_t total = M * G;
   if (total >= (static_cast<int64_t>(1) << 31)) return FP8Q_ERR_UNSUPPORTED;   // 32-bit group walk
-  int64_t grid = (total + 16 * GPT - 1) / (16 * GPT);
-  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
-  return launch(fp8q::quant_groups128_kernel<GPT>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream, x, M,
-                G, ldx, Xq, ldxq, x_scale, s16);
+  // Groups per half warp: 4, or 6 or 8 where that lets one pass of the
+  // resident CTAs (8 of 256 threads per SM) cover every group, so that no half
+  // warp waits on a second DRAM round trip.
+  const int64_t resident = static_cast<int64_t>(sms) * 8;
+  int gpt = 4;
+  if ((total + 63) / 64 > resident) gpt = (total + 95) / 96 <= resident ? 6 : 8;
+  int64_t grid = (total + 16 * gpt - 1) / (16 * gpt);
+  if (grid > resident) grid = resident;
+  const dim3 g1(static_cast<unsigned>(grid));
+  if (gpt == 4)
+    return launch(fp8q::quant_groups128_kernel<4>, g1, dim3(256), 0, stream, x, M, G, ldx, Xq, ldxq, x_scale, s16);
+  if (gpt == 6)
+    return launch(fp8q::quant_groups128_kernel<6>, g1, dim3(256), 0, stream, x, M, G, ldx, Xq, ldxq, x_scale, s16);
+  return launch(fp8q::quant_groups128_kernel<8>, g1, dim3(256), 0, stream, x, M, G, ldx, Xq, ldxq, x_scale, s16);
 }
 
 fp8q_status fp8_rmsnorm_quant_act(const void* X_bf16, const void* gamma_bf16, int64_t M, int64_t K, int64_t ldx,

@@ -36,7 +36,10 @@ def test_rows_bit_exact(M, K):
     P.assert_scales_equal(s, rs, f"rows {M}x{K}")
 
 
-@pytest.mark.parametrize("M,K", [(1, 128), (5, 384), (33, 3072), (300, 256)])
+@pytest.mark.parametrize("M,K", [(1, 128), (5, 384), (33, 3072), (300, 256),
+                                 (4100, 3072),    # 98,400 groups: 6 per half warp, one pass on 148 SMs
+                                 (5000, 3072),    # 120,000 groups: 8 per half warp, one pass
+                                 (9000, 3072)])   # 216,000 groups: 8 per half warp, a second pass
 def test_groups_bit_exact(M, K):
     x = synth.make_x(M, K, seed=7 * M + K)
     q, s = fq.fp8_quant_act(x.to(DEV), fq.BLOCK128)

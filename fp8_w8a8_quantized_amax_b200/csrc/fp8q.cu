@@ -255,12 +255,24 @@ constexpr int kDecodeMaxM = 64;
 
 int decode_nx(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
-void decode_shape(int64_t M, int64_t N, int64_t K, int sms, int* n_tiles, int64_t* total, int* G, int* nx) {
+bool decode_half_stages(int nx);
+
+// Stream-K split of a small-M problem: n_tiles weight tiles of 128 rows, KB K
+// blocks each, over G CTAs, one per SM.  Where the kernel is built for two
+// CTAs per SM (`two_per_sm`), KB is even and twice the tile count lies
+// between the SM count and 5/4 of it, G = 2 * n_tiles instead: every CTA
+// streams exactly half a tile.  Measured on the Llama-3.1-70B qkv_proj (80
+// tiles: 160 CTAs of 32 K blocks instead of 148 of 34-35 whose ranges cross
+// tiles), 0.59 -> 0.62 of HBM at M = 1 and 0.58 -> 0.61 at M = 8; the other
+// 70B decode shapes do not take it.
+void decode_shape(int64_t M, int64_t N, int64_t K, int sms, bool two_per_sm, int* n_tiles, int64_t* total, int* G,
+                  int* nx) {
   const int KB = static_cast<int>((K + 127) / 128);
   *n_tiles = static_cast<int>((N + 127) / 128);
   *total = static_cast<int64_t>(*n_tiles) * KB;
   *G = static_cast<int>(*total < sms ? *total : sms);
   *nx = decode_nx(M);
+  if (two_per_sm && KB % 2 == 0 && 2 * *n_tiles > sms && 8 * *n_tiles <= 5 * sms) *G = 2 * *n_tiles;
 }
 
 // Decode workspace: [n_tiles][4] arrival counters, padded to 16 bytes, then
@@ -718,7 +730,7 @@ size_t fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K, int mode) {
   }
   int n_tiles, G, nx;
   int64_t total;
-  decode_shape(M, N, K, sms, &n_tiles, &total, &G, &nx);
+  decode_shape(M, N, K, sms, decode_half_stages(decode_nx(M)), &n_tiles, &total, &G, &nx);
   return decode_workspace_bytes(n_tiles, G, nx);
 }
 
@@ -739,7 +751,7 @@ fp8q_status fp8_linear(const uint8_t* Xq, const float* x_scale, const uint8_t* W
   if (M <= kDecodeMaxM) {
     int n_tiles, G, nx;
     int64_t total;
-    decode_shape(M, N, K, sms, &n_tiles, &total, &G, &nx);
+    decode_shape(M, N, K, sms, decode_half_stages(decode_nx(M)), &n_tiles, &total, &G, &nx);
     if (!workspace || workspace_bytes < decode_workspace_bytes(n_tiles, G, nx)) return FP8Q_ERR_INVALID_ARG;
     if (!aligned(workspace, 16)) return FP8Q_ERR_MISALIGNED;
     CUtensorMap tw, tx;
@@ -912,7 +924,7 @@ size_t fp8_linear_w8a16_workspace_size(int64_t M, int64_t N, int64_t K) {
   if (current_device(&dev, &sms) != FP8Q_OK) return 0;
   int n_tiles, G, nx;
   int64_t total;
-  decode_shape(M, N, K, sms, &n_tiles, &total, &G, &nx);
+  decode_shape(M, N, K, sms, false, &n_tiles, &total, &G, &nx);
   return decode_workspace_bytes(n_tiles, G, nx);
 }
 
@@ -948,7 +960,7 @@ fp8q_status fp8_linear_w8a16(const void* X_bf16, int64_t ldx, const uint8_t* Wq,
   }
   int n_tiles, G, nx;
   int64_t total;
-  decode_shape(M, N, K, sms, &n_tiles, &total, &G, &nx);
+  decode_shape(M, N, K, sms, false, &n_tiles, &total, &G, &nx);
   if (!workspace || workspace_bytes < decode_workspace_bytes(n_tiles, G, nx)) return FP8Q_ERR_INVALID_ARG;
   if (!aligned(workspace, 16)) return FP8Q_ERR_MISALIGNED;
   CUtensorMap tw, tx;
@@ -1076,7 +1088,7 @@ fp8q_status fp8_linear_noalloc(const uint8_t* Xq, const float* x_scale, const ui
   if ((st = current_device(&dev, &sms)) != FP8Q_OK) return st;
   int n_tiles, G, nx;
   int64_t total;
-  decode_shape(M, N, K, sms, &n_tiles, &total, &G, &nx);
+  decode_shape(M, N, K, sms, decode_half_stages(decode_nx(M)), &n_tiles, &total, &G, &nx);
   if (decode_workspace_bytes(n_tiles, G, nx) > kNoAllocScratchBytes) return FP8Q_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   if ((st = noalloc_scratch(dev, &scratch)) != FP8Q_OK) return st;

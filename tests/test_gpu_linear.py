@@ -161,6 +161,18 @@ def test_decode_channel_ragged(M, N, K):
     check_full(M, N, K, fq.CHANNEL_TOKEN, seed=N)
 
 
+@pytest.mark.parametrize("M,N,K,mode", [
+    (1, 10240, 1024, fq.CHANNEL_TOKEN),    # 80 tiles, 8 K blocks: 160 CTAs of half a tile each
+    (16, 11776, 512, fq.CHANNEL_TOKEN),    # 92 tiles: 184 CTAs (the rule's upper edge on 148 SMs)
+    (8, 10240, 1152, fq.CHANNEL_TOKEN),    # 9 K blocks (odd): one CTA per SM, ranges cross tiles
+    (1, 10240, 1024, fq.BLOCK128),         # block scales on 160 CTAs, summed by the reduction kernel
+])
+def test_decode_half_tile_grid(M, N, K, mode):
+    # two CTAs per SM for 16-token tiles: where twice the tile count is a
+    # little over the SM count, every CTA streams exactly half a tile
+    check_full(M, N, K, mode, seed=N + K)
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 272, 384), (16, 1024, 2048), (40, 512, 1024), (64, 256, 128)])
 def test_decode_block(M, N, K):
     check_full(M, N, K, fq.BLOCK128, seed=K)

@@ -259,12 +259,14 @@ bool decode_half_stages(int nx);
 
 // Stream-K split of a small-M problem: n_tiles weight tiles of 128 rows, KB K
 // blocks each, over G CTAs, one per SM.  Where the kernel is built for two
-// CTAs per SM (`two_per_sm`), KB is even and twice the tile count lies
-// between the SM count and 5/4 of it, G = 2 * n_tiles instead: every CTA
-// streams exactly half a tile.  Measured on the Llama-3.1-70B qkv_proj (80
-// tiles: 160 CTAs of 32 K blocks instead of 148 of 34-35 whose ranges cross
-// tiles), 0.59 -> 0.62 of HBM at M = 1 and 0.58 -> 0.61 at M = 8; the other
-// 70B decode shapes do not take it.
+// CTAs per SM (`two_per_sm`), G = c * n_tiles instead for the smallest c >= 2
+// that divides KB and gives more CTAs than SMs but at most two per SM: every
+// CTA streams exactly 1/c of one tile.  Measured on the Llama-3.1-70B decode
+// shapes against one CTA per SM (ranges that cross tiles): qkv_proj (80
+// tiles, c = 2: 160 CTAs of 32 K blocks) 0.59 -> 0.62 of HBM at M = 1, 0.58
+// -> 0.61 at M = 8; down_proj (64 tiles of 224 K blocks, c = 4: 256 CTAs of
+// 56) 0.74 -> 0.77 at M = 1, 0.74 -> 0.76 at M = 8; gate/up (224 tiles) take
+// no c.
 void decode_shape(int64_t M, int64_t N, int64_t K, int sms, bool two_per_sm, int* n_tiles, int64_t* total, int* G,
                   int* nx) {
   const int KB = static_cast<int>((K + 127) / 128);
@@ -272,7 +274,12 @@ void decode_shape(int64_t M, int64_t N, int64_t K, int sms, bool two_per_sm, int
   *total = static_cast<int64_t>(*n_tiles) * KB;
   *G = static_cast<int>(*total < sms ? *total : sms);
   *nx = decode_nx(M);
-  if (two_per_sm && KB % 2 == 0 && 2 * *n_tiles > sms && 8 * *n_tiles <= 5 * sms) *G = 2 * *n_tiles;
+  if (two_per_sm)
+    for (int c = 2; c * *n_tiles <= 2 * sms; ++c)
+      if (c * *n_tiles > sms && KB % c == 0) {
+        *G = c * *n_tiles;
+        break;
+      }
 }
 
 // Decode workspace: [n_tiles][4] arrival counters, padded to 16 bytes, then

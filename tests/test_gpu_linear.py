@@ -163,13 +163,17 @@ def test_decode_channel_ragged(M, N, K):
 
 @pytest.mark.parametrize("M,N,K,mode", [
     (1, 10240, 1024, fq.CHANNEL_TOKEN),    # 80 tiles, 8 K blocks: 160 CTAs of half a tile each
-    (16, 11776, 512, fq.CHANNEL_TOKEN),    # 92 tiles: 184 CTAs (the rule's upper edge on 148 SMs)
-    (8, 10240, 1152, fq.CHANNEL_TOKEN),    # 9 K blocks (odd): one CTA per SM, ranges cross tiles
+    (16, 11776, 512, fq.CHANNEL_TOKEN),    # 92 tiles: 184 CTAs of half a tile
+    (8, 8192, 1536, fq.CHANNEL_TOKEN),     # 64 tiles, 12 K blocks: 192 CTAs of a third of a tile
+    (1, 8192, 512, fq.CHANNEL_TOKEN),      # 64 tiles, 4 K blocks (3 does not divide): 256 CTAs of one K block
+    (8, 10240, 1152, fq.CHANNEL_TOKEN),    # 80 tiles, 9 K blocks (odd): 240 CTAs of a third of a tile
+    (8, 10240, 896, fq.CHANNEL_TOKEN),     # 7 K blocks: no c divides them at two CTAs per SM, one CTA per SM
     (1, 10240, 1024, fq.BLOCK128),         # block scales on 160 CTAs, summed by the reduction kernel
 ])
-def test_decode_half_tile_grid(M, N, K, mode):
-    # two CTAs per SM for 16-token tiles: where twice the tile count is a
-    # little over the SM count, every CTA streams exactly half a tile
+def test_decode_tile_aligned_grid(M, N, K, mode):
+    # two CTAs per SM for 16-token tiles: where c CTAs per weight tile (c
+    # dividing the K blocks) fill the SMs at no more than two per SM, every
+    # CTA streams exactly 1/c of one tile
     check_full(M, N, K, mode, seed=N + K)
 
 

@@ -61,8 +61,9 @@ def T():
 
 # Shapes whose CTA 0 comes back to the withheld slot (8 slots): channel mode
 # with K = 128 (every step its own tile, 16 tiles per CTA on 148 SMs), and
-# block mode with 16 K blocks per CTA.
-CASES = [(4, 128 * 148 * 16, 128, fq.CHANNEL_TOKEN), (16, 128 * 148, 2048, fq.BLOCK128)]
+# block mode with 16 K blocks per CTA (148 tiles of 32 K blocks: two CTAs per
+# tile, 296 in all, with 16-token tiles built for two CTAs per SM).
+CASES = [(4, 128 * 148 * 16, 128, fq.CHANNEL_TOKEN), (16, 128 * 148, 4096, fq.BLOCK128)]
 # Two K blocks per tile, 12 or 13 steps per CTA on 148 SMs: CTA 0's first
 # segment is the first half of a tile that CTA 1 finishes, and CTA 0 has 7
 # segments, so its MMA warp never waits for a slot: only the epilogue's wait
